@@ -1,0 +1,208 @@
+"""CPU oracle for the HSTU layer forward (fp64).  TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` / ``--impl reference`` legs of
+``bench.py`` may import this package.  The product (``hstu_sequential_transduction_layer_b200``)
+never imports it and has no CPU fallback.
+
+Two independent implementations live here:
+
+* ``hstu_oracle.c`` -- the definition written out as plain fp64 loops (OpenMP over independent rows),
+  loaded through ctypes.  This is *the* oracle.
+* ``dense_ref.py``  -- a numpy fp64 restatement of the dense, padded HSTULayer sketch of
+  "4.4 推荐模型的 Scaling" (with its input LayerNorm removed and the bucketed bias filled in per
+  pair).  It exists only to pin the C oracle on tiny inputs.
+
+Parity pins of the C oracle (closed forms, invariants, brute force) are in ``tests/test_oracle_*.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional, Sequence
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hstu_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle with gcc (-O2, no fast-math, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+                               "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def bind(path: str):
+    """Load a compiled oracle library from `path` and declare its signatures."""
+    lib = ctypes.CDLL(path)
+    i64, i32, dp, ip = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p
+    f64 = ctypes.c_double
+    lib.oracle_layer_fwd.argtypes = [i64, ip, i32, i32, i32, i32, dp, ip, dp, dp, dp, dp, dp,
+                                     dp, dp, i32, dp, i32, dp, f64, f64, dp, dp, dp, dp]
+    lib.oracle_layer_fwd.restype = ctypes.c_int
+    lib.oracle_layer_rows.argtypes = [i64, ip, i32, i32, i32, i32, dp, ip, dp, dp, dp, dp, dp,
+                                      dp, dp, i32, dp, i32, dp, f64, f64, ip, i64, dp, dp]
+    lib.oracle_layer_rows.restype = ctypes.c_int
+    lib.oracle_token_embed.argtypes = [i64, i32, ip, ip, dp, dp, dp]
+    lib.oracle_token_embed.restype = None
+    lib.oracle_round_bf16.argtypes = [f64]
+    lib.oracle_round_bf16.restype = f64
+    lib.oracle_time_bucket.argtypes = [i64, i64, i32]
+    lib.oracle_time_bucket.restype = i32
+    lib.oracle_pos_bucket.argtypes = [i64, i64, i32]
+    lib.oracle_pos_bucket.restype = i32
+    lib.oracle_num_threads.argtypes = []
+    lib.oracle_num_threads.restype = ctypes.c_int
+    return lib
+
+
+def _load(lib=None):
+    global _lib
+    if lib is not None:
+        return lib
+    if _lib is None:
+        _lib = bind(build())
+    return _lib
+
+
+def _d(a: Optional[np.ndarray]):
+    """Contiguous fp64 copy (exact widening of the caller's fp32 / bf16-valued arrays)."""
+    if a is None:
+        return None
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _i(a: Optional[np.ndarray]):
+    if a is None:
+        return None
+    return np.ascontiguousarray(a, dtype=np.int64)
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def time_bucket(ti: int, tj: int, n_time_buckets: int) -> int:
+    return int(_load().oracle_time_bucket(int(ti), int(tj), int(n_time_buckets)))
+
+
+def pos_bucket(i: int, j: int, n_pos_buckets: int) -> int:
+    return int(_load().oracle_pos_bucket(int(i), int(j), int(n_pos_buckets)))
+
+
+def round_bf16(x: float) -> float:
+    return float(_load().oracle_round_bf16(float(x)))
+
+
+def layer_fwd(seq_offsets, X, W1, b1, W2, b2, ln_w, ln_b, *, num_heads: int, d_qk: int, d_v: int,
+              timestamps=None, pos_table=None, time_table=None, alibi_slopes=None,
+              scale: float, ln_eps: float = 1e-5, return_intermediates: bool = False, lib=None):
+    """Y = f2(LayerNorm(AV) * U) + X for one layer over a jagged batch (all rows).
+
+    With ``return_intermediates`` it also returns UVQK [T, n1], AV [T, H*dv] and G [T, H*dv].
+    ``lib`` selects another compiled copy of the oracle (the tests' planted-mistake variants)."""
+    lib = _load(lib)
+    off = _i(seq_offsets)
+    B = len(off) - 1
+    X = _d(X)
+    T, d = X.shape
+    H = int(num_heads)
+    n1 = 2 * H * d_v + 2 * H * d_qk
+    args = [_d(W1), _d(b1), _d(W2), _d(b2), _d(ln_w), _d(ln_b)]
+    ts = _i(timestamps)
+    pos = _d(pos_table)
+    tim = _d(time_table)
+    ali = _d(alibi_slopes)
+    P = 0 if pos is None else pos.shape[1]
+    Tb = 0 if tim is None else tim.shape[1]
+    Y = np.empty((T, d), np.float64)
+    uvqk = np.empty((T, n1), np.float64) if return_intermediates else None
+    av = np.empty((T, H * d_v), np.float64) if return_intermediates else None
+    g = np.empty((T, H * d_v), np.float64) if return_intermediates else None
+    rc = lib.oracle_layer_fwd(B, _p(off), d, H, d_qk, d_v, _p(X), _p(ts), *[_p(a) for a in args],
+                              _p(pos), P, _p(tim), Tb, _p(ali), float(scale), float(ln_eps),
+                              _p(Y), _p(uvqk), _p(av), _p(g))
+    if rc != 0:
+        raise MemoryError("oracle_layer_fwd failed")
+    if return_intermediates:
+        return Y, uvqk, av, g
+    return Y
+
+
+def layer_rows(seq_offsets, X, W1, b1, W2, b2, ln_w, ln_b, rows: Sequence[int], *, num_heads: int,
+               d_qk: int, d_v: int, timestamps=None, pos_table=None, time_table=None,
+               alibi_slopes=None, scale: float, ln_eps: float = 1e-5):
+    """The layer evaluated on a sample of output rows only (global token indices).
+
+    Returns (Y_rows [n, d], AV_rows [n, H*dv]).  Each row equals the corresponding row of
+    ``layer_fwd`` (same arithmetic in the same order)."""
+    lib = _load()
+    off = _i(seq_offsets)
+    B = len(off) - 1
+    X = _d(X)
+    T, d = X.shape
+    H = int(num_heads)
+    rows = _i(np.asarray(rows))
+    args = [_d(W1), _d(b1), _d(W2), _d(b2), _d(ln_w), _d(ln_b)]
+    ts = _i(timestamps)
+    pos = _d(pos_table)
+    tim = _d(time_table)
+    ali = _d(alibi_slopes)
+    P = 0 if pos is None else pos.shape[1]
+    Tb = 0 if tim is None else tim.shape[1]
+    Y = np.empty((len(rows), d), np.float64)
+    av = np.empty((len(rows), H * d_v), np.float64)
+    rc = lib.oracle_layer_rows(B, _p(off), d, H, d_qk, d_v, _p(X), _p(ts), *[_p(a) for a in args],
+                               _p(pos), P, _p(tim), Tb, _p(ali), float(scale), float(ln_eps),
+                               _p(rows), len(rows), _p(Y), _p(av))
+    if rc != 0:
+        raise MemoryError("oracle_layer_rows failed")
+    return Y, av
+
+
+def token_embed(item_ids, action_ids, item_table, action_table) -> np.ndarray:
+    """X = bf16(E_item[id] + E_act[a]) for every token, as fp64 values (GenRank token assembly).
+
+    ``item_table`` may be given as just the rows referenced (pass remapped ids accordingly)."""
+    lib = _load()
+    ii = _i(item_ids)
+    ai = _i(action_ids)
+    it = _d(item_table)
+    at = _d(action_table)
+    T = len(ii)
+    d = it.shape[1]
+    X = np.empty((T, d), np.float64)
+    lib.oracle_token_embed(T, d, _p(ii), _p(ai), _p(it), _p(at), _p(X))
+    return X
+
+
+def layer_fwd_inputs(inp, layer: int = 0, X=None, return_intermediates: bool = False):
+    """Convenience: run one layer of a ``workloads.Inputs`` (X defaults to the workload's X)."""
+    w = inp.workload
+    p = inp.layers[layer]
+    return layer_fwd(inp.seq_offsets, inp.X if X is None else X, p.W1, p.b1, p.W2, p.b2, p.ln_w,
+                     p.ln_b, num_heads=w.num_heads, d_qk=w.head_dim, d_v=w.head_dim,
+                     timestamps=inp.timestamps, pos_table=inp.pos_table,
+                     time_table=inp.time_table, alibi_slopes=inp.alibi_slopes, scale=inp.scale,
+                     ln_eps=inp.ln_eps, return_intermediates=return_intermediates)
+
+
+def layer_rows_inputs(inp, rows, layer: int = 0, X=None):
+    w = inp.workload
+    p = inp.layers[layer]
+    return layer_rows(inp.seq_offsets, inp.X if X is None else X, p.W1, p.b1, p.W2, p.b2, p.ln_w,
+                      p.ln_b, rows, num_heads=w.num_heads, d_qk=w.head_dim, d_v=w.head_dim,
+                      timestamps=inp.timestamps, pos_table=inp.pos_table,
+                      time_table=inp.time_table, alibi_slopes=inp.alibi_slopes, scale=inp.scale,
+                      ln_eps=inp.ln_eps)

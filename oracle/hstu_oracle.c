@@ -1,0 +1,301 @@
+/*
+ * HSTU layer forward -- CPU oracle in plain C, fp64 throughout.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the slow, obviously-correct definition that the CUDA path
+ * is checked against.  It is used by the tests, by `__graft_entry__.smoke()` and by the CPU-baseline
+ * leg of `bench.py`, and by nothing else.  It shares no code, header, table or helper with the CUDA
+ * path and includes nothing from it.
+ *
+ * What it computes (per layer, for every sequence s of a jagged batch and local token indices
+ * i, j in [0, n_s)), following "Actions Speak Louder than Words" (paper notes), section 3.1,
+ * Eqs. 1-3, and the HSTU-layer section of "4.4 推荐模型的 Scaling" (equations and the HSTULayer
+ * sketch):
+ *
+ *   Eq. 1   Z = X W1 + b1;  U | V | Q | K = SiLU(Z)         (column blocks, in that order)
+ *   Eq. 2   AV_i = sum_{j<=i} scale * SiLU(q_i . k_j + bias(i, j)) * v_j     (per head, no softmax)
+ *   Eq. 3   G_i = LayerNorm(AV_i) * U_i;   Y_i = G_i W2 + b2 + X_i           (residual between layers)
+ *
+ * bias(i, j) is either the relative attention bias rab^{p,t}
+ *   pos[h][min(i-j, P-1)] + time[h][min(Tb-1, floor(log2(1 + max(t_i - t_j, 0))))]
+ * or the GenRank ALiBi bias  -m_h * (i - j).
+ *
+ * Readings of the pages that this file fixes (the pages leave them open):
+ *   - `scale` multiplies SiLU's output (the sketch divides by a constant after SiLU);
+ *   - the causal mask is the summation range j <= i (the sketch zeroes masked weights after SiLU);
+ *   - LayerNorm spans all H*dv columns with biased variance and epsilon `ln_eps`;
+ *   - the time bucket is computed exactly on integer seconds (highest set bit of 1 + delta);
+ *   - the rab tables are per head; the position index is i - j clamped to P-1.
+ *
+ * Layouts: every matrix is row-major.  X [T, d], W1 [d, n1] (d_in x d_out) with
+ * n1 = 2*H*dv + 2*H*dqk, UVQK [T, n1] with columns [U: H*dv | V: H*dv | Q: H*dqk | K: H*dqk], each
+ * block head-major (head h owns columns h*hd .. h*hd+hd-1), AV and G [T, H*dv], W2 [H*dv, d],
+ * Y [T, d].  Tables: pos [H, P], time [H, Tb], alibi slopes [H].
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* SiLU(x) = x * sigmoid(x) = x / (1 + e^{-x}).  phi_1 and phi_2 of Eqs. 1-2. */
+static double silu(double x) { return x / (1.0 + exp(-x)); }
+
+/* floor(log2(v)) for v >= 1: the index of the highest set bit. */
+static int32_t floor_log2_u64(uint64_t v) {
+  int32_t b = 0;
+  while (v > 1) {
+    v >>= 1;
+    b++;
+  }
+  return b;
+}
+
+int32_t oracle_time_bucket(int64_t ti, int64_t tj, int32_t n_time_buckets) {
+  int64_t delta = ti - tj;
+  if (delta < 0) delta = 0;
+  int32_t b = floor_log2_u64((uint64_t)delta + 1u);
+  return b < n_time_buckets - 1 ? b : n_time_buckets - 1;
+}
+
+int32_t oracle_pos_bucket(int64_t i, int64_t j, int32_t n_pos_buckets) {
+  int64_t p = i - j;
+  if (p < 0) p = 0;
+  return p < n_pos_buckets - 1 ? (int32_t)p : n_pos_buckets - 1;
+}
+
+/* bias(i, j) for head h; i, j are local indices, ts points at the sequence's first timestamp. */
+static double bias_at(int32_t h, int64_t i, int64_t j, const int64_t* ts,
+                      const double* pos_table, int32_t P, const double* time_table, int32_t Tb,
+                      const double* alibi_slopes) {
+  if (alibi_slopes) return -alibi_slopes[h] * (double)(i - j);
+  double b = 0.0;
+  if (pos_table) b += pos_table[(int64_t)h * P + oracle_pos_bucket(i, j, P)];
+  if (time_table) b += time_table[(int64_t)h * Tb + oracle_time_bucket(ts[i], ts[j], Tb)];
+  return b;
+}
+
+/* ---------------------------------------------------------------------------------------------
+ * Eq. 1: one row of the pointwise projection, columns [c0, c1):  out[c] = SiLU(b1[c] + sum_k x[k] W1[k][c]).
+ * f1 is one affine map (weight W1, bias b1); phi_1 is SiLU; the result splits into U, V, Q, K.
+ * --------------------------------------------------------------------------------------------- */
+static void f1_row_cols(int32_t d, int32_t n1, const double* x, const double* W1, const double* b1,
+                        int32_t c0, int32_t c1, double* out /* indexed by c */) {
+  for (int32_t c = c0; c < c1; c++) out[c] = b1 ? b1[c] : 0.0;
+  for (int32_t k = 0; k < d; k++) {
+    const double xk = x[k];
+    const double* w = W1 + (int64_t)k * n1;
+    for (int32_t c = c0; c < c1; c++) out[c] += xk * w[c];
+  }
+  for (int32_t c = c0; c < c1; c++) out[c] = silu(out[c]);
+}
+
+void oracle_f1(int64_t T, int32_t d, int32_t n1, const double* X, const double* W1,
+               const double* b1, double* uvqk) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; t++) f1_row_cols(d, n1, X + t * d, W1, b1, 0, n1, uvqk + t * n1);
+}
+
+/* ---------------------------------------------------------------------------------------------
+ * Eq. 2: pointwise aggregated attention for one output row.
+ * AV_i[h] = sum_{j=0}^{i} scale * SiLU(q_i[h] . k_j[h] + bias_h(i, j)) * v_j[h].
+ * `uvqk_seq` points at the sequence's first row (row stride n1).
+ * --------------------------------------------------------------------------------------------- */
+static void attention_row(int64_t i, int32_t H, int32_t dqk, int32_t dv, int32_t n1,
+                          const double* uvqk_seq, const int64_t* ts, const double* pos_table,
+                          int32_t P, const double* time_table, int32_t Tb,
+                          const double* alibi_slopes, double scale, double* av_row) {
+  const int32_t offV = H * dv, offQ = 2 * H * dv, offK = 2 * H * dv + H * dqk;
+  for (int32_t h = 0; h < H; h++) {
+    double* acc = av_row + (int64_t)h * dv;
+    for (int32_t c = 0; c < dv; c++) acc[c] = 0.0;
+    const double* q = uvqk_seq + i * n1 + offQ + (int64_t)h * dqk;
+    for (int64_t j = 0; j <= i; j++) {
+      const double* k = uvqk_seq + j * n1 + offK + (int64_t)h * dqk;
+      const double* v = uvqk_seq + j * n1 + offV + (int64_t)h * dv;
+      double s = 0.0;
+      for (int32_t c = 0; c < dqk; c++) s += q[c] * k[c];
+      s += bias_at(h, i, j, ts, pos_table, P, time_table, Tb, alibi_slopes);
+      const double a = scale * silu(s);
+      for (int32_t c = 0; c < dv; c++) acc[c] += a * v[c];
+    }
+  }
+}
+
+void oracle_attention(int64_t B, const int64_t* seq_offsets, int32_t H, int32_t dqk, int32_t dv,
+                      const double* uvqk, const int64_t* timestamps, const double* pos_table,
+                      int32_t P, const double* time_table, int32_t Tb, const double* alibi_slopes,
+                      double scale, double* av) {
+  const int32_t n1 = 2 * H * dv + 2 * H * dqk;
+  const int64_t T = seq_offsets[B];
+  /* rows are independent; the row -> sequence map is a search over the offsets */
+#pragma omp parallel for schedule(dynamic, 16)
+  for (int64_t r = 0; r < T; r++) {
+    int64_t s = 0;
+    while (seq_offsets[s + 1] <= r) s++;
+    const int64_t start = seq_offsets[s];
+    attention_row(r - start, H, dqk, dv, n1, uvqk + start * n1,
+                  timestamps ? timestamps + start : NULL, pos_table, P, time_table, Tb,
+                  alibi_slopes, scale, av + r * (int64_t)H * dv);
+  }
+}
+
+/* ---------------------------------------------------------------------------------------------
+ * Eq. 3, first half: G = LayerNorm(AV) * U.  Norm is a layer normalisation; the sketch normalises
+ * the full d-wide row.  Mean and biased variance over the H*dv columns.
+ * --------------------------------------------------------------------------------------------- */
+static void ln_gate_row(int32_t w, const double* av, const double* u, const double* ln_w,
+                        const double* ln_b, double eps, double* g) {
+  double mean = 0.0;
+  for (int32_t c = 0; c < w; c++) mean += av[c];
+  mean /= (double)w;
+  double var = 0.0;
+  for (int32_t c = 0; c < w; c++) var += (av[c] - mean) * (av[c] - mean);
+  var /= (double)w;
+  const double rstd = 1.0 / sqrt(var + eps);
+  for (int32_t c = 0; c < w; c++) g[c] = ((av[c] - mean) * rstd * ln_w[c] + ln_b[c]) * u[c];
+}
+
+void oracle_ln_gate(int64_t T, int32_t H, int32_t dqk, int32_t dv, const double* av,
+                    const double* uvqk, const double* ln_w, const double* ln_b, double eps,
+                    double* g) {
+  const int32_t n1 = 2 * H * dv + 2 * H * dqk, w = H * dv;
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; t++)
+    ln_gate_row(w, av + t * w, uvqk + t * n1 /* U is block 0 */, ln_w, ln_b, eps, g + t * w);
+}
+
+/* ---------------------------------------------------------------------------------------------
+ * Eq. 3, second half, plus the residual connection between layers: Y = G W2 + b2 + X.
+ * --------------------------------------------------------------------------------------------- */
+static void f2_row(int32_t w, int32_t d, const double* g, const double* W2, const double* b2,
+                   const double* x, double* y) {
+  for (int32_t c = 0; c < d; c++) y[c] = b2 ? b2[c] : 0.0;
+  for (int32_t k = 0; k < w; k++) {
+    const double gk = g[k];
+    const double* wr = W2 + (int64_t)k * d;
+    for (int32_t c = 0; c < d; c++) y[c] += gk * wr[c];
+  }
+  for (int32_t c = 0; c < d; c++) y[c] += x[c];
+}
+
+void oracle_f2(int64_t T, int32_t w, int32_t d, const double* g, const double* W2,
+               const double* b2, const double* X, double* Y) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; t++) f2_row(w, d, g + t * w, W2, b2, X + t * d, Y + t * d);
+}
+
+/* ---------------------------------------------------------------------------------------------
+ * The whole layer.  Intermediates are returned when the caller passes buffers for them.
+ * Returns 0, or -1 on an allocation failure.
+ * --------------------------------------------------------------------------------------------- */
+int oracle_layer_fwd(int64_t B, const int64_t* seq_offsets, int32_t d, int32_t H, int32_t dqk,
+                     int32_t dv, const double* X, const int64_t* timestamps, const double* W1,
+                     const double* b1, const double* W2, const double* b2, const double* ln_w,
+                     const double* ln_b, const double* pos_table, int32_t P,
+                     const double* time_table, int32_t Tb, const double* alibi_slopes,
+                     double scale, double ln_eps, double* Y, double* uvqk_out, double* av_out,
+                     double* g_out) {
+  const int64_t T = seq_offsets[B];
+  const int32_t n1 = 2 * H * dv + 2 * H * dqk, w = H * dv;
+  double* uvqk = uvqk_out ? uvqk_out : (double*)malloc(sizeof(double) * (size_t)(T * n1 + 1));
+  double* av = av_out ? av_out : (double*)malloc(sizeof(double) * (size_t)(T * w + 1));
+  double* g = g_out ? g_out : (double*)malloc(sizeof(double) * (size_t)(T * w + 1));
+  if (!uvqk || !av || !g) return -1;
+  oracle_f1(T, d, n1, X, W1, b1, uvqk);
+  oracle_attention(B, seq_offsets, H, dqk, dv, uvqk, timestamps, pos_table, P, time_table, Tb,
+                   alibi_slopes, scale, av);
+  oracle_ln_gate(T, H, dqk, dv, av, uvqk, ln_w, ln_b, ln_eps, g);
+  oracle_f2(T, w, d, g, W2, b2, X, Y);
+  if (!uvqk_out) free(uvqk);
+  if (!av_out) free(av);
+  if (!g_out) free(g);
+  return 0;
+}
+
+/* ---------------------------------------------------------------------------------------------
+ * The layer on a sample of output rows (global token indices `rows[0..n_rows)`).  By causality,
+ * output row i of sequence s needs U and Q of row i and V and K of rows 0..i of s only, so each
+ * sampled row is evaluated exactly as oracle_layer_fwd would, computing just what it reads.
+ * Y_rows is [n_rows, d]; av_rows (nullable) is [n_rows, H*dv].
+ * --------------------------------------------------------------------------------------------- */
+int oracle_layer_rows(int64_t B, const int64_t* seq_offsets, int32_t d, int32_t H, int32_t dqk,
+                      int32_t dv, const double* X, const int64_t* timestamps, const double* W1,
+                      const double* b1, const double* W2, const double* b2, const double* ln_w,
+                      const double* ln_b, const double* pos_table, int32_t P,
+                      const double* time_table, int32_t Tb, const double* alibi_slopes,
+                      double scale, double ln_eps, const int64_t* rows, int64_t n_rows,
+                      double* Y_rows, double* av_rows) {
+  const int32_t n1 = 2 * H * dv + 2 * H * dqk, w = H * dv;
+  const int32_t offV = H * dv, offQ = 2 * H * dv, offK = 2 * H * dv + H * dqk;
+  for (int64_t s = 0; s < B; s++) {
+    const int64_t start = seq_offsets[s], n = seq_offsets[s + 1] - start;
+    int64_t last = -1; /* the largest sampled local index in this sequence */
+    for (int64_t r = 0; r < n_rows; r++)
+      if (rows[r] >= start && rows[r] < start + n && rows[r] - start > last) last = rows[r] - start;
+    if (last < 0) continue;
+    /* the sequence's rows 0..last: V and K for all of them, U and Q only where sampled */
+    double* uvqk = (double*)calloc((size_t)((last + 1) * n1), sizeof(double));
+    if (!uvqk) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j <= last; j++) {
+      f1_row_cols(d, n1, X + (start + j) * d, W1, b1, offV, offQ, uvqk + j * n1); /* V */
+      f1_row_cols(d, n1, X + (start + j) * d, W1, b1, offK, n1, uvqk + j * n1);   /* K */
+    }
+    for (int64_t r = 0; r < n_rows; r++) {
+      if (rows[r] < start || rows[r] >= start + n) continue;
+      const int64_t i = rows[r] - start;
+      double* ui = (double*)malloc(sizeof(double) * (size_t)n1);
+      double* avr = (double*)malloc(sizeof(double) * (size_t)w);
+      double* g = (double*)malloc(sizeof(double) * (size_t)w);
+      if (!ui || !avr || !g) return -1;
+      f1_row_cols(d, n1, X + (start + i) * d, W1, b1, 0, offV, ui);                 /* U */
+      f1_row_cols(d, n1, X + (start + i) * d, W1, b1, offQ, offK, uvqk + i * n1);   /* Q */
+      attention_row(i, H, dqk, dv, n1, uvqk, timestamps ? timestamps + start : NULL, pos_table,
+                    P, time_table, Tb, alibi_slopes, scale, avr);
+      ln_gate_row(w, avr, ui, ln_w, ln_b, ln_eps, g);
+      f2_row(w, d, g, W2, b2, X + (start + i) * d, Y_rows + r * d);
+      if (av_rows) memcpy(av_rows + r * w, avr, sizeof(double) * (size_t)w);
+      free(ui);
+      free(avr);
+      free(g);
+    }
+    free(uvqk);
+  }
+  return 0;
+}
+
+/* ---------------------------------------------------------------------------------------------
+ * Action-oriented token assembly (GenRank, "item-action organisation"): the token at each
+ * position is the sum of its item embedding and its action embedding, stored as bf16.
+ * --------------------------------------------------------------------------------------------- */
+
+/* Round to the nearest bf16 value (8 significant bits, ties to even), by definition: scale to an
+ * integer number of bf16 quanta and round half to even with rint() (default rounding mode). */
+double oracle_round_bf16(double x) {
+  if (x == 0.0 || !isfinite(x)) return x;
+  int e;
+  frexp(x, &e);               /* x = m * 2^e, 0.5 <= |m| < 1 */
+  int q = e - 8;              /* quantum 2^(e-8) keeps 8 significant bits */
+  if (q < -133) q = -133;     /* subnormal range: fixed quantum 2^-133 */
+  return ldexp(rint(ldexp(x, -q)), q);
+}
+
+void oracle_token_embed(int64_t T, int32_t d, const int64_t* item_ids, const int64_t* action_ids,
+                        const double* item_table, const double* action_table, double* X) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; t++)
+    for (int32_t c = 0; c < d; c++)
+      X[t * d + c] = oracle_round_bf16(item_table[item_ids[t] * d + c] +
+                                       action_table[action_ids[t] * d + c]);
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}

@@ -1,0 +1,117 @@
+"""Planted mistakes in the oracle must be caught by its pins (CPU only).
+
+Each case copies ``oracle/hstu_oracle.c``, plants one plausible mistake by a textual substitution (a
+flipped sign, a dropped term, a wrong index or range, transposed operands), compiles the copy into a
+temporary directory and runs the pins that do not depend on the oracle itself: the dense padded
+restatement of the sketch, the closed forms and causality.  The test passes only if every mutant
+fails at least one of them and the unmodified source passes all of them.
+"""
+import os
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle.dense_ref import hstu_layer_dense
+from workloads import random_case
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "hstu_oracle.c")
+
+MUTANTS = {
+    "silu_sign": ("return x / (1.0 + exp(-x));", "return x / (1.0 + exp(x));"),
+    "bias_dropped": ("s += bias_at(", "s += 0.0 * bias_at("),
+    "diagonal_excluded": ("for (int64_t j = 0; j <= i; j++) {", "for (int64_t j = 0; j < i; j++) {"),
+    "q_k_swapped": ("const double* q = uvqk_seq + i * n1 + offQ", "const double* q = uvqk_seq + i * n1 + offK"),
+    "u_is_v": ("uvqk + t * n1 /* U is block 0 */", "uvqk + t * n1 + H * dv"),
+    "pos_direction": ("int64_t p = i - j;", "int64_t p = j - i;"),
+    "time_bucket_off_by_one": ("floor_log2_u64((uint64_t)delta + 1u)", "floor_log2_u64((uint64_t)delta + 2u)"),
+    "time_delta_sign": ("int64_t delta = ti - tj;", "int64_t delta = tj - ti;"),
+    "unbiased_variance": ("var /= (double)w;", "var /= (double)(w - 1);"),
+    "eps_outside_sqrt": ("1.0 / sqrt(var + eps)", "1.0 / (sqrt(var) + eps)"),
+    "ln_w_b_swapped": ("* ln_w[c] + ln_b[c])", "* ln_b[c] + ln_w[c])"),
+    "residual_dropped": ("for (int32_t c = 0; c < d; c++) y[c] += x[c];",
+                         "for (int32_t c = 0; c < d; c++) y[c] += 0.0 * x[c];"),
+    "b1_dropped": ("out[c] = b1 ? b1[c] : 0.0;", "out[c] = 0.0;"),
+    "b2_dropped": ("y[c] = b2 ? b2[c] : 0.0;", "y[c] = 0.0;"),
+    "scale_inside_silu": ("scale * silu(s)", "silu(scale * s)"),
+    "alibi_sign": ("return -alibi_slopes[h] * (double)(i - j);", "return alibi_slopes[h] * (double)(i - j);"),
+    "v_head_offset": ("offV + (int64_t)h * dv;", "offV;"),
+    "gate_missing": ("+ ln_b[c]) * u[c];", "+ ln_b[c]);"),
+}
+
+
+def _silu(x):
+    return x / (1.0 + np.exp(-x))
+
+
+def _pins_pass(lib) -> bool:
+    """True when every independent pin holds for the given compiled oracle."""
+    def run(inp, **kw):
+        return _run_lib(inp, lib, **kw)
+
+    # dense restatement of the sketch on several small cases
+    for case in [dict(seed=1, lengths=[5], d=8, H=2, hd=4),
+                 dict(seed=2, lengths=[3, 16, 1], d=16, H=2, hd=8),
+                 dict(seed=4, lengths=[16, 9], d=8, H=1, hd=8, P=4, Tb=3),
+                 dict(seed=5, lengths=[11, 13], d=16, H=4, hd=4, alibi=True)]:
+        inp = random_case(**case)
+        w, p = inp.workload, inp.layers[0]
+        y = run(inp)
+        yd = hstu_layer_dense(inp.lengths, inp.X, p.W1, p.b1, p.W2, p.b2, p.ln_w, p.ln_b,
+                              num_heads=w.num_heads, d_qk=w.head_dim, d_v=w.head_dim,
+                              timestamps=inp.timestamps, pos_table=inp.pos_table,
+                              time_table=inp.time_table, alibi_slopes=inp.alibi_slopes,
+                              scale=inp.scale, ln_eps=inp.ln_eps)
+        if not np.max(np.abs(y - yd)) <= 1e-12 * max(1.0, np.max(np.abs(yd))):
+            return False
+    # closed form: Q = 0 and zero bias
+    inp = random_case(seed=11, lengths=[6, 10, 3], d=16, H=2, hd=8)
+    p = inp.layers[0]
+    p.W1[:, 32:48] = 0.0
+    p.b1[32:48] = 0.0
+    inp.pos_table[:] = 0.0
+    inp.time_table[:] = 0.0
+    X = inp.X.astype(np.float64)
+    U = _silu(X @ p.W1[:, :16].astype(np.float64) + p.b1[:16])
+    if not np.allclose(run(inp), (p.ln_b * U) @ p.W2.astype(np.float64) + p.b2 + X, rtol=1e-12, atol=1e-12):
+        return False
+    # causality
+    inp = random_case(seed=17, lengths=[12, 9], d=8, H=2, hd=4)
+    y0 = run(inp)
+    inp.X = inp.X.copy()
+    inp.X[6:12] += 3.0
+    if not np.array_equal(y0[:6], run(inp)[:6]):
+        return False
+    return True
+
+
+def _run_lib(inp, lib, **kw):
+    w, p = inp.workload, inp.layers[0]
+    return oracle.layer_fwd(inp.seq_offsets, inp.X, p.W1, p.b1, p.W2, p.b2, p.ln_w, p.ln_b,
+                            num_heads=w.num_heads, d_qk=w.head_dim, d_v=w.head_dim,
+                            timestamps=inp.timestamps, pos_table=inp.pos_table,
+                            time_table=inp.time_table, alibi_slopes=inp.alibi_slopes,
+                            scale=inp.scale, ln_eps=inp.ln_eps, lib=lib, **kw)
+
+
+def _compile(src_text: str, tmp_path, name: str):
+    c = tmp_path / f"{name}.c"
+    so = tmp_path / f"{name}.so"
+    c.write_text(src_text)
+    subprocess.check_call(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-o", str(so),
+                           str(c), "-lm"])
+    return oracle.bind(str(so))
+
+
+def test_unmodified_oracle_passes_the_independent_pins(tmp_path):
+    assert _pins_pass(_compile(open(SRC).read(), tmp_path, "orig"))
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(name, tmp_path):
+    src = open(SRC).read()
+    old, new = MUTANTS[name]
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    lib = _compile(src.replace(old, new), tmp_path, name)
+    assert not _pins_pass(lib), f"planted mistake {name} went unnoticed"
