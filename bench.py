@@ -1,0 +1,400 @@
+#!/usr/bin/env python3
+"""Throughput of the HSTU layer forward on B200: one JSON line on rank 0.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload long_seq] [--impl ours|reference]
+
+A step is one pass of the whole layer (f1 GEMM + SiLU + split, jagged attention with rab^{p,t},
+LayerNorm * U, f2 GEMM + residual) over one batch of the workload, with inputs resident in HBM.
+The default workload is `long_seq`: 8 sequences of 8192 tokens, d=512, 8 heads of 64, bf16 -- the
+encoder-efficiency shape of "Actions Speak Louder than Words" (paper notes, section 4.3), on
+synthetic seeded data.  Under torchrun every rank runs its own batch (sequences are independent;
+no collective on the data path), so the job's throughput is N x the per-rank batch over the slowest
+rank's device time ("scaling": "weak").
+
+`--impl reference` times the fp64 CPU oracle instead (the only reference implementation: the pages
+ship no code), on rank 0, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "HSTU layer fwd tokens/s; attention TFLOP/s as % of B200 BF16 dense peak"
+L2_FLUSH_BYTES = 256 << 20      # > 126 MB of L2
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def attention_flops(lengths, H, dqk, dv) -> float:
+    """Algorithmic attention FLOPs: 2*H*(dqk+dv) per causal pair (j <= i), masked half excluded."""
+    pairs = sum(int(n) * (int(n) + 1) // 2 for n in lengths)
+    return 2.0 * H * (dqk + dv) * pairs
+
+
+def gemm_flops(T, d, n1, wv):
+    return 2.0 * T * d * n1, 2.0 * T * wv * d
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = str(device_index)
+        try:  # nvidia-smi numbers GPUs by itself; address ours by its PCI bus id
+            import torch
+            p = torch.cuda.get_device_properties(device_index)
+            self.idx = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+        except Exception:
+            pass
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", self.idx, "-lms", "100"], stdout=open(self.path, "w"),
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        sm = []
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+            except ValueError:
+                pass
+            for k, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(k)
+        mx = rows[-1][2]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(mx) if mx.replace(".", "").isdigit() else mx,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------------------------
+# Our arm
+# ------------------------------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import hstu_sequential_transduction_layer_b200 as hstu
+    from workloads.device import to_device
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workloads.WORKLOADS[args.workload]
+    inp = workloads.make_inputs(w)
+    if w.token_embed:
+        raise SystemExit("bench.py times the layer on workloads with explicit X; "
+                         "use long_seq, retrieval or large")
+    H, hd, d = w.num_heads, w.head_dim, w.d_model
+    T = inp.T
+    D = to_device(inp, dev)
+    L = D["layers"][0]
+    max_len = int(inp.lengths.max())
+    shape = hstu.shape_for(D["X"], D["off"], H, hd, hd, max_len, D["pos"], D["tim"], inp.ln_eps)
+    n1 = 4 * d
+    wv = H * hd
+    uvqk = torch.empty((T, n1), dtype=torch.bfloat16, device=dev)
+    av = torch.empty((T, wv), dtype=torch.float32, device=dev)     # fp32 LayerNorm input
+    g = torch.empty((T, wv), dtype=torch.bfloat16, device=dev)
+    attn_ws = torch.empty(max(256, hstu.attention_workspace_size(shape)), dtype=torch.uint8,
+                          device=dev)
+    out = torch.empty_like(D["X"])
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        # the four entry points hstu_layer_fwd chains, with events between them
+        if evs:
+            evs[0].record(stream)
+        hstu.hstu_f1_fwd(shape, D["X"], L["W1"], L["b1"], uvqk, stream)
+        if evs:
+            evs[1].record(stream)
+        hstu.hstu_attention_fwd(shape, uvqk, D["off"], D["ts"], D["pos"], D["tim"], D["ali"],
+                                inp.scale, av, attn_ws, stream)
+        if evs:
+            evs[2].record(stream)
+        hstu.hstu_ln_gate_fwd(shape, av, uvqk, L["ln_w"], L["ln_b"], g, stream)
+        if evs:
+            evs[3].record(stream)
+        hstu.hstu_f2_fwd(shape, g, L["W2"], L["b2"], D["X"], out, stream)
+        if evs:
+            evs[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if hstu.device_status() != hstu.HSTU_OK:
+        raise SystemExit("device status error during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    launches0 = hstu.launch_count()
+    for k in range(args.steps):
+        flush.zero_()                      # L2 flush between timed steps (not timed)
+        step(evs[k])
+    torch.cuda.synchronize()
+    launches = hstu.launch_count() - launches0
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    per_kernel = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in evs])  # ms
+    step_ms = per_kernel.sum(axis=1)
+    total_ms = float(step_ms.sum())
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    if hstu.device_status() != hstu.HSTU_OK:
+        raise SystemExit("device status error in the timed region")
+
+    ms_per_step = total_ms / args.steps
+    tokens_per_s = world * T / (ms_per_step * 1e-3)
+    kern_ms = per_kernel.mean(axis=0)
+    peaks, peaks_src = load_peaks()
+    attn_fl = attention_flops(inp.lengths, H, hd, hd)
+    f1_fl, f2_fl = gemm_flops(T, d, n1, wv)
+    ln_bytes = 8.0 * wv * T          # AV (fp32) + U (bf16) read, G (bf16) written
+    tpk = peaks["bf16_tflops"]
+    kernels = {
+        "f1_gemm": {"ms": kern_ms[0], "TFLOP/s": f1_fl / kern_ms[0] / 1e9},
+        "attention": {"ms": kern_ms[1], "TFLOP/s": attn_fl / kern_ms[1] / 1e9},
+        "ln_gate": {"ms": kern_ms[2], "GB/s": ln_bytes / kern_ms[2] / 1e6},
+        "f2_gemm": {"ms": kern_ms[3], "TFLOP/s": f2_fl / kern_ms[3] / 1e9},
+    }
+    for k, v in kernels.items():
+        if "TFLOP/s" in v:
+            v["frac_of_bf16_peak"] = v["TFLOP/s"] / tpk
+        else:
+            v["frac_of_hbm"] = v["GB/s"] / peaks["hbm_gbs"]
+        for kk in list(v):
+            v[kk] = round(float(v[kk]), 4)
+    attn_tflops = attn_fl / kern_ms[1] / 1e9
+
+    e2e = run_e2e(args, hstu, torch, inp, D, shape, dev, stream, world)
+
+    result = {
+        "metric": METRIC, "value": round(tokens_per_s, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; shapes of the pages' long-sequence encoder benchmark)",
+        "config": {"workload": f"{w.name}: B={w.num_seqs} x n={max_len} jagged, d={d}, "
+                               f"H={H}x{hd}, rab P={w.n_pos_buckets}/Tb={w.n_time_buckets}, 1 layer",
+                   "global_batch_tokens": world * T, "seq_len": max_len,
+                   "parallelism": f"replicas over sequences x{world} (no collective)",
+                   "l2": "flushed between timed steps (256 MB write, outside the events)"},
+        "attention_tflops": round(attn_tflops, 2),
+        "attention_frac_of_bf16_peak": round(attn_tflops / tpk, 4),
+        "roofline": {"bound": "tensor", "kernel": "attention", "achieved": round(attn_tflops, 2),
+                     "peak": tpk, "unit": "TFLOP/s", "frac": round(attn_tflops / tpk, 4),
+                     "traffic": None, "peak_source": f"{peaks_src} bf16 burst (MEASURED_PEAKS.json)"
+                     if peaks_src == "measured" else "fallback 1590 TFLOP/s"},
+        "kernels": kernels,
+        "e2e": e2e,
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    return result
+
+
+def run_e2e(args, hstu, torch, inp, D, shape, dev, stream, world):
+    """Same metric through the public call hstu_layer_fwd with host buffers: the step's inputs are
+    copied from pinned host memory and the output read back inside the timed region."""
+    steps = max(1, min(args.steps, 20))
+    X_h = D["X"].cpu().pin_memory()
+    off_h = D["off"].cpu().pin_memory()
+    ts_h = D["ts"].cpu().pin_memory() if D["ts"] is not None else None
+    out_h = torch.empty_like(X_h).pin_memory()
+    X_d, off_d = torch.empty_like(D["X"]), torch.empty_like(D["off"])
+    ts_d = torch.empty_like(D["ts"]) if D["ts"] is not None else None
+    out_d = torch.empty_like(D["X"])
+    ws = hstu.alloc_workspace(shape, dev)
+    L = D["layers"][0]
+    max_len = int(inp.lengths.max())
+
+    def one():
+        X_d.copy_(X_h, non_blocking=True)
+        off_d.copy_(off_h, non_blocking=True)
+        if ts_d is not None:
+            ts_d.copy_(ts_h, non_blocking=True)
+        hstu.hstu_layer_fwd(X_d, off_d, ts_d, L["W1"], L["b1"], L["W2"], L["b2"], L["ln_w"],
+                            L["ln_b"], D["pos"], D["tim"], D["ali"], inp.scale,
+                            num_heads=inp.workload.num_heads, max_seq_len=max_len,
+                            ln_eps=inp.ln_eps, out=out_d, workspace=ws, stream=stream)
+        out_h.copy_(out_d, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    h2d = X_h.numel() * X_h.element_size() + off_h.numel() * 8 + (ts_h.numel() * 8 if ts_h is not None else 0)
+    d2h = out_h.numel() * out_h.element_size()
+    return {"value": round(world * inp.T / (ms * 1e-3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": round(ms, 4), "steps": steps}
+
+
+# ------------------------------------------------------------------------------------------------
+# The oracle on the host cores (cpu_baseline of our arm, and the whole reference arm)
+# ------------------------------------------------------------------------------------------------
+
+def oracle_sample_time(inp, seq: int, L: int):
+    import oracle
+    a = int(inp.seq_offsets[seq])
+    p = inp.layers[0]
+    w = inp.workload
+    t0 = time.perf_counter()
+    oracle.layer_fwd(np.array([0, L]), inp.X[a:a + L], p.W1, p.b1, p.W2, p.b2, p.ln_w, p.ln_b,
+                     num_heads=w.num_heads, d_qk=w.head_dim, d_v=w.head_dim,
+                     timestamps=None if inp.timestamps is None else inp.timestamps[a:a + L],
+                     pos_table=inp.pos_table, time_table=inp.time_table,
+                     alibi_slopes=inp.alibi_slopes, scale=inp.scale, ln_eps=inp.ln_eps)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(inp):
+    import oracle
+    oracle.build()
+    L = int(inp.lengths[0])
+    dt = oracle_sample_time(inp, 0, L)
+    return {"value": round(L / dt, 2), "unit": "tokens/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"one whole sequence ({L} tokens, all rows, 1 layer) of the workload; "
+                      f"{dt:.1f} s; C fp64 loops, OpenMP, -O2",
+            "host_cpus": len(os.sched_getaffinity(0))}
+
+
+def run_reference(args, rank, world):
+    import oracle
+    if rank != 0:
+        return None
+    oracle.build()
+    w = workloads.WORKLOADS[args.workload]
+    inp = workloads.make_inputs(w)
+    # size each step so the whole warm-up + timed run stays within about three minutes
+    n = int(inp.lengths[0])
+    budget = 180.0 / max(1, args.steps + args.warmup)
+    L = n
+    t_probe = oracle_sample_time(inp, 0, min(n, 1024))
+    while L > 256 and t_probe * (L / min(n, 1024)) ** 2 > budget:
+        L //= 2
+    for k in range(args.warmup):
+        oracle_sample_time(inp, k % len(inp.lengths), L)
+    times = [oracle_sample_time(inp, k % len(inp.lengths), L) for k in range(args.steps)]
+    ms = 1e3 * sum(times) / len(times)
+    value = L / (ms * 1e-3)
+    sample = (f"per step: the first {L} tokens of one sequence (a whole causal prefix) of "
+              f"{w.name}, 1 layer")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+            "config": {"workload": w.name, "seq_len": int(inp.lengths.max()), "sample_len": L},
+            "cpu_baseline": {"value": round(value, 2), "unit": "tokens/s",
+                             "cores": oracle.num_threads(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="long_seq", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    import torch
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                res["cpu_baseline"] = cpu_baseline(workloads.make_inputs(args.workload))
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,231 @@
+"""Python binding of libhstu_b200 (the C ABI in include/hstu.h): argument marshalling only.
+
+Every step of the HSTU layer forward runs in the library's CUDA kernels for sm_100a; this module
+passes device pointers, sizes and the current CUDA stream through ctypes.  PyTorch supplies device
+memory and streams.  There is no CPU implementation here: if the compiled library is missing,
+importing this package raises.
+
+The layer ("Actions Speak Louder than Words" paper notes, section 3.1, Eqs. 1-3):
+    [U|V|Q|K] = SiLU(X W1 + b1)
+    AV_i      = sum_{j<=i} scale * SiLU(q_i.k_j + rab^{p,t}(i, j)) v_j      (per head, jagged, causal)
+    Y         = (LayerNorm(AV) * U) W2 + b2 + X
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhstu_b200.so")
+
+HSTU_OK, HSTU_ERR_INVALID_ARG, HSTU_ERR_UNSUPPORTED, HSTU_ERR_CUDA = 0, 1, 2, 3
+HSTU_ERR_DEVICE_TIMEOUT, HSTU_ERR_DEVICE_BAD_OFFSETS = 4, 5
+HSTU_F32, HSTU_BF16 = 0, 1
+
+# Every symbol include/hstu.h declares.
+EXPORTED = ["hstu_layer_fwd", "hstu_layer_fwd_workspace_size", "hstu_f1_fwd", "hstu_attention_fwd",
+            "hstu_attention_workspace_size", "hstu_ln_gate_fwd", "hstu_f2_fwd",
+            "hstu_token_embed_fwd", "hstu_status_string", "hstu_get_device_status", "hstu_version",
+            "hstu_launch_count"]
+
+
+class HstuShape(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int64), ("total_tokens", ctypes.c_int64),
+                ("max_seq_len", ctypes.c_int64), ("d_model", ctypes.c_int32),
+                ("num_heads", ctypes.c_int32), ("d_qk", ctypes.c_int32), ("d_v", ctypes.c_int32),
+                ("n_pos_buckets", ctypes.c_int32), ("n_time_buckets", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("ln_eps", ctypes.c_float)]
+
+
+class HstuError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {status_string(code)}")
+
+
+def _load() -> ctypes.CDLL:
+    from . import build as _build
+    try:
+        _build.build()          # no-op unless a source is newer than the library
+    except Exception as e:      # no nvcc here: use the shipped library if there is one
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing and could not be built ({e}); "
+                              "this package has no CPU fallback") from e
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I64, I32, F32, S = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+    SH = ctypes.POINTER(HstuShape)
+    sig = {
+        "hstu_layer_fwd": ([SH, P, P, P, P, P, P, P, P, P, P, P, P, F32, P, P, S, P], ctypes.c_int),
+        "hstu_layer_fwd_workspace_size": ([SH], S),
+        "hstu_f1_fwd": ([SH, P, P, P, P, P], ctypes.c_int),
+        "hstu_attention_fwd": ([SH, P, P, P, P, P, P, F32, P, P, S, P], ctypes.c_int),
+        "hstu_attention_workspace_size": ([SH], S),
+        "hstu_ln_gate_fwd": ([SH, P, P, P, P, P, P], ctypes.c_int),
+        "hstu_f2_fwd": ([SH, P, P, P, P, P, P], ctypes.c_int),
+        "hstu_token_embed_fwd": ([I64, I32, P, P, P, I64, P, I64, P, P], ctypes.c_int),
+        "hstu_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "hstu_get_device_status": ([P], ctypes.c_int),
+        "hstu_version": ([], ctypes.c_char_p),
+        "hstu_launch_count": ([], ctypes.c_uint64),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+_lib = _load()
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return _lib.hstu_status_string(int(code)).decode()
+
+
+def version() -> str:
+    return _lib.hstu_version().decode()
+
+
+def launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(_lib.hstu_launch_count())
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != HSTU_OK:
+        raise HstuError(rc, what)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libhstu_b200 must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return HSTU_BF16
+    if t.dtype == torch.float32:
+        return HSTU_F32
+    raise ValueError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def make_shape(num_seqs: int, total_tokens: int, max_seq_len: int, d_model: int, num_heads: int,
+               d_qk: int, d_v: int, dtype: int, n_pos_buckets: int = 0, n_time_buckets: int = 0,
+               ln_eps: float = 1e-5) -> HstuShape:
+    return HstuShape(int(num_seqs), int(total_tokens), int(max_seq_len), int(d_model),
+                     int(num_heads), int(d_qk), int(d_v), int(n_pos_buckets), int(n_time_buckets),
+                     int(dtype), float(ln_eps))
+
+
+def shape_for(X: torch.Tensor, seq_offsets: torch.Tensor, num_heads: int, d_qk: int, d_v: int,
+              max_seq_len: int, pos_table=None, time_table=None, ln_eps: float = 1e-5) -> HstuShape:
+    return make_shape(seq_offsets.numel() - 1, X.shape[0], max_seq_len, X.shape[1], num_heads,
+                      d_qk, d_v, _dtype_code(X),
+                      0 if pos_table is None else pos_table.shape[1],
+                      0 if time_table is None else time_table.shape[1], ln_eps)
+
+
+def workspace_size(shape: HstuShape) -> int:
+    return int(_lib.hstu_layer_fwd_workspace_size(ctypes.byref(shape)))
+
+
+def attention_workspace_size(shape: HstuShape) -> int:
+    return int(_lib.hstu_attention_workspace_size(ctypes.byref(shape)))
+
+
+def alloc_workspace(shape: HstuShape, device) -> torch.Tensor:
+    n = workspace_size(shape)
+    if n == 0 and shape.total_tokens > 0:
+        raise HstuError(HSTU_ERR_INVALID_ARG, "hstu_layer_fwd_workspace_size")
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def hstu_layer_fwd(X: torch.Tensor, seq_offsets: torch.Tensor, timestamps: Optional[torch.Tensor],
+                   W1: torch.Tensor, b1: Optional[torch.Tensor], W2: torch.Tensor,
+                   b2: Optional[torch.Tensor], ln_w: torch.Tensor, ln_b: torch.Tensor,
+                   pos_table: Optional[torch.Tensor] = None,
+                   time_table: Optional[torch.Tensor] = None,
+                   alibi_slopes: Optional[torch.Tensor] = None, scale: Optional[float] = None, *,
+                   num_heads: int, d_qk: Optional[int] = None, d_v: Optional[int] = None,
+                   max_seq_len: int, ln_eps: float = 1e-5, out: Optional[torch.Tensor] = None,
+                   workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One HSTU layer on device tensors.  `scale` defaults to 1/max_seq_len."""
+    hd = X.shape[1] // num_heads
+    d_qk = hd if d_qk is None else d_qk
+    d_v = hd if d_v is None else d_v
+    shape = shape_for(X, seq_offsets, num_heads, d_qk, d_v, max_seq_len, pos_table, time_table,
+                      ln_eps)
+    if scale is None:
+        scale = 1.0 / max(1, max_seq_len)
+    if out is None:
+        out = torch.empty_like(X)
+    if workspace is None:
+        workspace = alloc_workspace(shape, X.device)
+    rc = _lib.hstu_layer_fwd(ctypes.byref(shape), _ptr(X), _ptr(seq_offsets), _ptr(timestamps),
+                             _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), _ptr(ln_w), _ptr(ln_b),
+                             _ptr(pos_table), _ptr(time_table), _ptr(alibi_slopes), float(scale),
+                             _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "hstu_layer_fwd")
+    return out
+
+
+def hstu_f1_fwd(shape: HstuShape, X, W1, b1, uvqk, stream=None):
+    _check(_lib.hstu_f1_fwd(ctypes.byref(shape), _ptr(X), _ptr(W1), _ptr(b1), _ptr(uvqk),
+                            _stream(stream)), "hstu_f1_fwd")
+    return uvqk
+
+
+def hstu_attention_fwd(shape: HstuShape, uvqk, seq_offsets, timestamps, pos_table, time_table,
+                       alibi_slopes, scale: float, av, workspace=None, stream=None):
+    if workspace is None:
+        workspace = torch.empty(max(256, attention_workspace_size(shape)), dtype=torch.uint8,
+                                device=uvqk.device)
+    _check(_lib.hstu_attention_fwd(ctypes.byref(shape), _ptr(uvqk), _ptr(seq_offsets),
+                                   _ptr(timestamps), _ptr(pos_table), _ptr(time_table),
+                                   _ptr(alibi_slopes), float(scale), _ptr(av), _ptr(workspace),
+                                   workspace.numel(), _stream(stream)), "hstu_attention_fwd")
+    return av
+
+
+def hstu_ln_gate_fwd(shape: HstuShape, av, uvqk, ln_w, ln_b, g, stream=None):
+    _check(_lib.hstu_ln_gate_fwd(ctypes.byref(shape), _ptr(av), _ptr(uvqk), _ptr(ln_w), _ptr(ln_b),
+                                 _ptr(g), _stream(stream)), "hstu_ln_gate_fwd")
+    return g
+
+
+def hstu_f2_fwd(shape: HstuShape, g, W2, b2, X, out, stream=None):
+    _check(_lib.hstu_f2_fwd(ctypes.byref(shape), _ptr(g), _ptr(W2), _ptr(b2), _ptr(X), _ptr(out),
+                            _stream(stream)), "hstu_f2_fwd")
+    return out
+
+
+def hstu_token_embed_fwd(item_ids, action_ids, item_table, action_table, out=None, stream=None):
+    T = item_ids.numel()
+    d = item_table.shape[1]
+    if out is None:
+        out = torch.empty((T, d), dtype=item_table.dtype, device=item_table.device)
+    _check(_lib.hstu_token_embed_fwd(T, d, _ptr(item_ids), _ptr(action_ids), _ptr(item_table),
+                                     item_table.shape[0], _ptr(action_table), action_table.shape[0],
+                                     _ptr(out), _stream(stream)), "hstu_token_embed_fwd")
+    return out
+
+
+def device_status(stream=None) -> int:
+    """Synchronises `stream`, then reads and clears the library's device status word."""
+    return int(_lib.hstu_get_device_status(_stream(stream)))

@@ -1,0 +1,319 @@
+// C ABI of libhstu_b200 (declared in include/hstu.h): argument validation, workspace layout and the
+// launch sequence of the HSTU layer forward.  Every step runs in this library's kernels.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "hbm_kernels.cuh"
+#include "simt_kernels.cuh"
+#include "tc_kernels.cuh"
+
+using namespace hstu;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+int64_t n1_of(const hstu_shape_t& s) { return 2LL * s.num_heads * s.d_v + 2LL * s.num_heads * s.d_qk; }
+int64_t wv_of(const hstu_shape_t& s) { return (int64_t)s.num_heads * s.d_v; }
+size_t esize(const hstu_shape_t& s) { return s.dtype == HSTU_BF16 ? 2 : 4; }
+
+bool aligned16(const void* p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+// Shape checks common to every entry point.
+hstu_status_t check_shape(const hstu_shape_t* s) {
+  if (!s) return HSTU_ERR_INVALID_ARG;
+  if (s->num_seqs < 0 || s->total_tokens < 0 || s->max_seq_len < 0) return HSTU_ERR_INVALID_ARG;
+  if (s->d_model <= 0 || s->num_heads <= 0 || s->d_qk <= 0 || s->d_v <= 0) return HSTU_ERR_INVALID_ARG;
+  if (s->dtype != HSTU_F32 && s->dtype != HSTU_BF16) return HSTU_ERR_INVALID_ARG;
+  if (!(s->ln_eps >= 0.0f) || !std::isfinite(s->ln_eps)) return HSTU_ERR_INVALID_ARG;
+  if (s->n_pos_buckets < 0 || s->n_time_buckets < 0) return HSTU_ERR_INVALID_ARG;
+  // keep every index product inside int64 and every row width inside int32
+  if (n1_of(*s) > (1LL << 30) || s->total_tokens > (1LL << 40)) return HSTU_ERR_INVALID_ARG;
+  if (s->dtype == HSTU_BF16) {
+    if (s->d_model % 64 != 0 || s->d_qk != s->d_v || (s->d_qk != 64 && s->d_qk != 128))
+      return HSTU_ERR_UNSUPPORTED;
+  } else {
+    if (s->d_qk > 256 || s->d_v > 256) return HSTU_ERR_UNSUPPORTED;
+  }
+  return HSTU_OK;
+}
+
+hstu_status_t check_bias(const hstu_shape_t* s, const int64_t* ts, const float* pos,
+                         const float* tim, const float* alibi, float scale) {
+  if (!std::isfinite(scale)) return HSTU_ERR_INVALID_ARG;
+  if (alibi && (pos || tim)) return HSTU_ERR_INVALID_ARG;
+  if (pos && s->n_pos_buckets <= 0) return HSTU_ERR_INVALID_ARG;
+  if (tim && (s->n_time_buckets <= 0 || !ts)) return HSTU_ERR_INVALID_ARG;
+  return HSTU_OK;
+}
+
+hstu_status_t launch_status() {
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Step launchers (shape already validated).
+// ------------------------------------------------------------------------------------------------
+
+hstu_status_t run_f1(const hstu_shape_t& s, const void* X, const void* W1, const void* b1,
+                     void* uvqk, cudaStream_t st) {
+  const int64_t T = s.total_tokens;
+  const int n1 = (int)n1_of(s), d = s.d_model;
+  if (T == 0) return HSTU_OK;
+  if (s.dtype == HSTU_BF16) return tc::launch_gemm_f1(T, n1, d, (const bf16*)X, (const bf16*)W1,
+                                                      (const bf16*)b1, (bf16*)uvqk, st);
+  dim3 grid((n1 + 63) / 64, (unsigned)((T + 63) / 64));
+  simt::gemm_kernel<float, simt::EPI_BIAS_SILU><<<grid, 256, 0, st>>>(
+      T, n1, d, (const float*)X, (const float*)W1, (const float*)b1, nullptr, (float*)uvqk);
+  return launch_status();
+}
+
+hstu_status_t run_attention(const hstu_shape_t& s, const void* uvqk, const int64_t* off,
+                            const int64_t* ts, const float* pos, const float* tim,
+                            const float* alibi, float scale, void* av, void* ws, size_t ws_bytes,
+                            cudaStream_t st) {
+  const int64_t T = s.total_tokens, B = s.num_seqs;
+  if (T == 0) return HSTU_OK;
+  check_offsets_kernel<<<(unsigned)((B + 1 + 255) / 256), 256, 0, st>>>(off, B, T);
+  if (launch_status() != HSTU_OK) return HSTU_ERR_CUDA;
+  if (s.dtype == HSTU_BF16)
+    return tc::launch_attention(T, B, s.num_heads, s.d_qk, s.max_seq_len, (const bf16*)uvqk, off,
+                                ts, pos, s.n_pos_buckets, tim, s.n_time_buckets, alibi, scale,
+                                (float*)av, ws, ws_bytes, st);
+  const int64_t warps = T * s.num_heads;
+  simt::attention_kernel<float, float><<<(unsigned)((warps * 32 + 255) / 256), 256, 0, st>>>(
+      T, B, s.num_heads, s.d_qk, s.d_v, (const float*)uvqk, off, ts, pos, s.n_pos_buckets, tim,
+      s.n_time_buckets, alibi, scale, (float*)av);
+  return launch_status();
+}
+
+hstu_status_t run_ln_gate(const hstu_shape_t& s, const void* av, const void* uvqk,
+                          const void* ln_w, const void* ln_b, void* g, cudaStream_t st) {
+  const int64_t T = s.total_tokens, wv = wv_of(s), n1 = n1_of(s);
+  if (T == 0) return HSTU_OK;
+  const unsigned blocks = (unsigned)((T * 32 + 255) / 256);
+  if (s.dtype == HSTU_BF16 && wv % 256 == 0 && wv <= 4096) {
+    const float* a = (const float*)av;
+    const bf16 *u = (const bf16*)uvqk, *w = (const bf16*)ln_w, *b = (const bf16*)ln_b;
+    bf16* o = (bf16*)g;
+    switch (wv / 256) {
+      case 1: ln_gate_bf16_kernel<1><<<blocks, 256, 0, st>>>(T, n1, a, u, w, b, s.ln_eps, o); break;
+      case 2: ln_gate_bf16_kernel<2><<<blocks, 256, 0, st>>>(T, n1, a, u, w, b, s.ln_eps, o); break;
+      case 4: ln_gate_bf16_kernel<4><<<blocks, 256, 0, st>>>(T, n1, a, u, w, b, s.ln_eps, o); break;
+      case 8: ln_gate_bf16_kernel<8><<<blocks, 256, 0, st>>>(T, n1, a, u, w, b, s.ln_eps, o); break;
+      case 16: ln_gate_bf16_kernel<16><<<blocks, 256, 0, st>>>(T, n1, a, u, w, b, s.ln_eps, o); break;
+      default:
+        simt::ln_gate_kernel<bf16, float><<<blocks, 256, 0, st>>>(T, (int)wv, n1, a, u, w, b, s.ln_eps, o);
+    }
+    return launch_status();
+  }
+  if (s.dtype == HSTU_BF16) {
+    simt::ln_gate_kernel<bf16, float><<<blocks, 256, 0, st>>>(T, (int)wv, n1, (const float*)av,
+                                                              (const bf16*)uvqk, (const bf16*)ln_w,
+                                                              (const bf16*)ln_b, s.ln_eps, (bf16*)g);
+  } else {
+    simt::ln_gate_kernel<float, float><<<blocks, 256, 0, st>>>(T, (int)wv, n1, (const float*)av,
+                                                               (const float*)uvqk, (const float*)ln_w,
+                                                               (const float*)ln_b, s.ln_eps, (float*)g);
+  }
+  return launch_status();
+}
+
+hstu_status_t run_f2(const hstu_shape_t& s, const void* g, const void* W2, const void* b2,
+                     const void* X, void* out, cudaStream_t st) {
+  const int64_t T = s.total_tokens;
+  const int d = s.d_model, wv = (int)wv_of(s);
+  if (T == 0) return HSTU_OK;
+  if (s.dtype == HSTU_BF16)
+    return tc::launch_gemm_f2(T, d, wv, (const bf16*)g, (const bf16*)W2, (const bf16*)b2,
+                              (const bf16*)X, (bf16*)out, st);
+  dim3 grid((d + 63) / 64, (unsigned)((T + 63) / 64));
+  simt::gemm_kernel<float, simt::EPI_BIAS_RESIDUAL><<<grid, 256, 0, st>>>(
+      T, d, wv, (const float*)g, (const float*)W2, (const float*)b2, (const float*)X, (float*)out);
+  return launch_status();
+}
+
+size_t attention_ws_bytes(const hstu_shape_t& s) {
+  return s.dtype == HSTU_BF16 ? tc::attention_workspace_bytes(s.total_tokens, s.num_seqs,
+                                                               s.num_heads)
+                              : 0;
+}
+
+struct Workspace {
+  void *uvqk, *av, *g, *attn;
+  size_t attn_bytes, total;
+};
+
+Workspace layout(const hstu_shape_t& s, void* base) {
+  Workspace w{};
+  const size_t T = (size_t)s.total_tokens, es = esize(s);
+  size_t o = 0;
+  char* b = static_cast<char*>(base);
+  w.uvqk = b ? b + o : nullptr;
+  o += align_up(T * (size_t)n1_of(s) * es);
+  w.av = b ? b + o : nullptr;  // AV is fp32 on both paths (LayerNorm input)
+  o += align_up(T * (size_t)wv_of(s) * 4);
+  w.g = b ? b + o : nullptr;
+  o += align_up(T * (size_t)wv_of(s) * es);
+  w.attn = b ? b + o : nullptr;
+  w.attn_bytes = attention_ws_bytes(s);
+  o += align_up(w.attn_bytes);
+  w.total = o;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* hstu_version(void) { return "0.1.0"; }
+
+uint64_t hstu_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* hstu_status_string(hstu_status_t st) {
+  switch (st) {
+    case HSTU_OK: return "HSTU_OK";
+    case HSTU_ERR_INVALID_ARG: return "HSTU_ERR_INVALID_ARG";
+    case HSTU_ERR_UNSUPPORTED: return "HSTU_ERR_UNSUPPORTED";
+    case HSTU_ERR_CUDA: return "HSTU_ERR_CUDA";
+    case HSTU_ERR_DEVICE_TIMEOUT: return "HSTU_ERR_DEVICE_TIMEOUT";
+    case HSTU_ERR_DEVICE_BAD_OFFSETS: return "HSTU_ERR_DEVICE_BAD_OFFSETS";
+  }
+  return "HSTU_ERR_UNKNOWN";
+}
+
+hstu_status_t hstu_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return HSTU_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, hstu::g_device_status, sizeof(int)) != cudaSuccess) return HSTU_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(hstu::g_device_status, &zero, sizeof(int)) != cudaSuccess) return HSTU_ERR_CUDA;
+  return static_cast<hstu_status_t>(v);
+}
+
+size_t hstu_layer_fwd_workspace_size(const hstu_shape_t* shape) {
+  if (check_shape(shape) != HSTU_OK) return 0;
+  return layout(*shape, nullptr).total;
+}
+
+size_t hstu_attention_workspace_size(const hstu_shape_t* shape) {
+  if (check_shape(shape) != HSTU_OK) return 0;
+  return attention_ws_bytes(*shape);
+}
+
+hstu_status_t hstu_f1_fwd(const hstu_shape_t* shape, const void* X, const void* W1, const void* b1,
+                          void* uvqk, void* stream) {
+  hstu_status_t rc = check_shape(shape);
+  if (rc != HSTU_OK) return rc;
+  if (shape->total_tokens > 0 && (!X || !W1 || !uvqk)) return HSTU_ERR_INVALID_ARG;
+  if (shape->dtype == HSTU_BF16 && !(aligned16(X) && aligned16(W1) && aligned16(b1) && aligned16(uvqk)))
+    return HSTU_ERR_INVALID_ARG;
+  return run_f1(*shape, X, W1, b1, uvqk, static_cast<cudaStream_t>(stream));
+}
+
+hstu_status_t hstu_attention_fwd(const hstu_shape_t* shape, const void* uvqk,
+                                 const int64_t* seq_offsets, const int64_t* timestamps,
+                                 const float* pos_table, const float* time_table,
+                                 const float* alibi_slopes, float scale, void* av, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  hstu_status_t rc = check_shape(shape);
+  if (rc != HSTU_OK) return rc;
+  if (shape->total_tokens == 0) return HSTU_OK;
+  rc = check_bias(shape, timestamps, pos_table, time_table, alibi_slopes, scale);
+  if (rc != HSTU_OK) return rc;
+  if (!uvqk || !av || !seq_offsets) return HSTU_ERR_INVALID_ARG;
+  if (shape->total_tokens > 0 && shape->num_seqs == 0) return HSTU_ERR_INVALID_ARG;
+  if (shape->dtype == HSTU_BF16 && !(aligned16(uvqk) && aligned16(av))) return HSTU_ERR_INVALID_ARG;
+  const size_t need = attention_ws_bytes(*shape);
+  if (need > 0 && (!workspace || workspace_bytes < need ||
+                   (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1))))
+    return HSTU_ERR_INVALID_ARG;
+  return run_attention(*shape, uvqk, seq_offsets, timestamps, pos_table, time_table, alibi_slopes,
+                       scale, av, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+hstu_status_t hstu_ln_gate_fwd(const hstu_shape_t* shape, const void* av, const void* uvqk,
+                               const void* ln_w, const void* ln_b, void* g, void* stream) {
+  hstu_status_t rc = check_shape(shape);
+  if (rc != HSTU_OK) return rc;
+  if (shape->total_tokens > 0 && (!av || !uvqk || !ln_w || !ln_b || !g)) return HSTU_ERR_INVALID_ARG;
+  if (shape->dtype == HSTU_BF16 &&
+      !(aligned16(av) && aligned16(uvqk) && aligned16(ln_w) && aligned16(ln_b) && aligned16(g)))
+    return HSTU_ERR_INVALID_ARG;
+  return run_ln_gate(*shape, av, uvqk, ln_w, ln_b, g, static_cast<cudaStream_t>(stream));
+}
+
+hstu_status_t hstu_f2_fwd(const hstu_shape_t* shape, const void* g, const void* W2, const void* b2,
+                          const void* X, void* out, void* stream) {
+  hstu_status_t rc = check_shape(shape);
+  if (rc != HSTU_OK) return rc;
+  if (shape->total_tokens > 0 && (!g || !W2 || !X || !out)) return HSTU_ERR_INVALID_ARG;
+  if (shape->dtype == HSTU_BF16 &&
+      !(aligned16(g) && aligned16(W2) && aligned16(b2) && aligned16(X) && aligned16(out)))
+    return HSTU_ERR_INVALID_ARG;
+  const size_t es = esize(*shape), T = (size_t)shape->total_tokens;
+  if (overlaps(out, T * shape->d_model * es, X, T * shape->d_model * es)) return HSTU_ERR_INVALID_ARG;
+  return run_f2(*shape, g, W2, b2, X, out, static_cast<cudaStream_t>(stream));
+}
+
+hstu_status_t hstu_layer_fwd(const hstu_shape_t* shape, const void* X, const int64_t* seq_offsets,
+                             const int64_t* timestamps, const void* W1, const void* b1,
+                             const void* W2, const void* b2, const void* ln_w, const void* ln_b,
+                             const float* pos_table, const float* time_table,
+                             const float* alibi_slopes, float scale, void* out, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  hstu_status_t rc = check_shape(shape);
+  if (rc != HSTU_OK) return rc;
+  const hstu_shape_t& s = *shape;
+  const int64_t T = s.total_tokens;
+  if (T == 0) return HSTU_OK;  // nothing to read or write; empty tensors may be NULL
+  rc = check_bias(shape, timestamps, pos_table, time_table, alibi_slopes, scale);
+  if (rc != HSTU_OK) return rc;
+  if (s.num_seqs == 0) return HSTU_ERR_INVALID_ARG;
+  if (!X || !seq_offsets || !W1 || !W2 || !ln_w || !ln_b || !out || !workspace)
+    return HSTU_ERR_INVALID_ARG;
+  if (s.dtype == HSTU_BF16 && !(aligned16(X) && aligned16(W1) && aligned16(b1) && aligned16(W2) &&
+                                aligned16(b2) && aligned16(ln_w) && aligned16(ln_b) && aligned16(out)))
+    return HSTU_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) return HSTU_ERR_INVALID_ARG;
+  const Workspace w = layout(s, workspace);
+  if (workspace_bytes < w.total) return HSTU_ERR_INVALID_ARG;
+  const size_t xbytes = (size_t)T * s.d_model * esize(s);
+  if (overlaps(out, xbytes, X, xbytes) || overlaps(out, xbytes, workspace, w.total) ||
+      overlaps(X, xbytes, workspace, w.total))
+    return HSTU_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = run_f1(s, X, W1, b1, w.uvqk, st)) != HSTU_OK) return rc;
+  if ((rc = run_attention(s, w.uvqk, seq_offsets, timestamps, pos_table, time_table, alibi_slopes,
+                          scale, w.av, w.attn, w.attn_bytes, st)) != HSTU_OK)
+    return rc;
+  if ((rc = run_ln_gate(s, w.av, w.uvqk, ln_w, ln_b, w.g, st)) != HSTU_OK) return rc;
+  return run_f2(s, w.g, W2, b2, X, out, st);
+}
+
+hstu_status_t hstu_token_embed_fwd(int64_t T, int32_t d, const int64_t* item_ids,
+                                   const int64_t* action_ids, const void* item_table,
+                                   int64_t n_items, const void* action_table, int64_t n_actions,
+                                   void* X, void* stream) {
+  if (T < 0 || d <= 0 || d % 8 != 0 || n_items <= 0 || n_actions <= 0) return HSTU_ERR_INVALID_ARG;
+  if (T == 0) return HSTU_OK;
+  if (!item_ids || !action_ids || !item_table || !action_table || !X) return HSTU_ERR_INVALID_ARG;
+  if (!aligned16(item_table) || !aligned16(action_table) || !aligned16(X)) return HSTU_ERR_INVALID_ARG;
+  const int64_t threads = T * (d / 8);
+  token_embed_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      T, d, item_ids, action_ids, (const bf16*)item_table, n_items, (const bf16*)action_table,
+      n_actions, (bf16*)X);
+  return launch_status();
+}
+
+}  // extern "C"

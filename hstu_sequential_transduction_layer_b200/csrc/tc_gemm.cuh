@@ -1,0 +1,236 @@
+// Persistent, warp-specialised tcgen05 GEMM for the two projections of the HSTU layer
+// ("Actions Speak Louder than Words" paper notes, section 3.1: f1 of Eq. 1 and f2 of Eq. 3):
+//
+//   C[M, N] = epilogue(A[M, K] . B[K, N]),  A row-major (K-major), B row-major (MN-major operand)
+//   EPI_BIAS_SILU:      C = SiLU(acc + bias)              f1: U|V|Q|K = SiLU(X W1 + b1)
+//   EPI_BIAS_RESIDUAL:  C = acc + bias + R                f2: Y = G W2 + b2 + X
+//
+// One CTA per SM (192 threads):
+//   warp 0      TMA producer: A tile 128x64 and B tile 64xBN per stage into a STAGES-deep ring, both
+//               128-byte swizzled; no multicast.
+//   warp 1      allocates TMEM (two BN-column fp32 accumulators) and issues tcgen05.mma (M=128,
+//               N=BN, K=16) from one thread; tcgen05.commit frees ring stages and publishes
+//               finished accumulators.
+//   warps 2-5   epilogue: tcgen05.ld 32 columns at a time from their TMEM lane quadrant, fused bias
+//               / SiLU / residual in fp32, bf16 stores.  The accumulator is double-buffered, so the
+//               epilogue of tile t overlaps the main loop of tile t+1.
+// Output tiles are visited in groups of up to 8 BN-wide column blocks over all row blocks, so that
+// the CTAs in flight share a few MB of A and B in L2.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace hstu {
+namespace tc {
+
+enum GemmEpilogue { EPI_BIAS_SILU = 0, EPI_BIAS_RESIDUAL = 1 };
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int BM = 128, BK = 64;
+  static constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BK * BN * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
+  static constexpr int TMEM_COLS = 2 * BN;
+};
+
+__device__ __forceinline__ void gemm_tile_coords(int64_t t, int tiles_n, int64_t tiles_m,
+                                                 int64_t& mb, int& nb) {
+  const int G = tiles_n < 8 ? tiles_n : 8;
+  const int64_t g = t / ((int64_t)G * tiles_m);
+  const int64_t r = t - g * (int64_t)G * tiles_m;
+  const int gw = min(G, tiles_n - (int)g * G);
+  mb = r / gw;
+  nb = (int)g * G + (int)(r % gw);
+}
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   int64_t M, int N, int K, const bf16* __restrict__ bias,
+                   const bf16* __restrict__ R, bf16* __restrict__ C) {
+  using Cfg = GemmCfg<BN>;
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::STAGES * Cfg::STAGE_BYTES);
+  uint64_t* empty = full + Cfg::STAGES;
+  uint64_t* tfull = empty + Cfg::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int tiles_n = N / BN;
+  const int64_t tiles_m = (M + Cfg::BM - 1) / Cfg::BM;
+  const int64_t num_tiles = tiles_m * tiles_n;
+  const int kblocks = K / Cfg::BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Cfg::STAGES; s++) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; a++) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      bool issued[Cfg::STAGES];
+      uint32_t issued_phase[Cfg::STAGES];
+      for (int s = 0; s < Cfg::STAGES; s++) issued[s] = false, issued_phase[s] = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        int64_t mb;
+        int nb;
+        gemm_tile_coords(t, tiles_n, tiles_m, mb, nb);
+        const int m0 = (int)(mb * Cfg::BM), n0 = nb * BN;
+        for (int kb = 0; kb < kblocks; kb++) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* a_s = smem + stage * Cfg::STAGE_BYTES;
+          uint8_t* b_s = a_s + Cfg::A_BYTES;
+          mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+          tma_load_2d(a_s, &tmA, &full[stage], kb * Cfg::BK, m0);
+#pragma unroll
+          for (int c = 0; c < BN / 64; c++)
+            tma_load_2d(b_s + c * (Cfg::BK * 128), &tmB, &full[stage], n0 + c * 64, kb * Cfg::BK);
+          issued[stage] = true;
+          issued_phase[stage] = phase;
+          if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok)  // copies still in flight must land before the CTA's shared memory goes away
+        for (int s = 0; s < Cfg::STAGES; s++)
+          if (issued[s]) mbar_drain(&full[s], issued_phase[s]);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(128, BN, false, true);
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < kblocks; kb++) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(smem + stage * Cfg::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + Cfg::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < Cfg::BK / 16; kk++) {
+            const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b_addr + kk * 2048, Cfg::BK * 128, 1024);
+            mma_ss(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        mma_commit(&tfull[acc]);
+        acc ^= 1u;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      // every issued MMA has finished reading shared memory before the CTA can exit
+      mma_commit(drain);
+      mbar_drain(drain, 0);
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    uint32_t acc = 0, acc_phase = 0;
+    for (int64_t t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      int64_t mb;
+      int nb;
+      gemm_tile_coords(t, tiles_n, tiles_m, mb, nb);
+      const int64_t row = mb * Cfg::BM + q * 32 + lane;
+      const int n0 = nb * BN;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
+      tc_fence_after();
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; c++) {
+        uint32_t r[32];
+        tmem_ld32(t_row + c * 32, r);
+        tmem_ld_wait();
+        const int n = n0 + c * 32;
+        uint4 bvec[4];
+        if (bias) {
+#pragma unroll
+          for (int v = 0; v < 4; v++) bvec[v] = __ldg(reinterpret_cast<const uint4*>(bias + n) + v);
+        } else {
+#pragma unroll
+          for (int v = 0; v < 4; v++) bvec[v] = make_uint4(0, 0, 0, 0);
+        }
+        if (row < M) {
+          uint4 rvec[4] = {};
+          if (EPI == EPI_BIAS_RESIDUAL) {
+#pragma unroll
+            for (int v = 0; v < 4; v++)
+              rvec[v] = __ldcs(reinterpret_cast<const uint4*>(R + row * N + n) + v);
+          }
+          uint4 out[4];
+#pragma unroll
+          for (int v = 0; v < 4; v++) {
+            const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bvec[v]);
+            const uint32_t* rw = reinterpret_cast<const uint32_t*>(&rvec[v]);
+            uint32_t* ow = reinterpret_cast<uint32_t*>(&out[v]);
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+              float lo = __uint_as_float(r[v * 8 + 2 * e]) + bf16_lo(bw[e]);
+              float hi = __uint_as_float(r[v * 8 + 2 * e + 1]) + bf16_hi(bw[e]);
+              if (EPI == EPI_BIAS_SILU) {
+                lo = silu_fast(lo);
+                hi = silu_fast(hi);
+              } else {
+                lo += bf16_lo(rw[e]);
+                hi += bf16_hi(rw[e]);
+              }
+              ow[e] = pack_bf16x2(lo, hi);
+            }
+          }
+#pragma unroll
+          for (int v = 0; v < 4; v++) reinterpret_cast<uint4*>(C + row * N + n)[v] = out[v];
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      acc ^= 1u;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+}  // namespace tc
+}  // namespace hstu

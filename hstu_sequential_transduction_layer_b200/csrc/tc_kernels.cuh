@@ -1,0 +1,171 @@
+// Host-side launchers of the bf16 tensor-core path: TMA tensor maps, the two GEMMs and the jagged
+// attention.
+#pragma once
+
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "tc_attention.cuh"
+#include "tc_gemm.cuh"
+
+namespace hstu {
+namespace tc {
+
+inline PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map over a row-major [outer, inner] matrix with row stride `ld` elements, a box of
+// box_inner x box_outer elements and 128-byte swizzling (box_inner * 2 must be 128).
+inline bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                          uint64_t ld, uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline int num_sms() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+template <int BN, int EPI>
+hstu_status_t launch_gemm_bn(int64_t M, int N, int K, const bf16* A, const bf16* B, const bf16* bias,
+                             const bf16* R, bf16* C, cudaStream_t st) {
+  using Cfg = GemmCfg<BN>;
+  CUtensorMap ta, tb;
+  if (!make_map_bf16(&ta, A, K, M, K, 64, 128)) return HSTU_ERR_CUDA;
+  if (!make_map_bf16(&tb, B, N, K, N, 64, 64)) return HSTU_ERR_CUDA;
+  auto kern = gemm_tc_kernel<BN, EPI>;
+  // set on every launch: the attribute is per device and the call is cheap
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
+      cudaSuccess)
+    return HSTU_ERR_CUDA;
+  const int64_t tiles = ((M + 127) / 128) * (N / BN);
+  const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+  kern<<<grid, 192, Cfg::SMEM, st>>>(ta, tb, M, N, K, bias, R, C);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+template <int EPI>
+hstu_status_t launch_gemm(int64_t M, int N, int K, const bf16* A, const bf16* B, const bf16* bias,
+                          const bf16* R, bf16* C, cudaStream_t st) {
+  if (M >= (1LL << 31) || K % 64 != 0 || N % 64 != 0) return HSTU_ERR_UNSUPPORTED;
+  if (N % 256 == 0) return launch_gemm_bn<256, EPI>(M, N, K, A, B, bias, R, C, st);
+  if (N % 128 == 0) return launch_gemm_bn<128, EPI>(M, N, K, A, B, bias, R, C, st);
+  return launch_gemm_bn<64, EPI>(M, N, K, A, B, bias, R, C, st);
+}
+
+// Eq. 1: uvqk[T, n1] = SiLU(X W1 + b1).
+inline hstu_status_t launch_gemm_f1(int64_t T, int n1, int d, const bf16* X, const bf16* W1,
+                                    const bf16* b1, bf16* uvqk, cudaStream_t st) {
+  return launch_gemm<EPI_BIAS_SILU>(T, n1, d, X, W1, b1, nullptr, uvqk, st);
+}
+
+// Eq. 3 + residual: out[T, d] = G W2 + b2 + X.
+inline hstu_status_t launch_gemm_f2(int64_t T, int d, int wv, const bf16* G, const bf16* W2,
+                                    const bf16* b2, const bf16* X, bf16* out, cudaStream_t st) {
+  return launch_gemm<EPI_BIAS_RESIDUAL>(T, d, wv, G, W2, b2, X, out, st);
+}
+
+// Attention workspace: header (256 B), per-sequence (start, length) pairs, then the item list (one
+// 8-byte entry per (sequence, 128-row query tile, head); at most H * (ceil(T/128) + B) of them).
+inline size_t attention_workspace_bytes(int64_t T, int64_t B, int H) {
+  const int64_t items = (int64_t)H * ((T + ATT_BM - 1) / ATT_BM + B);
+  return (size_t)(256 + ((16 * B + 255) / 256) * 256 + 8 * items);
+}
+
+inline AttnSchedule attention_schedule_view(void* ws, int64_t B) {
+  char* b = static_cast<char*>(ws);
+  AttnSchedule s;
+  s.header = reinterpret_cast<int64_t*>(b);
+  s.seqinfo = reinterpret_cast<int64_t*>(b + 256);
+  s.items = reinterpret_cast<int64_t*>(b + 256 + ((16 * B + 255) / 256) * 256);
+  return s;
+}
+
+template <int HD, int BIAS>
+hstu_status_t launch_attention_kernel(const CUtensorMap& tm, const AttnParams& prm,
+                                      const AttnSchedule& sch, int grid, cudaStream_t st) {
+  using Cfg = AttnCfg<HD>;
+  auto kern = attention_tc_kernel<HD, BIAS>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
+      cudaSuccess)
+    return HSTU_ERR_CUDA;
+  kern<<<grid, 192, Cfg::SMEM, st>>>(tm, prm, sch);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+// Eq. 2 on the tensor cores: builds the longest-first tile schedule on the device, then runs the
+// persistent attention kernel.  av is fp32 [T, H*hd].
+inline hstu_status_t launch_attention(int64_t T, int64_t B, int H, int hd, int64_t max_seq_len,
+                                      const bf16* uvqk, const int64_t* off, const int64_t* ts,
+                                      const float* pos, int P, const float* tim, int Tb,
+                                      const float* alibi, float scale, float* av, void* ws,
+                                      size_t ws_bytes, cudaStream_t st) {
+  if (T >= (1LL << 31) || H >= (1 << 15)) return HSTU_ERR_UNSUPPORTED;
+  if (ws_bytes < attention_workspace_bytes(T, B, H)) return HSTU_ERR_INVALID_ARG;
+  const int64_t max_len = max_seq_len > 0 ? max_seq_len : T;
+  const int64_t max_tiles64 = (max_len + ATT_BM - 1) / ATT_BM;
+  if (max_tiles64 > 16384) return HSTU_ERR_UNSUPPORTED;  // scheduler counters live in shared memory
+  const int max_tiles = (int)max_tiles64;
+  const AttnSchedule sch = attention_schedule_view(ws, B);
+  const size_t sched_smem = 2 * (size_t)(max_tiles + 1) * sizeof(int);
+  if (sched_smem > 48 * 1024 &&
+      cudaFuncSetAttribute(attn_schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)sched_smem) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  const int64_t capacity = (int64_t)H * ((T + ATT_BM - 1) / ATT_BM + B);
+  attn_schedule_kernel<<<1, 1024, sched_smem, st>>>(off, B, T, H, max_tiles, capacity, sch);
+  count_launch();
+  if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+
+  const int n1 = 4 * H * hd;
+  CUtensorMap tm;
+  if (!make_map_bf16(&tm, uvqk, n1, T, n1, 64, 128)) return HSTU_ERR_CUDA;
+  AttnParams prm;
+  prm.ts = ts;
+  prm.pos = pos;
+  prm.tim = tim;
+  prm.alibi = alibi;
+  prm.P = P;
+  prm.Tb = Tb;
+  prm.H = H;
+  prm.n1 = n1;
+  prm.scale = scale;
+  prm.av = av;
+  prm.T = T;
+  const int grid = (int)(capacity < num_sms() ? capacity : num_sms());
+  const int bias = alibi ? BIAS_ALIBI : ((pos || tim) ? BIAS_RAB : BIAS_NONE);
+  if (hd == 64) {
+    if (bias == BIAS_RAB) return launch_attention_kernel<64, BIAS_RAB>(tm, prm, sch, grid, st);
+    if (bias == BIAS_ALIBI) return launch_attention_kernel<64, BIAS_ALIBI>(tm, prm, sch, grid, st);
+    return launch_attention_kernel<64, BIAS_NONE>(tm, prm, sch, grid, st);
+  }
+  if (bias == BIAS_RAB) return launch_attention_kernel<128, BIAS_RAB>(tm, prm, sch, grid, st);
+  if (bias == BIAS_ALIBI) return launch_attention_kernel<128, BIAS_ALIBI>(tm, prm, sch, grid, st);
+  return launch_attention_kernel<128, BIAS_NONE>(tm, prm, sch, grid, st);
+}
+
+}  // namespace tc
+}  // namespace hstu

@@ -1,0 +1,173 @@
+/*
+ * hstu.h -- C ABI of the B200 (sm_100a) HSTU layer forward library, libhstu_b200.so.
+ *
+ * The layer (one "HSTU" block of "Actions Speak Louder than Words", paper notes, section 3.1,
+ * Eqs. 1-3; also the HSTU-layer section of "4.4 推荐模型的 Scaling") over a jagged batch of
+ * user-action sequences:
+ *
+ *   Eq. 1  [U | V | Q | K] = SiLU(X W1 + b1)                       pointwise projection
+ *   Eq. 2  AV_i = sum_{j <= i, same sequence} scale * SiLU(q_i . k_j + bias(i, j)) v_j
+ *                                                                   pointwise (no softmax) causal
+ *                                                                   attention, per head
+ *   Eq. 3  Y = (LayerNorm(AV) * U) W2 + b2 + X                     pointwise transformation plus the
+ *                                                                   residual joining stacked layers
+ *
+ * bias(i, j) (i, j local indices inside one sequence, i >= j) is one of
+ *   - the relative attention bias rab^{p,t} of section 3.1:
+ *       pos_table[h][min(i - j, P - 1)] + time_table[h][min(Tb - 1, floor(log2(1 + max(t_i - t_j, 0))))]
+ *     with either table optional (a missing table contributes 0);
+ *   - the ALiBi bias of the GenRank blog ("position & time bias"): -alibi_slopes[h] * (i - j);
+ *   - nothing (all three pointers NULL).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers (cudaMalloc'd or equivalent), owned by the caller.
+ *    The library allocates, frees and retains no memory; intermediates live in the caller's
+ *    workspace.  Every matrix is row-major and densely packed.
+ *  - `stream` is a cudaStream_t passed as void*; NULL means the legacy default stream.  Calls are
+ *    asynchronous: they only enqueue kernels and return.  They never synchronise.
+ *  - Errors checkable on the host (NULL pointers, bad dimensions, misalignment, aliasing) are
+ *    returned before anything is enqueued.  HSTU_ERR_CUDA reports a failed launch.  Problems that
+ *    only the device can see (offsets that are not monotone or exceed total_tokens, an mbarrier
+ *    wait that timed out) set bits of a device status word instead, which
+ *    hstu_get_device_status() reads and clears.  Kernels clamp indices so that bad offsets never
+ *    cause out-of-bounds accesses.
+ *  - dtype HSTU_BF16 is the tensor-core path: tcgen05 MMAs with fp32 accumulation, bf16 storage of
+ *    U, V, Q, K, of the attention weights fed to the AV product, of G and of the output; AV (the
+ *    LayerNorm input) is kept in fp32 and LayerNorm statistics are fp32.  dtype HSTU_F32 is the exact-arithmetic path (fp32
+ *    storage and fp32 FMA accumulation on CUDA cores, accurate expf), for small problems.
+ */
+#ifndef HSTU_B200_H_
+#define HSTU_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HSTU_OK = 0,
+  HSTU_ERR_INVALID_ARG = 1,    /* a NULL/misaligned pointer, a bad dimension, aliasing, a small workspace */
+  HSTU_ERR_UNSUPPORTED = 2,    /* valid arguments outside what the kernels implement (see hstu_layer_fwd) */
+  HSTU_ERR_CUDA = 3,           /* a CUDA runtime call or a kernel launch failed */
+  HSTU_ERR_DEVICE_TIMEOUT = 4, /* (device status) an mbarrier wait gave up after its time limit */
+  HSTU_ERR_DEVICE_BAD_OFFSETS = 5 /* (device status) seq_offsets not monotone / not ending at T */
+} hstu_status_t;
+
+typedef enum { HSTU_F32 = 0, HSTU_BF16 = 1 } hstu_dtype_t;
+
+/* Shape of one layer call. */
+typedef struct {
+  int64_t num_seqs;       /* B >= 0: number of sequences */
+  int64_t total_tokens;   /* T >= 0: sum of the sequence lengths (rows of X and out) */
+  int64_t max_seq_len;    /* >= the longest sequence; bounds the attention tile schedule */
+  int32_t d_model;        /* d: width of X, W1's rows, W2's columns and out */
+  int32_t num_heads;      /* H */
+  int32_t d_qk;           /* per-head width of Q and K */
+  int32_t d_v;            /* per-head width of V; AV, G, ln_w, ln_b are H*d_v wide */
+  int32_t n_pos_buckets;  /* P: columns of pos_table (ignored when pos_table is NULL) */
+  int32_t n_time_buckets; /* Tb: columns of time_table (ignored when time_table is NULL) */
+  int32_t dtype;          /* hstu_dtype_t of X, W1, b1, W2, b2, ln_w, ln_b, out and intermediates */
+  float ln_eps;           /* LayerNorm epsilon, added to the biased variance (e.g. 1e-5) */
+} hstu_shape_t;
+
+/*
+ * hstu_layer_fwd -- Y = f2(LayerNorm(AV) * U) + X for one layer (Eqs. 1-3 above).
+ *
+ *  X            [T, d]            input tokens (dtype)
+ *  seq_offsets  [B + 1] int64     jagged offsets: sequence s owns rows [off[s], off[s+1]);
+ *                                 off[0] = 0, non-decreasing, off[B] = T; empty sequences allowed
+ *  timestamps   [T] int64         per-token time in integer seconds; may be NULL unless time_table
+ *                                 is given.  Used only through t_i - t_j inside one sequence.
+ *  W1           [d, n1]           n1 = 2*H*d_v + 2*H*d_qk; columns are [U | V | Q | K] blocks, each
+ *                                 head-major (head h owns columns h*hd .. h*hd + hd - 1 of a block)
+ *  b1           [n1]              may be NULL (zero bias)
+ *  W2           [H*d_v, d]
+ *  b2           [d]               may be NULL (zero bias)
+ *  ln_w, ln_b   [H*d_v]           LayerNorm affine parameters (not NULL)
+ *  pos_table    [H, P] fp32       relative position bias, or NULL
+ *  time_table   [H, Tb] fp32      log2 time-difference bias, or NULL
+ *  alibi_slopes [H] fp32          ALiBi slopes m_h, or NULL; when given both tables must be NULL
+ *  scale        multiplier applied after SiLU (the pages normalise each weight by a constant such
+ *               as the sequence length; e.g. 1/max_len)
+ *  out          [T, d]            output (dtype); must not overlap X or the workspace
+ *  workspace    device buffer of at least hstu_layer_fwd_workspace_size(shape) bytes, 256-byte
+ *               aligned, reused freely by the call (holds UVQK, AV, G and the tile schedule)
+ *
+ * HSTU_BF16 requires: d % 64 == 0, d_qk == d_v in {64, 128}, every pointer 16-byte aligned.
+ * HSTU_F32 requires d_qk, d_v <= 256.  Other shapes return HSTU_ERR_UNSUPPORTED.  The bf16 path
+ * also requires T < 2^31 (32-bit TMA row coordinates).
+ */
+hstu_status_t hstu_layer_fwd(const hstu_shape_t* shape, const void* X, const int64_t* seq_offsets,
+                             const int64_t* timestamps, const void* W1, const void* b1,
+                             const void* W2, const void* b2, const void* ln_w, const void* ln_b,
+                             const float* pos_table, const float* time_table,
+                             const float* alibi_slopes, float scale, void* out, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace hstu_layer_fwd needs for `shape` (0 for an invalid shape). */
+size_t hstu_layer_fwd_workspace_size(const hstu_shape_t* shape);
+
+/*
+ * The four steps of hstu_layer_fwd, exposed one by one (same conventions, same kernels).
+ *
+ * hstu_f1_fwd         Eq. 1:  uvqk[T, n1] = SiLU(X W1 + b1).
+ * hstu_attention_fwd  Eq. 2:  av[T, H*d_v] from uvqk (reads its V, Q, K blocks).  av is fp32 for
+ *                     both dtypes: LayerNorm subtracts the row mean, which AV rows share to a large
+ *                     extent, so bf16 storage of AV would be amplified in G.  `workspace` holds the
+ *                     tile schedule: hstu_attention_workspace_size(shape) bytes, 256-byte aligned.
+ * hstu_ln_gate_fwd    Eq. 3 (first half): g[T, H*d_v] = LayerNorm(av) * U, with U = uvqk's block 0;
+ *                     av fp32, uvqk, ln_w, ln_b and g in dtype.
+ * hstu_f2_fwd         Eq. 3 (second half) + residual: out[T, d] = g W2 + b2 + X.
+ */
+hstu_status_t hstu_f1_fwd(const hstu_shape_t* shape, const void* X, const void* W1, const void* b1,
+                          void* uvqk, void* stream);
+hstu_status_t hstu_attention_fwd(const hstu_shape_t* shape, const void* uvqk,
+                                 const int64_t* seq_offsets, const int64_t* timestamps,
+                                 const float* pos_table, const float* time_table,
+                                 const float* alibi_slopes, float scale, void* av, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+size_t hstu_attention_workspace_size(const hstu_shape_t* shape);
+hstu_status_t hstu_ln_gate_fwd(const hstu_shape_t* shape, const void* av, const void* uvqk,
+                               const void* ln_w, const void* ln_b, void* g, void* stream);
+hstu_status_t hstu_f2_fwd(const hstu_shape_t* shape, const void* g, const void* W2, const void* b2,
+                          const void* X, void* out, void* stream);
+
+/*
+ * hstu_token_embed_fwd -- action-oriented token assembly of the GenRank blog ("item-action
+ * organisation"): X[t, :] = bf16(item_table[item_ids[t], :] + action_table[action_ids[t], :]).
+ *
+ *  item_ids, action_ids  [T] int64      indices; out-of-range ids set HSTU_ERR_DEVICE_BAD_OFFSETS in
+ *                                       the device status word and produce a zero row
+ *  item_table            [n_items, d] bf16
+ *  action_table          [n_actions, d] bf16
+ *  X                     [T, d] bf16 output
+ * Requires d % 8 == 0 and 16-byte aligned tables and output.
+ */
+hstu_status_t hstu_token_embed_fwd(int64_t T, int32_t d, const int64_t* item_ids,
+                                   const int64_t* action_ids, const void* item_table,
+                                   int64_t n_items, const void* action_table, int64_t n_actions,
+                                   void* X, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* hstu_status_string(hstu_status_t status);
+
+/*
+ * Reads the device status word of the current device after synchronising `stream`, clears it, and
+ * returns HSTU_OK or the first device-side error recorded since the last call.  This call blocks.
+ */
+hstu_status_t hstu_get_device_status(void* stream);
+
+/* Library version, e.g. "0.1.0". */
+const char* hstu_version(void);
+
+/* Number of kernels this library has launched in this process (all devices), for accounting. */
+uint64_t hstu_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HSTU_B200_H_ */

@@ -60,6 +60,14 @@ def bind(path: str):
     lib.oracle_pos_bucket.restype = i32
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_f1.argtypes = [i64, i32, i32, dp, dp, dp, dp]
+    lib.oracle_f1.restype = None
+    lib.oracle_attention.argtypes = [i64, ip, i32, i32, i32, dp, ip, dp, i32, dp, i32, dp, f64, dp]
+    lib.oracle_attention.restype = None
+    lib.oracle_ln_gate.argtypes = [i64, i32, i32, i32, dp, dp, dp, dp, f64, dp]
+    lib.oracle_ln_gate.restype = None
+    lib.oracle_f2.argtypes = [i64, i32, i32, dp, dp, dp, dp, dp]
+    lib.oracle_f2.restype = None
     return lib
 
 
@@ -206,3 +214,54 @@ def layer_rows_inputs(inp, rows, layer: int = 0, X=None):
                       timestamps=inp.timestamps, pos_table=inp.pos_table,
                       time_table=inp.time_table, alibi_slopes=inp.alibi_slopes, scale=inp.scale,
                       ln_eps=inp.ln_eps)
+
+
+# ------------------------------------------------------------------------------------------------
+# The layer's steps one at a time (for checking each kernel on its own inputs)
+# ------------------------------------------------------------------------------------------------
+
+def f1(X, W1, b1) -> np.ndarray:
+    """Eq. 1: SiLU(X W1 + b1) -> [T, n1]."""
+    X, W1 = _d(X), _d(W1)
+    b1 = _d(b1)
+    T, d = X.shape
+    n1 = W1.shape[1]
+    out = np.empty((T, n1), np.float64)
+    _load().oracle_f1(T, d, n1, _p(X), _p(W1), _p(b1), _p(out))
+    return out
+
+
+def attention(seq_offsets, uvqk, *, num_heads: int, d_qk: int, d_v: int, timestamps=None,
+              pos_table=None, time_table=None, alibi_slopes=None, scale: float) -> np.ndarray:
+    """Eq. 2 on a given UVQK [T, n1] -> AV [T, H*d_v]."""
+    off = _i(seq_offsets)
+    uvqk = _d(uvqk)
+    T = uvqk.shape[0]
+    ts, pos, tim, ali = _i(timestamps), _d(pos_table), _d(time_table), _d(alibi_slopes)
+    P = 0 if pos is None else pos.shape[1]
+    Tb = 0 if tim is None else tim.shape[1]
+    av = np.empty((T, num_heads * d_v), np.float64)
+    _load().oracle_attention(len(off) - 1, _p(off), num_heads, d_qk, d_v, _p(uvqk), _p(ts),
+                             _p(pos), P, _p(tim), Tb, _p(ali), float(scale), _p(av))
+    return av
+
+
+def ln_gate(av, uvqk, ln_w, ln_b, *, num_heads: int, d_qk: int, d_v: int,
+            ln_eps: float = 1e-5) -> np.ndarray:
+    """Eq. 3, first half: LayerNorm(AV) * U (U = block 0 of UVQK) -> [T, H*d_v]."""
+    av, uvqk, ln_w, ln_b = _d(av), _d(uvqk), _d(ln_w), _d(ln_b)
+    T = av.shape[0]
+    g = np.empty_like(av)
+    _load().oracle_ln_gate(T, num_heads, d_qk, d_v, _p(av), _p(uvqk), _p(ln_w), _p(ln_b),
+                           float(ln_eps), _p(g))
+    return g
+
+
+def f2(g, W2, b2, X) -> np.ndarray:
+    """Eq. 3, second half, plus the residual: G W2 + b2 + X -> [T, d]."""
+    g, W2, b2, X = _d(g), _d(W2), _d(b2), _d(X)
+    T, w = g.shape
+    d = W2.shape[1]
+    Y = np.empty((T, d), np.float64)
+    _load().oracle_f2(T, w, d, _p(g), _p(W2), _p(b2), _p(X), _p(Y))
+    return Y
