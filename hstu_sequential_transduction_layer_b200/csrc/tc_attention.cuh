@@ -36,6 +36,9 @@ enum AttnBias { BIAS_NONE = 0, BIAS_RAB = 1, BIAS_ALIBI = 2 };
 constexpr int ATT_BM = 128;       // query rows per item
 constexpr int ATT_BN = 128;       // keys per tile
 constexpr int ATT_TB_CAP = 512;   // time buckets staged in shared memory (more: read from global)
+constexpr int ATT_POS_CAP = 8192; // position buckets staged in shared memory (more: read from global)
+constexpr int ATT_THREADS = 320;  // producer warp, MMA warp, 8 pointwise warps
+constexpr int ATT_PW = 256;       // pointwise threads
 
 template <int HD>
 struct AttnCfg {
@@ -44,13 +47,17 @@ struct AttnCfg {
   static constexpr int KV_TILE = HD / 64 * BOX;             // K or V tile
   static constexpr int NST = HD == 64 ? 4 : 2;              // K/V ring depth
   static constexpr int STAGE_BYTES = 2 * KV_TILE;
-  static constexpr int TS_BYTES = 2 * ATT_BN * 8;           // key timestamps, double-buffered
-  static constexpr int TT_BYTES = 2 * ATT_TB_CAP * 4;       // time table, double-buffered
+  static constexpr int POS_BYTES = ATT_POS_CAP * 4;          // half position table
+  static constexpr int TT_BYTES = ATT_TB_CAP * 4;            // half time table
+  static constexpr int TS_BYTES = 2 * ATT_BN * 8;            // key timestamps, double-buffered
+  static constexpr int FLAG_BYTES = 64;                      // per-warp "keys sorted" flags
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM_TILES = Q_BYTES + NST * STAGE_BYTES;
-  static constexpr int SMEM = SMEM_TILES + TS_BYTES + TT_BYTES + BAR_BYTES + 1024;
-  static constexpr int TMEM_COLS = 512;                     // S0 | S1 | O
+  static constexpr int SMEM =
+      SMEM_TILES + POS_BYTES + TT_BYTES + TS_BYTES + FLAG_BYTES + BAR_BYTES + 1024;
+  static constexpr int TMEM_COLS = 512;   // S0 [0,128) | S1 [128,256) | O [256,256+hd) | P0 | P1
   static constexpr int O_COL = 256;
+  static constexpr int P_COL = 384;       // P_b (bf16 pairs, 64 columns each) at P_COL + 64 b
 };
 
 // Header of the attention workspace: item count, then per-sequence (start, length), then items.
@@ -137,8 +144,117 @@ __device__ __forceinline__ int time_bucket(int64_t ti, int64_t tj) {
   return 63 - __clzll((long long)((unsigned long long)dlt + 1ull));
 }
 
+// SiLU of x = 2h without the final multiplication by `scale` (applied to O in the epilogue):
+// SiLU(x) = x * sigmoid(x) = h + h * tanh(h) with h = x / 2; one MUFU operation.
+__device__ __forceinline__ float silu_from_half(float h) {
+  return fmaf(h, sm100::tanh_approx(h), h);
+}
+
+// All 128 pointwise threads arrive and wait (bounded) on a group barrier.
+__device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& count, volatile int* abort_flag) {
+  sm100::mbar_arrive(bar);
+  const bool ok = sm100::mbar_wait(bar, count & 1u, abort_flag);
+  count++;
+  return ok;
+}
+
+// How a pointwise warp forms the bias of its 32 rows x 64 keys of one tile.
+enum TileMode { TILE_GENERAL = 0, TILE_CONST = 1, TILE_TABLE = 2, TILE_ALIBI = 3 };
+
+// Fast path over 32 columns (col0 .. col0+31 of this warp's 64): h = S/2 + hb, P = SiLU(2h).
+//   hb = (SPLIT && col >= cstar ? hb1 : hb0)            time bias with at most one bucket change,
+//                                                        plus a constant position bias (TILE_CONST)
+//      + hpos[i - key]  (TILE_TABLE; prow = hpos + i - first key of the half)
+//   TILE_ALIBI: hb = hb0 + col * m/2 with hb0 = -(m/2) (i - first key of the half)
+template <int MODE, bool SPLIT>
+__device__ __forceinline__ void fast_chunk(const uint32_t (&sv)[32], int col0, float hb0, float hb1,
+                                           int cstar, const float* prow, float half_slope,
+                                           uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    float p2[2];
+#pragma unroll
+    for (int u = 0; u < 2; u++) {
+      const int col = col0 + e + u;
+      float hb = (SPLIT && col >= cstar) ? hb1 : hb0;
+      if (MODE == TILE_TABLE) hb += prow[-col];
+      if (MODE == TILE_ALIBI) hb = fmaf((float)col, half_slope, hb0);
+      p2[u] = silu_from_half(fmaf(__uint_as_float(sv[e + u]), 0.5f, hb));
+    }
+    pk[e / 2] = pack_bf16x2(p2[0], p2[1]);
+  }
+}
+
+template <int MODE, bool SPLIT>
+__device__ __forceinline__ void fast_tile(uint32_t s_col, uint32_t p_col, float hb0, float hb1,
+                                          int cstar, const float* prow, float half_slope) {
+  uint32_t sa[32], sb[32], pk[16];
+  sm100::tmem_ld32(s_col, sa);
+  sm100::tmem_ld32(s_col + 32, sb);
+  sm100::tmem_ld_wait(sa);
+  sm100::tmem_ld_wait(sb);
+  fast_chunk<MODE, SPLIT>(sa, 0, hb0, hb1, cstar, prow, half_slope, pk);
+  sm100::tmem_st16(p_col, pk);
+  fast_chunk<MODE, SPLIT>(sb, 32, hb0, hb1, cstar, prow, half_slope, pk);
+  sm100::tmem_st16(p_col + 16, pk);
+}
+
+// Exact path over this warp's 64 keys: clamped position bucket, per-element time bucket, causal mask.
+struct GeneralArgs {
+  int i, kbase, P, Tb, staged_n;
+  int64_t ti;
+  const int64_t* tsh;       // staged timestamps of this warp's 64 keys
+  const float *hpos, *htt, *pos_h, *tim_h;
+  float half_slope;
+  bool has_pos, has_time;
+};
+
+template <int BIAS>
+__device__ __forceinline__ void general_chunk(const uint32_t (&sv)[32], int col0,
+                                              const GeneralArgs& a, uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    float p2[2];
+#pragma unroll
+    for (int u = 0; u < 2; u++) {
+      const int col = col0 + e + u;
+      const int dist = a.i - (a.kbase + col);
+      float hb = 0.0f;
+      if (BIAS == BIAS_RAB) {
+        if (a.has_pos) {
+          const int pi = dist < 0 ? 0 : (dist < a.P - 1 ? dist : a.P - 1);
+          hb += pi < a.staged_n ? a.hpos[pi] : 0.5f * __ldg(a.pos_h + pi);
+        }
+        if (a.has_time) {
+          int b = time_bucket(a.ti, a.tsh[col]);
+          b = b < a.Tb - 1 ? b : a.Tb - 1;
+          hb += b < ATT_TB_CAP ? a.htt[b] : 0.5f * __ldg(a.tim_h + b);
+        }
+      } else if (BIAS == BIAS_ALIBI) {
+        hb = -a.half_slope * (float)dist;
+      }
+      const float h = fmaf(__uint_as_float(sv[e + u]), 0.5f, hb);
+      p2[u] = dist < 0 ? 0.0f : silu_from_half(h);
+    }
+    pk[e / 2] = pack_bf16x2(p2[0], p2[1]);
+  }
+}
+
+template <int BIAS>
+__device__ __forceinline__ void general_tile(uint32_t s_col, uint32_t p_col, const GeneralArgs& a) {
+  uint32_t sa[32], sb[32], pk[16];
+  sm100::tmem_ld32(s_col, sa);
+  sm100::tmem_ld32(s_col + 32, sb);
+  sm100::tmem_ld_wait(sa);
+  sm100::tmem_ld_wait(sb);
+  general_chunk<BIAS>(sa, 0, a, pk);
+  sm100::tmem_st16(p_col, pk);
+  general_chunk<BIAS>(sb, 32, a, pk);
+  sm100::tmem_st16(p_col + 16, pk);
+}
+
 template <int HD, int BIAS>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(ATT_THREADS, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnParams prm, AttnSchedule sch) {
   using Cfg = AttnCfg<HD>;
   using namespace sm100;
@@ -147,9 +263,11 @@ __global__ void __launch_bounds__(192, 1)
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* q_s = smem;
   uint8_t* kv_s = smem + Cfg::Q_BYTES;
-  int64_t* ts_s = reinterpret_cast<int64_t*>(smem + Cfg::SMEM_TILES);           // [2][128]
-  float* tt_s = reinterpret_cast<float*>(smem + Cfg::SMEM_TILES + Cfg::TS_BYTES);  // [2][cap]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::SMEM_TILES + Cfg::TS_BYTES + Cfg::TT_BYTES);
+  float* hpos_s = reinterpret_cast<float*>(smem + Cfg::SMEM_TILES);               // 0.5 * pos[h][.]
+  float* htt_s = hpos_s + ATT_POS_CAP;                                             // 0.5 * tim[h][.]
+  int64_t* ts_s = reinterpret_cast<int64_t*>(htt_s + ATT_TB_CAP);                  // [2][128]
+  int* flags_s = reinterpret_cast<int*>(ts_s + 2 * ATT_BN);                        // [2][4]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(flags_s) + Cfg::FLAG_BYTES);
   uint64_t* kv_full = bars;                  // [NST]
   uint64_t* kv_empty = kv_full + Cfg::NST;   // [NST]
   uint64_t* s_full = kv_empty + Cfg::NST;    // [2]
@@ -159,7 +277,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* q_empty = q_full + 1;
   uint64_t* o_full = q_empty + 1;
   uint64_t* o_empty = o_full + 1;
-  uint64_t* drain = o_empty + 1;
+  uint64_t* pw_bar = o_empty + 1;
+  uint64_t* drain = pw_bar + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -175,13 +294,14 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int b = 0; b < 2; b++) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 4);
-      mbar_init(&ts_full[b], 128);
+      mbar_init(&p_full[b], 8);
+      mbar_init(&ts_full[b], ATT_PW);
     }
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     mbar_init(o_full, 1);
-    mbar_init(o_empty, 4);
+    mbar_init(o_empty, 8);
+    mbar_init(pw_bar, ATT_PW);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -277,7 +397,7 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t v_addr = smem_u32(kv_s + (gj % Cfg::NST) * Cfg::STAGE_BYTES + Cfg::KV_TILE);
 #pragma unroll
           for (int kk = 0; kk < ATT_BN / 16; kk++)
-            mma_ts(tmem + Cfg::O_COL, tmem + (gj & 1u) * 128 + kk * 8,
+            mma_ts(tmem + Cfg::O_COL, tmem + Cfg::P_COL + (gj & 1u) * 64 + kk * 8,
                    sdesc_sw128(v_addr + kk * 2048, Cfg::BOX, 1024), idesc_o,
                    (j | kk) != 0 ? 1u : 0u);
           mma_commit(&kv_empty[gj % Cfg::NST]);
@@ -292,83 +412,144 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------------ pointwise warps
-    const int q = warp & 3;              // TMEM lane quadrant
-    const int tid = threadIdx.x - 64;    // 0..127 among the pointwise warps
-    const int r = q * 32 + lane;         // query row inside the tile
+    // Two warps per TMEM lane quadrant: warp (q, half) handles query rows q*32.. and the keys
+    // half*64 .. half*64+63 of every tile.
+    const int pw = warp - 2;              // 0..7
+    const int q = warp & 3;               // TMEM lane quadrant
+    const int half = pw >> 2;             // which 64 keys of a tile
+    const int tid = threadIdx.x - 64;     // 0..255
+    const int r = q * 32 + lane;          // query row inside the tile
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    uint32_t g = 0, k = 0;
+    const bool has_pos = BIAS == BIAS_RAB && prm.pos != nullptr;
+    const bool has_time = BIAS == BIAS_RAB && prm.tim != nullptr;
+    const int P = prm.P, Tb = prm.Tb;
+    uint32_t g = 0, k = 0, pw_cnt = 0;
+    int staged_head = -1, staged_n = 0;  // what hpos_s / htt_s hold
     for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x, k++) {
       const int64_t item = sch.items[it];
       const int64_t seq = item & 0xffffffffLL;
       const int qt = (int)((item >> 32) & 0xffff), h = (int)(item >> 48);
       const int64_t row0 = sch.seqinfo[2 * seq], n = sch.seqinfo[2 * seq + 1];
-      const int i = qt * ATT_BM + r;                  // local query index
+      const int q0 = qt * ATT_BM;
+      const int i = q0 + r;                        // local query index of this thread's row
       const int nk = qt + 1;
-      float* tt = tt_s + (k & 1u) * ATT_TB_CAP;
-      int64_t ti = 0;
-      const float* pos_h = nullptr;
-      const float* tim_h = nullptr;
-      float slope = 0.0f;
-      if (BIAS == BIAS_RAB) {
-        if (prm.tim) {
-          tim_h = prm.tim + (int64_t)h * prm.Tb;
-          for (int e = tid; e < prm.Tb && e < ATT_TB_CAP; e += 128) tt[e] = tim_h[e];
-          ti = prm.ts[row0 + (i < n ? i : n - 1)];
-        }
-        if (prm.pos) pos_h = prm.pos + (int64_t)h * prm.P;
-      } else if (BIAS == BIAS_ALIBI) {
-        slope = prm.alibi[h];
+      const float* pos_h = has_pos ? prm.pos + (int64_t)h * P : nullptr;
+      const float* tim_h = has_time ? prm.tim + (int64_t)h * Tb : nullptr;
+      // stage the halved bias tables of this head (the first 128*(qt+1) position buckets suffice)
+      const int need = min(min(P, (qt + 1) * ATT_BN), ATT_POS_CAP);
+      if ((has_pos || has_time) && (h != staged_head || need > staged_n)) {
+        if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;   // earlier items are done reading
+        if (has_pos)
+          for (int e = tid; e < need; e += ATT_PW) hpos_s[e] = 0.5f * __ldg(pos_h + e);
+        if (has_time)
+          for (int e = tid; e < Tb && e < ATT_TB_CAP; e += ATT_PW) htt_s[e] = 0.5f * __ldg(tim_h + e);
+        staged_head = h;
+        staged_n = need;
+        if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;   // tables visible to all
+      }
+      const int64_t ti = has_time ? prm.ts[row0 + (i < n ? i : n - 1)] : 0;
+      const float half_slope = BIAS == BIAS_ALIBI ? 0.5f * prm.alibi[h] : 0.0f;
+      // key timestamps of the next tile, loaded one tile ahead (threads 0..127: one key each)
+      int64_t t_c = 0, t_n = 0;
+      if (has_time && tid < ATT_BN) {
+        const int kj = tid;
+        t_c = prm.ts[row0 + (kj < n ? kj : n - 1)];
+        t_n = prm.ts[row0 + (kj + 1 < n ? kj + 1 : n - 1)];
       }
       bool ok = true;
       for (int j = 0; j < nk; j++) {
         const uint32_t gj = g + j;
         const int key0 = j * ATT_BN;
-        if (BIAS == BIAS_RAB && prm.tim) {
-          int64_t* tsb = ts_s + (gj & 1u) * ATT_BN;
-          const int kj = key0 + tid;
-          tsb[tid] = prm.ts[row0 + (kj < n ? kj : n - 1)];
+        const int kbase = key0 + half * 64;       // first key of this warp's half
+        const bool diag = (j == qt);
+        const int64_t* tsh = ts_s + (gj & 1u) * ATT_BN + half * 64;
+        int mode = TILE_GENERAL;
+        bool split = false;
+        float hb0 = 0.0f, hb1 = 0.0f;
+        int cstar = 64;
+        bool time_fast = true;
+        if (has_time) {
+          if (tid < ATT_BN) {
+            ts_s[(gj & 1u) * ATT_BN + tid] = t_c;
+            const bool sorted = __all_sync(0xffffffffu, tid == ATT_BN - 1 || t_c <= t_n);
+            if (lane == 0) flags_s[(gj & 1u) * 4 + pw] = sorted ? 1 : 0;
+          }
           mbar_arrive(&ts_full[gj & 1u]);
+          if (tid < ATT_BN && j + 1 < nk) {   // prefetch the next tile's keys
+            const int kj = key0 + ATT_BN + tid;
+            t_c = prm.ts[row0 + (kj < n ? kj : n - 1)];
+            t_n = prm.ts[row0 + (kj + 1 < n ? kj + 1 : n - 1)];
+          }
           if (!mbar_wait(&ts_full[gj & 1u], (gj >> 1) & 1u, abort_flag)) { ok = false; break; }
+          const int* fl = flags_s + (gj & 1u) * 4 + 2 * half;
+          const bool sorted = (fl[0] & fl[1]) != 0;
+          const int bf = time_bucket(ti, tsh[0]), bl = time_bucket(ti, tsh[63]);
+          time_fast = __all_sync(0xffffffffu, sorted && bf - bl <= 1 && bf < 62);
+          if (time_fast) {
+            if (bf != bl) {
+              // keys are sorted, so the bucket steps down once: find the first key in the lower one
+              const int64_t thr = ti + 1 - (1LL << bf);
+              int lo = 1, hi = 63;
+              while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (tsh[mid] > thr) hi = mid; else lo = mid + 1;
+              }
+              cstar = lo;
+            }
+            split = __any_sync(0xffffffffu, bf != bl);
+            const int b0 = bf < Tb - 1 ? bf : Tb - 1, b1 = bl < Tb - 1 ? bl : Tb - 1;
+            hb0 = b0 < ATT_TB_CAP ? htt_s[b0] : 0.5f * __ldg(tim_h + b0);
+            hb1 = b1 < ATT_TB_CAP ? htt_s[b1] : 0.5f * __ldg(tim_h + b1);
+          }
         }
+        if (!diag && time_fast) {
+          if (BIAS == BIAS_ALIBI) {
+            mode = TILE_ALIBI;
+            hb0 = -half_slope * (float)(i - kbase);
+          } else if (!has_pos) {
+            mode = TILE_CONST;
+          } else {
+            const int min_d = q0 - (kbase + 63), max_d = q0 + ATT_BM - 1 - kbase;
+            if (min_d >= P - 1) {
+              mode = TILE_CONST;
+              const float hp = P - 1 < staged_n ? hpos_s[P - 1] : 0.5f * __ldg(pos_h + P - 1);
+              hb0 += hp;
+              hb1 += hp;
+            } else if (max_d <= P - 1 && max_d < staged_n) {
+              mode = TILE_TABLE;
+            }
+          }
+        }
+        const float* prow = hpos_s + (i - kbase);
         if (!mbar_wait(&s_full[gj & 1u], (gj >> 1) & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t s_col = t_lane + (gj & 1u) * 128;
-        const int64_t* tsb = ts_s + (gj & 1u) * ATT_BN;
-        const bool diag = (j == qt);
-#pragma unroll 1
-        for (int c = 0; c < 4; c++) {
-          uint32_t sv[32];
-          tmem_ld32(s_col + c * 32, sv);
-          tmem_ld_wait();
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float pv[2];
-#pragma unroll
-            for (int u = 0; u < 2; u++) {
-              const int jj = key0 + c * 32 + e + u;   // local key index
-              float x = __uint_as_float(sv[e + u]);
-              const int dist = i - jj;
-              if (BIAS == BIAS_RAB) {
-                if (pos_h) {
-                  const int pi = dist < 0 ? 0 : (dist < prm.P - 1 ? dist : prm.P - 1);
-                  x += __ldg(pos_h + pi);
-                }
-                if (tim_h) {
-                  int b = time_bucket(ti, tsb[c * 32 + e + u]);
-                  b = b < prm.Tb - 1 ? b : prm.Tb - 1;
-                  x += (b < ATT_TB_CAP) ? tt[b] : __ldg(tim_h + b);
-                }
-              } else if (BIAS == BIAS_ALIBI) {
-                x = fmaf(-slope, (float)dist, x);
-              }
-              float p = prm.scale * silu_fast(x);
-              if (diag && jj > i) p = 0.0f;
-              pv[u] = p;
-            }
-            pk[e / 2] = pack_bf16x2(pv[0], pv[1]);
-          }
-          tmem_st16(s_col + c * 16, pk);
+        const uint32_t s_col = t_lane + (gj & 1u) * 128 + half * 64;
+        const uint32_t p_col = t_lane + Cfg::P_COL + (gj & 1u) * 64 + half * 32;
+        if (mode == TILE_TABLE) {
+          if (split) fast_tile<TILE_TABLE, true>(s_col, p_col, hb0, hb1, cstar, prow, half_slope);
+          else fast_tile<TILE_TABLE, false>(s_col, p_col, hb0, hb1, cstar, prow, half_slope);
+        } else if (mode == TILE_CONST) {
+          if (split) fast_tile<TILE_CONST, true>(s_col, p_col, hb0, hb1, cstar, prow, half_slope);
+          else fast_tile<TILE_CONST, false>(s_col, p_col, hb0, hb1, cstar, prow, half_slope);
+        } else if (mode == TILE_ALIBI) {
+          fast_tile<TILE_ALIBI, false>(s_col, p_col, hb0, hb1, cstar, prow, half_slope);
+        } else {
+          GeneralArgs a;
+          a.i = i;
+          a.kbase = kbase;
+          a.P = P;
+          a.Tb = Tb;
+          a.staged_n = staged_n;
+          a.ti = ti;
+          a.tsh = tsh;
+          a.hpos = hpos_s;
+          a.htt = htt_s;
+          a.pos_h = pos_h;
+          a.tim_h = tim_h;
+          a.half_slope = half_slope;
+          a.has_pos = has_pos;
+          a.has_time = has_time;
+          general_tile<BIAS>(s_col, p_col, a);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -377,21 +558,22 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (!ok) break;
       g += nk;
-      // epilogue: O rows -> AV
+      // epilogue: AV rows = scale * O (this warp's half of the head's columns)
       if (!mbar_wait(o_full, k & 1u, abort_flag)) break;
       tc_fence_after();
       const bool valid = i < n;
-      float* dst = prm.av + (row0 + i) * (int64_t)(H * HD) + h * HD;
-#pragma unroll 1
-      for (int c = 0; c < HD / 32; c++) {
+      float* dst = prm.av + (row0 + i) * (int64_t)(H * HD) + h * HD + half * (HD / 2);
+#pragma unroll
+      for (int c = 0; c < HD / 64; c++) {
         uint32_t ov[32];
-        tmem_ld32(t_lane + Cfg::O_COL + c * 32, ov);
-        tmem_ld_wait();
+        tmem_ld32(t_lane + Cfg::O_COL + half * (HD / 2) + c * 32, ov);
+        tmem_ld_wait(ov);
         if (valid) {
 #pragma unroll
           for (int v = 0; v < 8; v++)
-            reinterpret_cast<uint4*>(dst + c * 32)[v] =
-                make_uint4(ov[4 * v], ov[4 * v + 1], ov[4 * v + 2], ov[4 * v + 3]);
+            reinterpret_cast<float4*>(dst + c * 32)[v] =
+                make_float4(prm.scale * __uint_as_float(ov[4 * v]), prm.scale * __uint_as_float(ov[4 * v + 1]),
+                            prm.scale * __uint_as_float(ov[4 * v + 2]), prm.scale * __uint_as_float(ov[4 * v + 3]));
         }
       }
       tc_fence_before();

@@ -111,7 +111,7 @@ hstu_status_t launch_attention_kernel(const CUtensorMap& tm, const AttnParams& p
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
       cudaSuccess)
     return HSTU_ERR_CUDA;
-  kern<<<grid, 192, Cfg::SMEM, st>>>(tm, prm, sch);
+  kern<<<grid, ATT_THREADS, Cfg::SMEM, st>>>(tm, prm, sch);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
