@@ -88,9 +88,13 @@ inline hstu_status_t launch_gemm_f2(int64_t T, int d, int wv, const bf16* G, con
 }
 
 // Attention workspace: header (256 B), per-sequence (start, length) pairs, then the item list (one
-// 8-byte entry per (sequence, 128-row query tile, head); at most H * (ceil(T/128) + B) of them).
+// 8-byte entry per (sequence, pair of 128-row query tiles, head); at most H * (ceil(T/256) + B)).
+inline int64_t attention_capacity(int64_t T, int64_t B, int H) {
+  return (int64_t)H * ((T + ATT_ITEM_ROWS - 1) / ATT_ITEM_ROWS + B);
+}
+
 inline size_t attention_workspace_bytes(int64_t T, int64_t B, int H) {
-  const int64_t items = (int64_t)H * ((T + ATT_BM - 1) / ATT_BM + B);
+  const int64_t items = attention_capacity(T, B, H);
   return (size_t)(256 + ((16 * B + 255) / 256) * 256 + 8 * items);
 }
 
@@ -126,17 +130,17 @@ inline hstu_status_t launch_attention(int64_t T, int64_t B, int H, int hd, int64
   if (T >= (1LL << 31) || H >= (1 << 15)) return HSTU_ERR_UNSUPPORTED;
   if (ws_bytes < attention_workspace_bytes(T, B, H)) return HSTU_ERR_INVALID_ARG;
   const int64_t max_len = max_seq_len > 0 ? max_seq_len : T;
-  const int64_t max_tiles64 = (max_len + ATT_BM - 1) / ATT_BM;
-  if (max_tiles64 > 16384) return HSTU_ERR_UNSUPPORTED;  // scheduler counters live in shared memory
-  const int max_tiles = (int)max_tiles64;
+  const int64_t max_pairs64 = (max_len + ATT_ITEM_ROWS - 1) / ATT_ITEM_ROWS;
+  if (max_pairs64 > 16384) return HSTU_ERR_UNSUPPORTED;  // scheduler counters live in shared memory
+  const int max_pairs = (int)max_pairs64;
   const AttnSchedule sch = attention_schedule_view(ws, B);
-  const size_t sched_smem = 2 * (size_t)(max_tiles + 1) * sizeof(int);
+  const size_t sched_smem = 2 * (size_t)(max_pairs + 1) * sizeof(int);
   if (sched_smem > 48 * 1024 &&
       cudaFuncSetAttribute(attn_schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)sched_smem) != cudaSuccess)
     return HSTU_ERR_CUDA;
-  const int64_t capacity = (int64_t)H * ((T + ATT_BM - 1) / ATT_BM + B);
-  attn_schedule_kernel<<<1, 1024, sched_smem, st>>>(off, B, T, H, max_tiles, capacity, sch);
+  const int64_t capacity = attention_capacity(T, B, H);
+  attn_schedule_kernel<<<1, 1024, sched_smem, st>>>(off, B, T, H, max_pairs, capacity, sch);
   count_launch();
   if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
 
