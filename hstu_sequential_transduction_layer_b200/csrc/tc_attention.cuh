@@ -54,10 +54,12 @@ struct AttnCfg {
   static constexpr int POS_CAP = HD == 64 ? 8192 : 7168;    // position buckets staged (half values)
   static constexpr int OFF_KV = 2 * Q_BYTES;
   static constexpr int OFF_TS = OFF_KV + NST * STAGE_BYTES;          // [NST][128] int64
-  static constexpr int OFF_FLAG = OFF_TS + NST * ATT_BN * 8;         // [NST] int
+  static constexpr int OFF_TS32 = OFF_TS + NST * ATT_BN * 8;         // [NST][128] int32, relative
+  static constexpr int OFF_FLAG = OFF_TS32 + NST * ATT_BN * 4;       // [NST] int
   static constexpr int OFF_POS = OFF_FLAG + 64;                      // [POS_CAP] float
   static constexpr int OFF_TT = OFF_POS + POS_CAP * 4;               // [TB_CAP] float
-  static constexpr int OFF_BAR = OFF_TT + ATT_TB_CAP * 4;
+  static constexpr int OFF_CLZ = OFF_TT + ATT_TB_CAP * 4;            // [32] float
+  static constexpr int OFF_BAR = OFF_CLZ + 32 * 4;
   static constexpr int SMEM = OFF_BAR + 256;
   static constexpr int TMEM_COLS = 512;
   // TMEM columns.  hd = 64: S_A | S_B | O_A | O_B | P_A | P_B (128, 128, 64, 64, 64, 64), P apart
@@ -164,7 +166,11 @@ __device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& count, volat
 }
 
 // How a pointwise warp forms the bias of its 32 rows x 128 keys of one tile.
-enum TileMode { TILE_GENERAL = 0, TILE_FAST = 1 };
+enum TileMode { TILE_GENERAL = 0, TILE_FAST = 1, TILE_GEN32 = 2 };
+
+// Key-tile flags written by the producer next to the staged timestamps.
+constexpr int KEYS_SORTED = 1;   // non-decreasing along the tile
+constexpr int KEYS_REL32 = 2;    // every key's timestamp is within +-2^30 of the sequence's first
 
 // Fast path over 32 columns (col0 + e, e = 0..31): h = S/2 + hb, P = SiLU(2h).
 //   BIAS_RAB:   hb = hpos_ext[i - key] + (SPLIT && col >= cstar ? hb1 : hb0), where hpos_ext holds
@@ -231,12 +237,40 @@ __device__ __forceinline__ void general_chunk(const uint32_t (&sv)[32], int dist
   }
 }
 
+// Exact path with 32-bit timestamps relative to the sequence's first one: the time bucket
+// floor(log2(1 + max(ti - tj, 0))) is 31 - clz(max(ti1 - tj, 1)) with ti1 = ti + 1, and hclz[c]
+// holds the halved time bias of bucket min(31 - c, Tb - 1).  Causal mask as in general_chunk.
+__device__ __forceinline__ void general32_chunk(const uint32_t (&sv)[32], int dist0, int P,
+                                                int staged_n, int ti1, const int* tsk32,
+                                                const float* hpos, const float* hclz,
+                                                const float* pos_h, uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    float p2[2];
+#pragma unroll
+    for (int u = 0; u < 2; u++) {
+      const int dist = dist0 - (e + u);
+      float hb = 0.0f;
+      if (pos_h) {
+        const int pi = dist < 0 ? 0 : dist;   // the staged table already clamps to P-1
+        hb = pi < staged_n ? hpos[pi] : 0.5f * __ldg(pos_h + (pi < P - 1 ? pi : P - 1));
+      }
+      const int d1 = max(ti1 - tsk32[e + u], 1);
+      hb += hclz[__clz(d1)];
+      const float h = fmaf(__uint_as_float(sv[e + u]), 0.5f, hb);
+      p2[u] = dist < 0 ? 0.0f : silu_from_half(h);
+    }
+    pk[e / 2] = pack_bf16x2(p2[0], p2[1]);
+  }
+}
+
 // Per-tile state of one pointwise thread.
 struct TileArgs {
-  int i, key0, P, Tb, staged_n, cstar;
+  int i, key0, P, Tb, staged_n, cstar, ti1;
   int64_t ti;
   const int64_t* tsk;       // staged timestamps of the tile's 128 keys
-  const float *hpos, *htt, *pos_h, *tim_h;
+  const int* tsk32;         // the same, relative to the sequence's first timestamp
+  const float *hpos, *htt, *hclz, *pos_h, *tim_h;
   float hb0, hb1, half_slope;
 };
 
@@ -246,6 +280,9 @@ __device__ __forceinline__ void do_chunk(const uint32_t (&sv)[32], int col0, con
   if (MODE == TILE_GENERAL) {
     general_chunk<BIAS>(sv, a.i - a.key0 - col0, a.P, a.Tb, a.staged_n, a.ti, a.tsk + col0, a.hpos,
                         a.htt, a.pos_h, a.tim_h, a.half_slope, pk);
+  } else if (MODE == TILE_GEN32) {
+    general32_chunk(sv, a.i - a.key0 - col0, a.P, a.staged_n, a.ti1, a.tsk32 + col0, a.hpos, a.hclz,
+                    a.pos_h, pk);
   } else if (BIAS == BIAS_ALIBI) {
     fast_chunk<BIAS, false>(sv, fmaf((float)col0, a.half_slope, a.hb0), 0.0f, 0, nullptr,
                             a.half_slope, pk);
@@ -313,6 +350,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   uint8_t* q_s = smem;                                            // [2][Q_BYTES]: A, B
   uint8_t* kv_s = smem + Cfg::OFF_KV;
   int64_t* ts_ring = reinterpret_cast<int64_t*>(smem + Cfg::OFF_TS);
+  int* ts32_ring = reinterpret_cast<int*>(smem + Cfg::OFF_TS32);
+  float* hclz_s = reinterpret_cast<float*>(smem + Cfg::OFF_CLZ);
   int* flag_ring = reinterpret_cast<int*>(smem + Cfg::OFF_FLAG);
   float* hpos_s = reinterpret_cast<float*>(smem + Cfg::OFF_POS);  // 0.5 * pos[h][.]
   float* htt_s = reinterpret_cast<float*>(smem + Cfg::OFF_TT);    // 0.5 * tim[h][.]
@@ -407,20 +446,28 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         if (has_time) {
-          // the tile's key timestamps (clamped to the sequence) and whether they are sorted
+          // the tile's key timestamps (clamped to the sequence), also relative to the sequence's
+          // first one as int32, and whether they are sorted and fit
+          const int64_t t0 = prm.ts[row0];
           int64_t* dst = ts_ring + st * ATT_BN;
+          int* dst32 = ts32_ring + st * ATT_BN;
           int64_t t4[4];
+          bool fits = true;
 #pragma unroll
           for (int e = 0; e < 4; e++) {
             const int64_t kj = (int64_t)j * ATT_BN + 4 * lane + e;
             t4[e] = prm.ts[row0 + (kj < n ? kj : n - 1)];
             dst[4 * lane + e] = t4[e];
+            const int64_t rel = t4[e] - t0;
+            fits = fits && rel > -(1LL << 30) && rel < (1LL << 30);
+            dst32[4 * lane + e] = (int)rel;
           }
           const int64_t next = __shfl_down_sync(0xffffffffu, t4[0], 1);
           const bool mine = t4[0] <= t4[1] && t4[1] <= t4[2] && t4[2] <= t4[3] &&
                             (lane == 31 || t4[3] <= next);
           const bool sorted = __all_sync(0xffffffffu, mine);
-          if (lane == 0) flag_ring[st] = sorted ? 1 : 0;
+          const bool rel32 = __all_sync(0xffffffffu, fits);
+          if (lane == 0) flag_ring[st] = (sorted ? KEYS_SORTED : 0) | (rel32 ? KEYS_REL32 : 0);
         }
         __syncwarp();
         if (lane == 0) {
@@ -563,8 +610,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         // hpos_s[d] = pos[h][min(d, P-1)] / 2 for every distance d < need (zeros without a table)
         for (int e = tid; e < need; e += ATT_PW)
           hpos_s[e] = has_pos ? 0.5f * __ldg(pos_h + (e < P - 1 ? e : P - 1)) : 0.0f;
-        if (has_time)
+        if (has_time) {
           for (int e = tid; e < Tb && e < ATT_TB_CAP; e += ATT_PW) htt_s[e] = 0.5f * __ldg(tim_h + e);
+          if (tid < 32) hclz_s[tid] = 0.5f * __ldg(tim_h + (31 - tid < Tb - 1 ? 31 - tid : Tb - 1));
+        }
         staged_head = h;
         staged_n = need;
         if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;   // tables visible to all
@@ -577,6 +626,9 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       const int q0 = qt * ATT_BM;
       const int i = q0 + r;                        // local query index of this thread's row
       const int64_t ti = has_time ? prm.ts[row0 + (i < n ? i : n - 1)] : 0;
+      const int64_t ti_rel = has_time ? ti - prm.ts[row0] : 0;
+      const bool row_rel32 = ti_rel > -(1LL << 30) && ti_rel < (1LL << 30);
+      const int ti1 = (int)ti_rel + 1;
       const float half_slope = BIAS == BIAS_ALIBI ? 0.5f * prm.alibi[h] : 0.0f;
       bool ok = true;
       for (int j = 0; j <= qt; j++) {
@@ -584,6 +636,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         const int key0 = j * ATT_BN;
         const bool diag = (j == qt);
         const int64_t* tsk = ts_ring + (gj % Cfg::NST) * ATT_BN;
+        const int* tsk32 = ts32_ring + (gj % Cfg::NST) * ATT_BN;
+        bool rel32 = false;
         // ---- per-tile bias set-up (overlaps the tensor core's work on S)
         bool split = false;
         float hb0 = 0.0f, hb1 = 0.0f;
@@ -592,17 +646,34 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         if (has_time) {
           // the tile's timestamps arrived with its K/V stage
           if (!mbar_wait(&kv_full[gj % Cfg::NST], (gj / Cfg::NST) & 1u, abort_flag)) { ok = false; break; }
-          const bool sorted = flag_ring[gj % Cfg::NST] != 0;
-          const int bf = time_bucket(ti, tsk[0]), bl = time_bucket(ti, tsk[ATT_BN - 1]);
+          const int flags = flag_ring[gj % Cfg::NST];
+          const bool sorted = (flags & KEYS_SORTED) != 0;
+          rel32 = __all_sync(0xffffffffu, (flags & KEYS_REL32) && row_rel32);
+          int bf, bl;
+          if (rel32) {
+            bf = 31 - __clz(max(ti1 - tsk32[0], 1));
+            bl = 31 - __clz(max(ti1 - tsk32[ATT_BN - 1], 1));
+          } else {
+            bf = time_bucket(ti, tsk[0]);
+            bl = time_bucket(ti, tsk[ATT_BN - 1]);
+          }
           time_fast = __all_sync(0xffffffffu, sorted && bf - bl <= 1 && bf < 62);
           if (time_fast) {
             if (bf != bl) {
               // the keys are sorted, so the bucket steps down once: find the first key in the lower one
-              const int64_t thr = ti + 1 - (1LL << bf);
               int lo = 1, hi = ATT_BN - 1;
-              while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if (tsk[mid] > thr) hi = mid; else lo = mid + 1;
+              if (rel32) {
+                const int thr = ti1 - (1 << bf);
+                while (lo < hi) {
+                  const int mid = (lo + hi) >> 1;
+                  if (tsk32[mid] > thr) hi = mid; else lo = mid + 1;
+                }
+              } else {
+                const int64_t thr = ti + 1 - (1LL << bf);
+                while (lo < hi) {
+                  const int mid = (lo + hi) >> 1;
+                  if (tsk[mid] > thr) hi = mid; else lo = mid + 1;
+                }
               }
               cstar = lo;
             }
@@ -623,6 +694,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             mode = TILE_FAST;
           }
         }
+        if (mode == TILE_GENERAL && has_time && rel32) mode = TILE_GEN32;
         TileArgs ta;
         ta.i = i;
         ta.key0 = key0;
@@ -631,7 +703,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         ta.staged_n = staged_n;
         ta.cstar = cstar;
         ta.ti = ti;
+        ta.ti1 = ti1;
         ta.tsk = tsk;
+        ta.tsk32 = tsk32;
+        ta.hclz = hclz_s;
         ta.hpos = hpos_s;
         ta.htt = htt_s;
         ta.pos_h = pos_h;
@@ -656,6 +731,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
           if (mode == TILE_FAST) {
             if (split) pointwise_tile_sep<BIAS, TILE_FAST, true>(s_col, p_col, ta, wait_pf, consumed);
             else pointwise_tile_sep<BIAS, TILE_FAST, false>(s_col, p_col, ta, wait_pf, consumed);
+          } else if (BIAS == BIAS_RAB && mode == TILE_GEN32) {
+            pointwise_tile_sep<BIAS, TILE_GEN32, false>(s_col, p_col, ta, wait_pf, consumed);
           } else {
             pointwise_tile_sep<BIAS, TILE_GENERAL, false>(s_col, p_col, ta, wait_pf, consumed);
           }
@@ -663,6 +740,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         } else if (mode == TILE_FAST) {
           if (split) pointwise_tile<BIAS, TILE_FAST, true>(s_col, ta);
           else pointwise_tile<BIAS, TILE_FAST, false>(s_col, ta);
+        } else if (BIAS == BIAS_RAB && mode == TILE_GEN32) {
+          pointwise_tile<BIAS, TILE_GEN32, false>(s_col, ta);
         } else {
           pointwise_tile<BIAS, TILE_GENERAL, false>(s_col, ta);
         }
