@@ -29,7 +29,7 @@ HSTU_F32, HSTU_BF16 = 0, 1
 EXPORTED = ["hstu_layer_fwd", "hstu_layer_fwd_workspace_size", "hstu_f1_fwd", "hstu_attention_fwd",
             "hstu_attention_workspace_size", "hstu_ln_gate_fwd", "hstu_f2_fwd",
             "hstu_token_embed_fwd", "hstu_status_string", "hstu_get_device_status", "hstu_version",
-            "hstu_launch_count"]
+            "hstu_launch_count", "hstu_attention_fwd_noalloc"]
 
 
 class HstuShape(ctypes.Structure):
@@ -63,6 +63,7 @@ def _load() -> ctypes.CDLL:
         "hstu_f1_fwd": ([SH, P, P, P, P, P], ctypes.c_int),
         "hstu_attention_fwd": ([SH, P, P, P, P, P, P, F32, P, P, S, P], ctypes.c_int),
         "hstu_attention_workspace_size": ([SH], S),
+        "hstu_attention_fwd_noalloc": ([SH, P, P, P, P, P, P, F32, P, P], ctypes.c_int),
         "hstu_ln_gate_fwd": ([SH, P, P, P, P, P, P], ctypes.c_int),
         "hstu_f2_fwd": ([SH, P, P, P, P, P, P], ctypes.c_int),
         "hstu_token_embed_fwd": ([I64, I32, P, P, P, I64, P, I64, P, P], ctypes.c_int),
@@ -200,6 +201,17 @@ def hstu_attention_fwd(shape: HstuShape, uvqk, seq_offsets, timestamps, pos_tabl
                                    _ptr(timestamps), _ptr(pos_table), _ptr(time_table),
                                    _ptr(alibi_slopes), float(scale), _ptr(av), _ptr(workspace),
                                    workspace.numel(), _stream(stream)), "hstu_attention_fwd")
+    return av
+
+
+def hstu_attention_fwd_noalloc(shape: HstuShape, uvqk, seq_offsets, timestamps, pos_table,
+                               time_table, alibi_slopes, scale: float, av, stream=None):
+    """hstu_attention_fwd with the tile schedule in the library's fixed device scratch array (no
+    workspace argument, nothing allocated).  Calls that overlap on the GPU share that array and race."""
+    _check(_lib.hstu_attention_fwd_noalloc(ctypes.byref(shape), _ptr(uvqk), _ptr(seq_offsets),
+                                           _ptr(timestamps), _ptr(pos_table), _ptr(time_table),
+                                           _ptr(alibi_slopes), float(scale), _ptr(av),
+                                           _stream(stream)), "hstu_attention_fwd_noalloc")
     return av
 
 

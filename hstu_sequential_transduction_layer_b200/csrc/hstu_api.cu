@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "hbm_kernels.cuh"
@@ -11,7 +12,31 @@
 
 using namespace hstu;
 
+// Scratch of hstu_attention_fwd_noalloc: room for the attention tile schedule, in a fixed device
+// array that every GPU loading this library holds until the process exits.  Host code must not
+// use the array's name as a device address; it looks the address up with cudaGetSymbolAddress.
+static constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
 namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device (looked up once per device).
+hstu_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HSTU_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return HSTU_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return HSTU_OK;
+}
 
 constexpr size_t kAlign = 256;
 size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
@@ -240,6 +265,27 @@ hstu_status_t hstu_attention_fwd(const hstu_shape_t* shape, const void* uvqk,
     return HSTU_ERR_INVALID_ARG;
   return run_attention(*shape, uvqk, seq_offsets, timestamps, pos_table, time_table, alibi_slopes,
                        scale, av, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+hstu_status_t hstu_attention_fwd_noalloc(const hstu_shape_t* shape, const void* uvqk,
+                                         const int64_t* seq_offsets, const int64_t* timestamps,
+                                         const float* pos_table, const float* time_table,
+                                         const float* alibi_slopes, float scale, void* av,
+                                         void* stream) {
+  hstu_status_t rc = check_shape(shape);
+  if (rc != HSTU_OK) return rc;
+  if (shape->total_tokens == 0) return HSTU_OK;
+  rc = check_bias(shape, timestamps, pos_table, time_table, alibi_slopes, scale);
+  if (rc != HSTU_OK) return rc;
+  if (!uvqk || !av || !seq_offsets) return HSTU_ERR_INVALID_ARG;
+  if (shape->num_seqs == 0) return HSTU_ERR_INVALID_ARG;
+  if (shape->dtype == HSTU_BF16 && !(aligned16(uvqk) && aligned16(av))) return HSTU_ERR_INVALID_ARG;
+  const size_t need = attention_ws_bytes(*shape);
+  if (need > kNoAllocScratchBytes) return HSTU_ERR_UNSUPPORTED;  // schedule larger than the scratch
+  void* scratch = nullptr;
+  if (need > 0 && (rc = noalloc_scratch(&scratch)) != HSTU_OK) return rc;
+  return run_attention(*shape, uvqk, seq_offsets, timestamps, pos_table, time_table, alibi_slopes,
+                       scale, av, scratch, kNoAllocScratchBytes, static_cast<cudaStream_t>(stream));
 }
 
 hstu_status_t hstu_ln_gate_fwd(const hstu_shape_t* shape, const void* av, const void* uvqk,

@@ -130,6 +130,30 @@ hstu_status_t hstu_attention_fwd(const hstu_shape_t* shape, const void* uvqk,
                                  const float* alibi_slopes, float scale, void* av, void* workspace,
                                  size_t workspace_bytes, void* stream);
 size_t hstu_attention_workspace_size(const hstu_shape_t* shape);
+
+/*
+ * hstu_attention_fwd_noalloc -- hstu_attention_fwd without a caller-provided workspace.
+ *
+ * The paper has no counterpart: this entry point exists for callers that cannot allocate device
+ * memory around the call -- for example code whose device memory is owned by a pool or framework
+ * allocator it cannot call into, or a latency-critical path where a cudaMalloc (which may
+ * synchronise the device) is not acceptable.  Arguments, layouts and results are those of
+ * hstu_attention_fwd; it allocates nothing and calls no allocating routine.
+ *
+ * The attention tile schedule lives instead in a fixed 8 MiB device array inside this library,
+ * which every GPU that loads the library keeps until the process exits.  The first call on a device
+ * looks the array's address up (cudaGetSymbolAddress); make that first call before any stream
+ * capture.  Shapes whose schedule needs more than 8 MiB (hstu_attention_workspace_size(shape) >
+ * 8 MiB) are rejected with HSTU_ERR_UNSUPPORTED before anything is enqueued.  All calls share the
+ * one array and each call rewrites the part it uses, so calls whose executions overlap on the GPU
+ * (different streams, or different host threads, on the same device) race: serialise them.
+ */
+hstu_status_t hstu_attention_fwd_noalloc(const hstu_shape_t* shape, const void* uvqk,
+                                         const int64_t* seq_offsets, const int64_t* timestamps,
+                                         const float* pos_table, const float* time_table,
+                                         const float* alibi_slopes, float scale, void* av,
+                                         void* stream);
+
 hstu_status_t hstu_ln_gate_fwd(const hstu_shape_t* shape, const void* av, const void* uvqk,
                                const void* ln_w, const void* ln_b, void* g, void* stream);
 hstu_status_t hstu_f2_fwd(const hstu_shape_t* shape, const void* g, const void* W2, const void* b2,
