@@ -3,7 +3,7 @@
  *
  * TEST INFRASTRUCTURE ONLY.  This file is the slow, obviously-correct definition that the CUDA path
  * is checked against.  It is used by the tests, by `__graft_entry__.smoke()` and by the CPU-baseline
- * leg of `bench.py`, and by nothing else.  It shares no code, header, table or helper with the CUDA
+ * and reference legs of `bench.py`, and by nothing else.  It shares no code, header, table or helper with the CUDA
  * path and includes nothing from it.
  *
  * What it computes (per layer, for every sequence s of a jagged batch and local token indices
