@@ -46,6 +46,26 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
+def profiled_traffic(workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was captured on this
+    workload from the kernel source as it is now (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"attention_tc_kernel_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path):
+        if ":" in line and not line.startswith(("|", " ", "#")):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    src = os.path.join(ROOT, fields.get("kernel_source", ""))
+    if not os.path.isfile(src) or "traffic_bytes_per_launch" not in fields:
+        return None
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != fields.get("source_sha256"):
+        return None
+    return int(fields["traffic_bytes_per_launch"])
+
+
 def attention_flops(lengths, H, dqk, dv) -> float:
     """Algorithmic attention FLOPs: 2*H*(dqk+dv) per causal pair (j <= i), masked half excluded."""
     pairs = sum(int(n) * (int(n) + 1) // 2 for n in lengths)
@@ -57,7 +77,7 @@ def gemm_flops(T, d, n1, wv):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled every 100 ms while the timed region runs."""
+    """nvidia-smi clocks and throttle reasons, sampled every 20 ms while the timed region runs."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -79,7 +99,7 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", self.idx, "-lms", "100"], stdout=open(self.path, "w"),
+                 "-i", self.idx, "-lms", "20"], stdout=open(self.path, "w"),
                 stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -239,7 +259,8 @@ def run_ours(args, rank, world, local_rank):
         "attention_frac_of_bf16_peak": round(attn_tflops / tpk, 4),
         "roofline": {"bound": "tensor", "kernel": "attention", "achieved": round(attn_tflops, 2),
                      "peak": tpk, "unit": "TFLOP/s", "frac": round(attn_tflops / tpk, 4),
-                     "traffic": None, "peak_source": f"{peaks_src} bf16 burst (MEASURED_PEAKS.json)"
+                     "traffic": profiled_traffic(args.workload),
+                     "peak_source": f"{peaks_src} bf16 burst (MEASURED_PEAKS.json)"
                      if peaks_src == "measured" else "fallback 1590 TFLOP/s"},
         "kernels": kernels,
         "e2e": e2e,
@@ -362,7 +383,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long_seq", choices=sorted(workloads.WORKLOADS))
