@@ -139,6 +139,24 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------------------
+# Ranks: each rank runs its own batch of sequences (sequences never interact, so there is no
+# exchange on the path); the job's time is the slowest rank's and its work the sum of the ranks'.
+# ------------------------------------------------------------------------------------------------
+
+def combine_over_ranks(local_ms: float, local_tokens: int, world: int, device):
+    """(max over ranks of the timed milliseconds, sum over ranks of the tokens processed).
+    Every rank must call it, in the same order, at the same point of the run."""
+    if world <= 1:
+        return float(local_ms), int(local_tokens)
+    import torch
+    t = torch.tensor([float(local_ms)], dtype=torch.float64, device=device)
+    n = torch.tensor([int(local_tokens)], dtype=torch.int64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    torch.distributed.all_reduce(n, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item()), int(n.item())
+
+
+# ------------------------------------------------------------------------------------------------
 # Our arm
 # ------------------------------------------------------------------------------------------------
 
@@ -213,15 +231,12 @@ def run_ours(args, rank, world, local_rank):
     per_kernel = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in evs])  # ms
     step_ms = per_kernel.sum(axis=1)
     total_ms = float(step_ms.sum())
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms, job_tokens = combine_over_ranks(total_ms, T, world, dev)
     if hstu.device_status() != hstu.HSTU_OK:
         raise SystemExit("device status error in the timed region")
 
     ms_per_step = total_ms / args.steps
-    tokens_per_s = world * T / (ms_per_step * 1e-3)
+    tokens_per_s = job_tokens / (ms_per_step * 1e-3)
     kern_ms = per_kernel.mean(axis=0)
     peaks, peaks_src = load_peaks()
     attn_fl = attention_flops(inp.lengths, H, hd, hd)
@@ -252,7 +267,7 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic (seeded; shapes of the pages' long-sequence encoder benchmark)",
         "config": {"workload": f"{w.name}: B={w.num_seqs} x n={max_len} jagged, d={d}, "
                                f"H={H}x{hd}, rab P={w.n_pos_buckets}/Tb={w.n_time_buckets}, 1 layer",
-                   "global_batch_tokens": world * T, "seq_len": max_len,
+                   "global_batch_tokens": job_tokens, "seq_len": max_len,
                    "parallelism": f"replicas over sequences x{world} (no collective)",
                    "l2": "flushed between timed steps (256 MB write, outside the events)"},
         "attention_tflops": round(attn_tflops, 2),
@@ -306,14 +321,10 @@ def run_e2e(args, hstu, torch, inp, D, shape, dev, stream, world):
         one()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / steps
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms, job_tokens = combine_over_ranks(e0.elapsed_time(e1) / steps, inp.T, world, dev)
     h2d = X_h.numel() * X_h.element_size() + off_h.numel() * 8 + (ts_h.numel() * 8 if ts_h is not None else 0)
     d2h = out_h.numel() * out_h.element_size()
-    return {"value": round(world * inp.T / (ms * 1e-3), 1), "unit": "tokens/s",
+    return {"value": round(job_tokens / (ms * 1e-3), 1), "unit": "tokens/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": round(ms, 4), "steps": steps}
 
