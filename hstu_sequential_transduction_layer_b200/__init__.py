@@ -29,7 +29,7 @@ HSTU_F32, HSTU_BF16 = 0, 1
 EXPORTED = ["hstu_layer_fwd", "hstu_layer_fwd_workspace_size", "hstu_f1_fwd", "hstu_attention_fwd",
             "hstu_attention_workspace_size", "hstu_ln_gate_fwd", "hstu_f2_fwd",
             "hstu_token_embed_fwd", "hstu_status_string", "hstu_get_device_status", "hstu_version",
-            "hstu_launch_count", "hstu_attention_fwd_noalloc"]
+            "hstu_launch_count", "hstu_attention_fwd_noalloc", "hstu_selftest_bounded_wait"]
 
 
 class HstuShape(ctypes.Structure):
@@ -71,6 +71,7 @@ def _load() -> ctypes.CDLL:
         "hstu_get_device_status": ([P], ctypes.c_int),
         "hstu_version": ([], ctypes.c_char_p),
         "hstu_launch_count": ([], ctypes.c_uint64),
+        "hstu_selftest_bounded_wait": ([ctypes.c_uint64, P, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -92,6 +93,14 @@ def status_string(code: int) -> str:
 
 def version() -> str:
     return _lib.hstu_version().decode()
+
+
+def selftest_bounded_wait(limit_ns: int, result, stream=None) -> None:
+    """Runs the device self-test of the library's bounded mbarrier wait (see the C header):
+    `result` is a CUDA int64 tensor of 4 elements; the device status word is left set to
+    HSTU_ERR_DEVICE_TIMEOUT for the caller to read with device_status()."""
+    _check(_lib.hstu_selftest_bounded_wait(int(limit_ns), _ptr(result), _stream(stream)),
+           "hstu_selftest_bounded_wait")
 
 
 def launch_count() -> int:

@@ -131,12 +131,15 @@ hstu_status_t run_ln_gate(const hstu_shape_t& s, const void* av, const void* uvq
     const float* a = (const float*)av;
     const bf16 *u = (const bf16*)uvqk, *w = (const bf16*)ln_w, *b = (const bf16*)ln_b;
     bf16* o = (bf16*)g;
+    // rows of up to 512 elements: one warp per row; wider rows: 2, 4 or 8 warps per row, so that
+    // every lane holds 16 elements and all its loads are in flight at once
+    auto rows_blocks = [&](int rows_per_block) { return (unsigned)((T + rows_per_block - 1) / rows_per_block); };
     switch (wv / 256) {
-      case 1: ln_gate_bf16_kernel<1><<<blocks, 256, 0, st>>>(T, n1, a, u, w, b, s.ln_eps, o); break;
-      case 2: ln_gate_bf16_kernel<2><<<blocks, 256, 0, st>>>(T, n1, a, u, w, b, s.ln_eps, o); break;
-      case 4: ln_gate_bf16_kernel<4><<<blocks, 256, 0, st>>>(T, n1, a, u, w, b, s.ln_eps, o); break;
-      case 8: ln_gate_bf16_kernel<8><<<blocks, 256, 0, st>>>(T, n1, a, u, w, b, s.ln_eps, o); break;
-      case 16: ln_gate_bf16_kernel<16><<<blocks, 256, 0, st>>>(T, n1, a, u, w, b, s.ln_eps, o); break;
+      case 1: ln_gate_bf16_kernel<1, 1><<<rows_blocks(8), 256, 0, st>>>(T, n1, a, u, w, b, s.ln_eps, o); break;
+      case 2: ln_gate_bf16_kernel<2, 1><<<rows_blocks(8), 256, 0, st>>>(T, n1, a, u, w, b, s.ln_eps, o); break;
+      case 4: ln_gate_bf16_kernel<2, 2><<<rows_blocks(4), 256, 0, st>>>(T, n1, a, u, w, b, s.ln_eps, o); break;
+      case 8: ln_gate_bf16_kernel<2, 4><<<rows_blocks(2), 256, 0, st>>>(T, n1, a, u, w, b, s.ln_eps, o); break;
+      case 16: ln_gate_bf16_kernel<2, 8><<<rows_blocks(1), 256, 0, st>>>(T, n1, a, u, w, b, s.ln_eps, o); break;
       default:
         simt::ln_gate_kernel<bf16, float><<<blocks, 256, 0, st>>>(T, (int)wv, n1, a, u, w, b, s.ln_eps, o);
     }
@@ -198,6 +201,35 @@ Workspace layout(const hstu_shape_t& s, void* base) {
 }
 
 }  // namespace
+
+// Self-test of the bounded wait every pipelined kernel uses: one warp waits on an mbarrier that
+// nothing arrives on.  The wait must give up after limit_ns, raise the CTA's abort flag and report
+// HSTU_ERR_DEVICE_TIMEOUT; a second wait must then return at once because the flag is up.
+// result[0], result[1]: the two waits' return values (0 = gave up); result[2]: nanoseconds the
+// first wait took; result[3]: nanoseconds the second took.
+static constexpr uint64_t kSelftestMaxWaitNs = 1000000000ull;
+__global__ void selftest_bounded_wait_kernel(uint64_t limit_ns, long long* result) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    sm100::fence_mbar_init();
+    abort_flag = 0;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    volatile int* flag = &abort_flag;
+    const uint64_t t0 = sm100::globaltimer();
+    const bool first = sm100::mbar_wait(&bar, 0, flag, limit_ns);
+    const uint64_t t1 = sm100::globaltimer();
+    const bool second = sm100::mbar_wait(&bar, 0, flag, limit_ns);
+    const uint64_t t2 = sm100::globaltimer();
+    result[0] = first;
+    result[1] = second;
+    result[2] = (long long)(t1 - t0);
+    result[3] = (long long)(t2 - t1);
+  }
+}
 
 extern "C" {
 
@@ -359,6 +391,12 @@ hstu_status_t hstu_token_embed_fwd(int64_t T, int32_t d, const int64_t* item_ids
   token_embed_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
       T, d, item_ids, action_ids, (const bf16*)item_table, n_items, (const bf16*)action_table,
       n_actions, (bf16*)X);
+  return launch_status();
+}
+
+hstu_status_t hstu_selftest_bounded_wait(uint64_t limit_ns, long long* result, void* stream) {
+  if (limit_ns == 0 || limit_ns > kSelftestMaxWaitNs || !result) return HSTU_ERR_INVALID_ARG;
+  selftest_bounded_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, result);
   return launch_status();
 }
 

@@ -70,13 +70,14 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // Bounded wait on the phase with the given parity.  On time-out it raises the CTA's abort flag and
 // reports HSTU_ERR_DEVICE_TIMEOUT; once the flag is up every later wait returns false at once.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait_suspend(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort_flag = 1;
       report(HSTU_ERR_DEVICE_TIMEOUT);
       return false;

@@ -160,6 +160,22 @@ hstu_status_t hstu_f2_fwd(const hstu_shape_t* shape, const void* g, const void* 
                           const void* X, void* out, void* stream);
 
 /*
+ * hstu_selftest_bounded_wait -- checks, on the device, the bounded wait that every pipelined kernel
+ * of this library uses on its mbarriers.
+ *
+ * The paper has no counterpart: it is a diagnostic of this library's failure detection.  One warp
+ * waits on a barrier that nothing completes; the wait must give up after limit_ns nanoseconds
+ * (0 < limit_ns <= 1e9, else HSTU_ERR_INVALID_ARG before any launch), raise the block's abort flag
+ * and set HSTU_ERR_DEVICE_TIMEOUT in the device status word, and a second wait must return at once
+ * because the flag is up.  Nothing faults and the context stays usable; read (and clear) the status
+ * with hstu_get_device_status afterwards.
+ *
+ *  result   device pointer to 4 int64, written by the kernel: the two waits' outcomes (1 = the
+ *           barrier completed, 0 = gave up), then the nanoseconds each wait took.
+ */
+hstu_status_t hstu_selftest_bounded_wait(uint64_t limit_ns, long long* result, void* stream);
+
+/*
  * hstu_token_embed_fwd -- action-oriented token assembly of the GenRank blog ("item-action
  * organisation"): X[t, :] = bf16(item_table[item_ids[t], :] + action_table[action_ids[t], :]).
  *
