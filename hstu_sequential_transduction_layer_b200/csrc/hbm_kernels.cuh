@@ -7,39 +7,60 @@
 
 namespace hstu {
 
-// Eq. 3, first half ("Actions Speak Louder than Words" paper notes, section 3.1): one warp per
-// token row.  AV arrives in fp32 (see the attention epilogue) and U in bf16.  Lane l owns the
-// 8-element groups l, l+32, ..., l+32*(VPL-1) of the row, so every vector access of a warp covers a
-// contiguous span.  The AV row stays in registers between the mean pass and the variance pass
-// (two-pass biased variance over all H*d_v columns); U, ln_w and ln_b stream in the output pass.
-template <int VPL>
+// Eq. 3, first half ("Actions Speak Louder than Words" paper notes, section 3.1): WPR warps per
+// token row (8 / WPR rows per 256-thread block).  AV arrives in fp32 (see the attention epilogue) and
+// U in bf16.  Lane l of the row's warp w owns the 8-element groups (w*32 + l) + k*32*WPR, k < G, so
+// every vector access of a warp covers a contiguous span.  All of a lane's AV and U bytes are
+// requested up front; the AV values stay in registers between the mean pass and the variance pass
+// (two-pass biased variance over all H*d_v columns), partial sums of a row's warps meet in shared
+// memory.  Row width W = G * WPR * 256 elements.
+template <int G, int WPR>
 __global__ void __launch_bounds__(256) ln_gate_bf16_kernel(int64_t T, int64_t ldu,
                                                            const float* __restrict__ av,
                                                            const bf16* __restrict__ u,
                                                            const bf16* __restrict__ ln_w,
                                                            const bf16* __restrict__ ln_b,
                                                            float eps, bf16* __restrict__ g) {
-  constexpr int W = VPL * 256;  // row width in elements
-  const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32;
-  const int lane = threadIdx.x % 32;
-  if (row >= T) return;
+  constexpr int W = G * WPR * 256;
+  constexpr int ROWS = 8 / WPR;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int rsub = warp / WPR, wsub = warp % WPR;
+  const int64_t row = (int64_t)blockIdx.x * ROWS + rsub;
+  const bool live = row < T;
+  if (WPR == 1 && !live) return;  // no block-wide barrier below in that case
+  __shared__ float red[2][8];
   const float4* x4 = reinterpret_cast<const float4*>(av + row * W);
   const uint4* u4 = reinterpret_cast<const uint4*>(u + row * ldu);
-  float4 x[2 * VPL];
+  float4 x[2 * G];
+  uint4 uv[G];
 #pragma unroll
-  for (int k = 0; k < VPL; k++) {
-    x[2 * k] = __ldcs(x4 + 2 * (lane + 32 * k));
-    x[2 * k + 1] = __ldcs(x4 + 2 * (lane + 32 * k) + 1);
+  for (int k = 0; k < G; k++) {
+    const int grp = wsub * 32 + lane + k * 32 * WPR;
+    if (live) {
+      x[2 * k] = __ldcs(x4 + 2 * grp);
+      x[2 * k + 1] = __ldcs(x4 + 2 * grp + 1);
+      uv[k] = __ldcs(u4 + grp);
+    } else {
+      x[2 * k] = x[2 * k + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+      uv[k] = make_uint4(0, 0, 0, 0);
+    }
   }
   float sum = 0.0f;
 #pragma unroll
-  for (int k = 0; k < 2 * VPL; k++) sum += (x[k].x + x[k].y) + (x[k].z + x[k].w);
+  for (int k = 0; k < 2 * G; k++) sum += (x[k].x + x[k].y) + (x[k].z + x[k].w);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if constexpr (WPR > 1) {
+    if (lane == 0) red[0][warp] = sum;
+    __syncthreads();
+    sum = 0.0f;
+#pragma unroll
+    for (int w = 0; w < WPR; w++) sum += red[0][rsub * WPR + w];
+  }
   const float mean = sum * (1.0f / (float)W);
   float sq = 0.0f;
 #pragma unroll
-  for (int k = 0; k < 2 * VPL; k++) {
+  for (int k = 0; k < 2 * G; k++) {
     const float a = x[k].x - mean, b = x[k].y - mean, c = x[k].z - mean, d = x[k].w - mean;
     sq = fmaf(a, a, sq);
     sq = fmaf(b, b, sq);
@@ -48,17 +69,25 @@ __global__ void __launch_bounds__(256) ln_gate_bf16_kernel(int64_t T, int64_t ld
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+  if constexpr (WPR > 1) {
+    if (lane == 0) red[1][warp] = sq;
+    __syncthreads();
+    sq = 0.0f;
+#pragma unroll
+    for (int w = 0; w < WPR; w++) sq += red[1][rsub * WPR + w];
+  }
+  if (!live) return;
   const float rstd = rsqrtf(sq * (1.0f / (float)W) + eps);
   uint4* g4 = reinterpret_cast<uint4*>(g + row * W);
   const uint4* w4 = reinterpret_cast<const uint4*>(ln_w);
   const uint4* b4 = reinterpret_cast<const uint4*>(ln_b);
 #pragma unroll
-  for (int k = 0; k < VPL; k++) {
-    const uint4 uv = __ldcs(u4 + lane + 32 * k);
-    const uint4 wv = __ldg(w4 + lane + 32 * k), bv = __ldg(b4 + lane + 32 * k);
+  for (int k = 0; k < G; k++) {
+    const int grp = wsub * 32 + lane + k * 32 * WPR;
+    const uint4 wv = __ldg(w4 + grp), bv = __ldg(b4 + grp);
     const float xs[8] = {x[2 * k].x, x[2 * k].y, x[2 * k].z, x[2 * k].w,
                          x[2 * k + 1].x, x[2 * k + 1].y, x[2 * k + 1].z, x[2 * k + 1].w};
-    const uint32_t* us = reinterpret_cast<const uint32_t*>(&uv);
+    const uint32_t* us = reinterpret_cast<const uint32_t*>(&uv[k]);
     const uint32_t* ws = reinterpret_cast<const uint32_t*>(&wv);
     const uint32_t* bs = reinterpret_cast<const uint32_t*>(&bv);
     uint4 out;
@@ -69,7 +98,7 @@ __global__ void __launch_bounds__(256) ln_gate_bf16_kernel(int64_t T, int64_t ld
       const float hi = fmaf((xs[2 * e + 1] - mean) * rstd, bf16_hi(ws[e]), bf16_hi(bs[e])) * bf16_hi(us[e]);
       os[e] = pack_bf16x2(lo, hi);
     }
-    __stcs(g4 + lane + 32 * k, out);
+    __stcs(g4 + grp, out);
   }
 }
 

@@ -5,15 +5,16 @@
 //   EPI_BIAS_SILU:      C = SiLU(acc + bias)              f1: U|V|Q|K = SiLU(X W1 + b1)
 //   EPI_BIAS_RESIDUAL:  C = acc + bias + R                f2: Y = G W2 + b2 + X
 //
-// One CTA per SM (192 threads):
+// One CTA per SM (320 threads):
 //   warp 0      TMA producer: A tile 128x64 and B tile 64xBN per stage into a STAGES-deep ring, both
 //               128-byte swizzled; no multicast.
 //   warp 1      allocates TMEM (two BN-column fp32 accumulators) and issues tcgen05.mma (M=128,
 //               N=BN, K=16) from one thread; tcgen05.commit frees ring stages and publishes
 //               finished accumulators.
-//   warps 2-5   epilogue: tcgen05.ld 32 columns at a time from their TMEM lane quadrant, fused bias
-//               / SiLU / residual in fp32, bf16 stores.  The accumulator is double-buffered, so the
-//               epilogue of tile t overlaps the main loop of tile t+1.
+//   warps 2-9   epilogue, two warps per TMEM lane quadrant, each on half of the tile's columns:
+//               tcgen05.ld 32 columns at a time (the next load in flight during the math), fused
+//               bias / SiLU / residual in fp32, bf16 stores.  The accumulator is double-buffered, so
+//               the epilogue of tile t overlaps the main loop of tile t+1.
 // Output tiles are visited in groups of up to 8 BN-wide column blocks over all row blocks, so that
 // the CTAs in flight share a few MB of A and B in L2.
 #pragma once
@@ -47,8 +48,60 @@ __device__ __forceinline__ void gemm_tile_coords(int64_t t, int tiles_n, int64_t
   nb = (int)g * G + (int)(r % gw);
 }
 
+// SiLU for bf16 outputs with one MUFU op: x * sigmoid(x) = h + h * tanh(h), h = x / 2.  The
+// absolute error is about |x| * 2^-12 (that of tanh.approx), below the bf16 rounding of the result.
+__device__ __forceinline__ float silu_tanh(float x) {
+  const float h = 0.5f * x;
+  return fmaf(h, sm100::tanh_approx(h), h);
+}
+
+// Bias (+ SiLU | + residual) of 32 consecutive columns n .. n+31 of one row, stored as bf16.
+template <int EPI>
+__device__ __forceinline__ void gemm_epilogue_chunk(const uint32_t (&r)[32], const bf16* __restrict__ bias,
+                                                    const bf16* __restrict__ R, bf16* __restrict__ C,
+                                                    int64_t row, int64_t M, int N, int n) {
+  uint4 bvec[4];
+  if (bias) {
+#pragma unroll
+    for (int v = 0; v < 4; v++) bvec[v] = __ldg(reinterpret_cast<const uint4*>(bias + n) + v);
+  } else {
+#pragma unroll
+    for (int v = 0; v < 4; v++) bvec[v] = make_uint4(0, 0, 0, 0);
+  }
+  if (row >= M) return;
+  uint4 rvec[4] = {};
+  if (EPI == EPI_BIAS_RESIDUAL) {
+#pragma unroll
+    for (int v = 0; v < 4; v++) rvec[v] = __ldcs(reinterpret_cast<const uint4*>(R + row * N + n) + v);
+  }
+  uint4 out[4];
+#pragma unroll
+  for (int v = 0; v < 4; v++) {
+    const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bvec[v]);
+    const uint32_t* rw = reinterpret_cast<const uint32_t*>(&rvec[v]);
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&out[v]);
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      float lo = __uint_as_float(r[v * 8 + 2 * e]) + bf16_lo(bw[e]);
+      float hi = __uint_as_float(r[v * 8 + 2 * e + 1]) + bf16_hi(bw[e]);
+      if (EPI == EPI_BIAS_SILU) {
+        lo = silu_tanh(lo);
+        hi = silu_tanh(hi);
+      } else {
+        lo += bf16_lo(rw[e]);
+        hi += bf16_hi(rw[e]);
+      }
+      ow[e] = pack_bf16x2(lo, hi);
+    }
+  }
+#pragma unroll
+  for (int v = 0; v < 4; v++) reinterpret_cast<uint4*>(C + row * N + n)[v] = out[v];
+}
+
+constexpr int kGemmThreads = 320;  // producer warp, MMA warp, 8 epilogue warps
+
 template <int BN, int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int64_t M, int N, int K, const bf16* __restrict__ bias,
                    const bf16* __restrict__ R, bf16* __restrict__ C) {
@@ -78,7 +131,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; a++) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], 8);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -160,65 +213,38 @@ __global__ void __launch_bounds__(192, 1)
     }
     __syncwarp();
   } else {
-    const int q = warp & 3;  // TMEM lane quadrant this warp may access
+    // Epilogue warps 2..9: warp w reads TMEM lane quadrant w % 4 (rows q*32 .. q*32+31 of the
+    // tile) and covers one half of the tile's columns; two warps share each quadrant.
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
+    constexpr int HALF = BN / 2, CHUNKS = HALF / 32;
     uint32_t acc = 0, acc_phase = 0;
     for (int64_t t = blockIdx.x; t < num_tiles; t += gridDim.x) {
       int64_t mb;
       int nb;
       gemm_tile_coords(t, tiles_n, tiles_m, mb, nb);
       const int64_t row = mb * Cfg::BM + q * 32 + lane;
-      const int n0 = nb * BN;
+      const int n0 = nb * BN + half * HALF;
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; c++) {
-        uint32_t r[32];
-        tmem_ld32(t_row + c * 32, r);
-        tmem_ld_wait();
-        const int n = n0 + c * 32;
-        uint4 bvec[4];
-        if (bias) {
+      const uint32_t t_row =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + half * HALF;
+      // the next chunk's TMEM load is in flight while this chunk is converted and stored
+      uint32_t ra[32], rb[32];
+      tmem_ld32(t_row, ra);
 #pragma unroll
-          for (int v = 0; v < 4; v++) bvec[v] = __ldg(reinterpret_cast<const uint4*>(bias + n) + v);
-        } else {
-#pragma unroll
-          for (int v = 0; v < 4; v++) bvec[v] = make_uint4(0, 0, 0, 0);
+      for (int c = 0; c < CHUNKS; c++) {
+        uint32_t(&cur)[32] = (c & 1) ? rb : ra;
+        uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
+        tmem_ld_wait(cur);
+        if (c + 1 < CHUNKS) tmem_ld32(t_row + (c + 1) * 32, nxt);
+        if (c + 1 == CHUNKS) {  // every TMEM read of this accumulator is done: release it early
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[acc]);
         }
-        if (row < M) {
-          uint4 rvec[4] = {};
-          if (EPI == EPI_BIAS_RESIDUAL) {
-#pragma unroll
-            for (int v = 0; v < 4; v++)
-              rvec[v] = __ldcs(reinterpret_cast<const uint4*>(R + row * N + n) + v);
-          }
-          uint4 out[4];
-#pragma unroll
-          for (int v = 0; v < 4; v++) {
-            const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bvec[v]);
-            const uint32_t* rw = reinterpret_cast<const uint32_t*>(&rvec[v]);
-            uint32_t* ow = reinterpret_cast<uint32_t*>(&out[v]);
-#pragma unroll
-            for (int e = 0; e < 4; e++) {
-              float lo = __uint_as_float(r[v * 8 + 2 * e]) + bf16_lo(bw[e]);
-              float hi = __uint_as_float(r[v * 8 + 2 * e + 1]) + bf16_hi(bw[e]);
-              if (EPI == EPI_BIAS_SILU) {
-                lo = silu_fast(lo);
-                hi = silu_fast(hi);
-              } else {
-                lo += bf16_lo(rw[e]);
-                hi += bf16_hi(rw[e]);
-              }
-              ow[e] = pack_bf16x2(lo, hi);
-            }
-          }
-#pragma unroll
-          for (int v = 0; v < 4; v++) reinterpret_cast<uint4*>(C + row * N + n)[v] = out[v];
-        }
+        gemm_epilogue_chunk<EPI>(cur, bias, R, C, row, M, N, n0 + c * 32);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
       acc ^= 1u;
       if (acc == 0) acc_phase ^= 1u;
     }

@@ -61,7 +61,7 @@ hstu_status_t launch_gemm_bn(int64_t M, int N, int K, const bf16* A, const bf16*
     return HSTU_ERR_CUDA;
   const int64_t tiles = ((M + 127) / 128) * (N / BN);
   const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
-  kern<<<grid, 192, Cfg::SMEM, st>>>(ta, tb, M, N, K, bias, R, C);
+  kern<<<grid, kGemmThreads, Cfg::SMEM, st>>>(ta, tb, M, N, K, bias, R, C);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
