@@ -41,8 +41,9 @@ constexpr int ATT_BM = 128;       // query rows per query tile
 constexpr int ATT_BN = 128;       // keys per key tile
 constexpr int ATT_ITEM_ROWS = 2 * ATT_BM;  // query rows per work item (a pair of query tiles)
 constexpr int ATT_TB_CAP = 256;   // time buckets staged in shared memory (more: read from global)
-constexpr int ATT_THREADS = 384;  // producer, 2 MMA issuers, idle warp, 2 pointwise warpgroups
-constexpr int ATT_PW = 256;       // pointwise threads
+constexpr int ATT_THREADS = 640;  // producer, 2 MMA issuers, idle warp, 4 pointwise warpgroups
+constexpr int ATT_PW = 512;       // pointwise threads
+constexpr int ATT_PW_WARPS = 8;   // pointwise warps per query tile
 
 template <int HD>
 struct AttnCfg {
@@ -292,53 +293,40 @@ __device__ __forceinline__ void do_chunk(const uint32_t (&sv)[32], int col0, con
   }
 }
 
-// One warp's 32 rows x 128 keys, as two iterations over a pair of 32-column chunks with statically
-// double-buffered registers: the next chunk's TMEM load is in flight while one is computed.  P
-// (bf16 pairs) overwrites S columns [0, 64) of the same lanes, which this thread has already read.
+// One warp's 32 rows x 64 keys (columns col0 .. col0+63 of the S tile), as two 32-column chunks.
+// P (bf16 pairs) of the 64 keys overwrites the first 32 of these S columns, which this thread has
+// already read.  The next chunk's TMEM load is issued before the current chunk's P is stored.
 template <int BIAS, int MODE, bool SPLIT>
-__device__ __forceinline__ void pointwise_tile(uint32_t s_col, const TileArgs& a) {
-  uint32_t sa[32], sb[32], pk[16];
-  sm100::tmem_ld32(s_col, sa);
-  sm100::tmem_ld_wait(sa);
-#pragma unroll 1
-  for (int cc = 0; cc < 4; cc += 2) {
-    sm100::tmem_ld32(s_col + (cc + 1) * 32, sb);
-    do_chunk<BIAS, MODE, SPLIT>(sa, cc * 32, a, pk);
-    sm100::tmem_st16(s_col + cc * 16, pk);
-    sm100::tmem_ld_wait(sb);
-    if (cc == 0) sm100::tmem_ld32(s_col + 2 * 32, sa);
-    do_chunk<BIAS, MODE, SPLIT>(sb, (cc + 1) * 32, a, pk);
-    sm100::tmem_st16(s_col + (cc + 1) * 16, pk);
-    if (cc == 0) sm100::tmem_ld_wait(sa);
-  }
+__device__ __forceinline__ void pointwise_tile(uint32_t s_col, int col0, const TileArgs& a) {
+  uint32_t sv[32], pk[16];
+  sm100::tmem_ld32(s_col, sv);
+  sm100::tmem_ld_wait(sv);
+  do_chunk<BIAS, MODE, SPLIT>(sv, col0, a, pk);
+  sm100::tmem_ld32(s_col + 32, sv);
+  sm100::tmem_st16(s_col, pk);
+  sm100::tmem_ld_wait(sv);
+  do_chunk<BIAS, MODE, SPLIT>(sv, col0 + 32, a, pk);
+  sm100::tmem_st16(s_col + 16, pk);
 }
 
-// Separate-P form (hd = 64): P goes to its own TMEM columns.  All of S is in registers half-way
-// through the tile, and `s_consumed()` is called then, so that the next S can be computed while the
-// rest of P is.  `p_free()` is called before the first P store: the previous tile's PV must have read
-// the P columns.
+// Separate-P form (hd = 64): P goes to its own TMEM columns.  `s_consumed()` is called as soon as
+// the warp's S columns are in registers, so that the next S can be computed while P is; `p_free()`
+// is called before the first P store: the previous tile's PV must have read the P columns.
 template <int BIAS, int MODE, bool SPLIT, class PFree, class SConsumed>
-__device__ __forceinline__ void pointwise_tile_sep(uint32_t s_col, uint32_t p_col, const TileArgs& a,
-                                                   PFree p_free, SConsumed s_consumed) {
-  uint32_t sa[32], sb[32], pk[16];
-  sm100::tmem_ld32(s_col, sa);
-  sm100::tmem_ld_wait(sa);
-  sm100::tmem_ld32(s_col + 32, sb);
-  do_chunk<BIAS, MODE, SPLIT>(sa, 0, a, pk);
+__device__ __forceinline__ void pointwise_tile_sep(uint32_t s_col, uint32_t p_col, int col0,
+                                                   const TileArgs& a, PFree p_free,
+                                                   SConsumed s_consumed) {
+  uint32_t sv[32], pk[16];
+  sm100::tmem_ld32(s_col, sv);
+  sm100::tmem_ld_wait(sv);
+  do_chunk<BIAS, MODE, SPLIT>(sv, col0, a, pk);
+  sm100::tmem_ld32(s_col + 32, sv);
   p_free();
   sm100::tmem_st16(p_col, pk);
-  sm100::tmem_ld_wait(sb);
-  sm100::tmem_ld32(s_col + 64, sa);
-  do_chunk<BIAS, MODE, SPLIT>(sb, 32, a, pk);
-  sm100::tmem_st16(p_col + 16, pk);
-  sm100::tmem_ld_wait(sa);
-  sm100::tmem_ld32(s_col + 96, sb);
-  sm100::tmem_ld_wait(sb);
+  sm100::tmem_ld_wait(sv);
   s_consumed();
-  do_chunk<BIAS, MODE, SPLIT>(sa, 64, a, pk);
-  sm100::tmem_st16(p_col + 32, pk);
-  do_chunk<BIAS, MODE, SPLIT>(sb, 96, a, pk);
-  sm100::tmem_st16(p_col + 48, pk);
+  do_chunk<BIAS, MODE, SPLIT>(sv, col0 + 32, a, pk);
+  sm100::tmem_st16(p_col + 16, pk);
 }
 
 template <int HD, int BIAS>
@@ -387,10 +375,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     }
     for (int x = 0; x < 2; x++) {
       mbar_init(&s_full[x], 1);
-      mbar_init(&p_full[x], 4);
+      mbar_init(&p_full[x], ATT_PW_WARPS);
       mbar_init(&o_full[x], 1);
-      mbar_init(&o_empty[x], 4);
-      mbar_init(&s_free[x], 4);
+      mbar_init(&o_empty[x], ATT_PW_WARPS);
+      mbar_init(&s_free[x], ATT_PW_WARPS);
       mbar_init(&p_free[x], 1);
     }
     mbar_init(q_full, 1);
@@ -518,9 +506,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       auto issue_pv = [&](uint32_t gg, bool accumulate) {
         const uint32_t v_addr = smem_u32(kv_s + (gg % Cfg::NST) * Cfg::STAGE_BYTES + Cfg::KV_TILE);
 #pragma unroll
-        for (int kk = 0; kk < ATT_BN / 16; kk++)
-          mma_ts(o_tmem, p_tmem + kk * 8, sdesc_sw128(v_addr + kk * 2048, Cfg::BOX, 1024), idesc_o,
+        for (int kk = 0; kk < ATT_BN / 16; kk++) {
+          // P of keys 16kk .. 16kk+15: 8 columns; with P aliased into S, the P of keys 64..127 sits
+          // at S column 64 (the first S column the second half's warps read)
+          const uint32_t pc = Cfg::SEP_P ? kk * 8 : (kk & 3) * 8 + (kk >> 2) * 64;
+          mma_ts(o_tmem, p_tmem + pc, sdesc_sw128(v_addr + kk * 2048, Cfg::BOX, 1024), idesc_o,
                  (accumulate || kk > 0) ? 1u : 0u);
+        }
       };
       for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x, k++) {
         const int64_t item = sch.items[it];
@@ -584,12 +576,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ pointwise warpgroups
-    const int x = (warp - 4) >> 2;        // 0: query tile A, 1: query tile B
+    const int x = (warp - 4) >> 3;        // 0: query tile A, 1: query tile B
+    const int half = (warp >> 2) & 1;     // key columns [64 half, 64 half + 64) of each S tile
     const int q = warp & 3;               // TMEM lane quadrant
-    const int tid = threadIdx.x - 128;    // 0..255 over both warpgroups
+    const int tid = threadIdx.x - 128;    // 0..511 over the four warpgroups
     const int r = q * 32 + lane;          // query row inside the tile
+    const int col0 = half * 64;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    const uint32_t s_col = t_lane + x * 128;
+    const uint32_t s_col = t_lane + x * 128 + col0;
     const bool has_pos = BIAS == BIAS_RAB && prm.pos != nullptr;
     const int P = prm.P, Tb = prm.Tb;
     uint32_t g = 0, kx = 0, gx = 0, pw_cnt = 0;
@@ -727,23 +721,23 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_free[x]);
           };
-          const uint32_t p_col = t_lane + Cfg::P_COL + x * 64;
+          const uint32_t p_col = t_lane + Cfg::P_COL + x * 64 + half * 32;
           if (mode == TILE_FAST) {
-            if (split) pointwise_tile_sep<BIAS, TILE_FAST, true>(s_col, p_col, ta, wait_pf, consumed);
-            else pointwise_tile_sep<BIAS, TILE_FAST, false>(s_col, p_col, ta, wait_pf, consumed);
+            if (split) pointwise_tile_sep<BIAS, TILE_FAST, true>(s_col, p_col, col0, ta, wait_pf, consumed);
+            else pointwise_tile_sep<BIAS, TILE_FAST, false>(s_col, p_col, col0, ta, wait_pf, consumed);
           } else if (BIAS == BIAS_RAB && mode == TILE_GEN32) {
-            pointwise_tile_sep<BIAS, TILE_GEN32, false>(s_col, p_col, ta, wait_pf, consumed);
+            pointwise_tile_sep<BIAS, TILE_GEN32, false>(s_col, p_col, col0, ta, wait_pf, consumed);
           } else {
-            pointwise_tile_sep<BIAS, TILE_GENERAL, false>(s_col, p_col, ta, wait_pf, consumed);
+            pointwise_tile_sep<BIAS, TILE_GENERAL, false>(s_col, p_col, col0, ta, wait_pf, consumed);
           }
           if (!pf_ok) { ok = false; break; }
         } else if (mode == TILE_FAST) {
-          if (split) pointwise_tile<BIAS, TILE_FAST, true>(s_col, ta);
-          else pointwise_tile<BIAS, TILE_FAST, false>(s_col, ta);
+          if (split) pointwise_tile<BIAS, TILE_FAST, true>(s_col, col0, ta);
+          else pointwise_tile<BIAS, TILE_FAST, false>(s_col, col0, ta);
         } else if (BIAS == BIAS_RAB && mode == TILE_GEN32) {
-          pointwise_tile<BIAS, TILE_GEN32, false>(s_col, ta);
+          pointwise_tile<BIAS, TILE_GEN32, false>(s_col, col0, ta);
         } else {
-          pointwise_tile<BIAS, TILE_GENERAL, false>(s_col, ta);
+          pointwise_tile<BIAS, TILE_GENERAL, false>(s_col, col0, ta);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -757,11 +751,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       if (!mbar_wait(&o_full[x], kx & 1u, abort_flag)) break;
       tc_fence_after();
       const bool valid = i < n;
-      float* dst = prm.av + (row0 + i) * (int64_t)(H * HD) + h * HD;
+      // this warp's half of the head's columns
+      float* dst = prm.av + (row0 + i) * (int64_t)(H * HD) + h * HD + half * (HD / 2);
 #pragma unroll
-      for (int c = 0; c < HD / 32; c++) {
+      for (int c = 0; c < HD / 64; c++) {
         uint32_t ov[32];
-        tmem_ld32(t_lane + Cfg::O_COL + x * Cfg::O_STRIDE + c * 32, ov);
+        tmem_ld32(t_lane + Cfg::O_COL + x * Cfg::O_STRIDE + half * (HD / 2) + c * 32, ov);
         tmem_ld_wait(ov);
         if (valid) {
 #pragma unroll
