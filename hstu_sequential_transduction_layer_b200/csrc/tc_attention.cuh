@@ -9,8 +9,12 @@
 //
 // Work decomposition: one work item = (sequence, pair of adjacent 128-row query tiles A = 2m and
 // B = 2m+1, head).  Every K/V tile an item loads serves both query tiles.  A scheduling kernel builds
-// the item list on the device from seq_offsets, heaviest first (pair m reads 2m+2 key tiles), and
-// the persistent attention CTAs take items round-robin.  Sequences are never padded: tiles that
+// the item list on the device from seq_offsets: batches of a few (sequence, head) groups, heaviest
+// pair first inside a batch (pair m reads 2m+2 key tiles).  When the K/V of the whole batch of
+// sequences is small against L2, the list is one batch and CTA b takes items b, b + grid, ...;
+// otherwise each CTA's producer claims the next item from a global counter whenever it starts one,
+// and hands it to the CTA's other warps through a small ring in shared memory, so that the CTAs
+// running at the same time stay inside one or two batches whose K/V fit in L2.  Sequences are never padded: tiles that
 // straddle a sequence end read the next rows (or TMA zero fill past T) and the causal mask, which
 // coincides with the length mask for valid rows, removes them; rows past the end are not stored.
 //
@@ -44,6 +48,8 @@ constexpr int ATT_TB_CAP = 256;   // time buckets staged in shared memory (more:
 constexpr int ATT_THREADS = 640;  // producer, 2 MMA issuers, idle warp, 4 pointwise warpgroups
 constexpr int ATT_PW = 512;       // pointwise threads
 constexpr int ATT_PW_WARPS = 8;   // pointwise warps per query tile
+constexpr int ATT_ITEM_RING = 4;  // work items handed from the producer to the other roles
+constexpr int ATT_ITEM_READERS = 2 + 2 * ATT_PW_WARPS;  // MMA issuers and pointwise warps
 
 template <int HD>
 struct AttnCfg {
@@ -61,7 +67,7 @@ struct AttnCfg {
   static constexpr int OFF_TT = OFF_POS + POS_CAP * 4;               // [TB_CAP] float
   static constexpr int OFF_CLZ = OFF_TT + ATT_TB_CAP * 4;            // [32] float
   static constexpr int OFF_BAR = OFF_CLZ + 32 * 4;
-  static constexpr int SMEM = OFF_BAR + 256;
+  static constexpr int SMEM = OFF_BAR + 512;
   static constexpr int TMEM_COLS = 512;
   // TMEM columns.  hd = 64: S_A | S_B | O_A | O_B | P_A | P_B (128, 128, 64, 64, 64, 64), P apart
   // from S so that S(j+1) can be computed while P(j) still waits for its PV product.  hd = 128:
@@ -71,24 +77,76 @@ struct AttnCfg {
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
-// Header of the attention workspace: item count, then per-sequence (start, length), then items.
+// Header of the attention workspace: [0] item count, [1] next item to hand out (the persistent CTAs
+// take items from this counter in list order), then per-sequence (start, length), then items.
 struct AttnSchedule {
-  int64_t* header;    // [0] = number of items
+  int64_t* header;
   int64_t* seqinfo;   // [2*B]: start row, length (clamped to [0, T])
   int64_t* items;     // packed: seq | pair << 32 | head << 48
 };
 
-// Builds the item list, heaviest (largest query-tile pair index) first.  One CTA; dynamic shared
-// memory holds 2 * (max_pairs + 1) counters.  Bad offsets are clamped (and reported) so that every
-// item addresses rows inside [0, T).
+// Builds the item list.  Sequences are ranked by decreasing number of query-tile pairs p; group
+// g = rank * H + h is one (sequence, head); consecutive groups form batches of `gb` groups, sized by
+// the host so that a batch's K and V fit in L2 with room to spare.  The list holds the batches in
+// order, and inside a batch the items by decreasing pair index m (heaviest first: pair m reads 2m+2
+// key tiles), groups in order for equal m.  CTAs take items from the list in order as they become
+// free: the CTAs running at the same time work on one or two batches, whose K/V stay in L2, each
+// batch starts with its big items, and the list ends with the smallest items of the shortest
+// sequences (load balance).  One CTA; dynamic shared memory holds three arrays over p.  Bad offsets
+// are clamped (and reported) so that every item addresses rows inside [0, T).
+struct SchedTables {
+  const int* ge;                   // ge[p]: sequences with at least p pairs (p = 1 .. max_pairs + 1)
+  const unsigned long long* pge;   // pge[p]: pairs summed over the sequences with at least p pairs
+  int max_pairs;
+};
+
+// Pairs of the sequence at rank r (0 <= r < ge[1]): the largest p with ge[p] > r.
+__device__ __forceinline__ int pairs_at_rank(const SchedTables& t, uint32_t r) {
+  int lo = 1, hi = t.max_pairs;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if ((uint32_t)t.ge[mid] > r) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Pairs summed over the sequences of rank < r.
+__device__ __forceinline__ unsigned long long pairs_before_rank(const SchedTables& t, uint32_t r) {
+  if ((int)r >= t.ge[1]) return t.pge[1];
+  const int p = pairs_at_rank(t, r);
+  return t.pge[p + 1] + (unsigned long long)(r - (uint32_t)t.ge[p + 1]) * p;
+}
+
+// Items of the groups before group g (g <= number of groups < 2^31).
+__device__ __forceinline__ unsigned long long items_before_group(const SchedTables& t, uint32_t g,
+                                                                 uint32_t H) {
+  const uint32_t r = g / H, h = g - r * H;
+  const unsigned long long before = pairs_before_rank(t, r) * H;
+  return (int)r < t.ge[1] ? before + (unsigned long long)h * pairs_at_rank(t, r) : before;
+}
+
+// Sum over the groups before group g of max(0, pairs - m - 1): the items of those groups whose
+// pair index exceeds m.  Only the first ge[m + 2] ranks have more than m + 1 pairs.
+__device__ __forceinline__ unsigned long long items_above_before_group(const SchedTables& t,
+                                                                       uint32_t g, uint32_t H,
+                                                                       int m) {
+  const uint32_t r = g / H, h = g - r * H;
+  const uint32_t c = (uint32_t)t.ge[m + 2];
+  const uint32_t rr = r < c ? r : c;
+  unsigned long long v = (pairs_before_rank(t, rr) - (unsigned long long)(m + 1) * rr) * H;
+  if (r < c) v += (unsigned long long)h * (unsigned long long)(pairs_at_rank(t, r) - m - 1);
+  return v;
+}
+
 __global__ void __launch_bounds__(1024) attn_schedule_kernel(const int64_t* __restrict__ off,
                                                              int64_t B, int64_t T, int H,
-                                                             int max_pairs, int64_t capacity,
-                                                             AttnSchedule sch) {
-  extern __shared__ int sched_smem[];
-  int* cnt = sched_smem;                // cnt[m]: sequences with more than m query-tile pairs
-  int* cursor = sched_smem + max_pairs + 1;
-  for (int q = threadIdx.x; q <= max_pairs; q += blockDim.x) cnt[q] = 0, cursor[q] = 0;
+                                                             int max_pairs, int gb,
+                                                             int64_t capacity, AttnSchedule sch) {
+  extern __shared__ unsigned long long sched_smem[];
+  unsigned long long* pge = sched_smem;                               // [max_pairs + 2]
+  int* ge = reinterpret_cast<int*>(sched_smem + max_pairs + 2);       // [max_pairs + 2]
+  int* cnt = ge + max_pairs + 2;                                      // [max_pairs + 2]
+  for (int q = threadIdx.x; q < max_pairs + 2; q += blockDim.x) cnt[q] = 0, ge[q] = 0, pge[q] = 0;
   __syncthreads();
   for (int64_t s = threadIdx.x; s < B; s += blockDim.x) {
     const int64_t a = clamp64(off[s], 0, T);
@@ -102,34 +160,75 @@ __global__ void __launch_bounds__(1024) attn_schedule_kernel(const int64_t* __re
     }
     sch.seqinfo[2 * s] = a;
     sch.seqinfo[2 * s + 1] = n;
-    if (pairs > 0) atomicAdd(&cnt[pairs - 1], 1);
+    atomicAdd(&cnt[pairs], 1);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    int run = 0;  // suffix sums: cnt[m] = #sequences with pairs > m
-    for (int m = max_pairs - 1; m >= 0; m--) {
-      run += cnt[m];
-      cnt[m] = run;
+    int run = 0;
+    unsigned long long prun = 0;
+    for (int p = max_pairs; p >= 1; p--) {
+      run += cnt[p];
+      prun += (unsigned long long)cnt[p] * p;
+      ge[p] = run;
+      pge[p] = prun;
+      cnt[p] = 0;  // reused below as the rank cursor of pair count p
     }
-    int64_t base = 0;  // first slot (in sequences) of pair index m, for m descending
-    for (int m = max_pairs - 1; m >= 0; m--) {
-      cursor[m] = (int)base;
-      base += cnt[m];
-    }
+    const unsigned long long total = prun * (unsigned long long)H;
     // valid offsets give at most H * (ceil(T/256) + B) items, the list's capacity; overlapping
     // (invalid) offsets could give more: those are reported and the excess is dropped
-    if (base * H > capacity) report(HSTU_ERR_DEVICE_BAD_OFFSETS);
-    sch.header[0] = base * H < capacity ? base * H : capacity;
+    if ((int64_t)total > capacity) report(HSTU_ERR_DEVICE_BAD_OFFSETS);
+    sch.header[0] = (int64_t)total < capacity ? (int64_t)total : capacity;
+    sch.header[1] = 0;
   }
   __syncthreads();
-  for (int64_t s = threadIdx.x; s < B; s += blockDim.x) {
+  const SchedTables tab{ge, pge, max_pairs};
+  // 32-bit index arithmetic: the host guarantees B * H < 2^31
+  const uint32_t H32 = (uint32_t)H;
+  const uint32_t ngroups = (uint32_t)ge[1] * H32;
+  const uint32_t gbe = (uint32_t)gb < ngroups ? (uint32_t)gb : (ngroups > 0 ? ngroups : 1u);
+  if (gbe >= ngroups) {
+    // one batch: the items with pair index m follow the H * sum over ranks of max(0, p - m - 1)
+    // items with a larger one, in group order; one thread per sequence
+    for (int64_t s = threadIdx.x; s < B; s += blockDim.x) {
+      const int64_t n = sch.seqinfo[2 * s + 1];
+      const int p = (int)((n + ATT_ITEM_ROWS - 1) / ATT_ITEM_ROWS);
+      if (p == 0) continue;
+      const uint32_t g = (uint32_t)(ge[p + 1] + atomicAdd(&cnt[p], 1)) * H32;
+      for (int m = 0; m < p; m++) {
+        const unsigned long long above =
+            (pge[m + 2] - (unsigned long long)(m + 1) * (unsigned long long)ge[m + 2]) * H32;
+        for (uint32_t h = 0; h < H32; h++) {
+          const unsigned long long slot = above + g + h;
+          if ((int64_t)slot < capacity)
+            sch.items[slot] = (int64_t)s | ((int64_t)m << 32) | ((int64_t)h << 48);
+        }
+      }
+    }
+    return;
+  }
+  // several batches: one warp per sequence writes its H * pairs items
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int64_t s = warp; s < B; s += blockDim.x / 32) {
     const int64_t n = sch.seqinfo[2 * s + 1];
-    const int pairs = (int)((n + ATT_ITEM_ROWS - 1) / ATT_ITEM_ROWS);
-    for (int m = 0; m < pairs; m++) {
-      const int slot = atomicAdd(&cursor[m], 1);
-      for (int h = 0; h < H; h++)
-        if ((int64_t)slot * H + h < capacity)
-          sch.items[(int64_t)slot * H + h] = (int64_t)s | ((int64_t)m << 32) | ((int64_t)h << 48);
+    const int p = (int)((n + ATT_ITEM_ROWS - 1) / ATT_ITEM_ROWS);
+    if (p == 0) continue;
+    uint32_t rank = 0;
+    if (lane == 0) rank = (uint32_t)(ge[p + 1] + atomicAdd(&cnt[p], 1));
+    rank = __shfl_sync(0xffffffffu, rank, 0);
+    for (uint32_t e = lane; e < (uint32_t)p * H32; e += 32) {
+      const uint32_t h = e / (uint32_t)p;
+      const int m = p - 1 - (int)(e - h * (uint32_t)p);
+      const uint32_t g = rank * H32 + h;
+      // the batch [g0, g1) holding g; inside it, the items with a larger pair index come first,
+      // then those with pair index m of the batch's groups before g (all have more than m pairs)
+      const uint32_t g0 = gbe >= ngroups ? 0u : g / gbe * gbe;
+      const uint32_t g1 = ngroups - g0 > gbe ? g0 + gbe : ngroups;
+      const unsigned long long above =
+          items_above_before_group(tab, g1, H32, m) - items_above_before_group(tab, g0, H32, m);
+      const unsigned long long slot =
+          (g0 == 0 ? 0ull : items_before_group(tab, g0, H32)) + above + (g - g0);
+      if ((int64_t)slot < capacity)
+        sch.items[slot] = (int64_t)s | ((int64_t)m << 32) | ((int64_t)h << 48);
     }
   }
 }
@@ -143,6 +242,7 @@ struct AttnParams {
   float scale;
   float* av;                // [T, H*hd] fp32
   int64_t T;
+  int dynamic;              // 1: CTAs claim items from the list's counter; 0: CTA b takes b, b+grid, ...
 };
 
 // floor(log2(1 + max(ti - tj, 0))), exact on integers.
@@ -329,6 +429,40 @@ __device__ __forceinline__ void pointwise_tile_sep(uint32_t s_col, uint32_t p_co
   sm100::tmem_st16(p_col + 16, pk);
 }
 
+// Producer side (one thread): claims the next unhandled entry of the item list (or -1 past its end)
+// and hands it over as item k in ring slot k % ATT_ITEM_RING, once every reader has taken the slot's
+// previous item.  False if the CTA aborted.
+__device__ __forceinline__ bool publish_item(uint32_t k, uint64_t* item_full, uint64_t* item_empty,
+                                             int64_t* ring, const AttnSchedule& sch,
+                                             int64_t n_items, volatile int* abort_flag,
+                                             int64_t& item) {
+  const uint32_t slot = k % ATT_ITEM_RING, ph = (k / ATT_ITEM_RING) & 1u;
+  if (!sm100::mbar_wait(&item_empty[slot], ph ^ 1u, abort_flag)) return false;
+  const unsigned long long it =
+      atomicAdd(reinterpret_cast<unsigned long long*>(sch.header + 1), 1ull);
+  item = (int64_t)it < n_items ? sch.items[it] : -1;
+  ring[slot] = item;
+  sm100::mbar_arrive(&item_full[slot]);
+  return true;
+}
+
+// Static assignment: the CTA's k-th item is list entry blockIdx.x + k * gridDim.x (-1 past the end).
+__device__ __forceinline__ int64_t static_item(uint32_t k, const AttnSchedule& sch, int64_t n_items) {
+  const int64_t it = (int64_t)blockIdx.x + (int64_t)k * gridDim.x;
+  return it < n_items ? sch.items[it] : -1;
+}
+
+// Reader side (one thread per reading warp): waits for item k, reads it and releases the slot.
+// -1: no more items, or the CTA aborted.
+__device__ __forceinline__ int64_t read_item(uint32_t k, uint64_t* item_full, uint64_t* item_empty,
+                                             const int64_t* ring, volatile int* abort_flag) {
+  const uint32_t slot = k % ATT_ITEM_RING, ph = (k / ATT_ITEM_RING) & 1u;
+  if (!sm100::mbar_wait(&item_full[slot], ph, abort_flag)) return -1;
+  const int64_t item = *reinterpret_cast<const volatile int64_t*>(ring + slot);
+  sm100::mbar_arrive(&item_empty[slot]);
+  return item;
+}
+
 template <int HD, int BIAS>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
     attention_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnParams prm, AttnSchedule sch) {
@@ -356,7 +490,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   uint64_t* q_empty = q_full + 1;
   uint64_t* pw_bar = q_empty + 1;
   uint64_t* drain = pw_bar + 1;             // [2]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 2);
+  uint64_t* item_full = drain + 2;          // [ATT_ITEM_RING] the producer published an item
+  uint64_t* item_empty = item_full + ATT_ITEM_RING;  // [ATT_ITEM_RING] every consumer has read it
+  int64_t* item_ring = reinterpret_cast<int64_t*>(item_empty + ATT_ITEM_RING);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_ring + ATT_ITEM_RING);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -386,6 +523,10 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     mbar_init(pw_bar, ATT_PW);
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
+    for (int r = 0; r < ATT_ITEM_RING; r++) {
+      mbar_init(&item_full[r], 1);
+      mbar_init(&item_empty[r], ATT_ITEM_READERS);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tm);
@@ -405,8 +546,17 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     int q_par = -1, kv_par[Cfg::NST];   // parity of the last fill issued (-1: none)
     for (int s = 0; s < Cfg::NST; s++) kv_par[s] = -1;
     bool ok = true;
-    for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x, k++) {
-      const int64_t item = sch.items[it];
+    for (; ok; k++) {
+      int64_t item = -1;
+      if (prm.dynamic) {
+        if (lane == 0)
+          ok = publish_item(k, item_full, item_empty, item_ring, sch, n_items, abort_flag, item);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        item = __shfl_sync(0xffffffffu, item, 0);
+      } else {
+        item = static_item(k, sch, n_items);
+      }
+      if (!ok || item < 0) break;
       const int64_t seq = item & 0xffffffffLL;
       const int m = (int)((item >> 32) & 0xffff), h = (int)(item >> 48);
       const int64_t row0 = sch.seqinfo[2 * seq], n = sch.seqinfo[2 * seq + 1];
@@ -514,8 +664,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                  (accumulate || kk > 0) ? 1u : 0u);
         }
       };
-      for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x, k++) {
-        const int64_t item = sch.items[it];
+      for (; ok; k++) {
+        const int64_t item = prm.dynamic
+                                 ? read_item(k, item_full, item_empty, item_ring, abort_flag)
+                                 : static_item(k, sch, n_items);
+        if (item < 0) break;
         const int64_t seq = item & 0xffffffffLL;
         const int m = (int)((item >> 32) & 0xffff);
         const int64_t n = sch.seqinfo[2 * seq + 1];
@@ -588,8 +741,15 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     const int P = prm.P, Tb = prm.Tb;
     uint32_t g = 0, kx = 0, gx = 0, pw_cnt = 0;
     int staged_head = -1, staged_n = 0;  // what hpos_s / htt_s hold
-    for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x) {
-      const int64_t item = sch.items[it];
+    for (uint32_t k = 0;; k++) {
+      int64_t item = -1;
+      if (prm.dynamic) {
+        if (lane == 0) item = read_item(k, item_full, item_empty, item_ring, abort_flag);
+        item = __shfl_sync(0xffffffffu, item, 0);
+      } else {
+        item = static_item(k, sch, n_items);
+      }
+      if (item < 0) break;
       const int64_t seq = item & 0xffffffffLL;
       const int m = (int)((item >> 32) & 0xffff), h = (int)(item >> 48);
       const int64_t row0 = sch.seqinfo[2 * seq], n = sch.seqinfo[2 * seq + 1];

@@ -120,27 +120,34 @@ hstu_status_t launch_attention_kernel(const CUtensorMap& tm, const AttnParams& p
   return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
 
-// Eq. 2 on the tensor cores: builds the longest-first tile schedule on the device, then runs the
+// Eq. 2 on the tensor cores: builds the batched, heaviest-first tile schedule on the device, then runs the
 // persistent attention kernel.  av is fp32 [T, H*hd].
 inline hstu_status_t launch_attention(int64_t T, int64_t B, int H, int hd, int64_t max_seq_len,
                                       const bf16* uvqk, const int64_t* off, const int64_t* ts,
                                       const float* pos, int P, const float* tim, int Tb,
                                       const float* alibi, float scale, float* av, void* ws,
                                       size_t ws_bytes, cudaStream_t st) {
-  if (T >= (1LL << 31) || H >= (1 << 15)) return HSTU_ERR_UNSUPPORTED;
+  if (T >= (1LL << 31) || H >= (1 << 15) || B * (int64_t)H >= (1LL << 31)) return HSTU_ERR_UNSUPPORTED;
   if (ws_bytes < attention_workspace_bytes(T, B, H)) return HSTU_ERR_INVALID_ARG;
   const int64_t max_len = max_seq_len > 0 ? max_seq_len : T;
   const int64_t max_pairs64 = (max_len + ATT_ITEM_ROWS - 1) / ATT_ITEM_ROWS;
-  if (max_pairs64 > 16384) return HSTU_ERR_UNSUPPORTED;  // scheduler counters live in shared memory
+  if (max_pairs64 > 12288) return HSTU_ERR_UNSUPPORTED;  // scheduler tables live in shared memory
   const int max_pairs = (int)max_pairs64;
   const AttnSchedule sch = attention_schedule_view(ws, B);
-  const size_t sched_smem = 2 * (size_t)(max_pairs + 1) * sizeof(int);
+  const size_t sched_smem = (size_t)(max_pairs + 2) * (sizeof(unsigned long long) + 2 * sizeof(int));
+  // K and V take 4 * hd bytes per row and head.  Up to 256 MB in all (about twice L2), one batch
+  // taken statically in heaviest-first order keeps enough of them in L2; beyond that, batches of
+  // (sequence, head) groups whose K/V stay within 32 MB (a quarter of L2), claimed dynamically.
+  const bool dynamic = 4.0 * hd * (double)T * H > 256.0 * (1 << 20);
+  const int64_t kv_bytes_per_group = 4LL * hd * (max_pairs64 * ATT_ITEM_ROWS);
+  const int64_t gb64 = (32LL << 20) / kv_bytes_per_group;
+  const int gb = !dynamic ? (1 << 30) : (int)(gb64 < 1 ? 1 : (gb64 > 256 ? 256 : gb64));
   if (sched_smem > 48 * 1024 &&
       cudaFuncSetAttribute(attn_schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)sched_smem) != cudaSuccess)
     return HSTU_ERR_CUDA;
   const int64_t capacity = attention_capacity(T, B, H);
-  attn_schedule_kernel<<<1, 1024, sched_smem, st>>>(off, B, T, H, max_pairs, capacity, sch);
+  attn_schedule_kernel<<<1, 1024, sched_smem, st>>>(off, B, T, H, max_pairs, gb, capacity, sch);
   count_launch();
   if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
 
@@ -159,6 +166,7 @@ inline hstu_status_t launch_attention(int64_t T, int64_t B, int H, int hd, int64
   prm.scale = scale;
   prm.av = av;
   prm.T = T;
+  prm.dynamic = dynamic ? 1 : 0;
   const int grid = (int)(capacity < num_sms() ? capacity : num_sms());
   const int bias = alibi ? BIAS_ALIBI : ((pos || tim) ? BIAS_RAB : BIAS_NONE);
   if (hd == 64) {

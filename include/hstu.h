@@ -98,7 +98,8 @@ typedef struct {
  *
  * HSTU_BF16 requires: d % 64 == 0, d_qk == d_v in {64, 128}, every pointer 16-byte aligned.
  * HSTU_F32 requires d_qk, d_v <= 256.  Other shapes return HSTU_ERR_UNSUPPORTED.  The bf16 path
- * also requires T < 2^31 (32-bit TMA row coordinates).
+ * also requires T < 2^31 (32-bit TMA row coordinates), num_seqs * num_heads < 2^31 and
+ * max_seq_len <= 3,145,728 (its tile scheduler keeps per-length tables in shared memory).
  */
 hstu_status_t hstu_layer_fwd(const hstu_shape_t* shape, const void* X, const int64_t* seq_offsets,
                              const int64_t* timestamps, const void* W1, const void* b1,
