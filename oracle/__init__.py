@@ -64,6 +64,9 @@ def bind(path: str):
     lib.oracle_f1.restype = None
     lib.oracle_attention.argtypes = [i64, ip, i32, i32, i32, dp, ip, dp, i32, dp, i32, dp, f64, dp]
     lib.oracle_attention.restype = None
+    lib.oracle_candidate_attention.argtypes = [i64, ip, ip, i32, i32, i32, dp, ip, dp, ip, dp, i32,
+                                               dp, i32, dp, f64, dp]
+    lib.oracle_candidate_attention.restype = None
     lib.oracle_ln_gate.argtypes = [i64, i32, i32, i32, dp, dp, dp, dp, f64, dp]
     lib.oracle_ln_gate.restype = None
     lib.oracle_f2.argtypes = [i64, i32, i32, dp, dp, dp, dp, dp]
@@ -244,6 +247,40 @@ def attention(seq_offsets, uvqk, *, num_heads: int, d_qk: int, d_v: int, timesta
     _load().oracle_attention(len(off) - 1, _p(off), num_heads, d_qk, d_v, _p(uvqk), _p(ts),
                              _p(pos), P, _p(tim), Tb, _p(ali), float(scale), _p(av))
     return av
+
+
+def candidate_attention(hist_offsets, uvqk_hist, cand_offsets, uvqk_cand, *, num_heads: int,
+                        d_qk: int, d_v: int, hist_timestamps=None, cand_timestamps=None,
+                        pos_table=None, time_table=None, alibi_slopes=None,
+                        scale: float, lib=None) -> np.ndarray:
+    """M-FALCON candidate attention: every candidate row of user b sees b's history (its K and V
+    taken from uvqk_hist) and itself, at position n_b -> AV of the candidates [T_cand, H*d_v]."""
+    hoff, coff = _i(hist_offsets), _i(cand_offsets)
+    uh, uc = _d(uvqk_hist), _d(uvqk_cand)
+    hts, cts = _i(hist_timestamps), _i(cand_timestamps)
+    pos, tim, ali = _d(pos_table), _d(time_table), _d(alibi_slopes)
+    P = 0 if pos is None else pos.shape[1]
+    Tb = 0 if tim is None else tim.shape[1]
+    av = np.empty((uc.shape[0], num_heads * d_v), np.float64)
+    _load(lib).oracle_candidate_attention(len(hoff) - 1, _p(hoff), _p(coff), num_heads, d_qk, d_v,
+                                       _p(uh), _p(hts), _p(uc), _p(cts), _p(pos), P, _p(tim), Tb,
+                                       _p(ali), float(scale), _p(av))
+    return av
+
+
+def candidate_layer_fwd(hist_offsets, uvqk_hist, cand_offsets, X_cand, W1, b1, W2, b2, ln_w,
+                        ln_b, *, num_heads: int, d_qk: int, d_v: int, hist_timestamps=None,
+                        cand_timestamps=None, pos_table=None, time_table=None,
+                        alibi_slopes=None, scale: float, ln_eps: float = 1e-5) -> np.ndarray:
+    """One HSTU layer over the candidates (Eqs. 1-3 with the candidate attention above), given the
+    history's UVQK of the same layer -> Y of the candidates [T_cand, d]."""
+    uc = f1(X_cand, W1, b1)
+    av = candidate_attention(hist_offsets, uvqk_hist, cand_offsets, uc, num_heads=num_heads,
+                             d_qk=d_qk, d_v=d_v, hist_timestamps=hist_timestamps,
+                             cand_timestamps=cand_timestamps, pos_table=pos_table,
+                             time_table=time_table, alibi_slopes=alibi_slopes, scale=scale)
+    g = ln_gate(av, uc, ln_w, ln_b, num_heads=num_heads, d_qk=d_qk, d_v=d_v, ln_eps=ln_eps)
+    return f2(g, W2, b2, X_cand)
 
 
 def ln_gate(av, uvqk, ln_w, ln_b, *, num_heads: int, d_qk: int, d_v: int,

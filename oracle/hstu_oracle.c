@@ -143,6 +143,71 @@ void oracle_attention(int64_t B, const int64_t* seq_offsets, int32_t H, int32_t 
 }
 
 /* ---------------------------------------------------------------------------------------------
+ * M-FALCON candidate scoring ("Actions Speak Louder than Words" paper notes, section 3.6; the
+ * efficiency paragraph of "4.4 推荐模型的 Scaling"): m candidates are appended after a user's n
+ * history tokens and scored in one pass; the attention mask lets each candidate see the history
+ * but no other candidate, and the relative bias is modified for candidates.  Readings fixed here:
+ *   - a candidate also sees itself (the causal mask keeps its diagonal; only the other
+ *     candidates are removed);
+ *   - every candidate takes the position n it would have as the single item appended after the
+ *     history, so its position bias towards history token j uses n - j and towards itself 0, and
+ *     its time bias uses its own timestamp t_c: bucket of t_c - t_j, and of 0 for itself;
+ *   - with ALiBi the bias is -m_h (n - j), and 0 for itself.
+ * Hence, per head,
+ *   AV_c = sum_{j<n} scale * SiLU(q_c . k_j + bias(n, j)) v_j + scale * SiLU(q_c . k_c + bias(n, n)) v_c
+ * which, for a single candidate, is the causal attention row of the sequence [history, candidate]
+ * at index n.  Micro-batching the candidates and caching the history's K and V change neither.
+ * --------------------------------------------------------------------------------------------- */
+
+/* Bias between a query at position pi with timestamp ti and a key at position pj, timestamp tj. */
+static double bias_pt(int32_t h, int64_t pi, int64_t pj, int64_t ti, int64_t tj,
+                      const double* pos_table, int32_t P, const double* time_table, int32_t Tb,
+                      const double* alibi_slopes) {
+  if (alibi_slopes) return -alibi_slopes[h] * (double)(pi - pj);
+  double b = 0.0;
+  if (pos_table) b += pos_table[(int64_t)h * P + oracle_pos_bucket(pi, pj, P)];
+  if (time_table) b += time_table[(int64_t)h * Tb + oracle_time_bucket(ti, tj, Tb)];
+  return b;
+}
+
+void oracle_candidate_attention(int64_t B, const int64_t* hist_offsets,
+                                const int64_t* cand_offsets, int32_t H, int32_t dqk, int32_t dv,
+                                const double* uvqk_hist, const int64_t* hist_ts,
+                                const double* uvqk_cand, const int64_t* cand_ts,
+                                const double* pos_table, int32_t P, const double* time_table,
+                                int32_t Tb, const double* alibi_slopes, double scale,
+                                double* av_cand) {
+  const int32_t n1 = 2 * H * dv + 2 * H * dqk;
+  const int32_t offV = H * dv, offQ = 2 * H * dv, offK = 2 * H * dv + H * dqk;
+  const int64_t Tc = cand_offsets[B];
+#pragma omp parallel for schedule(dynamic, 4)
+  for (int64_t c = 0; c < Tc; c++) {
+    int64_t b = 0;
+    while (cand_offsets[b + 1] <= c) b++;
+    const int64_t h0 = hist_offsets[b], n = hist_offsets[b + 1] - hist_offsets[b];
+    const int64_t tc = cand_ts ? cand_ts[c] : 0;
+    const double* crow = uvqk_cand + c * n1;
+    for (int32_t h = 0; h < H; h++) {
+      double* acc = av_cand + c * (int64_t)H * dv + (int64_t)h * dv;
+      for (int32_t e = 0; e < dv; e++) acc[e] = 0.0;
+      const double* q = crow + offQ + (int64_t)h * dqk;
+      /* keys 0 .. n-1: the history; key n: the candidate itself */
+      for (int64_t j = 0; j <= n; j++) {
+        const double* krow = j < n ? uvqk_hist + (h0 + j) * n1 : crow;
+        const double* k = krow + offK + (int64_t)h * dqk;
+        const double* v = krow + offV + (int64_t)h * dv;
+        const int64_t tj = j < n ? (hist_ts ? hist_ts[h0 + j] : 0) : tc;
+        double sc = 0.0;
+        for (int32_t e = 0; e < dqk; e++) sc += q[e] * k[e];
+        sc += bias_pt(h, n, j, tc, tj, pos_table, P, time_table, Tb, alibi_slopes);
+        const double a = scale * silu(sc);
+        for (int32_t e = 0; e < dv; e++) acc[e] += a * v[e];
+      }
+    }
+  }
+}
+
+/* ---------------------------------------------------------------------------------------------
  * Eq. 3, first half: G = LayerNorm(AV) * U.  Norm is a layer normalisation; the sketch normalises
  * the full d-wide row.  Mean and biased variance over the H*dv columns.
  * --------------------------------------------------------------------------------------------- */

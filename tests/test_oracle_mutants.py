@@ -41,8 +41,50 @@ MUTANTS = {
 }
 
 
+# planted in the M-FALCON candidate code: caught by the candidate pin below
+CANDIDATE_MUTANTS = {
+    "cand_self_excluded": ("for (int64_t j = 0; j <= n; j++) {", "for (int64_t j = 0; j < n; j++) {"),
+    "cand_position_from_own_index": ("sc += bias_pt(h, n, j,", "sc += bias_pt(h, n + (c - cand_offsets[b]), j,"),
+    "cand_time_of_last_history": ("const int64_t tc = cand_ts ? cand_ts[c] : 0;",
+                                  "const int64_t tc = (cand_ts && n > 0) ? hist_ts[h0 + n - 1] : 0;"),
+    "cand_alibi_unmodified": ("if (alibi_slopes) return -alibi_slopes[h] * (double)(pi - pj);",
+                              "if (alibi_slopes) return -alibi_slopes[h] * (double)(pi - pj + 1);"),
+}
+
+
 def _silu(x):
     return x / (1.0 + np.exp(-x))
+
+
+def _candidate_pins_pass(lib) -> bool:
+    """Each candidate's AV from `lib` equals the row after its history of the (unmodified, separately
+    pinned) causal oracle on [history, candidate]; with rab and with ALiBi."""
+    rng = np.random.default_rng(23)
+    H, hd = 2, 4
+    n1 = 4 * H * hd
+    for alibi in (False, True):
+        hist, cand = [4, 0, 7], [3, 2, 2]
+        hoff = np.concatenate([[0], np.cumsum(hist)]).astype(np.int64)
+        coff = np.concatenate([[0], np.cumsum(cand)]).astype(np.int64)
+        uh, uc = rng.normal(0, 0.8, (hoff[-1], n1)), rng.normal(0, 0.8, (coff[-1], n1))
+        hts = np.cumsum(rng.integers(0, 300, hoff[-1])).astype(np.int64)
+        cts = hts[-1] + rng.integers(1, 5000, coff[-1]).astype(np.int64)
+        kw = dict(num_heads=H, d_qk=hd, d_v=hd, scale=0.5)
+        if alibi:
+            kw["alibi_slopes"] = np.array([0.25, 0.5])
+        else:
+            kw.update(pos_table=rng.normal(0, 0.5, (H, 8)), time_table=rng.normal(0, 0.5, (H, 16)))
+        av = oracle.candidate_attention(hoff, uh, coff, uc, hist_timestamps=hts, cand_timestamps=cts,
+                                        lib=lib, **kw)
+        for b in range(len(hist)):
+            for c in range(coff[b], coff[b + 1]):
+                seq = np.vstack([uh[hoff[b]:hoff[b + 1]], uc[c][None, :]])
+                ts = np.concatenate([hts[hoff[b]:hoff[b + 1]], [cts[c]]]).astype(np.int64)
+                ref = oracle.attention(np.array([0, len(seq)]), seq,
+                                       timestamps=None if alibi else ts, **kw)[-1]
+                if not np.allclose(av[c], ref, rtol=1e-12, atol=1e-12):
+                    return False
+    return True
 
 
 def _pins_pass(lib) -> bool:
@@ -105,7 +147,18 @@ def _compile(src_text: str, tmp_path, name: str):
 
 
 def test_unmodified_oracle_passes_the_independent_pins(tmp_path):
-    assert _pins_pass(_compile(open(SRC).read(), tmp_path, "orig"))
+    lib = _compile(open(SRC).read(), tmp_path, "orig")
+    assert _pins_pass(lib)
+    assert _candidate_pins_pass(lib)
+
+
+@pytest.mark.parametrize("name", sorted(CANDIDATE_MUTANTS))
+def test_planted_candidate_mistake_is_caught(name, tmp_path):
+    src = open(SRC).read()
+    old, new = CANDIDATE_MUTANTS[name]
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    lib = _compile(src.replace(old, new), tmp_path, name)
+    assert not _candidate_pins_pass(lib), f"planted mistake {name} went unnoticed"
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
