@@ -29,7 +29,9 @@ HSTU_F32, HSTU_BF16 = 0, 1
 EXPORTED = ["hstu_layer_fwd", "hstu_layer_fwd_workspace_size", "hstu_f1_fwd", "hstu_attention_fwd",
             "hstu_attention_workspace_size", "hstu_ln_gate_fwd", "hstu_f2_fwd",
             "hstu_token_embed_fwd", "hstu_status_string", "hstu_get_device_status", "hstu_version",
-            "hstu_launch_count", "hstu_attention_fwd_noalloc", "hstu_selftest_bounded_wait"]
+            "hstu_launch_count", "hstu_attention_fwd_noalloc", "hstu_selftest_bounded_wait",
+            "hstu_candidate_workspace_size", "hstu_candidate_attention_fwd",
+            "hstu_candidate_layer_workspace_size", "hstu_candidate_layer_fwd"]
 
 
 class HstuShape(ctypes.Structure):
@@ -72,6 +74,12 @@ def _load() -> ctypes.CDLL:
         "hstu_version": ([], ctypes.c_char_p),
         "hstu_launch_count": ([], ctypes.c_uint64),
         "hstu_selftest_bounded_wait": ([ctypes.c_uint64, P, P], ctypes.c_int),
+        "hstu_candidate_workspace_size": ([SH, I64], S),
+        "hstu_candidate_attention_fwd": ([SH, P, P, P, I64, I64, P, P, P, P, P, P, F32, P, P, S, P],
+                                         ctypes.c_int),
+        "hstu_candidate_layer_workspace_size": ([SH, I64], S),
+        "hstu_candidate_layer_fwd": ([SH, P, P, P, I64, I64, P, P, P, P, P, P, P, P, P, P, P, P, F32,
+                                      P, P, S, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -222,6 +230,49 @@ def hstu_attention_fwd_noalloc(shape: HstuShape, uvqk, seq_offsets, timestamps, 
                                            _ptr(alibi_slopes), float(scale), _ptr(av),
                                            _stream(stream)), "hstu_attention_fwd_noalloc")
     return av
+
+
+def candidate_workspace_size(shape: HstuShape, num_candidates: int) -> int:
+    return int(_lib.hstu_candidate_workspace_size(ctypes.byref(shape), int(num_candidates)))
+
+
+def hstu_candidate_attention_fwd(shape: HstuShape, uvqk_hist, hist_offsets, hist_timestamps,
+                                 uvqk_cand, cand_offsets, cand_timestamps, pos_table, time_table,
+                                 alibi_slopes, scale: float, av_cand, max_candidates: int,
+                                 workspace=None, stream=None):
+    """M-FALCON candidate attention (see the C header): `shape` is the history's shape."""
+    Tc = int(uvqk_cand.shape[0])
+    if workspace is None:
+        workspace = torch.empty(max(256, candidate_workspace_size(shape, Tc)), dtype=torch.uint8,
+                                device=uvqk_cand.device)
+    _check(_lib.hstu_candidate_attention_fwd(
+        ctypes.byref(shape), _ptr(uvqk_hist), _ptr(hist_offsets), _ptr(hist_timestamps), Tc,
+        int(max_candidates), _ptr(uvqk_cand), _ptr(cand_offsets), _ptr(cand_timestamps),
+        _ptr(pos_table), _ptr(time_table), _ptr(alibi_slopes), float(scale), _ptr(av_cand),
+        _ptr(workspace), workspace.numel(), _stream(stream)), "hstu_candidate_attention_fwd")
+    return av_cand
+
+
+def candidate_layer_workspace_size(shape: HstuShape, num_candidates: int) -> int:
+    return int(_lib.hstu_candidate_layer_workspace_size(ctypes.byref(shape), int(num_candidates)))
+
+
+def hstu_candidate_layer_fwd(shape: HstuShape, uvqk_hist, hist_offsets, hist_timestamps, X_cand,
+                             cand_offsets, cand_timestamps, W1, b1, W2, b2, ln_w, ln_b, pos_table,
+                             time_table, alibi_slopes, scale: float, out_cand, max_candidates: int,
+                             workspace=None, stream=None):
+    """One HSTU layer over the candidates given the history's UVQK of the same layer."""
+    Tc = int(X_cand.shape[0])
+    if workspace is None:
+        workspace = torch.empty(max(256, candidate_layer_workspace_size(shape, Tc)),
+                                dtype=torch.uint8, device=X_cand.device)
+    _check(_lib.hstu_candidate_layer_fwd(
+        ctypes.byref(shape), _ptr(uvqk_hist), _ptr(hist_offsets), _ptr(hist_timestamps), Tc,
+        int(max_candidates), _ptr(X_cand), _ptr(cand_offsets), _ptr(cand_timestamps), _ptr(W1),
+        _ptr(b1), _ptr(W2), _ptr(b2), _ptr(ln_w), _ptr(ln_b), _ptr(pos_table), _ptr(time_table),
+        _ptr(alibi_slopes), float(scale), _ptr(out_cand), _ptr(workspace), workspace.numel(),
+        _stream(stream)), "hstu_candidate_layer_fwd")
+    return out_cand
 
 
 def hstu_ln_gate_fwd(shape: HstuShape, av, uvqk, ln_w, ln_b, g, stream=None):

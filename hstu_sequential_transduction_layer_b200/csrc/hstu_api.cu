@@ -200,6 +200,76 @@ Workspace layout(const hstu_shape_t& s, void* base) {
   return w;
 }
 
+// M-FALCON candidate path: the candidates' shape is the history's with their own token count.
+hstu_shape_t candidate_shape(const hstu_shape_t& s, int64_t Tc, int64_t max_cand) {
+  hstu_shape_t c = s;
+  c.total_tokens = Tc;
+  c.max_seq_len = max_cand;
+  return c;
+}
+
+// Checks of hstu_candidate_attention_fwd's arguments (also used by the candidate layer).
+hstu_status_t check_candidates(const hstu_shape_t* shape, const void* uvqk_hist,
+                               const int64_t* hist_offsets, const int64_t* hist_ts, int64_t Tc,
+                               int64_t max_cand, const int64_t* cand_offsets, const int64_t* cand_ts,
+                               const float* pos, const float* tim, const float* alibi, float scale) {
+  hstu_status_t rc = check_shape(shape);
+  if (rc != HSTU_OK) return rc;
+  const hstu_shape_t& s = *shape;
+  if (s.dtype != HSTU_BF16) return HSTU_ERR_UNSUPPORTED;
+  if (Tc < 0 || max_cand < 0 || Tc > (1LL << 40)) return HSTU_ERR_INVALID_ARG;
+  // a user's candidate-tile pairs are numbered in 16 bits; the schedule uses 32-bit group indices
+  if (max_cand > 65535LL * 256 || s.num_seqs * (int64_t)s.num_heads >= (1LL << 31))
+    return HSTU_ERR_UNSUPPORTED;
+  if (Tc == 0) return HSTU_OK;
+  if ((rc = check_bias(shape, hist_ts, pos, tim, alibi, scale)) != HSTU_OK) return rc;
+  if (tim && !cand_ts) return HSTU_ERR_INVALID_ARG;
+  if (s.num_seqs == 0 || !hist_offsets || !cand_offsets) return HSTU_ERR_INVALID_ARG;
+  if (s.total_tokens > 0 && !uvqk_hist) return HSTU_ERR_INVALID_ARG;
+  if (!aligned16(uvqk_hist)) return HSTU_ERR_INVALID_ARG;
+  return HSTU_OK;
+}
+
+hstu_status_t run_candidate_attention(const hstu_shape_t& s, const void* uvqk_hist,
+                                      const int64_t* hoff, const int64_t* hts, int64_t Tc,
+                                      int64_t max_cand, const void* uvqk_cand, const int64_t* coff,
+                                      const int64_t* cts, const float* pos, const float* tim,
+                                      const float* alibi, float scale, void* av, void* ws,
+                                      size_t ws_bytes, cudaStream_t st) {
+  const int64_t B = s.num_seqs, Th = s.total_tokens;
+  check_offsets_kernel<<<(unsigned)((B + 1 + 255) / 256), 256, 0, st>>>(hoff, B, Th);
+  if (launch_status() != HSTU_OK) return HSTU_ERR_CUDA;
+  check_offsets_kernel<<<(unsigned)((B + 1 + 255) / 256), 256, 0, st>>>(coff, B, Tc);
+  if (launch_status() != HSTU_OK) return HSTU_ERR_CUDA;
+  (void)max_cand;
+  return tc::launch_candidate_attention(Th, Tc, B, s.num_heads, s.d_qk, s.max_seq_len,
+                                        (const bf16*)uvqk_hist, hoff, hts, (const bf16*)uvqk_cand,
+                                        coff, cts, pos, s.n_pos_buckets, tim, s.n_time_buckets,
+                                        alibi, scale, (float*)av, ws, ws_bytes, st);
+}
+
+struct CandWorkspace {
+  void *uvqk, *av, *g, *attn;
+  size_t attn_bytes, total;
+};
+
+CandWorkspace cand_layout(const hstu_shape_t& s, int64_t Tc, void* base) {
+  CandWorkspace w{};
+  size_t o = 0;
+  char* b = static_cast<char*>(base);
+  w.uvqk = b ? b + o : nullptr;
+  o += align_up((size_t)Tc * (size_t)n1_of(s) * 2);
+  w.av = b ? b + o : nullptr;
+  o += align_up((size_t)Tc * (size_t)wv_of(s) * 4);
+  w.g = b ? b + o : nullptr;
+  o += align_up((size_t)Tc * (size_t)wv_of(s) * 2);
+  w.attn = b ? b + o : nullptr;
+  w.attn_bytes = tc::candidate_workspace_bytes(Tc, s.num_seqs, s.num_heads);
+  o += align_up(w.attn_bytes);
+  w.total = o;
+  return w;
+}
+
 }  // namespace
 
 // Self-test of the bounded wait every pipelined kernel uses: one warp waits on an mbarrier that
@@ -392,6 +462,83 @@ hstu_status_t hstu_token_embed_fwd(int64_t T, int32_t d, const int64_t* item_ids
       T, d, item_ids, action_ids, (const bf16*)item_table, n_items, (const bf16*)action_table,
       n_actions, (bf16*)X);
   return launch_status();
+}
+
+size_t hstu_candidate_workspace_size(const hstu_shape_t* shape, int64_t num_candidates) {
+  if (check_shape(shape) != HSTU_OK || num_candidates < 0) return 0;
+  return tc::candidate_workspace_bytes(num_candidates, shape->num_seqs, shape->num_heads);
+}
+
+hstu_status_t hstu_candidate_attention_fwd(const hstu_shape_t* shape, const void* uvqk_hist,
+                                           const int64_t* hist_offsets,
+                                           const int64_t* hist_timestamps, int64_t num_candidates,
+                                           int64_t max_candidates, const void* uvqk_cand,
+                                           const int64_t* cand_offsets,
+                                           const int64_t* cand_timestamps, const float* pos_table,
+                                           const float* time_table, const float* alibi_slopes,
+                                           float scale, void* av_cand, void* workspace,
+                                           size_t workspace_bytes, void* stream) {
+  hstu_status_t rc = check_candidates(shape, uvqk_hist, hist_offsets, hist_timestamps,
+                                      num_candidates, max_candidates, cand_offsets,
+                                      cand_timestamps, pos_table, time_table, alibi_slopes, scale);
+  if (rc != HSTU_OK || num_candidates == 0) return rc;
+  const hstu_shape_t& s = *shape;
+  if (!uvqk_cand || !av_cand || !workspace) return HSTU_ERR_INVALID_ARG;
+  if (!aligned16(uvqk_cand) || !aligned16(av_cand)) return HSTU_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) return HSTU_ERR_INVALID_ARG;
+  if (workspace_bytes < tc::candidate_workspace_bytes(num_candidates, s.num_seqs, s.num_heads))
+    return HSTU_ERR_INVALID_ARG;
+  const size_t avb = (size_t)num_candidates * wv_of(s) * 4;
+  if (overlaps(av_cand, avb, uvqk_cand, (size_t)num_candidates * n1_of(s) * 2) ||
+      overlaps(av_cand, avb, workspace, workspace_bytes) ||
+      overlaps(av_cand, avb, uvqk_hist, (size_t)s.total_tokens * n1_of(s) * 2))
+    return HSTU_ERR_INVALID_ARG;
+  return run_candidate_attention(s, uvqk_hist, hist_offsets, hist_timestamps, num_candidates,
+                                 max_candidates, uvqk_cand, cand_offsets, cand_timestamps,
+                                 pos_table, time_table, alibi_slopes, scale, av_cand, workspace,
+                                 workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+size_t hstu_candidate_layer_workspace_size(const hstu_shape_t* shape, int64_t num_candidates) {
+  if (check_shape(shape) != HSTU_OK || num_candidates < 0) return 0;
+  return cand_layout(*shape, num_candidates, nullptr).total;
+}
+
+hstu_status_t hstu_candidate_layer_fwd(const hstu_shape_t* shape, const void* uvqk_hist,
+                                       const int64_t* hist_offsets, const int64_t* hist_timestamps,
+                                       int64_t num_candidates, int64_t max_candidates,
+                                       const void* X_cand, const int64_t* cand_offsets,
+                                       const int64_t* cand_timestamps, const void* W1,
+                                       const void* b1, const void* W2, const void* b2,
+                                       const void* ln_w, const void* ln_b, const float* pos_table,
+                                       const float* time_table, const float* alibi_slopes,
+                                       float scale, void* out_cand, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  hstu_status_t rc = check_candidates(shape, uvqk_hist, hist_offsets, hist_timestamps,
+                                      num_candidates, max_candidates, cand_offsets,
+                                      cand_timestamps, pos_table, time_table, alibi_slopes, scale);
+  if (rc != HSTU_OK || num_candidates == 0) return rc;
+  const hstu_shape_t c = candidate_shape(*shape, num_candidates, max_candidates);
+  if (!X_cand || !W1 || !W2 || !ln_w || !ln_b || !out_cand || !workspace) return HSTU_ERR_INVALID_ARG;
+  if (!(aligned16(X_cand) && aligned16(W1) && aligned16(b1) && aligned16(W2) && aligned16(b2) &&
+        aligned16(ln_w) && aligned16(ln_b) && aligned16(out_cand)))
+    return HSTU_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) return HSTU_ERR_INVALID_ARG;
+  const CandWorkspace w = cand_layout(c, num_candidates, workspace);
+  if (workspace_bytes < w.total) return HSTU_ERR_INVALID_ARG;
+  const size_t xbytes = (size_t)num_candidates * c.d_model * 2;
+  if (overlaps(out_cand, xbytes, X_cand, xbytes) || overlaps(out_cand, xbytes, workspace, w.total) ||
+      overlaps(X_cand, xbytes, workspace, w.total))
+    return HSTU_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((rc = run_f1(c, X_cand, W1, b1, w.uvqk, st)) != HSTU_OK) return rc;
+  if ((rc = run_candidate_attention(*shape, uvqk_hist, hist_offsets, hist_timestamps,
+                                    num_candidates, max_candidates, w.uvqk, cand_offsets,
+                                    cand_timestamps, pos_table, time_table, alibi_slopes, scale,
+                                    w.av, w.attn, w.attn_bytes, st)) != HSTU_OK)
+    return rc;
+  if ((rc = run_ln_gate(c, w.av, w.uvqk, ln_w, ln_b, w.g, st)) != HSTU_OK) return rc;
+  return run_f2(c, w.g, W2, b2, X_cand, out_cand, st);
 }
 
 hstu_status_t hstu_selftest_bounded_wait(uint64_t limit_ns, long long* result, void* stream) {

@@ -233,6 +233,70 @@ __global__ void __launch_bounds__(1024) attn_schedule_kernel(const int64_t* __re
   }
 }
 
+// M-FALCON candidate schedule: one item per (user, pair of 128-row candidate tiles, head).  An
+// item reads all of its user's history tiles, so users go by decreasing number of history tiles
+// (heaviest first) and a user's items stay together (they share the history's K/V in L2).  One
+// CTA; dynamic shared memory holds 2 * (max_tiles + 1) counters.  Per user the schedule keeps
+// (candidate start, candidate count, history start, history length), clamped like the causal one.
+__global__ void __launch_bounds__(1024) cand_schedule_kernel(const int64_t* __restrict__ hoff,
+                                                             const int64_t* __restrict__ coff,
+                                                             int64_t B, int64_t Th, int64_t Tc,
+                                                             int H, int max_tiles,
+                                                             int64_t capacity, AttnSchedule sch) {
+  extern __shared__ unsigned long long cand_smem[];
+  unsigned long long* items_at = cand_smem;                 // items of users with t history tiles
+  unsigned long long* cursor = cand_smem + max_tiles + 1;   // first slot of those items
+  for (int t = threadIdx.x; t <= max_tiles; t += blockDim.x) items_at[t] = 0, cursor[t] = 0;
+  __syncthreads();
+  for (int64_t s = threadIdx.x; s < B; s += blockDim.x) {
+    const int64_t ha = clamp64(hoff[s], 0, Th);
+    int64_t nh = clamp64(hoff[s + 1], 0, Th) - ha;
+    const int64_t ca = clamp64(coff[s], 0, Tc);
+    int64_t nc = clamp64(coff[s + 1], 0, Tc) - ca;
+    if (nh < 0) nh = 0;
+    if (nc < 0) nc = 0;
+    int tiles = (int)((nh + ATT_BN - 1) / ATT_BN);
+    if (tiles > max_tiles) {  // longer than the stated maximum history: clamp and report
+      report(HSTU_ERR_DEVICE_BAD_OFFSETS);
+      tiles = max_tiles;
+      nh = (int64_t)max_tiles * ATT_BN;
+    }
+    sch.seqinfo[4 * s] = ca;
+    sch.seqinfo[4 * s + 1] = nc;
+    sch.seqinfo[4 * s + 2] = ha;
+    sch.seqinfo[4 * s + 3] = nh;
+    const int64_t pairs = (nc + ATT_ITEM_ROWS - 1) / ATT_ITEM_ROWS;
+    atomicAdd(&items_at[tiles], (unsigned long long)(pairs * H));
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long base = 0;
+    for (int t = max_tiles; t >= 0; t--) {
+      cursor[t] = base;
+      base += items_at[t];
+    }
+    if ((int64_t)base > capacity) report(HSTU_ERR_DEVICE_BAD_OFFSETS);
+    sch.header[0] = (int64_t)base < capacity ? (int64_t)base : capacity;
+    sch.header[1] = 0;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  for (int64_t s = warp; s < B; s += blockDim.x / 32) {
+    const int64_t nc = sch.seqinfo[4 * s + 1], nh = sch.seqinfo[4 * s + 3];
+    const int pairs = (int)((nc + ATT_ITEM_ROWS - 1) / ATT_ITEM_ROWS);
+    if (pairs == 0) continue;
+    const int tiles = (int)((nh + ATT_BN - 1) / ATT_BN);
+    unsigned long long slot = 0;
+    if (lane == 0) slot = atomicAdd(&cursor[tiles], (unsigned long long)pairs * H);
+    slot = __shfl_sync(0xffffffffu, slot, 0);
+    for (uint32_t e = lane; e < (uint32_t)pairs * (uint32_t)H; e += 32) {
+      const uint32_t h = e / (uint32_t)pairs, m = e - h * (uint32_t)pairs;
+      if ((int64_t)(slot + e) < capacity)
+        sch.items[slot + e] = (int64_t)s | ((int64_t)m << 32) | ((int64_t)h << 48);
+    }
+  }
+}
+
 struct AttnParams {
   const int64_t* ts;        // timestamps [T] or null
   const float* pos;         // [H, P] or null
@@ -243,7 +307,45 @@ struct AttnParams {
   float* av;                // [T, H*hd] fp32
   int64_t T;
   int dynamic;              // 1: CTAs claim items from the list's counter; 0: CTA b takes b, b+grid, ...
+  // candidate mode only: the candidates' timestamps [T_cand] and UVQK rows (for each candidate's
+  // own term); ts, the K/V tensor map and the schedule's key rows are then the history's
+  const int64_t* cts;
+  const bf16* cand_uvqk;
 };
+
+// Geometry of one work item.  Causal mode: queries and keys are the same sequence, query tile x of
+// pair m reads key tiles 0 .. 2m + x.  Candidate mode (M-FALCON): the queries are a user's
+// candidates, the keys its history (all tiles, for both query tiles), and every candidate sits at
+// position n_hist.  The schedule stores (start, length) per sequence, or (candidate start, count,
+// history start, length) per user.
+struct ItemGeom {
+  int64_t qrow0, nq;        // first query row, number of query rows of the sequence / user
+  int64_t krow0, nkr;       // first key row, number of key rows
+  int m, h, nk;             // pair index, head, key tiles the item loads
+  bool has_b;               // the pair has its second query tile
+};
+
+template <bool CAND>
+__device__ __forceinline__ ItemGeom item_geom(int64_t item, const AttnSchedule& sch) {
+  ItemGeom g;
+  const int64_t seq = item & 0xffffffffLL;
+  g.m = (int)((item >> 32) & 0xffff);
+  g.h = (int)(item >> 48);
+  if (CAND) {
+    g.qrow0 = sch.seqinfo[4 * seq];
+    g.nq = sch.seqinfo[4 * seq + 1];
+    g.krow0 = sch.seqinfo[4 * seq + 2];
+    g.nkr = sch.seqinfo[4 * seq + 3];
+    g.has_b = (2 * g.m + 1) * ATT_BM < g.nq;
+    g.nk = (int)((g.nkr + ATT_BN - 1) / ATT_BN);
+  } else {
+    g.qrow0 = g.krow0 = sch.seqinfo[2 * seq];
+    g.nq = g.nkr = sch.seqinfo[2 * seq + 1];
+    g.has_b = (2 * g.m + 1) * ATT_BM < g.nq;
+    g.nk = g.has_b ? 2 * g.m + 2 : 2 * g.m + 1;
+  }
+  return g;
+}
 
 // floor(log2(1 + max(ti - tj, 0))), exact on integers.
 __device__ __forceinline__ int time_bucket(int64_t ti, int64_t tj) {
@@ -303,10 +405,12 @@ __device__ __forceinline__ void fast_chunk(const uint32_t (&sv)[32], float hb0, 
   }
 }
 
-// Exact path over 32 columns: clamped position bucket, per-element time bucket, causal mask.
-// dist0 = i - (key0 + col0); tsk points at this chunk's staged key timestamps.
+// Exact path over 32 columns: clamped position bucket, per-element time bucket, mask.
+// dist0 = i - (key0 + col0) with i the row's position; keys at distance < dmin are masked (0: the
+// causal mask j <= i; 1: a candidate sees history keys j < n_hist only); tsk points at this chunk's
+// staged key timestamps.
 template <int BIAS>
-__device__ __forceinline__ void general_chunk(const uint32_t (&sv)[32], int dist0, int P, int Tb,
+__device__ __forceinline__ void general_chunk(const uint32_t (&sv)[32], int dist0, int dmin, int P, int Tb,
                                               int staged_n, int64_t ti, const int64_t* tsk,
                                               const float* hpos, const float* htt,
                                               const float* pos_h, const float* tim_h,
@@ -332,7 +436,7 @@ __device__ __forceinline__ void general_chunk(const uint32_t (&sv)[32], int dist
         hb = -half_slope * (float)dist;
       }
       const float h = fmaf(__uint_as_float(sv[e + u]), 0.5f, hb);
-      p2[u] = dist < 0 ? 0.0f : silu_from_half(h);
+      p2[u] = dist < dmin ? 0.0f : silu_from_half(h);
     }
     pk[e / 2] = pack_bf16x2(p2[0], p2[1]);
   }
@@ -340,8 +444,8 @@ __device__ __forceinline__ void general_chunk(const uint32_t (&sv)[32], int dist
 
 // Exact path with 32-bit timestamps relative to the sequence's first one: the time bucket
 // floor(log2(1 + max(ti - tj, 0))) is 31 - clz(max(ti1 - tj, 1)) with ti1 = ti + 1, and hclz[c]
-// holds the halved time bias of bucket min(31 - c, Tb - 1).  Causal mask as in general_chunk.
-__device__ __forceinline__ void general32_chunk(const uint32_t (&sv)[32], int dist0, int P,
+// holds the halved time bias of bucket min(31 - c, Tb - 1).  Mask as in general_chunk.
+__device__ __forceinline__ void general32_chunk(const uint32_t (&sv)[32], int dist0, int dmin, int P,
                                                 int staged_n, int ti1, const int* tsk32,
                                                 const float* hpos, const float* hclz,
                                                 const float* pos_h, uint32_t (&pk)[16]) {
@@ -359,7 +463,7 @@ __device__ __forceinline__ void general32_chunk(const uint32_t (&sv)[32], int di
       const int d1 = max(ti1 - tsk32[e + u], 1);
       hb += hclz[__clz(d1)];
       const float h = fmaf(__uint_as_float(sv[e + u]), 0.5f, hb);
-      p2[u] = dist < 0 ? 0.0f : silu_from_half(h);
+      p2[u] = dist < dmin ? 0.0f : silu_from_half(h);
     }
     pk[e / 2] = pack_bf16x2(p2[0], p2[1]);
   }
@@ -367,7 +471,7 @@ __device__ __forceinline__ void general32_chunk(const uint32_t (&sv)[32], int di
 
 // Per-tile state of one pointwise thread.
 struct TileArgs {
-  int i, key0, P, Tb, staged_n, cstar, ti1;
+  int i, key0, P, Tb, staged_n, cstar, ti1, dmin;
   int64_t ti;
   const int64_t* tsk;       // staged timestamps of the tile's 128 keys
   const int* tsk32;         // the same, relative to the sequence's first timestamp
@@ -379,10 +483,10 @@ template <int BIAS, int MODE, bool SPLIT>
 __device__ __forceinline__ void do_chunk(const uint32_t (&sv)[32], int col0, const TileArgs& a,
                                          uint32_t (&pk)[16]) {
   if (MODE == TILE_GENERAL) {
-    general_chunk<BIAS>(sv, a.i - a.key0 - col0, a.P, a.Tb, a.staged_n, a.ti, a.tsk + col0, a.hpos,
+    general_chunk<BIAS>(sv, a.i - a.key0 - col0, a.dmin, a.P, a.Tb, a.staged_n, a.ti, a.tsk + col0, a.hpos,
                         a.htt, a.pos_h, a.tim_h, a.half_slope, pk);
   } else if (MODE == TILE_GEN32) {
-    general32_chunk(sv, a.i - a.key0 - col0, a.P, a.staged_n, a.ti1, a.tsk32 + col0, a.hpos, a.hclz,
+    general32_chunk(sv, a.i - a.key0 - col0, a.dmin, a.P, a.staged_n, a.ti1, a.tsk32 + col0, a.hpos, a.hclz,
                     a.pos_h, pk);
   } else if (BIAS == BIAS_ALIBI) {
     fast_chunk<BIAS, false>(sv, fmaf((float)col0, a.half_slope, a.hb0), 0.0f, 0, nullptr,
@@ -463,9 +567,10 @@ __device__ __forceinline__ int64_t read_item(uint32_t k, uint64_t* item_full, ui
   return item;
 }
 
-template <int HD, int BIAS>
+template <int HD, int BIAS, bool CAND>
 __global__ void __launch_bounds__(ATT_THREADS, 1)
-    attention_tc_kernel(const __grid_constant__ CUtensorMap tm, AttnParams prm, AttnSchedule sch) {
+    attention_tc_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tmq,
+                        AttnParams prm, AttnSchedule sch) {
   using Cfg = AttnCfg<HD>;
   using namespace sm100;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -530,6 +635,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tm);
+    if (CAND) prefetch_tensormap(&tmq);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
@@ -557,22 +663,21 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         item = static_item(k, sch, n_items);
       }
       if (!ok || item < 0) break;
-      const int64_t seq = item & 0xffffffffLL;
-      const int m = (int)((item >> 32) & 0xffff), h = (int)(item >> 48);
-      const int64_t row0 = sch.seqinfo[2 * seq], n = sch.seqinfo[2 * seq + 1];
-      const bool has_b = (2 * m + 1) * ATT_BM < n;
-      const int nk = has_b ? 2 * m + 2 : 2 * m + 1;
+      const ItemGeom ig = item_geom<CAND>(item, sch);
+      const int m = ig.m, h = ig.h, nk = ig.nk;
+      const int64_t row0 = ig.krow0, n = ig.nkr;   // key rows
+      const bool has_b = ig.has_b;
       if (lane == 0) {
         ok = mbar_wait(q_empty, (k & 1u) ^ 1u, abort_flag);
         if (ok) {
           mbar_arrive_expect_tx(q_full, (has_b ? 2 : 1) * Cfg::Q_BYTES);
 #pragma unroll
           for (int b = 0; b < HD / 64; b++) {
-            tma_load_2d(q_s + b * Cfg::BOX, &tm, q_full, col_q + h * HD + b * 64,
-                        (int)row0 + 2 * m * ATT_BM);
+            tma_load_2d(q_s + b * Cfg::BOX, &tmq, q_full, col_q + h * HD + b * 64,
+                        (int)ig.qrow0 + 2 * m * ATT_BM);
             if (has_b)
-              tma_load_2d(q_s + Cfg::Q_BYTES + b * Cfg::BOX, &tm, q_full, col_q + h * HD + b * 64,
-                          (int)row0 + (2 * m + 1) * ATT_BM);
+              tma_load_2d(q_s + Cfg::Q_BYTES + b * Cfg::BOX, &tmq, q_full, col_q + h * HD + b * 64,
+                          (int)ig.qrow0 + (2 * m + 1) * ATT_BM);
           }
           q_par = (int)(k & 1u);
         }
@@ -669,13 +774,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
                                  ? read_item(k, item_full, item_empty, item_ring, abort_flag)
                                  : static_item(k, sch, n_items);
         if (item < 0) break;
-        const int64_t seq = item & 0xffffffffLL;
-        const int m = (int)((item >> 32) & 0xffff);
-        const int64_t n = sch.seqinfo[2 * seq + 1];
-        const bool has_b = (2 * m + 1) * ATT_BM < n;
-        const int nk = has_b ? 2 * m + 2 : 2 * m + 1;
-        const int last = 2 * m + x;                   // this query tile's last (diagonal) key tile
-        const bool mine = x == 0 || has_b;
+        const ItemGeom ig = item_geom<CAND>(item, sch);
+        const int m = ig.m, nk = ig.nk;
+        const bool has_b = ig.has_b;
+        // this query tile's last key tile: the diagonal one, or the history's last
+        const int last = CAND ? nk - 1 : 2 * m + x;
+        // a candidate item without history has no key tile: its query tiles take no MMA
+        const bool mine = (x == 0 || has_b) && nk > 0;
         if (!mbar_wait(q_full, k & 1u, abort_flag)) break;
         int j = 0;
         if (mine) {
@@ -750,15 +855,16 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         item = static_item(k, sch, n_items);
       }
       if (item < 0) break;
-      const int64_t seq = item & 0xffffffffLL;
-      const int m = (int)((item >> 32) & 0xffff), h = (int)(item >> 48);
-      const int64_t row0 = sch.seqinfo[2 * seq], n = sch.seqinfo[2 * seq + 1];
-      const bool has_b = (2 * m + 1) * ATT_BM < n;
-      const int nk = has_b ? 2 * m + 2 : 2 * m + 1;
+      const ItemGeom ig = item_geom<CAND>(item, sch);
+      const int m = ig.m, h = ig.h, nk = ig.nk;
+      const int64_t row0 = ig.krow0, n = ig.nkr;   // key rows (the query rows too, in causal mode)
+      const bool has_b = ig.has_b;
       const float* pos_h = has_pos ? prm.pos + (int64_t)h * P : nullptr;
       const float* tim_h = has_time ? prm.tim + (int64_t)h * Tb : nullptr;
-      // stage the halved bias tables of this head (the first 128*nk position buckets suffice)
-      const int need = min(nk * ATT_BN, Cfg::POS_CAP);
+      // stage the halved bias tables of this head: the first 128*nk position buckets suffice, or
+      // n_hist + 1 for candidates (distances 0 .. n_hist)
+      const int need = CAND ? (int)(n + 1 < Cfg::POS_CAP ? n + 1 : Cfg::POS_CAP)
+                            : min(nk * ATT_BN, Cfg::POS_CAP);
       if (BIAS == BIAS_RAB && (h != staged_head || need > staged_n)) {
         if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;   // earlier items are done reading
         // hpos_s[d] = pos[h][min(d, P-1)] / 2 for every distance d < need (zeros without a table)
@@ -779,16 +885,22 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       }
       const int q0 = qt * ATT_BM;
       const int i = q0 + r;                        // local query index of this thread's row
-      const int64_t ti = has_time ? prm.ts[row0 + (i < n ? i : n - 1)] : 0;
-      const int64_t ti_rel = has_time ? ti - prm.ts[row0] : 0;
+      const int ipos = CAND ? (int)n : i;          // the row's position for the bias
+      int64_t ti = 0;
+      if (has_time)
+        ti = CAND ? prm.cts[ig.qrow0 + (i < ig.nq ? i : ig.nq - 1)] : prm.ts[row0 + (i < n ? i : n - 1)];
+      const int64_t ti_rel = has_time && n > 0 ? ti - prm.ts[row0] : 0;
       const bool row_rel32 = ti_rel > -(1LL << 30) && ti_rel < (1LL << 30);
       const int ti1 = (int)ti_rel + 1;
       const float half_slope = BIAS == BIAS_ALIBI ? 0.5f * prm.alibi[h] : 0.0f;
       bool ok = true;
-      for (int j = 0; j <= qt; j++) {
+      const int last = CAND ? nk - 1 : qt;
+      for (int j = 0; j <= last; j++) {
         const uint32_t gj = g + j;
         const int key0 = j * ATT_BN;
-        const bool diag = (j == qt);
+        // tiles that need the per-element mask: the diagonal one, or the history's last when it
+        // is partial
+        const bool diag = CAND ? (j == nk - 1 && (n % ATT_BN) != 0) : (j == qt);
         const int64_t* tsk = ts_ring + (gj % Cfg::NST) * ATT_BN;
         const int* tsk32 = ts32_ring + (gj % Cfg::NST) * ATT_BN;
         bool rel32 = false;
@@ -841,16 +953,17 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         if (!diag && time_fast) {
           if (BIAS == BIAS_ALIBI) {
             mode = TILE_FAST;
-            hb0 = -half_slope * (float)(i - key0);
+            hb0 = -half_slope * (float)(ipos - key0);
           } else if (BIAS == BIAS_NONE) {
             mode = TILE_FAST;
-          } else if (q0 + ATT_BM - 1 - key0 < staged_n) {   // every distance of the tile is staged
+          } else if ((CAND ? ipos : q0 + ATT_BM - 1) - key0 < staged_n) {  // all distances staged
             mode = TILE_FAST;
           }
         }
         if (mode == TILE_GENERAL && has_time && rel32) mode = TILE_GEN32;
         TileArgs ta;
-        ta.i = i;
+        ta.i = ipos;
+        ta.dmin = CAND ? 1 : 0;
         ta.key0 = key0;
         ta.P = P;
         ta.Tb = Tb;
@@ -907,29 +1020,74 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       }
       if (!ok) break;
       g += nk;
-      // epilogue: AV rows = scale * O
-      if (!mbar_wait(&o_full[x], kx & 1u, abort_flag)) break;
-      tc_fence_after();
-      const bool valid = i < n;
+      // epilogue: AV rows = scale * O, plus in candidate mode the candidate's own term
+      // scale * SiLU(q_c . k_c + bias at distance 0 and time difference 0) * v_c
+      const bool has_o = !CAND || nk > 0;   // a candidate without history has no PV product
+      if (has_o) {
+        if (!mbar_wait(&o_full[x], kx & 1u, abort_flag)) break;
+        tc_fence_after();
+      }
+      const bool valid = i < ig.nq;
       // this warp's half of the head's columns
-      float* dst = prm.av + (row0 + i) * (int64_t)(H * HD) + h * HD + half * (HD / 2);
+      float* dst = prm.av + (ig.qrow0 + i) * (int64_t)(H * HD) + h * HD + half * (HD / 2);
+      float self_p = 0.0f;
+      const bf16* v_self = nullptr;
+      if (CAND) {
+        const bf16* crow =
+            prm.cand_uvqk + (ig.qrow0 + (i < ig.nq ? i : ig.nq - 1)) * (int64_t)prm.n1;
+        const uint4* q4 = reinterpret_cast<const uint4*>(crow + col_q + h * HD);
+        const uint4* k4 = reinterpret_cast<const uint4*>(crow + col_k + h * HD);
+        float sdot = 0.0f;
+#pragma unroll
+        for (int e = 0; e < HD / 8; e++) {
+          const uint4 qa = __ldg(q4 + e), ka = __ldg(k4 + e);
+          const uint32_t* qw = reinterpret_cast<const uint32_t*>(&qa);
+          const uint32_t* kw = reinterpret_cast<const uint32_t*>(&ka);
+#pragma unroll
+          for (int w = 0; w < 4; w++)
+            sdot = fmaf(bf16_hi(qw[w]), bf16_hi(kw[w]), fmaf(bf16_lo(qw[w]), bf16_lo(kw[w]), sdot));
+        }
+        // the staged tables hold half values; distance 0 and time bucket 0
+        const float bias0 =
+            BIAS == BIAS_RAB ? 2.0f * (hpos_s[0] + (has_time ? htt_s[0] : 0.0f)) : 0.0f;
+        const float xs = sdot + bias0;
+        self_p = prm.scale * __fdividef(xs, 1.0f + __expf(-xs));
+        v_self = crow + col_v + h * HD + half * (HD / 2);
+      }
 #pragma unroll
       for (int c = 0; c < HD / 64; c++) {
         uint32_t ov[32];
-        tmem_ld32(t_lane + Cfg::O_COL + x * Cfg::O_STRIDE + half * (HD / 2) + c * 32, ov);
-        tmem_ld_wait(ov);
+        if (has_o) {
+          tmem_ld32(t_lane + Cfg::O_COL + x * Cfg::O_STRIDE + half * (HD / 2) + c * 32, ov);
+          tmem_ld_wait(ov);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; e++) ov[e] = 0u;
+        }
         if (valid) {
 #pragma unroll
-          for (int v = 0; v < 8; v++)
-            reinterpret_cast<float4*>(dst + c * 32)[v] =
-                make_float4(prm.scale * __uint_as_float(ov[4 * v]), prm.scale * __uint_as_float(ov[4 * v + 1]),
-                            prm.scale * __uint_as_float(ov[4 * v + 2]), prm.scale * __uint_as_float(ov[4 * v + 3]));
+          for (int v = 0; v < 8; v++) {
+            float4 o = make_float4(prm.scale * __uint_as_float(ov[4 * v]),
+                                   prm.scale * __uint_as_float(ov[4 * v + 1]),
+                                   prm.scale * __uint_as_float(ov[4 * v + 2]),
+                                   prm.scale * __uint_as_float(ov[4 * v + 3]));
+            if (CAND) {
+              const uint2 vv = __ldg(reinterpret_cast<const uint2*>(v_self + c * 32) + v);
+              o.x = fmaf(self_p, bf16_lo(vv.x), o.x);
+              o.y = fmaf(self_p, bf16_hi(vv.x), o.y);
+              o.z = fmaf(self_p, bf16_lo(vv.y), o.z);
+              o.w = fmaf(self_p, bf16_hi(vv.y), o.w);
+            }
+            reinterpret_cast<float4*>(dst + c * 32)[v] = o;
+          }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty[x]);
-      kx++;
+      if (has_o) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&o_empty[x]);
+        kx++;
+      }
     }
   }
 

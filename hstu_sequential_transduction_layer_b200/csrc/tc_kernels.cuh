@@ -107,15 +107,16 @@ inline AttnSchedule attention_schedule_view(void* ws, int64_t B) {
   return s;
 }
 
-template <int HD, int BIAS>
-hstu_status_t launch_attention_kernel(const CUtensorMap& tm, const AttnParams& prm,
-                                      const AttnSchedule& sch, int grid, cudaStream_t st) {
+template <int HD, int BIAS, bool CAND = false>
+hstu_status_t launch_attention_kernel(const CUtensorMap& tm, const CUtensorMap& tmq,
+                                      const AttnParams& prm, const AttnSchedule& sch, int grid,
+                                      cudaStream_t st) {
   using Cfg = AttnCfg<HD>;
-  auto kern = attention_tc_kernel<HD, BIAS>;
+  auto kern = attention_tc_kernel<HD, BIAS, CAND>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
       cudaSuccess)
     return HSTU_ERR_CUDA;
-  kern<<<grid, ATT_THREADS, Cfg::SMEM, st>>>(tm, prm, sch);
+  kern<<<grid, ATT_THREADS, Cfg::SMEM, st>>>(tm, tmq, prm, sch);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
@@ -167,16 +168,93 @@ inline hstu_status_t launch_attention(int64_t T, int64_t B, int H, int hd, int64
   prm.av = av;
   prm.T = T;
   prm.dynamic = dynamic ? 1 : 0;
+  prm.cts = nullptr;
+  prm.cand_uvqk = nullptr;
   const int grid = (int)(capacity < num_sms() ? capacity : num_sms());
   const int bias = alibi ? BIAS_ALIBI : ((pos || tim) ? BIAS_RAB : BIAS_NONE);
   if (hd == 64) {
-    if (bias == BIAS_RAB) return launch_attention_kernel<64, BIAS_RAB>(tm, prm, sch, grid, st);
-    if (bias == BIAS_ALIBI) return launch_attention_kernel<64, BIAS_ALIBI>(tm, prm, sch, grid, st);
-    return launch_attention_kernel<64, BIAS_NONE>(tm, prm, sch, grid, st);
+    if (bias == BIAS_RAB) return launch_attention_kernel<64, BIAS_RAB>(tm, tm, prm, sch, grid, st);
+    if (bias == BIAS_ALIBI) return launch_attention_kernel<64, BIAS_ALIBI>(tm, tm, prm, sch, grid, st);
+    return launch_attention_kernel<64, BIAS_NONE>(tm, tm, prm, sch, grid, st);
   }
-  if (bias == BIAS_RAB) return launch_attention_kernel<128, BIAS_RAB>(tm, prm, sch, grid, st);
-  if (bias == BIAS_ALIBI) return launch_attention_kernel<128, BIAS_ALIBI>(tm, prm, sch, grid, st);
-  return launch_attention_kernel<128, BIAS_NONE>(tm, prm, sch, grid, st);
+  if (bias == BIAS_RAB) return launch_attention_kernel<128, BIAS_RAB>(tm, tm, prm, sch, grid, st);
+  if (bias == BIAS_ALIBI) return launch_attention_kernel<128, BIAS_ALIBI>(tm, tm, prm, sch, grid, st);
+  return launch_attention_kernel<128, BIAS_NONE>(tm, tm, prm, sch, grid, st);
+}
+
+// M-FALCON candidate attention workspace: header (256 B), per-user (candidate start, count,
+// history start, length), then one 8-byte entry per (user, pair of candidate tiles, head); at most
+// H * (ceil(Tc/256) + B) entries.
+inline int64_t candidate_capacity(int64_t Tc, int64_t B, int H) {
+  return (int64_t)H * ((Tc + ATT_ITEM_ROWS - 1) / ATT_ITEM_ROWS + B);
+}
+
+inline size_t candidate_workspace_bytes(int64_t Tc, int64_t B, int H) {
+  return (size_t)(256 + ((32 * B + 255) / 256) * 256 + 8 * candidate_capacity(Tc, B, H));
+}
+
+// Candidates of user b attend to b's history (K/V in uvqk_hist rows hoff[b] .. hoff[b+1]) and to
+// themselves; av_cand is fp32 [Tc, H*hd].  The history's UVQK is the one its own layer forward
+// produced (the encoder-level K/V cache).
+inline hstu_status_t launch_candidate_attention(
+    int64_t Th, int64_t Tc, int64_t B, int H, int hd, int64_t max_hist_len, const bf16* uvqk_hist,
+    const int64_t* hoff, const int64_t* hts, const bf16* uvqk_cand, const int64_t* coff,
+    const int64_t* cts, const float* pos, int P, const float* tim, int Tb, const float* alibi,
+    float scale, float* av, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (Th >= (1LL << 31) || Tc >= (1LL << 31) || H >= (1 << 15)) return HSTU_ERR_UNSUPPORTED;
+  if (ws_bytes < candidate_workspace_bytes(Tc, B, H)) return HSTU_ERR_INVALID_ARG;
+  const int64_t max_tiles64 = ((max_hist_len > 0 ? max_hist_len : Th) + ATT_BN - 1) / ATT_BN;
+  if (max_tiles64 > 12288) return HSTU_ERR_UNSUPPORTED;  // schedule counters in shared memory
+  const int max_tiles = (int)max_tiles64;
+  char* b = static_cast<char*>(ws);
+  AttnSchedule sch;
+  sch.header = reinterpret_cast<int64_t*>(b);
+  sch.seqinfo = reinterpret_cast<int64_t*>(b + 256);
+  sch.items = reinterpret_cast<int64_t*>(b + 256 + ((32 * B + 255) / 256) * 256);
+  const size_t sched_smem = 2 * (size_t)(max_tiles + 1) * sizeof(unsigned long long);
+  if (sched_smem > 48 * 1024 &&
+      cudaFuncSetAttribute(cand_schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)sched_smem) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  const int64_t capacity = candidate_capacity(Tc, B, H);
+  cand_schedule_kernel<<<1, 1024, sched_smem, st>>>(hoff, coff, B, Th, Tc, H, max_tiles, capacity,
+                                                    sch);
+  count_launch();
+  if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+
+  const int n1 = 4 * H * hd;
+  CUtensorMap tmk, tmq;
+  if (!make_map_bf16(&tmq, uvqk_cand, n1, Tc, n1, 64, 128)) return HSTU_ERR_CUDA;
+  if (Th > 0) {
+    if (!make_map_bf16(&tmk, uvqk_hist, n1, Th, n1, 64, 128)) return HSTU_ERR_CUDA;
+  } else {
+    tmk = tmq;  // no history anywhere: no key tile is ever loaded
+  }
+  AttnParams prm;
+  prm.ts = hts;
+  prm.pos = pos;
+  prm.tim = tim;
+  prm.alibi = alibi;
+  prm.P = P;
+  prm.Tb = Tb;
+  prm.H = H;
+  prm.n1 = n1;
+  prm.scale = scale;
+  prm.av = av;
+  prm.T = Tc;
+  prm.dynamic = 0;
+  prm.cts = cts;
+  prm.cand_uvqk = uvqk_cand;
+  const int grid = (int)(capacity < num_sms() ? capacity : num_sms());
+  const int bias = alibi ? BIAS_ALIBI : ((pos || tim) ? BIAS_RAB : BIAS_NONE);
+  if (hd == 64) {
+    if (bias == BIAS_RAB) return launch_attention_kernel<64, BIAS_RAB, true>(tmk, tmq, prm, sch, grid, st);
+    if (bias == BIAS_ALIBI) return launch_attention_kernel<64, BIAS_ALIBI, true>(tmk, tmq, prm, sch, grid, st);
+    return launch_attention_kernel<64, BIAS_NONE, true>(tmk, tmq, prm, sch, grid, st);
+  }
+  if (bias == BIAS_RAB) return launch_attention_kernel<128, BIAS_RAB, true>(tmk, tmq, prm, sch, grid, st);
+  if (bias == BIAS_ALIBI) return launch_attention_kernel<128, BIAS_ALIBI, true>(tmk, tmq, prm, sch, grid, st);
+  return launch_attention_kernel<128, BIAS_NONE, true>(tmk, tmq, prm, sch, grid, st);
 }
 
 }  // namespace tc

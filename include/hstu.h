@@ -161,6 +161,63 @@ hstu_status_t hstu_f2_fwd(const hstu_shape_t* shape, const void* g, const void* 
                           const void* X, void* out, void* stream);
 
 /*
+ * M-FALCON candidate scoring ("Actions Speak Louder than Words" paper notes, section 3.6; the
+ * efficiency paragraph of "4.4 推荐模型的 Scaling").  A user's m candidates are scored in one pass
+ * after its n history tokens: each candidate attends to the whole history and to itself, never to
+ * another candidate, and sits at position n (the place of the single next item) for the relative
+ * bias, with its own timestamp.  Per head:
+ *   AV_c = sum_{j<n} scale * SiLU(q_c . k_j + bias(n, j)) v_j + scale * SiLU(q_c . k_c + bias(n, n)) v_c
+ * with bias the rab^{p,t} buckets of distance n - j and time t_c - t_j (0 and 0 for the candidate
+ * itself), or ALiBi -m_h (n - j).  The history's K and V are read from its own UVQK, the one this
+ * layer's forward over the history produced (the encoder-level K/V cache): candidates can be
+ * scored in micro-batches of any size against the same cache with the same result.  bf16 only.
+ *
+ *  shape            the HISTORY's shape: num_seqs = users B, total_tokens = history tokens Th,
+ *                   max_seq_len >= the longest history; dims, tables and dtype (HSTU_BF16) as for
+ *                   hstu_layer_fwd
+ *  uvqk_hist        [Th, 4*H*hd] bf16, the history's f1 output of this layer
+ *  hist_offsets     [B+1] int64 history offsets; hist_timestamps [Th] (NULL without a time table)
+ *  num_candidates   Tc, all users' candidates; max_candidates >= the largest count of one user
+ *                   (at most 16,776,960)
+ *  uvqk_cand        [Tc, 4*H*hd] bf16, the candidates' f1 output
+ *  cand_offsets     [B+1] int64 candidate offsets (user b owns rows cand_offsets[b] ..
+ *                   cand_offsets[b+1]); cand_timestamps [Tc] (required with a time table)
+ *  av_cand          [Tc, H*hd] fp32 output; must not overlap the inputs or the workspace
+ *  workspace        hstu_candidate_workspace_size(shape, Tc) bytes, 256-byte aligned
+ * Errors as for hstu_attention_fwd; users with an empty history score their candidates from the
+ * candidates' own terms alone.
+ */
+size_t hstu_candidate_workspace_size(const hstu_shape_t* shape, int64_t num_candidates);
+hstu_status_t hstu_candidate_attention_fwd(const hstu_shape_t* shape, const void* uvqk_hist,
+                                           const int64_t* hist_offsets,
+                                           const int64_t* hist_timestamps, int64_t num_candidates,
+                                           int64_t max_candidates, const void* uvqk_cand,
+                                           const int64_t* cand_offsets,
+                                           const int64_t* cand_timestamps, const float* pos_table,
+                                           const float* time_table, const float* alibi_slopes,
+                                           float scale, void* av_cand, void* workspace,
+                                           size_t workspace_bytes, void* stream);
+
+/*
+ * hstu_candidate_layer_fwd -- one HSTU layer over the candidates (Eqs. 1-3 with the candidate
+ * attention above): out_cand = f2(LayerNorm(AV_c) * U_c) + X_cand, with U|V|Q|K of the candidates
+ * from f1 of X_cand [Tc, d].  Other arguments as for hstu_candidate_attention_fwd and
+ * hstu_layer_fwd; workspace: hstu_candidate_layer_workspace_size(shape, Tc) bytes (holds the
+ * candidates' UVQK, AV, G and the schedule).
+ */
+size_t hstu_candidate_layer_workspace_size(const hstu_shape_t* shape, int64_t num_candidates);
+hstu_status_t hstu_candidate_layer_fwd(const hstu_shape_t* shape, const void* uvqk_hist,
+                                       const int64_t* hist_offsets, const int64_t* hist_timestamps,
+                                       int64_t num_candidates, int64_t max_candidates,
+                                       const void* X_cand, const int64_t* cand_offsets,
+                                       const int64_t* cand_timestamps, const void* W1,
+                                       const void* b1, const void* W2, const void* b2,
+                                       const void* ln_w, const void* ln_b, const float* pos_table,
+                                       const float* time_table, const float* alibi_slopes,
+                                       float scale, void* out_cand, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
+/*
  * hstu_selftest_bounded_wait -- checks, on the device, the bounded wait that every pipelined kernel
  * of this library uses on its mbarriers.
  *

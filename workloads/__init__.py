@@ -268,3 +268,40 @@ def random_case(seed: int, lengths, d: int, H: int, hd: int, P: int = 16, Tb: in
     if scale is not None:
         inp.scale = scale
     return inp
+
+
+# ----------------------------------------------------------------------------------------------
+# M-FALCON candidates
+# ----------------------------------------------------------------------------------------------
+
+
+@dataclasses.dataclass
+class Candidates:
+    """Candidates appended after each user's history (one user = one sequence of an Inputs)."""
+    counts: np.ndarray                 # [B] candidates per user
+    offsets: np.ndarray                # [B+1]
+    X: np.ndarray                      # [Tc, d], drawn like the history's X
+    timestamps: Optional[np.ndarray]   # [Tc] int64, or None when the history has none
+
+
+def draw_candidates(inp: Inputs, counts, spread_s: int = 0, stream: int = 20) -> Candidates:
+    """Candidate tokens for every user of `inp`: N(0,1) embeddings (rounded like the workload's X),
+    scored at a request time one Exp(gap_mean) gap after the user's last history event; with
+    `spread_s` > 0 each candidate gets its own time up to `spread_s` seconds later."""
+    w = inp.workload
+    counts = np.asarray(counts, dtype=np.int64)
+    assert len(counts) == len(inp.lengths)
+    off = offsets_from_lengths(counts)
+    rng = _stream(w.index, stream)
+    X = _round_like(w, rng.standard_normal((int(off[-1]), w.d_model), dtype=np.float32))
+    ts = None
+    if inp.timestamps is not None:
+        ts = np.zeros(int(off[-1]), dtype=np.int64)
+        gap = w.gap_mean_s if w.gap_mean_s > 0 else 60.0
+        for b in range(len(counts)):
+            a, e = inp.seq_offsets[b], inp.seq_offsets[b + 1]
+            last = int(inp.timestamps[e - 1]) if e > a else 0
+            t = last + int(np.floor(rng.exponential(gap)))
+            extra = rng.integers(0, spread_s + 1, size=int(counts[b])) if spread_s > 0 else 0
+            ts[off[b]:off[b + 1]] = t + extra
+    return Candidates(counts, off, X, ts)
