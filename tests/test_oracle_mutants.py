@@ -36,7 +36,7 @@ MUTANTS = {
     "b2_dropped": ("y[c] = b2 ? b2[c] : 0.0;", "y[c] = 0.0;"),
     "scale_inside_silu": ("scale * silu(s)", "silu(scale * s)"),
     "alibi_sign": ("return -alibi_slopes[h] * (double)(i - j);", "return alibi_slopes[h] * (double)(i - j);"),
-    "v_head_offset": ("offV + (int64_t)h * dv;", "offV;"),
+    "v_head_offset": ("uvqk_seq + j * n1 + offV + (int64_t)h * dv;", "uvqk_seq + j * n1 + offV;"),
     "gate_missing": ("+ ln_b[c]) * u[c];", "+ ln_b[c]);"),
 }
 
