@@ -330,6 +330,198 @@ def run_e2e(args, hstu, torch, inp, D, shape, dev, stream, world):
 
 
 # ------------------------------------------------------------------------------------------------
+# M-FALCON candidate scoring (--candidates M): M candidates per user scored after the workload's
+# sequences, which serve as the users' histories.  The history's UVQK (the K/V cache) is computed
+# once before the timed region; a step is one candidate layer (f1, candidate attention, LayerNorm*U,
+# f2) over every user's candidates.
+# ------------------------------------------------------------------------------------------------
+
+CAND_METRIC = "HSTU candidate scoring throughput (M-FALCON, one layer over cached history K/V)"
+
+
+def run_candidates(args, rank, world, local_rank):
+    import torch
+    import hstu_sequential_transduction_layer_b200 as hstu
+    from workloads.device import to_device, tensor
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workloads.WORKLOADS[args.workload]
+    inp = workloads.make_inputs(w)
+    if w.token_embed:
+        raise SystemExit("candidate scoring is timed on workloads with explicit X")
+    M = args.candidates
+    cand = workloads.draw_candidates(inp, np.full(len(inp.lengths), M))
+    H, hd, d = w.num_heads, w.head_dim, w.d_model
+    Tc = int(cand.offsets[-1])
+    D = to_device(inp, dev)
+    L = D["layers"][0]
+    shape = hstu.shape_for(D["X"], D["off"], H, hd, hd, int(inp.lengths.max()), D["pos"], D["tim"],
+                           inp.ln_eps)
+    cshape = hstu.make_shape(len(inp.lengths), Tc, M, d, H, hd, hd, hstu.HSTU_BF16,
+                             shape.n_pos_buckets, shape.n_time_buckets, inp.ln_eps)
+    n1, wv = 4 * H * hd, H * hd
+    uvqk_hist = torch.empty((inp.T, n1), dtype=torch.bfloat16, device=dev)
+    hstu.hstu_f1_fwd(shape, D["X"], L["W1"], L["b1"], uvqk_hist)       # the history's K/V cache
+    Xc = tensor(cand.X, "bf16", dev)
+    coff = tensor(cand.offsets, "i64", dev)
+    cts = tensor(cand.timestamps, "i64", dev) if cand.timestamps is not None else None
+    uvqk_c = torch.empty((Tc, n1), dtype=torch.bfloat16, device=dev)
+    av = torch.empty((Tc, wv), dtype=torch.float32, device=dev)
+    g = torch.empty((Tc, wv), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((Tc, d), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(max(256, hstu.candidate_workspace_size(shape, Tc)), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        hstu.hstu_f1_fwd(cshape, Xc, L["W1"], L["b1"], uvqk_c, stream)
+        if evs:
+            evs[1].record(stream)
+        hstu.hstu_candidate_attention_fwd(shape, uvqk_hist, D["off"], D["ts"], uvqk_c, coff, cts,
+                                          D["pos"], D["tim"], D["ali"], inp.scale, av,
+                                          max_candidates=M, workspace=ws, stream=stream)
+        if evs:
+            evs[2].record(stream)
+        hstu.hstu_ln_gate_fwd(cshape, av, uvqk_c, L["ln_w"], L["ln_b"], g, stream)
+        if evs:
+            evs[3].record(stream)
+        hstu.hstu_f2_fwd(cshape, g, L["W2"], L["b2"], Xc, out, stream)
+        if evs:
+            evs[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if hstu.device_status() != hstu.HSTU_OK:
+        raise SystemExit("device status error during warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    launches0 = hstu.launch_count()
+    for k in range(args.steps):
+        flush.zero_()
+        step(evs[k])
+    torch.cuda.synchronize()
+    launches = hstu.launch_count() - launches0
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    per_kernel = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in evs])
+    total_ms, job_cands = combine_over_ranks(float(per_kernel.sum()), Tc, world, dev)
+    if hstu.device_status() != hstu.HSTU_OK:
+        raise SystemExit("device status error in the timed region")
+    ms_per_step = total_ms / args.steps
+    kern_ms = per_kernel.mean(axis=0)
+    peaks, peaks_src = load_peaks()
+    tpk = peaks["bf16_tflops"]
+    # algorithmic attention work: every candidate against its history plus itself
+    pairs = float(np.sum(cand.counts * (inp.lengths + 1)))
+    attn_fl = 2.0 * H * (2 * hd) * pairs
+    f1_fl, f2_fl = gemm_flops(Tc, d, n1, wv)
+    kernels = {
+        "f1_gemm": {"ms": kern_ms[0], "TFLOP/s": f1_fl / kern_ms[0] / 1e9},
+        "candidate_attention": {"ms": kern_ms[1], "TFLOP/s": attn_fl / kern_ms[1] / 1e9},
+        "ln_gate": {"ms": kern_ms[2], "GB/s": 8.0 * wv * Tc / kern_ms[2] / 1e6},
+        "f2_gemm": {"ms": kern_ms[3], "TFLOP/s": f2_fl / kern_ms[3] / 1e9},
+    }
+    for v in kernels.values():
+        for kk in list(v):
+            v[kk] = round(float(v[kk]), 4)
+    attn_tflops = attn_fl / kern_ms[1] / 1e9
+
+    # end to end through hstu_candidate_layer_fwd: candidate X, offsets and timestamps copied in
+    # from pinned host memory and the scores' inputs (Y) copied out, the history cache on the device
+    Xh = Xc.cpu().pin_memory()
+    offh = coff.cpu().pin_memory()
+    tsh = cts.cpu().pin_memory() if cts is not None else None
+    outh = torch.empty_like(Xh).pin_memory()
+    Xd, offd = torch.empty_like(Xc), torch.empty_like(coff)
+    tsd = torch.empty_like(cts) if cts is not None else None
+    lws = torch.empty(max(256, hstu.candidate_layer_workspace_size(shape, Tc)), dtype=torch.uint8,
+                      device=dev)
+
+    def one():
+        Xd.copy_(Xh, non_blocking=True)
+        offd.copy_(offh, non_blocking=True)
+        if tsd is not None:
+            tsd.copy_(tsh, non_blocking=True)
+        hstu.hstu_candidate_layer_fwd(shape, uvqk_hist, D["off"], D["ts"], Xd, offd, tsd, L["W1"],
+                                      L["b1"], L["W2"], L["b2"], L["ln_w"], L["ln_b"], D["pos"],
+                                      D["tim"], D["ali"], inp.scale, out, max_candidates=M,
+                                      workspace=lws, stream=stream)
+        outh.copy_(out, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e2e_steps = max(1, min(args.steps, 20))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ems, _ = combine_over_ranks(e0.elapsed_time(e1) / e2e_steps, Tc, world, dev)
+    h2d = Xh.numel() * 2 + offh.numel() * 8 + (tsh.numel() * 8 if tsh is not None else 0)
+
+    return {
+        "metric": CAND_METRIC, "value": round(job_cands / (ms_per_step * 1e-3), 1),
+        "unit": "candidates/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded; users' histories from the workload, N(0,1) candidates)",
+        "config": {"workload": f"{w.name} histories (B={len(inp.lengths)}, n={int(inp.lengths.max())}, "
+                               f"d={d}, H={H}x{hd}) + {M} candidates per user, 1 layer",
+                   "candidates_per_step": job_cands,
+                   "l2": "flushed between timed steps (256 MB write, outside the events)"},
+        "roofline": {"bound": "tensor", "kernel": "candidate_attention",
+                     "achieved": round(attn_tflops, 2), "peak": tpk, "unit": "TFLOP/s",
+                     "frac": round(attn_tflops / tpk, 4), "traffic": None,
+                     "peak_source": f"{peaks_src} bf16 burst (MEASURED_PEAKS.json)"
+                     if peaks_src == "measured" else "fallback 1590 TFLOP/s"},
+        "kernels": kernels,
+        "e2e": {"value": round(job_cands / (ems * 1e-3), 1), "unit": "candidates/s",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(outh.numel() * 2),
+                "ms_per_step": round(ems, 4), "steps": e2e_steps},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+
+
+def candidate_cpu_baseline(args):
+    """The oracle's candidate layer on one user's first 32 candidates against its full history."""
+    import oracle
+    oracle.build()
+    w = workloads.WORKLOADS[args.workload]
+    inp = workloads.make_inputs(w)
+    M = min(args.candidates, 32)
+    cand = workloads.draw_candidates(inp, np.full(len(inp.lengths), args.candidates))
+    p = inp.layers[0]
+    n = int(inp.lengths[0])
+    t0 = time.perf_counter()
+    uh = oracle.f1(inp.X[:n], p.W1, p.b1)
+    t1 = time.perf_counter()
+    oracle.candidate_layer_fwd(np.array([0, n]), uh, np.array([0, M]), cand.X[:M], p.W1, p.b1,
+                               p.W2, p.b2, p.ln_w, p.ln_b, num_heads=w.num_heads, d_qk=w.head_dim,
+                               d_v=w.head_dim, hist_timestamps=None if inp.timestamps is None
+                               else inp.timestamps[:n],
+                               cand_timestamps=None if cand.timestamps is None
+                               else cand.timestamps[:M], pos_table=inp.pos_table,
+                               time_table=inp.time_table, alibi_slopes=inp.alibi_slopes,
+                               scale=inp.scale, ln_eps=inp.ln_eps)
+    dt = time.perf_counter() - t1
+    return {"value": round(M / dt, 2), "unit": "candidates/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{M} candidates of one user against its {n}-token history (cache built in "
+                      f"{t1 - t0:.1f} s, not counted); {dt:.1f} s; C fp64 loops, OpenMP, -O2"}
+
+
+# ------------------------------------------------------------------------------------------------
 # The oracle on the host cores (cpu_baseline of our arm, and the whole reference arm)
 # ------------------------------------------------------------------------------------------------
 
@@ -399,6 +591,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long_seq", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--candidates", type=int, default=0,
+                    help="time M-FALCON scoring of this many candidates per user instead")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -418,6 +612,13 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
+        if args.candidates > 0:
+            res = run_candidates(args, rank, world, local_rank)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                res["cpu_baseline"] = candidate_cpu_baseline(args)
+            if rank == 0:
+                print(json.dumps(res), flush=True)
+            return
         res = run_ours(args, rank, world, local_rank)
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:
