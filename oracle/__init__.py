@@ -67,6 +67,8 @@ def bind(path: str):
     lib.oracle_candidate_attention.argtypes = [i64, ip, ip, i32, i32, i32, dp, ip, dp, ip, dp, i32,
                                                dp, i32, dp, f64, dp]
     lib.oracle_candidate_attention.restype = None
+    lib.oracle_stochastic_length.argtypes = [i64, ip, i64, f64, dp, ip, ip, ip]
+    lib.oracle_stochastic_length.restype = i64
     lib.oracle_ln_gate.argtypes = [i64, i32, i32, i32, dp, dp, dp, dp, f64, dp]
     lib.oracle_ln_gate.restype = None
     lib.oracle_f2.argtypes = [i64, i32, i32, dp, dp, dp, dp, dp]
@@ -281,6 +283,20 @@ def candidate_layer_fwd(hist_offsets, uvqk_hist, cand_offsets, X_cand, W1, b1, W
                              time_table=time_table, alibi_slopes=alibi_slopes, scale=scale)
     g = ln_gate(av, uc, ln_w, ln_b, num_heads=num_heads, d_qk=d_qk, d_v=d_v, ln_eps=ln_eps)
     return f2(g, W2, b2, X_cand)
+
+
+def stochastic_length(seq_offsets, max_len: int, alpha: float, u, keys, lib=None):
+    """Stochastic Length: -> (new_offsets [B+1], index [T_new]) with index[r] the source row of the
+    subsampled batch's row r.  u: [B] uniforms in [0, 1); keys: [T] uint32."""
+    off = _i(seq_offsets)
+    B = len(off) - 1
+    u = _d(u)
+    keys = np.ascontiguousarray(keys, dtype=np.uint32)
+    new_off = np.empty(B + 1, np.int64)
+    index = np.empty(max(1, int(off[-1])), np.int64)
+    n = _load(lib).oracle_stochastic_length(B, _p(off), int(max_len), float(alpha), _p(u),
+                                            _p(keys), _p(new_off), _p(index))
+    return new_off, index[:n]
 
 
 def ln_gate(av, uvqk, ln_w, ln_b, *, num_heads: int, d_qk: int, d_v: int,

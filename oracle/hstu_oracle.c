@@ -208,6 +208,66 @@ void oracle_candidate_attention(int64_t B, const int64_t* hist_offsets,
 }
 
 /* ---------------------------------------------------------------------------------------------
+ * Stochastic Length ("Actions Speak Louder than Words" paper notes, section 3.3).  With
+ * N_c = the longest sequence (passed in) and alpha in (1, 2], a sequence of n tokens is kept whole
+ * when n <= N_c^(alpha/2); otherwise, with probability 1 - N_c^alpha / n^2, it is replaced by a
+ * subsequence of floor(N_c^(alpha/2)) of its tokens (and kept whole with probability
+ * N_c^alpha / n^2).  Readings fixed here (the pages leave them open):
+ *   - the subsequence is a uniformly random subset of that size, kept in the original order;
+ *   - the method's random draws are inputs: u[s] uniform in [0, 1) per sequence (subsample when
+ *     u[s] >= N_c^alpha / n^2) and keys[t] uniform 32-bit words per token (the subset is the
+ *     floor(N_c^(alpha/2)) tokens with the smallest (key, position) pairs, which is a uniform
+ *     random subset when the keys are i.i.d.).
+ * Output: the new offsets [B+1] and, for the new batch's row r, the source row index[r]; returns
+ * the new token count.
+ * --------------------------------------------------------------------------------------------- */
+typedef struct {
+  uint32_t key;
+  int64_t pos;
+} sl_entry;
+
+static int sl_by_key(const void* a, const void* b) {
+  const sl_entry* x = (const sl_entry*)a;
+  const sl_entry* y = (const sl_entry*)b;
+  if (x->key != y->key) return x->key < y->key ? -1 : 1;
+  return x->pos < y->pos ? -1 : (x->pos > y->pos ? 1 : 0);
+}
+
+static int sl_by_pos(const void* a, const void* b) {
+  const sl_entry* x = (const sl_entry*)a;
+  const sl_entry* y = (const sl_entry*)b;
+  return x->pos < y->pos ? -1 : (x->pos > y->pos ? 1 : 0);
+}
+
+int64_t oracle_stochastic_length(int64_t B, const int64_t* seq_offsets, int64_t max_len,
+                                 double alpha, const double* u, const uint32_t* keys,
+                                 int64_t* new_offsets, int64_t* index) {
+  const double lf = pow((double)max_len, alpha / 2.0);   /* N_c^(alpha/2) */
+  const int64_t L = (int64_t)floor(lf);
+  int64_t r = 0;
+  new_offsets[0] = 0;
+  for (int64_t s = 0; s < B; s++) {
+    const int64_t a = seq_offsets[s], n = seq_offsets[s + 1] - seq_offsets[s];
+    const int sub = (double)n > lf && u[s] >= (lf * lf) / ((double)n * (double)n);
+    if (!sub) {
+      for (int64_t i = 0; i < n; i++) index[r++] = a + i;
+    } else {
+      sl_entry* e = (sl_entry*)malloc((size_t)n * sizeof(sl_entry));
+      for (int64_t i = 0; i < n; i++) {
+        e[i].key = keys[a + i];
+        e[i].pos = i;
+      }
+      qsort(e, (size_t)n, sizeof(sl_entry), sl_by_key);   /* the L smallest come first */
+      qsort(e, (size_t)L, sizeof(sl_entry), sl_by_pos);   /* back to sequence order */
+      for (int64_t k = 0; k < L; k++) index[r++] = a + e[k].pos;
+      free(e);
+    }
+    new_offsets[s + 1] = r;
+  }
+  return r;
+}
+
+/* ---------------------------------------------------------------------------------------------
  * Eq. 3, first half: G = LayerNorm(AV) * U.  Norm is a layer normalisation; the sketch normalises
  * the full d-wide row.  Mean and biased variance over the H*dv columns.
  * --------------------------------------------------------------------------------------------- */

@@ -52,6 +52,40 @@ CANDIDATE_MUTANTS = {
 }
 
 
+# planted in the Stochastic Length code: caught by the pins below
+SL_MUTANTS = {
+    "sl_probability_inverted": ("u[s] >= (lf * lf) / ((double)n * (double)n)",
+                                "u[s] < (lf * lf) / ((double)n * (double)n)"),
+    "sl_length_rounded_up": ("const int64_t L = (int64_t)floor(lf);", "const int64_t L = (int64_t)ceil(lf);"),
+    "sl_largest_keys": ("if (x->key != y->key) return x->key < y->key ? -1 : 1;",
+                        "if (x->key != y->key) return x->key > y->key ? -1 : 1;"),
+    "sl_order_lost": ("qsort(e, (size_t)L, sizeof(sl_entry), sl_by_pos);", "(void)sl_by_pos;"),
+}
+
+
+def _sl_pins_pass(lib) -> bool:
+    """The Stochastic Length pins: the page's 4096 -> 776 at alpha 1.6, closed forms with known key
+    order, and the cut probability by Monte Carlo."""
+    from workloads import draw_stochastic_length_randoms
+    off = np.array([0, 4096, 7096], np.int64)
+    keys = np.random.default_rng(1).integers(0, 1 << 32, 7096, dtype=np.uint64).astype(np.uint32)
+    no, _ = oracle.stochastic_length(off, 4096, 1.6, np.array([0.999999, 0.999999]), keys, lib=lib)
+    if list(np.diff(no)) != [776, 776]:
+        return False
+    n = 600
+    perm = np.random.default_rng(2).permutation(n).astype(np.uint32)
+    no, idx = oracle.stochastic_length(np.array([0, n]), 1000, 1.5, np.array([0.99]), perm, lib=lib)
+    if no[-1] != 177 or not np.array_equal(idx, np.flatnonzero(perm < 177)):
+        return False
+    trials, n = 2000, 1200
+    off = np.arange(trials + 1, dtype=np.int64) * n
+    u, keys = draw_stochastic_length_randoms(off, seed=7)
+    no, _ = oracle.stochastic_length(off, 4096, 1.6, u, keys, lib=lib)
+    p = 1 - (4096 ** 0.8) ** 2 / n ** 2
+    cut = np.mean(np.diff(no) < n)
+    return abs(cut - p) < 4 * np.sqrt(p * (1 - p) / trials)
+
+
 def _silu(x):
     return x / (1.0 + np.exp(-x))
 
@@ -150,6 +184,16 @@ def test_unmodified_oracle_passes_the_independent_pins(tmp_path):
     lib = _compile(open(SRC).read(), tmp_path, "orig")
     assert _pins_pass(lib)
     assert _candidate_pins_pass(lib)
+    assert _sl_pins_pass(lib)
+
+
+@pytest.mark.parametrize("name", sorted(SL_MUTANTS))
+def test_planted_stochastic_length_mistake_is_caught(name, tmp_path):
+    src = open(SRC).read()
+    old, new = SL_MUTANTS[name]
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    lib = _compile(src.replace(old, new), tmp_path, name)
+    assert not _sl_pins_pass(lib), f"planted mistake {name} went unnoticed"
 
 
 @pytest.mark.parametrize("name", sorted(CANDIDATE_MUTANTS))

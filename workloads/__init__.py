@@ -305,3 +305,13 @@ def draw_candidates(inp: Inputs, counts, spread_s: int = 0, stream: int = 20) ->
             extra = rng.integers(0, spread_s + 1, size=int(counts[b])) if spread_s > 0 else 0
             ts[off[b]:off[b + 1]] = t + extra
     return Candidates(counts, off, X, ts)
+
+
+def draw_stochastic_length_randoms(seq_offsets: np.ndarray, seed: int):
+    """The Stochastic Length draws, as inputs: one uniform in [0, 1) per sequence (float64) and one
+    uniform 32-bit key per token (uint32)."""
+    rng = np.random.default_rng(np.random.SeedSequence([seed, 30]))
+    B = len(seq_offsets) - 1
+    u = rng.random(B)
+    keys = rng.integers(0, 1 << 32, size=int(seq_offsets[-1]), dtype=np.uint64).astype(np.uint32)
+    return u, keys
