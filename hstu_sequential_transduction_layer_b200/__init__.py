@@ -31,7 +31,8 @@ EXPORTED = ["hstu_layer_fwd", "hstu_layer_fwd_workspace_size", "hstu_f1_fwd", "h
             "hstu_token_embed_fwd", "hstu_status_string", "hstu_get_device_status", "hstu_version",
             "hstu_launch_count", "hstu_attention_fwd_noalloc", "hstu_selftest_bounded_wait",
             "hstu_candidate_workspace_size", "hstu_candidate_attention_fwd",
-            "hstu_candidate_layer_workspace_size", "hstu_candidate_layer_fwd"]
+            "hstu_candidate_layer_workspace_size", "hstu_candidate_layer_fwd",
+            "hstu_stochastic_length_workspace_size", "hstu_stochastic_length", "hstu_gather_rows"]
 
 
 class HstuShape(ctypes.Structure):
@@ -78,6 +79,10 @@ def _load() -> ctypes.CDLL:
         "hstu_candidate_attention_fwd": ([SH, P, P, P, I64, I64, P, P, P, P, P, P, F32, P, P, S, P],
                                          ctypes.c_int),
         "hstu_candidate_layer_workspace_size": ([SH, I64], S),
+        "hstu_stochastic_length_workspace_size": ([I64], S),
+        "hstu_stochastic_length": ([I64, I64, P, I64, ctypes.c_double, P, P, P, P, P, S, P],
+                                   ctypes.c_int),
+        "hstu_gather_rows": ([I64, P, I64, P, P, I64, P, P], ctypes.c_int),
         "hstu_candidate_layer_fwd": ([SH, P, P, P, I64, I64, P, P, P, P, P, P, P, P, P, P, P, P, F32,
                                       P, P, S, P], ctypes.c_int),
     }
@@ -273,6 +278,30 @@ def hstu_candidate_layer_fwd(shape: HstuShape, uvqk_hist, hist_offsets, hist_tim
         _ptr(alibi_slopes), float(scale), _ptr(out_cand), _ptr(workspace), workspace.numel(),
         _stream(stream)), "hstu_candidate_layer_fwd")
     return out_cand
+
+
+def hstu_stochastic_length(seq_offsets, max_len: int, alpha: float, u, keys, new_offsets, index,
+                           workspace=None, stream=None):
+    """Stochastic Length on the device (see the C header); returns (new_offsets, index)."""
+    B = int(seq_offsets.numel()) - 1
+    T = int(keys.numel())
+    if workspace is None:
+        workspace = torch.empty(max(256, int(_lib.hstu_stochastic_length_workspace_size(B))),
+                                dtype=torch.uint8, device=seq_offsets.device)
+    _check(_lib.hstu_stochastic_length(B, T, _ptr(seq_offsets), int(max_len), float(alpha),
+                                       _ptr(u), _ptr(keys), _ptr(new_offsets), _ptr(index),
+                                       _ptr(workspace), workspace.numel(), _stream(stream)),
+           "hstu_stochastic_length")
+    return new_offsets, index
+
+
+def hstu_gather_rows(index, src, dst, row_count=None, stream=None):
+    """dst[r] = src[index[r]] for r < row_count (a device int64 scalar) or all of dst's rows."""
+    max_rows = int(dst.shape[0])
+    row_bytes = int(dst[0].numel() * dst.element_size()) if dst.dim() > 1 else dst.element_size()
+    _check(_lib.hstu_gather_rows(max_rows, _ptr(row_count), row_bytes, _ptr(index), _ptr(src),
+                                 int(src.shape[0]), _ptr(dst), _stream(stream)), "hstu_gather_rows")
+    return dst
 
 
 def hstu_ln_gate_fwd(shape: HstuShape, av, uvqk, ln_w, ln_b, g, stream=None):

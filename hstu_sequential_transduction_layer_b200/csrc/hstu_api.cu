@@ -7,6 +7,7 @@
 
 #include "common.cuh"
 #include "hbm_kernels.cuh"
+#include "sl_kernels.cuh"
 #include "simt_kernels.cuh"
 #include "tc_kernels.cuh"
 
@@ -539,6 +540,60 @@ hstu_status_t hstu_candidate_layer_fwd(const hstu_shape_t* shape, const void* uv
     return rc;
   if ((rc = run_ln_gate(c, w.av, w.uvqk, ln_w, ln_b, w.g, st)) != HSTU_OK) return rc;
   return run_f2(c, w.g, W2, b2, X_cand, out_cand, st);
+}
+
+size_t hstu_stochastic_length_workspace_size(int64_t num_seqs) {
+  return num_seqs < 0 ? 0 : align_up((size_t)num_seqs * sizeof(int32_t) + 1);
+}
+
+hstu_status_t hstu_stochastic_length(int64_t num_seqs, int64_t total_tokens,
+                                     const int64_t* seq_offsets, int64_t max_len, double alpha,
+                                     const double* u, const uint32_t* keys, int64_t* new_offsets,
+                                     int64_t* index, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  const int64_t B = num_seqs, T = total_tokens;
+  if (B < 0 || T < 0 || max_len < 0 || T > (1LL << 40)) return HSTU_ERR_INVALID_ARG;
+  if (!(alpha > 0.0 && alpha <= 2.0)) return HSTU_ERR_INVALID_ARG;
+  if (!new_offsets) return HSTU_ERR_INVALID_ARG;
+  if (B > 0 && (!seq_offsets || !u || !workspace)) return HSTU_ERR_INVALID_ARG;
+  if (T > 0 && (!keys || !index)) return HSTU_ERR_INVALID_ARG;
+  if (workspace_bytes < hstu_stochastic_length_workspace_size(B)) return HSTU_ERR_INVALID_ARG;
+  // N_c^(alpha/2) and its floor, computed once on the host in fp64 (the same pow as the oracle's)
+  const double lf = std::pow((double)max_len, alpha / 2.0);
+  const int64_t L = (int64_t)std::floor(lf);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* cut = static_cast<int32_t*>(workspace);
+  sl::sl_plan_kernel<<<1, sl::SL_THREADS, 0, st>>>(seq_offsets, B, T, lf, L, u, cut, new_offsets);
+  if (launch_status() != HSTU_OK) return HSTU_ERR_CUDA;
+  if (B == 0 || T == 0) return HSTU_OK;
+  const int64_t grid = B < 4096 ? B : 4096;
+  sl::sl_select_kernel<<<(unsigned)grid, sl::SL_THREADS, 0, st>>>(seq_offsets, B, T, L, keys, cut,
+                                                                  new_offsets, index);
+  return launch_status();
+}
+
+hstu_status_t hstu_gather_rows(int64_t max_rows, const int64_t* row_count, int64_t row_bytes,
+                               const int64_t* index, const void* src, int64_t src_rows, void* dst,
+                               void* stream) {
+  if (max_rows < 0 || src_rows < 0 || row_bytes <= 0 || row_bytes % 8 != 0 ||
+      row_bytes > (1LL << 30) || max_rows > (1LL << 40))
+    return HSTU_ERR_INVALID_ARG;
+  if (max_rows == 0) return HSTU_OK;
+  if (!index || !src || !dst) return HSTU_ERR_INVALID_ARG;
+  if (overlaps(dst, (size_t)max_rows * row_bytes, src, (size_t)src_rows * row_bytes))
+    return HSTU_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool v16 = row_bytes % 16 == 0 && aligned16(src) && aligned16(dst);
+  const int units = (int)(row_bytes / (v16 ? 16 : 8));
+  const int64_t threads = max_rows * units;
+  const unsigned blocks = (unsigned)((threads + 255) / 256);
+  if (v16)
+    sl::gather_rows16_kernel<<<blocks, 256, 0, st>>>(max_rows, row_count, units, index,
+                                                     (const uint4*)src, src_rows, (uint4*)dst);
+  else
+    sl::gather_rows8_kernel<<<blocks, 256, 0, st>>>(max_rows, row_count, units, index,
+                                                    (const uint2*)src, src_rows, (uint2*)dst);
+  return launch_status();
 }
 
 hstu_status_t hstu_selftest_bounded_wait(uint64_t limit_ns, long long* result, void* stream) {

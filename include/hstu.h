@@ -218,6 +218,44 @@ hstu_status_t hstu_candidate_layer_fwd(const hstu_shape_t* shape, const void* uv
                                        size_t workspace_bytes, void* stream);
 
 /*
+ * Stochastic Length ("Actions Speak Louder than Words" paper notes, section 3.3): shortens the
+ * long sequences of a jagged batch before the layers run.  With N_c = max_len and
+ * Lf = N_c^(alpha/2) (computed on the host in fp64), sequence s of n tokens is cut when n > Lf and
+ * u[s] >= Lf^2 / n^2 (probability 1 - N_c^alpha / n^2 for u uniform), to the floor(Lf) tokens
+ * with the smallest (keys[t], position) pairs, kept in their original order (a uniformly random
+ * subset for i.i.d. keys); otherwise it is kept whole.  The method's random draws are the
+ * caller's inputs, so results are reproducible.
+ *
+ *  num_seqs, total_tokens   B and T of the input batch; seq_offsets [B+1] int64 (device)
+ *  max_len                  N_c (the batch's or the configuration's longest sequence)
+ *  alpha                    in (0, 2] (the pages use (1, 2]); else HSTU_ERR_INVALID_ARG
+ *  u                        [B] fp64 in [0, 1) (device); keys [T] uint32 (device)
+ *  new_offsets              [B+1] int64 output (device); new_offsets[B] is the new token count
+ *  index                    [T] int64 output (device): index[r] is the source row of new row r,
+ *                           r < new_offsets[B]
+ *  workspace                hstu_stochastic_length_workspace_size(B) bytes of device memory
+ * Asynchronous on `stream`; bad offsets are clamped and reported in the device status word.
+ */
+size_t hstu_stochastic_length_workspace_size(int64_t num_seqs);
+hstu_status_t hstu_stochastic_length(int64_t num_seqs, int64_t total_tokens,
+                                     const int64_t* seq_offsets, int64_t max_len, double alpha,
+                                     const double* u, const uint32_t* keys, int64_t* new_offsets,
+                                     int64_t* index, void* workspace, size_t workspace_bytes,
+                                     void* stream);
+
+/*
+ * hstu_gather_rows -- dst[r] = src[index[r]] for rows of row_bytes bytes (a multiple of 8), for
+ * r < *row_count when row_count (a device int64, e.g. new_offsets + B of hstu_stochastic_length)
+ * is given, else r < max_rows; dst holds max_rows rows.  Builds the shortened batch (X rows,
+ * timestamps) without a host round trip.  An index outside [0, src_rows) gives a zero row and
+ * HSTU_ERR_DEVICE_BAD_OFFSETS in the device status word.  The paper has no counterpart: it is
+ * the data movement that Stochastic Length implies.
+ */
+hstu_status_t hstu_gather_rows(int64_t max_rows, const int64_t* row_count, int64_t row_bytes,
+                               const int64_t* index, const void* src, int64_t src_rows, void* dst,
+                               void* stream);
+
+/*
  * hstu_selftest_bounded_wait -- checks, on the device, the bounded wait that every pipelined kernel
  * of this library uses on its mbarriers.
  *
