@@ -522,6 +522,103 @@ def candidate_cpu_baseline(args):
 
 
 # ------------------------------------------------------------------------------------------------
+# Stochastic Length (--stochastic-length ALPHA): a step shortens the workload's batch on the device
+# (cut decisions and new offsets, per-sequence selection) and gathers the shortened batch's X rows
+# and timestamps, the new token count read on the device.
+# ------------------------------------------------------------------------------------------------
+
+SL_METRIC = "Stochastic Length subsampling throughput (input tokens, incl. the gather of X and timestamps)"
+
+
+def run_stochastic_length(args, rank, world, local_rank):
+    import torch
+    import hstu_sequential_transduction_layer_b200 as hstu
+    from workloads.device import tensor
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workloads.WORKLOADS[args.workload]
+    inp = workloads.make_inputs(w)
+    if w.token_embed:
+        raise SystemExit("Stochastic Length is timed on workloads with explicit X")
+    alpha = args.stochastic_length
+    B, T, d = len(inp.lengths), inp.T, w.d_model
+    max_len = int(inp.lengths.max())
+    u, keys = workloads.draw_stochastic_length_randoms(inp.seq_offsets, seed=w.index)
+    off = tensor(inp.seq_offsets, "i64", dev)
+    u_d = torch.from_numpy(u).to(dev)
+    k_d = torch.from_numpy(keys.view(np.int32)).to(dev)
+    X = tensor(inp.X, "bf16", dev)
+    ts = tensor(inp.timestamps, "i64", dev)
+    new_off = torch.empty(B + 1, dtype=torch.int64, device=dev)
+    index = torch.empty(T, dtype=torch.int64, device=dev)
+    Xn = torch.empty_like(X)
+    tsn = torch.empty_like(ts) if ts is not None else None
+    ws = torch.empty(max(256, int(hstu.library().hstu_stochastic_length_workspace_size(B))),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        hstu.hstu_stochastic_length(off, max_len, alpha, u_d, k_d, new_off, index, ws, stream)
+        if evs:
+            evs[1].record(stream)
+        hstu.hstu_gather_rows(index, X, Xn, row_count=new_off[B:], stream=stream)
+        if tsn is not None:
+            hstu.hstu_gather_rows(index, ts, tsn, row_count=new_off[B:], stream=stream)
+        if evs:
+            evs[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if hstu.device_status() != hstu.HSTU_OK:
+        raise SystemExit("device status error during warm-up")
+    T_new = int(new_off[B].item())
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    torch.cuda.synchronize()
+    sampler.start()
+    launches0 = hstu.launch_count()
+    for k in range(args.steps):
+        flush.zero_()
+        step(evs[k])
+    torch.cuda.synchronize()
+    launches = hstu.launch_count() - launches0
+    clocks = sampler.stop()
+    per = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2])] for e in evs])
+    total_ms, job_tokens = combine_over_ranks(float(per.sum()), T, world, dev)
+    ms = total_ms / args.steps
+    sel_ms, gat_ms = per.mean(axis=0)
+    peaks, peaks_src = load_peaks()
+    # algorithmic bytes: the selection reads offsets, draws and the cut sequences' keys (four
+    # passes of the radix select and one of the compaction) and writes the index; the gather reads
+    # the index and the kept rows and writes them
+    cut_tokens = int(sum(n for n, m in zip(inp.lengths, np.diff(new_off.cpu().numpy())) if m < n))
+    sel_bytes = 8.0 * (B + 1) * 2 + 8.0 * B + 4.0 * 5 * cut_tokens + 8.0 * T_new
+    row_bytes = 2 * d + (8 if tsn is not None else 0)
+    gat_bytes = 8.0 * T_new * (2 if tsn is not None else 1) + 2.0 * row_bytes * T_new
+    gbs = gat_bytes / gat_ms / 1e6
+    return {
+        "metric": SL_METRIC, "value": round(job_tokens / (ms * 1e-3), 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u32/i64/bf16 rows",
+        "data": "synthetic (seeded lengths, draws and rows of the workload)",
+        "config": {"workload": f"{w.name}: B={B}, T={T}, N_c={max_len}, alpha={alpha}, d={d}",
+                   "tokens_kept": T_new, "l2": "flushed between timed steps (outside the events)"},
+        "roofline": {"bound": "hbm", "kernel": "gather_rows", "achieved": round(gbs, 1),
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                     "traffic": None, "peak_source": f"{peaks_src} copy (MEASURED_PEAKS.json)"},
+        "kernels": {"plan_and_select": {"ms": round(float(sel_ms), 4),
+                                        "GB/s": round(sel_bytes / sel_ms / 1e6, 1)},
+                    "gather": {"ms": round(float(gat_ms), 4), "GB/s": round(gbs, 1)}},
+        "gpu_launches": int(launches), "clocks": clocks,
+    }
+
+
+# ------------------------------------------------------------------------------------------------
 # The oracle on the host cores (cpu_baseline of our arm, and the whole reference arm)
 # ------------------------------------------------------------------------------------------------
 
@@ -591,6 +688,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long_seq", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--stochastic-length", type=float, default=0.0,
+                    help="time Stochastic Length subsampling with this alpha instead")
     ap.add_argument("--candidates", type=int, default=0,
                     help="time M-FALCON scoring of this many candidates per user instead")
     args = ap.parse_args()
@@ -612,6 +711,11 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
+        if args.stochastic_length > 0:
+            res = run_stochastic_length(args, rank, world, local_rank)
+            if rank == 0:
+                print(json.dumps(res), flush=True)
+            return
         if args.candidates > 0:
             res = run_candidates(args, rank, world, local_rank)
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
