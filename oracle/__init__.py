@@ -67,6 +67,9 @@ def bind(path: str):
     lib.oracle_candidate_attention.argtypes = [i64, ip, ip, i32, i32, i32, dp, ip, dp, ip, dp, i32,
                                                dp, i32, dp, f64, dp]
     lib.oracle_candidate_attention.restype = None
+    lib.oracle_attention_bwd.argtypes = [i64, ip, i32, i32, i32, dp, ip, dp, i32, dp, i32, dp, f64,
+                                         dp, dp, dp, dp, dp, dp]
+    lib.oracle_attention_bwd.restype = None
     lib.oracle_stochastic_length.argtypes = [i64, ip, i64, f64, dp, ip, ip, ip]
     lib.oracle_stochastic_length.restype = i64
     lib.oracle_ln_gate.argtypes = [i64, i32, i32, i32, dp, dp, dp, dp, f64, dp]
@@ -283,6 +286,25 @@ def candidate_layer_fwd(hist_offsets, uvqk_hist, cand_offsets, X_cand, W1, b1, W
                              time_table=time_table, alibi_slopes=alibi_slopes, scale=scale)
     g = ln_gate(av, uc, ln_w, ln_b, num_heads=num_heads, d_qk=d_qk, d_v=d_v, ln_eps=ln_eps)
     return f2(g, W2, b2, X_cand)
+
+
+def attention_bwd(seq_offsets, uvqk, dav, *, num_heads: int, d_qk: int, d_v: int, timestamps=None,
+                  pos_table=None, time_table=None, alibi_slopes=None, scale: float, lib=None):
+    """Backward of Eq. 2: -> dict of dq, dk, dv [T, H*hd] and dpos [H, P], dtime [H, Tb] (or None)."""
+    off, uvqk, dav = _i(seq_offsets), _d(uvqk), _d(dav)
+    T = uvqk.shape[0]
+    ts, pos, tim, ali = _i(timestamps), _d(pos_table), _d(time_table), _d(alibi_slopes)
+    P = 0 if pos is None else pos.shape[1]
+    Tb = 0 if tim is None else tim.shape[1]
+    dq = np.empty((T, num_heads * d_qk))
+    dk = np.empty((T, num_heads * d_qk))
+    dv = np.empty((T, num_heads * d_v))
+    dpos = None if pos is None else np.empty((num_heads, P))
+    dtime = None if tim is None else np.empty((num_heads, Tb))
+    _load(lib).oracle_attention_bwd(len(off) - 1, _p(off), num_heads, d_qk, d_v, _p(uvqk), _p(ts),
+                                    _p(pos), P, _p(tim), Tb, _p(ali), float(scale), _p(dav),
+                                    _p(dq), _p(dk), _p(dv), _p(dpos), _p(dtime))
+    return {"dq": dq, "dk": dk, "dv": dv, "dpos": dpos, "dtime": dtime}
 
 
 def stochastic_length(seq_offsets, max_len: int, alpha: float, u, keys, lib=None):

@@ -143,6 +143,70 @@ void oracle_attention(int64_t B, const int64_t* seq_offsets, int32_t H, int32_t 
 }
 
 /* ---------------------------------------------------------------------------------------------
+ * Backward of Eq. 2 (training; "Actions Speak Louder than Words" paper notes, sections 3.4-3.5 and
+ * the training-speed figures of section 4): given dAV = dL/dAV, with x_ij = q_i . k_j + bias(i, j)
+ * and a_ij = scale * SiLU(x_ij) for j <= i (per head),
+ *   dv_j   = sum_{i >= j} a_ij dAV_i
+ *   dx_ij  = scale * SiLU'(x_ij) * (dAV_i . v_j),  SiLU'(x) = s(x) (1 + x (1 - s(x))), s = sigmoid
+ *   dq_i   = sum_{j <= i} dx_ij k_j,   dk_j = sum_{i >= j} dx_ij q_i
+ *   dpos[h][p] = sum of dx_ij over the pairs whose position bucket is p; dtime likewise.
+ * ALiBi slopes are fixed hyperparameters: no gradient.  Outputs are [T, H*hd] (dq, dk, dv) and the
+ * table shapes, fully overwritten.
+ * --------------------------------------------------------------------------------------------- */
+static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+void oracle_attention_bwd(int64_t B, const int64_t* seq_offsets, int32_t H, int32_t dqk, int32_t dv,
+                          const double* uvqk, const int64_t* timestamps, const double* pos_table,
+                          int32_t P, const double* time_table, int32_t Tb,
+                          const double* alibi_slopes, double scale, const double* dav, double* dq,
+                          double* dk, double* dvv, double* dpos, double* dtime) {
+  const int32_t n1 = 2 * H * dv + 2 * H * dqk;
+  const int32_t offV = H * dv, offQ = 2 * H * dv, offK = 2 * H * dv + H * dqk;
+  const int64_t T = seq_offsets[B];
+  memset(dq, 0, sizeof(double) * (size_t)T * H * dqk);
+  memset(dk, 0, sizeof(double) * (size_t)T * H * dqk);
+  memset(dvv, 0, sizeof(double) * (size_t)T * H * dv);
+  if (dpos) memset(dpos, 0, sizeof(double) * (size_t)H * P);
+  if (dtime) memset(dtime, 0, sizeof(double) * (size_t)H * Tb);
+  /* one (sequence, head) at a time; its pairs touch only its rows and head columns */
+  for (int64_t s = 0; s < B; s++) {
+    const int64_t a0 = seq_offsets[s], n = seq_offsets[s + 1] - seq_offsets[s];
+    const double* u = uvqk + a0 * n1;
+    const int64_t* ts = timestamps ? timestamps + a0 : NULL;
+    for (int32_t h = 0; h < H; h++) {
+      for (int64_t i = 0; i < n; i++) {
+        const double* q = u + i * n1 + offQ + (int64_t)h * dqk;
+        const double* g = dav + (a0 + i) * (int64_t)H * dv + (int64_t)h * dv;
+        for (int64_t j = 0; j <= i; j++) {
+          const double* k = u + j * n1 + offK + (int64_t)h * dqk;
+          const double* v = u + j * n1 + offV + (int64_t)h * dv;
+          double x = 0.0, gv = 0.0;
+          for (int32_t c = 0; c < dqk; c++) x += q[c] * k[c];
+          x += bias_at(h, i, j, ts, pos_table, P, time_table, Tb, alibi_slopes);
+          for (int32_t c = 0; c < dv; c++) gv += g[c] * v[c];
+          const double sg = sigmoid(x);
+          const double a = scale * x * sg;
+          const double dx = scale * sg * (1.0 + x * (1.0 - sg)) * gv;
+          double* dvj = dvv + (a0 + j) * (int64_t)H * dv + (int64_t)h * dv;
+          for (int32_t c = 0; c < dv; c++) dvj[c] += a * g[c];
+          double* dqi = dq + (a0 + i) * (int64_t)H * dqk + (int64_t)h * dqk;
+          double* dkj = dk + (a0 + j) * (int64_t)H * dqk + (int64_t)h * dqk;
+          for (int32_t c = 0; c < dqk; c++) {
+            dqi[c] += dx * k[c];
+            dkj[c] += dx * q[c];
+          }
+          if (!alibi_slopes) {
+            if (pos_table && dpos) dpos[(int64_t)h * P + oracle_pos_bucket(i, j, P)] += dx;
+            if (time_table && dtime)
+              dtime[(int64_t)h * Tb + oracle_time_bucket(ts[i], ts[j], Tb)] += dx;
+          }
+        }
+      }
+    }
+  }
+}
+
+/* ---------------------------------------------------------------------------------------------
  * M-FALCON candidate scoring ("Actions Speak Louder than Words" paper notes, section 3.6; the
  * efficiency paragraph of "4.4 推荐模型的 Scaling"): m candidates are appended after a user's n
  * history tokens and scored in one pass; the attention mask lets each candidate see the history

@@ -86,6 +86,51 @@ def _sl_pins_pass(lib) -> bool:
     return abs(cut - p) < 4 * np.sqrt(p * (1 - p) / trials)
 
 
+# planted in the attention backward: caught by finite differences of the forward
+BWD_MUTANTS = {
+    "bwd_silu_derivative": ("sg * (1.0 + x * (1.0 - sg)) * gv", "sg * (1.0 + x * sg) * gv"),
+    "bwd_dk_from_k": ("dkj[c] += dx * q[c];", "dkj[c] += dx * k[c];"),
+    "bwd_dv_unscaled": ("const double a = scale * x * sg;", "const double a = x * sg;"),
+    "bwd_time_bucket_of_key": ("oracle_time_bucket(ts[i], ts[j], Tb)] += dx;", "oracle_time_bucket(ts[j], ts[i], Tb)] += dx;"),
+}
+
+
+def _bwd_pins_pass(lib) -> bool:
+    """Backward of Eq. 2 from `lib` against central differences of the (unmodified) forward."""
+    rng = np.random.default_rng(4)
+    H, hd = 2, 4
+    n1 = 4 * H * hd
+    off = np.array([0, 4, 11], np.int64)
+    uvqk = rng.normal(0, 0.6, (11, n1))
+    dav = rng.normal(0, 1.0, (11, H * hd))
+    ts = np.concatenate([np.cumsum(rng.integers(0, 9, 4)), np.cumsum(rng.integers(0, 9, 7))]).astype(np.int64)
+    kw = dict(num_heads=H, d_qk=hd, d_v=hd, timestamps=ts, pos_table=rng.normal(0, 0.3, (H, 6)),
+              time_table=rng.normal(0, 0.3, (H, 4)), scale=0.7)
+    got = oracle.attention_bwd(off, uvqk, dav, lib=lib, **kw)
+    eps = 1e-6
+
+    def loss():
+        return float(np.sum(dav * oracle.attention(off, uvqk, **kw)))
+
+    for arr, key, sl in ((uvqk, "dv", slice(H * hd, 2 * H * hd)), (uvqk, "dq", slice(2 * H * hd, 3 * H * hd)),
+                         (uvqk, "dk", slice(3 * H * hd, 4 * H * hd)), (kw["time_table"], "dtime", None)):
+        g = np.zeros_like(arr)
+        for idx in np.ndindex(*arr.shape):
+            if sl is not None and not (sl.start <= idx[1] < sl.stop):
+                continue
+            old = arr[idx]
+            arr[idx] = old + eps
+            fp = loss()
+            arr[idx] = old - eps
+            fm = loss()
+            arr[idx] = old
+            g[idx] = (fp - fm) / (2 * eps)
+        ref = g[:, sl] if sl is not None else g
+        if not np.allclose(got[key], ref, rtol=1e-6, atol=1e-8):
+            return False
+    return True
+
+
 def _silu(x):
     return x / (1.0 + np.exp(-x))
 
@@ -185,6 +230,16 @@ def test_unmodified_oracle_passes_the_independent_pins(tmp_path):
     assert _pins_pass(lib)
     assert _candidate_pins_pass(lib)
     assert _sl_pins_pass(lib)
+    assert _bwd_pins_pass(lib)
+
+
+@pytest.mark.parametrize("name", sorted(BWD_MUTANTS))
+def test_planted_backward_mistake_is_caught(name, tmp_path):
+    src = open(SRC).read()
+    old, new = BWD_MUTANTS[name]
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    lib = _compile(src.replace(old, new), tmp_path, name)
+    assert not _bwd_pins_pass(lib), f"planted mistake {name} went unnoticed"
 
 
 @pytest.mark.parametrize("name", sorted(SL_MUTANTS))
