@@ -32,7 +32,8 @@ EXPORTED = ["hstu_layer_fwd", "hstu_layer_fwd_workspace_size", "hstu_f1_fwd", "h
             "hstu_launch_count", "hstu_attention_fwd_noalloc", "hstu_selftest_bounded_wait",
             "hstu_candidate_workspace_size", "hstu_candidate_attention_fwd",
             "hstu_candidate_layer_workspace_size", "hstu_candidate_layer_fwd",
-            "hstu_stochastic_length_workspace_size", "hstu_stochastic_length", "hstu_gather_rows"]
+            "hstu_stochastic_length_workspace_size", "hstu_stochastic_length", "hstu_gather_rows",
+            "hstu_attention_bwd_workspace_size", "hstu_attention_bwd"]
 
 
 class HstuShape(ctypes.Structure):
@@ -83,6 +84,8 @@ def _load() -> ctypes.CDLL:
         "hstu_stochastic_length": ([I64, I64, P, I64, ctypes.c_double, P, P, P, P, P, S, P],
                                    ctypes.c_int),
         "hstu_gather_rows": ([I64, P, I64, P, P, I64, P, P], ctypes.c_int),
+        "hstu_attention_bwd_workspace_size": ([SH], S),
+        "hstu_attention_bwd": ([SH, P, P, P, P, P, P, F32, P, P, P, P, P, P, P, S, P], ctypes.c_int),
         "hstu_candidate_layer_fwd": ([SH, P, P, P, I64, I64, P, P, P, P, P, P, P, P, P, P, P, P, F32,
                                       P, P, S, P], ctypes.c_int),
     }
@@ -278,6 +281,21 @@ def hstu_candidate_layer_fwd(shape: HstuShape, uvqk_hist, hist_offsets, hist_tim
         _ptr(alibi_slopes), float(scale), _ptr(out_cand), _ptr(workspace), workspace.numel(),
         _stream(stream)), "hstu_candidate_layer_fwd")
     return out_cand
+
+
+def hstu_attention_bwd(shape: HstuShape, uvqk, seq_offsets, timestamps, pos_table, time_table,
+                       alibi_slopes, scale: float, dav, dq, dk, dv, dpos_table=None,
+                       dtime_table=None, workspace=None, stream=None):
+    """Backward of Eq. 2 (see the C header): fills dq, dk, dv and the table gradients."""
+    if workspace is None:
+        workspace = torch.empty(max(256, int(_lib.hstu_attention_bwd_workspace_size(ctypes.byref(shape)))),
+                                dtype=torch.uint8, device=uvqk.device)
+    _check(_lib.hstu_attention_bwd(ctypes.byref(shape), _ptr(uvqk), _ptr(seq_offsets), _ptr(timestamps),
+                                   _ptr(pos_table), _ptr(time_table), _ptr(alibi_slopes), float(scale),
+                                   _ptr(dav), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dpos_table),
+                                   _ptr(dtime_table), _ptr(workspace), workspace.numel(),
+                                   _stream(stream)), "hstu_attention_bwd")
+    return dq, dk, dv
 
 
 def hstu_stochastic_length(seq_offsets, max_len: int, alpha: float, u, keys, new_offsets, index,

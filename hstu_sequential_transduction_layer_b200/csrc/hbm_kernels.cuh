@@ -134,6 +134,12 @@ __global__ void __launch_bounds__(256) token_embed_kernel(int64_t T, int d,
   __stcs(reinterpret_cast<uint4*>(X + t * d) + c, out);
 }
 
+// out[0 .. n) = 0 (fp32 accumulators of the backward pass).
+__global__ void __launch_bounds__(256) zero_f32_kernel(float* __restrict__ out, int64_t n) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = 0.0f;
+}
+
 // Device-side check of the jagged offsets: off[0] == 0, non-decreasing, off[B] == T.
 __global__ void check_offsets_kernel(const int64_t* __restrict__ off, int64_t B, int64_t T) {
   const int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;

@@ -542,6 +542,56 @@ hstu_status_t hstu_candidate_layer_fwd(const hstu_shape_t* shape, const void* uv
   return run_f2(c, w.g, W2, b2, X_cand, out_cand, st);
 }
 
+size_t hstu_attention_bwd_workspace_size(const hstu_shape_t* shape) {
+  if (check_shape(shape) != HSTU_OK) return 0;
+  return tc::attention_bwd_workspace_bytes(shape->total_tokens, shape->num_seqs, shape->num_heads);
+}
+
+hstu_status_t hstu_attention_bwd(const hstu_shape_t* shape, const void* uvqk,
+                                 const int64_t* seq_offsets, const int64_t* timestamps,
+                                 const float* pos_table, const float* time_table,
+                                 const float* alibi_slopes, float scale, const void* dav, float* dq,
+                                 float* dk, float* dv, float* dpos_table, float* dtime_table,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  hstu_status_t rc = check_shape(shape);
+  if (rc != HSTU_OK) return rc;
+  const hstu_shape_t& s = *shape;
+  if (s.dtype != HSTU_BF16 || s.d_qk != 64 || s.d_v != 64) return HSTU_ERR_UNSUPPORTED;
+  if (s.num_seqs * (int64_t)s.num_heads >= (1LL << 31)) return HSTU_ERR_UNSUPPORTED;
+  if ((rc = check_bias(shape, timestamps, pos_table, time_table, alibi_slopes, scale)) != HSTU_OK)
+    return rc;
+  if ((pos_table && !dpos_table) || (time_table && !dtime_table)) return HSTU_ERR_INVALID_ARG;
+  const int64_t T = s.total_tokens, B = s.num_seqs;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  auto zero = [&](float* p, int64_t n) {
+    if (!p || n <= 0) return HSTU_OK;
+    zero_f32_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p, n);
+    return launch_status();
+  };
+  const int64_t w = (int64_t)s.num_heads * 64;
+  if (pos_table && (rc = zero(dpos_table, (int64_t)s.num_heads * s.n_pos_buckets)) != HSTU_OK) return rc;
+  if (time_table && (rc = zero(dtime_table, (int64_t)s.num_heads * s.n_time_buckets)) != HSTU_OK)
+    return rc;
+  if (T == 0) return HSTU_OK;
+  if (B == 0 || !uvqk || !seq_offsets || !dav || !dq || !dk || !dv || !workspace)
+    return HSTU_ERR_INVALID_ARG;
+  if (!(aligned16(uvqk) && aligned16(dav) && aligned16(dq) && aligned16(dk) && aligned16(dv)))
+    return HSTU_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) return HSTU_ERR_INVALID_ARG;
+  const size_t gb = (size_t)T * w * 4;
+  if (overlaps(dq, gb, dk, gb) || overlaps(dq, gb, dv, gb) || overlaps(dk, gb, dv, gb) ||
+      overlaps(dq, gb, workspace, workspace_bytes) || overlaps(dk, gb, workspace, workspace_bytes) ||
+      overlaps(dv, gb, workspace, workspace_bytes))
+    return HSTU_ERR_INVALID_ARG;
+  if ((rc = zero(dq, T * w)) != HSTU_OK) return rc;
+  check_offsets_kernel<<<(unsigned)((B + 1 + 255) / 256), 256, 0, st>>>(seq_offsets, B, T);
+  if (launch_status() != HSTU_OK) return HSTU_ERR_CUDA;
+  return tc::launch_attention_bwd(T, B, s.num_heads, s.max_seq_len, (const bf16*)uvqk, seq_offsets,
+                                  timestamps, pos_table, s.n_pos_buckets, time_table,
+                                  s.n_time_buckets, alibi_slopes, scale, (const bf16*)dav, dq, dk,
+                                  dv, dpos_table, dtime_table, workspace, workspace_bytes, st);
+}
+
 size_t hstu_stochastic_length_workspace_size(int64_t num_seqs) {
   return num_seqs < 0 ? 0 : align_up((size_t)num_seqs * sizeof(int32_t) + 1);
 }

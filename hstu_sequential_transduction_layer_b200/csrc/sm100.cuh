@@ -190,6 +190,19 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
       : "memory");
 }
 
+// Makes this thread's generic-proxy shared-memory writes visible to the async proxy (tcgen05.mma
+// operands read through shared-memory descriptors, TMA stores).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 16-byte vector reduction (add) of four fp32 values into global memory.
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
 // tanh via the MUFU approximation (max relative error about 2^-11).
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;

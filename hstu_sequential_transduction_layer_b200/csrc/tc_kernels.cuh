@@ -7,6 +7,7 @@
 #include <mutex>
 
 #include "tc_attention.cuh"
+#include "tc_attention_bwd.cuh"
 #include "tc_gemm.cuh"
 
 namespace hstu {
@@ -180,6 +181,66 @@ inline hstu_status_t launch_attention(int64_t T, int64_t B, int H, int hd, int64
   if (bias == BIAS_RAB) return launch_attention_kernel<128, BIAS_RAB>(tm, tm, prm, sch, grid, st);
   if (bias == BIAS_ALIBI) return launch_attention_kernel<128, BIAS_ALIBI>(tm, tm, prm, sch, grid, st);
   return launch_attention_kernel<128, BIAS_NONE>(tm, tm, prm, sch, grid, st);
+}
+
+// Attention backward workspace: header (256 B), per-sequence (start, length), then one entry per
+// (sequence, key tile, head): at most H * (ceil(T/128) + B).
+inline int64_t attention_bwd_capacity(int64_t T, int64_t B, int H) {
+  return (int64_t)H * ((T + ATT_BN - 1) / ATT_BN + B);
+}
+
+inline size_t attention_bwd_workspace_bytes(int64_t T, int64_t B, int H) {
+  return (size_t)(256 + ((16 * B + 255) / 256) * 256 + 8 * attention_bwd_capacity(T, B, H));
+}
+
+// Backward of Eq. 2 (head dim 64): dq, dpos and dtime are accumulated and must be zero on entry.
+inline hstu_status_t launch_attention_bwd(int64_t T, int64_t B, int H, int64_t max_seq_len,
+                                          const bf16* uvqk, const int64_t* off, const int64_t* ts,
+                                          const float* pos, int P, const float* tim, int Tb,
+                                          const float* alibi, float scale, const bf16* dav, float* dq,
+                                          float* dk, float* dv, float* dpos, float* dtime, void* ws,
+                                          size_t ws_bytes, cudaStream_t st) {
+  if (T >= (1LL << 31) || H >= (1 << 15)) return HSTU_ERR_UNSUPPORTED;
+  if (ws_bytes < attention_bwd_workspace_bytes(T, B, H)) return HSTU_ERR_INVALID_ARG;
+  const int64_t max_tiles64 = ((max_seq_len > 0 ? max_seq_len : T) + ATT_BN - 1) / ATT_BN;
+  if (max_tiles64 > 12288) return HSTU_ERR_UNSUPPORTED;
+  const int max_tiles = (int)max_tiles64;
+  const AttnSchedule sch = attention_schedule_view(ws, B);
+  const size_t sched_smem = 2 * (size_t)(max_tiles + 2) * sizeof(unsigned long long);
+  if (sched_smem > 48 * 1024 &&
+      cudaFuncSetAttribute(bwd_schedule_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)sched_smem) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  const int64_t capacity = attention_bwd_capacity(T, B, H);
+  bwd_schedule_kernel<<<1, 1024, sched_smem, st>>>(off, B, T, H, max_tiles, capacity, sch);
+  count_launch();
+  if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+  const int n1 = 4 * H * 64;
+  CUtensorMap tm, tdo;
+  if (!make_map_bf16(&tm, uvqk, n1, T, n1, 64, 128)) return HSTU_ERR_CUDA;
+  if (!make_map_bf16(&tdo, dav, (uint64_t)H * 64, T, (uint64_t)H * 64, 64, 128)) return HSTU_ERR_CUDA;
+  BwdParams prm;
+  prm.ts = ts;
+  prm.pos = pos;
+  prm.tim = tim;
+  prm.alibi = alibi;
+  prm.P = P;
+  prm.Tb = Tb;
+  prm.H = H;
+  prm.n1 = n1;
+  prm.scale = scale;
+  prm.dq = dq;
+  prm.dk = dk;
+  prm.dv = dv;
+  prm.dpos = dpos;
+  prm.dtime = dtime;
+  if (cudaFuncSetAttribute(attention_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           BwdCfg::SMEM) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  const int grid = (int)(capacity < num_sms() ? capacity : num_sms());
+  attention_bwd_kernel<<<grid, BWD_THREADS, BwdCfg::SMEM, st>>>(tm, tdo, prm, sch);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
 
 // M-FALCON candidate attention workspace: header (256 B), per-user (candidate start, count,

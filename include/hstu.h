@@ -161,6 +161,28 @@ hstu_status_t hstu_f2_fwd(const hstu_shape_t* shape, const void* g, const void* 
                           const void* X, void* out, void* stream);
 
 /*
+ * hstu_attention_bwd -- backward of Eq. 2 (training): given dAV = dL/dAV, the gradients of the
+ * loss with respect to Q, K, V and the rab tables.  With x_ij = q_i . k_j + bias(i, j),
+ *   dv_j = sum_{i>=j} scale*SiLU(x_ij) dAV_i,   dx_ij = scale*SiLU'(x_ij) (dAV_i . v_j),
+ *   dq_i = sum_{j<=i} dx_ij k_j,   dk_j = sum_{i>=j} dx_ij q_i,
+ *   dpos[h][p], dtime[h][b] = sums of dx_ij over the pairs in bucket p, b (ALiBi slopes: none).
+ * bf16 with d_qk = d_v = 64 (else HSTU_ERR_UNSUPPORTED); the forward's arguments, plus
+ *  dav            [T, H*64] bf16, the incoming gradient
+ *  dq, dk, dv     [T, H*64] fp32 outputs (16-byte aligned, not overlapping)
+ *  dpos_table     [H, P] fp32 output, required when pos_table is given (else ignored)
+ *  dtime_table    [H, Tb] fp32 output, required when time_table is given (else ignored)
+ *  workspace      hstu_attention_bwd_workspace_size(shape) bytes, 256-byte aligned
+ * All outputs are overwritten.  Asynchronous on `stream`.
+ */
+size_t hstu_attention_bwd_workspace_size(const hstu_shape_t* shape);
+hstu_status_t hstu_attention_bwd(const hstu_shape_t* shape, const void* uvqk,
+                                 const int64_t* seq_offsets, const int64_t* timestamps,
+                                 const float* pos_table, const float* time_table,
+                                 const float* alibi_slopes, float scale, const void* dav, float* dq,
+                                 float* dk, float* dv, float* dpos_table, float* dtime_table,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * M-FALCON candidate scoring ("Actions Speak Louder than Words" paper notes, section 3.6; the
  * efficiency paragraph of "4.4 推荐模型的 Scaling").  A user's m candidates are scored in one pass
  * after its n history tokens: each candidate attends to the whole history and to itself, never to
