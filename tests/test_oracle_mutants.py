@@ -21,7 +21,8 @@ SRC = os.path.join(os.path.dirname(oracle.__file__), "hstu_oracle.c")
 MUTANTS = {
     "silu_sign": ("return x / (1.0 + exp(-x));", "return x / (1.0 + exp(x));"),
     "bias_dropped": ("s += bias_at(", "s += 0.0 * bias_at("),
-    "diagonal_excluded": ("for (int64_t j = 0; j <= i; j++) {", "for (int64_t j = 0; j < i; j++) {"),
+    "diagonal_excluded": ("(int64_t)h * dqk;\n    for (int64_t j = 0; j <= i; j++) {",
+                          "(int64_t)h * dqk;\n    for (int64_t j = 0; j < i; j++) {"),
     "q_k_swapped": ("const double* q = uvqk_seq + i * n1 + offQ", "const double* q = uvqk_seq + i * n1 + offK"),
     "u_is_v": ("uvqk + t * n1 /* U is block 0 */", "uvqk + t * n1 + H * dv"),
     "pos_direction": ("int64_t p = i - j;", "int64_t p = j - i;"),
