@@ -522,6 +522,89 @@ def candidate_cpu_baseline(args):
 
 
 # ------------------------------------------------------------------------------------------------
+# Attention backward (--backward): dQ, dK, dV and the rab-table gradients for the workload's
+# attention given a seeded dAV; the layer's UVQK is computed once before the timed region.
+# ------------------------------------------------------------------------------------------------
+
+BWD_METRIC = "HSTU attention backward throughput (dQ, dK, dV and rab-table gradients)"
+
+
+def run_backward(args, rank, world, local_rank):
+    import torch
+    import hstu_sequential_transduction_layer_b200 as hstu
+    from workloads.device import to_device, tensor
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workloads.WORKLOADS[args.workload]
+    if w.head_dim != 64 or w.token_embed:
+        raise SystemExit("the attention backward is implemented for head dim 64 (long_seq, retrieval)")
+    inp = workloads.make_inputs(w)
+    H, hd, d, T = w.num_heads, w.head_dim, w.d_model, inp.T
+    D = to_device(inp, dev)
+    L = D["layers"][0]
+    shape = hstu.shape_for(D["X"], D["off"], H, hd, hd, int(inp.lengths.max()), D["pos"], D["tim"],
+                           inp.ln_eps)
+    uvqk = torch.empty((T, 4 * H * hd), dtype=torch.bfloat16, device=dev)
+    hstu.hstu_f1_fwd(shape, D["X"], L["W1"], L["b1"], uvqk)
+    rng = np.random.default_rng(w.index + 500)
+    dav = tensor(rng.standard_normal((T, H * hd), dtype=np.float32), "bf16", dev)
+    dq, dk, dv = (torch.empty((T, H * hd), dtype=torch.float32, device=dev) for _ in range(3))
+    dpos = torch.empty_like(D["pos"]) if D["pos"] is not None else None
+    dtim = torch.empty_like(D["tim"]) if D["tim"] is not None else None
+    ws = torch.empty(max(256, int(hstu.library().hstu_attention_bwd_workspace_size(shape))),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        hstu.hstu_attention_bwd(shape, uvqk, D["off"], D["ts"], D["pos"], D["tim"], D["ali"],
+                                inp.scale, dav, dq, dk, dv, dpos, dtim, ws, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if hstu.device_status() != hstu.HSTU_OK:
+        raise SystemExit("device status error during warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    torch.cuda.synchronize()
+    sampler.start()
+    launches0 = hstu.launch_count()
+    for k in range(args.steps):
+        flush.zero_()
+        evs[k][0].record(stream)
+        step()
+        evs[k][1].record(stream)
+    torch.cuda.synchronize()
+    launches = hstu.launch_count() - launches0
+    clocks = sampler.stop()
+    total_ms, job_tokens = combine_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evs), T, world, dev)
+    if hstu.device_status() != hstu.HSTU_OK:
+        raise SystemExit("device status error in the timed region")
+    ms = total_ms / args.steps
+    peaks, peaks_src = load_peaks()
+    tpk = peaks["bf16_tflops"]
+    # five products per causal pair and head: S, dP, dV, dK, dQ, 2*hd FLOP each
+    pairs = float(np.sum(inp.lengths * (inp.lengths + 1) // 2))
+    fl = 2.0 * H * 5 * hd * pairs
+    tf = fl / ms / 1e9
+    return {
+        "metric": BWD_METRIC, "value": round(job_tokens / (ms * 1e-3), 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded inputs of the workload, N(0,1) incoming gradient)",
+        "config": {"workload": f"{w.name}: B={len(inp.lengths)}, n={int(inp.lengths.max())}, "
+                               f"H={H}x{hd}, rab P={w.n_pos_buckets}/Tb={w.n_time_buckets}",
+                   "l2": "flushed between timed steps (outside the events)"},
+        "roofline": {"bound": "tensor", "kernel": "attention_bwd", "achieved": round(tf, 2),
+                     "peak": tpk, "unit": "TFLOP/s", "frac": round(tf / tpk, 4), "traffic": None,
+                     "peak_source": f"{peaks_src} bf16 burst (MEASURED_PEAKS.json)"},
+        "gpu_launches": int(launches), "clocks": clocks,
+    }
+
+
+# ------------------------------------------------------------------------------------------------
 # Stochastic Length (--stochastic-length ALPHA): a step shortens the workload's batch on the device
 # (cut decisions and new offsets, per-sequence selection) and gathers the shortened batch's X rows
 # and timestamps, the new token count read on the device.
@@ -688,6 +771,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long_seq", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the attention backward instead")
     ap.add_argument("--stochastic-length", type=float, default=0.0,
                     help="time Stochastic Length subsampling with this alpha instead")
     ap.add_argument("--candidates", type=int, default=0,
@@ -711,6 +796,11 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
+        if args.backward:
+            res = run_backward(args, rank, world, local_rank)
+            if rank == 0:
+                print(json.dumps(res), flush=True)
+            return
         if args.stochastic_length > 0:
             res = run_stochastic_length(args, rank, world, local_rank)
             if rank == 0:

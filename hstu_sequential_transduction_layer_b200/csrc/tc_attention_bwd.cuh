@@ -12,28 +12,33 @@
 //   pointwise: P^T = scale*SiLU(S^T + bias^T), dS^T = scale*SiLU'(.) * dP^T, masked to j <= i
 //   dV_j += P^T dAV_i,  dK_j += dS^T Q_i                   (P^T, dS^T read from TMEM)
 //   dQ_i partial = dS K_j                                  (dS from shared memory, MN-major A)
-// and the dQ partial is added to global dQ (fp32) with 16-byte vector reductions.  The position and
-// time table gradients collect dx in shared memory (one atomic add per score for the position
-// bucket, one per run of equal time buckets along a row) and are flushed to global memory per item.
+// and the dQ partial is added to global dQ (fp32) with 16-byte vector reductions.  Table gradients:
+// each pointwise warp writes its 32 x 32 block of dx skewed into shared memory (row r, column
+// (c - r) mod 32), so that every column holds two diagonals, whose sums (one bucket each, all
+// distances along a diagonal being equal) go to the global position gradient with one reduction
+// per diagonal; the time-bucket gradient accumulates per row and chunk in two registers (the
+// chunk's first bucket and the next one), in shared memory per item, then to global memory.
 // dV and dK are owned by the item and stored directly.
 //
-// Per CTA (384 threads, one per SM): warp 0 producer (TMA of K_j, V_j, and Q_i, dAV_i per query tile
-// into a 2-deep ring; key and query timestamps), warp 1 single-thread MMA issuer, warps 2-3 idle,
-// warps 4-11 pointwise (two per TMEM lane quadrant, each on 64 of the 128 query columns).
+// Per CTA (320 threads, one per SM): warp 0 producer (TMA of K_j, V_j, and Q_i, dAV_i per query tile
+// into a 2-deep ring; key and query timestamps), warp 1 single-thread MMA issuer, warps 2-9
+// pointwise (two per TMEM lane quadrant, each on 64 of the 128 query columns).
 // TMEM: S^T [0,128) | dP^T [128,256) | dV [256,320) | dK [320,384) | dQ partial [384,448); P^T and
 // dS^T (bf16) overwrite the S^T / dP^T columns each warp has read (a warp's 64 queries pack into 32
 // columns at the start of its own 64).
 #pragma once
+
+#include <type_traits>
 
 #include "tc_attention.cuh"
 
 namespace hstu {
 namespace tc {
 
-constexpr int BWD_THREADS = 384;
+constexpr int BWD_THREADS = 320;
 constexpr int BWD_PW = 256;          // pointwise threads
 constexpr int BWD_PW_WARPS = 8;
-constexpr int BWD_POS_CAP = 8192;    // position buckets staged (and accumulated) in shared memory
+constexpr int BWD_POS_CAP = 8192;    // position buckets staged in shared memory
 constexpr int BWD_TB_CAP = 256;
 
 struct BwdCfg {
@@ -46,9 +51,12 @@ struct BwdCfg {
   static constexpr int OFF_DS = OFF_DO + NST * BOX;         // dS^T, two 16 KB panels (MN-major A)
   static constexpr int OFF_QTS = OFF_DS + 2 * BOX;          // [NST][128] int64 query timestamps
   static constexpr int OFF_KTS = OFF_QTS + NST * 128 * 8;   // [128] int64 key timestamps
-  static constexpr int OFF_POS = OFF_KTS + 128 * 8;         // [POS_CAP] float position table
-  static constexpr int OFF_DPOS = OFF_POS + BWD_POS_CAP * 4;  // [POS_CAP] float its gradient
-  static constexpr int OFF_TT = OFF_DPOS + BWD_POS_CAP * 4;   // [TB_CAP] float time table
+  static constexpr int OFF_QTS32 = OFF_KTS + 128 * 8;       // [NST][128] int32, relative
+  static constexpr int OFF_KTS32 = OFF_QTS32 + NST * 128 * 4;  // [128] int32, relative
+  static constexpr int OFF_TFLAG = OFF_KTS32 + 128 * 4;     // [NST] query fits, [NST] key fits
+  static constexpr int OFF_XP = OFF_TFLAG + 64;             // [8 warps][32][32] float: dx blocks
+  static constexpr int OFF_POS = OFF_XP + BWD_PW_WARPS * 32 * 32 * 4;  // [POS_CAP] float pos table
+  static constexpr int OFF_TT = OFF_POS + BWD_POS_CAP * 4;    // [TB_CAP] float time table
   static constexpr int OFF_DTT = OFF_TT + BWD_TB_CAP * 4;     // [TB_CAP] float its gradient
   static constexpr int OFF_BAR = OFF_DTT + BWD_TB_CAP * 4;
   static constexpr int SMEM = OFF_BAR + 256;
@@ -132,6 +140,10 @@ __device__ __forceinline__ void silu_and_grad(float x, float& silu, float& dsilu
   dsilu = sg * fmaf(x, 1.0f - sg, 1.0f);
 }
 
+// Bias modes of the backward kernel (compile-time): position table, time table, ALiBi.
+constexpr int BWD_POS = 1, BWD_TIME = 2, BWD_ALIBI = 4;
+
+template <int BM>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     attention_bwd_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tdo,
                          BwdParams prm, AttnSchedule sch) {
@@ -143,8 +155,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   uint8_t* ds_s = smem + Cfg::OFF_DS;
   int64_t* qts = reinterpret_cast<int64_t*>(smem + Cfg::OFF_QTS);
   int64_t* kts = reinterpret_cast<int64_t*>(smem + Cfg::OFF_KTS);
+  int* qts32 = reinterpret_cast<int*>(smem + Cfg::OFF_QTS32);
+  int* kts32 = reinterpret_cast<int*>(smem + Cfg::OFF_KTS32);
+  int* tflag = reinterpret_cast<int*>(smem + Cfg::OFF_TFLAG);   // [0]: keys fit; [1 + st]: queries
+  float* xp_s = reinterpret_cast<float*>(smem + Cfg::OFF_XP);
   float* pos_s = reinterpret_cast<float*>(smem + Cfg::OFF_POS);
-  float* dpos_s = reinterpret_cast<float*>(smem + Cfg::OFF_DPOS);
   float* tt_s = reinterpret_cast<float*>(smem + Cfg::OFF_TT);
   float* dtt_s = reinterpret_cast<float*>(smem + Cfg::OFF_DTT);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
@@ -166,8 +181,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int H = prm.H;
   const int col_v = H * 64, col_q = 2 * H * 64, col_k = 3 * H * 64;
-  const bool has_time = prm.tim != nullptr && prm.alibi == nullptr;
-  const bool has_pos = prm.pos != nullptr && prm.alibi == nullptr;
+  constexpr bool has_time = (BM & BWD_TIME) != 0;
+  constexpr bool has_pos = (BM & BWD_POS) != 0;
+  constexpr bool alibi = (BM & BWD_ALIBI) != 0;
   const bool aligned = (smem_u32(smem) & 1023u) == 0;
   const int64_t n_items = aligned ? sch.header[0] : 0;
 
@@ -192,7 +208,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     prefetch_tensormap(&tm);
     prefetch_tensormap(&tdo);
   }
-  for (int e = threadIdx.x; e < BWD_POS_CAP; e += BWD_THREADS) dpos_s[e] = 0.0f;
   for (int e = threadIdx.x; e < BWD_TB_CAP; e += BWD_THREADS) dtt_s[e] = 0.0f;
   if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
@@ -224,6 +239,17 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           const int64_t j = k0 + 4 * lane + e;
           kts[4 * lane + e] = prm.ts[row0 + (j < n ? j : n - 1)];
         }
+        // the same relative to the sequence's first timestamp, as int32 when every one fits
+        const int64_t t0 = prm.ts[row0];
+        bool fits = true;
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+          const int64_t rel = kts[4 * lane + e] - t0;
+          fits = fits && rel > -(1LL << 30) && rel < (1LL << 30);
+          kts32[4 * lane + e] = (int)rel;
+        }
+        fits = __all_sync(0xffffffffu, fits);
+        if (lane == 0) tflag[0] = fits ? 1 : 0;
       }
       __syncwarp();
       if (lane == 0) {
@@ -243,6 +269,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             const int64_t qi = (int64_t)i * ATT_BM + 4 * lane + e;
             qts[st * 128 + 4 * lane + e] = prm.ts[row0 + (qi < n ? qi : n - 1)];
           }
+          const int64_t t0 = prm.ts[row0];
+          bool fits = true;
+#pragma unroll
+          for (int e = 0; e < 4; e++) {
+            const int64_t rel = qts[st * 128 + 4 * lane + e] - t0;
+            fits = fits && rel > -(1LL << 30) && rel < (1LL << 30);
+            qts32[st * 128 + 4 * lane + e] = (int)rel;
+          }
+          fits = __all_sync(0xffffffffu, fits);
+          if (lane == 0) tflag[1 + st] = fits ? 1 : 0;
         }
         __syncwarp();
         if (lane == 0) {
@@ -332,13 +368,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       mbar_drain(drain, 0);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp >= 2) {
     // ------------------------------------------------------------------ pointwise warps
-    const int pw = warp - 4;
+    const int pw = warp - 2;
     const int half = pw >> 2;            // query columns [64 half, 64 half + 64)
     const int q = warp & 3;              // TMEM lane quadrant
     const int r = q * 32 + lane;         // key row of S^T / dP^T, query row of the dQ partial
-    const int tid = threadIdx.x - 128;
+    const int tid = threadIdx.x - 64;
     const int c0 = half * 64;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const int P = prm.P, Tb = prm.Tb;
@@ -357,7 +393,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const int k0 = jt * ATT_BN;
       const float* pos_h = has_pos ? prm.pos + (int64_t)h * P : nullptr;
       const float* tim_h = has_time ? prm.tim + (int64_t)h * Tb : nullptr;
-      const float slope = prm.alibi ? prm.alibi[h] : 0.0f;
+      const float slope = alibi ? prm.alibi[h] : 0.0f;
       if ((has_pos || has_time) && h != staged_head) {
         if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;
         if (has_pos)
@@ -371,17 +407,18 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const int j = k0 + r;                       // this thread's key (local index)
       const bool kvalid = j < n;
       const int64_t tj = has_time ? kts[r] : 0;
+      const int tj1 = has_time ? kts32[r] - 1 : 0;   // relative key time minus one
+      const bool keys_rel32 = has_time && tflag[0] != 0;
+      float* xp = xp_s + pw * (32 * 32);          // this warp's 32 x 32 block of dx, skewed
       for (int i = jt; i < nt; i++, g++, t++) {
         const uint32_t st = g % Cfg::NST;
         const int q0 = i * ATT_BM;
         const int64_t* qt_s = qts + st * 128;
+        const int* qt32 = qts32 + st * 128;
         // the stage's query timestamps are published with its Q/dAV tiles
         if (has_time && !mbar_wait(&q_full[st], (g / Cfg::NST) & 1u, abort_flag)) { ok = false; break; }
         if (!mbar_wait(sp_full, t & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        // every distance of this tile at least P-1: one bucket
-        const bool all_clamped = has_pos && q0 - (k0 + ATT_BN - 1) >= P - 1;
-        float clamped_acc = 0.0f;
 #pragma unroll 1
         for (int ch = 0; ch < 2; ch++) {
           const int cc = c0 + ch * 32;
@@ -390,8 +427,17 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           tmem_ld32(t_lane + Cfg::DP_COL + cc, dpv);
           tmem_ld_wait(sv);
           tmem_ld_wait(dpv);
-          int run_b = -1;
-          float run_acc = 0.0f;
+          // time-bucket gradient: the chunk's buckets along a row are those of its first query
+          // and the next one up (queries are later in time along the row); others go directly
+          int tb_first = 0;
+          float acc_lo = 0.0f, acc_hi = 0.0f;
+          if (has_time) {
+            const int b = time_bucket(qt_s[cc], tj);
+            tb_first = b < Tb - 1 ? b : Tb - 1;
+          }
+          // the element loop, with 32-bit time buckets when the tile's timestamps fit
+          auto elements = [&](auto rel_tag) {
+            constexpr bool REL32 = decltype(rel_tag)::value;
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             float a2[2], d2[2];
@@ -401,19 +447,22 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
               const int dist = iq - j;
               const bool valid = kvalid && iq < n && dist >= 0;
               float bias = 0.0f;
-              int pb = 0, tb = -1;
-              if (prm.alibi) {
-                bias = -slope * (float)dist;
-              } else {
-                if (has_pos) {
-                  pb = dist < 0 ? 0 : (dist < P - 1 ? dist : P - 1);
-                  bias += pb < BWD_POS_CAP ? pos_s[pb] : __ldg(pos_h + pb);
-                }
-                if (has_time) {
+              int tb = 0;
+              if (alibi) bias = -slope * (float)dist;
+              if (has_pos) {
+                const int pb = dist < 0 ? 0 : (dist < P - 1 ? dist : P - 1);
+                bias += pb < BWD_POS_CAP ? pos_s[pb] : __ldg(pos_h + pb);
+              }
+              if (has_time) {
+                if (REL32) {
+                  // floor(log2(1 + max(ti - tj, 0))) = 31 - clz(max(ti - tj, 0) + 1)
+                  const int dd = qt32[cc + e + u] - tj1;
+                  tb = 31 - __clz(dd > 1 ? dd : 1);
+                } else {
                   tb = time_bucket(qt_s[cc + e + u], tj);
-                  tb = tb < Tb - 1 ? tb : Tb - 1;
-                  bias += tb < BWD_TB_CAP ? tt_s[tb] : __ldg(tim_h + tb);
                 }
+                tb = tb < Tb - 1 ? tb : Tb - 1;
+                bias += tt_s[tb];
               }
               float sl, dsl;
               silu_and_grad(__uint_as_float(sv[e + u]) + bias, sl, dsl);
@@ -421,29 +470,65 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
               const float dx = valid ? scale * dsl * __uint_as_float(dpv[e + u]) : 0.0f;
               a2[u] = av;
               d2[u] = dx;
-              if (valid && has_pos) {
-                if (all_clamped) clamped_acc += dx;
-                else if (pb < BWD_POS_CAP) atomicAdd(&dpos_s[pb], dx);
-                else atomicAdd(prm.dpos + (int64_t)h * P + pb, dx);
-              }
-              if (valid && has_time) {
-                if (tb != run_b) {
-                  if (run_b >= 0) {
-                    if (run_b < BWD_TB_CAP) atomicAdd(&dtt_s[run_b], run_acc);
-                    else atomicAdd(prm.dtime + (int64_t)h * Tb + run_b, run_acc);
-                  }
-                  run_b = tb;
-                  run_acc = 0.0f;
+              // row `lane`, column (c - lane) mod 32: diagonal c - lane becomes a column
+              if (has_pos) xp[lane * 32 + ((e + u - lane) & 31)] = dx;
+              if (has_time) {
+                const int db = tb - tb_first;
+                acc_lo += db == 0 ? dx : 0.0f;
+                acc_hi += db == 1 ? dx : 0.0f;
+                // rare (a step of two or more buckets inside a chunk, near the diagonal): a
+                // warp vote keeps the shared-memory atomic off the common path
+                const bool far = valid && (db < 0 || db > 1);
+                if (__any_sync(0xffffffffu, far)) {
+                  if (far) atomicAdd(&dtt_s[tb], dx);
                 }
-                run_acc += dx;
               }
             }
             pk[e / 2] = pack_bf16x2(a2[0], a2[1]);
             dk[e / 2] = pack_bf16x2(d2[0], d2[1]);
           }
-          if (run_b >= 0) {
-            if (run_b < BWD_TB_CAP) atomicAdd(&dtt_s[run_b], run_acc);
-            else atomicAdd(prm.dtime + (int64_t)h * Tb + run_b, run_acc);
+          };
+          if (has_time && keys_rel32 && tflag[1 + st] != 0) elements(std::true_type{});
+          else elements(std::false_type{});
+          if (has_time) {
+            // one atomic per run of lanes with the same first bucket: the rows of a warp are 32
+            // consecutive keys, so equal first buckets are contiguous; a segmented inclusive scan
+            // leaves each run's sums in its last lane
+            const int prev = __shfl_up_sync(0xffffffffu, tb_first, 1);
+            const unsigned heads = __ballot_sync(0xffffffffu, lane == 0 || prev != tb_first);
+            const int seg0 = 31 - __clz(heads & (0xffffffffu >> (31 - lane)));
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+              const float lo = __shfl_up_sync(0xffffffffu, acc_lo, o);
+              const float hi = __shfl_up_sync(0xffffffffu, acc_hi, o);
+              if (lane - o >= seg0) {
+                acc_lo += lo;
+                acc_hi += hi;
+              }
+            }
+            const bool last = lane == 31 || ((heads >> (lane + 1)) & 1u);
+            if (last) {
+              if (acc_lo != 0.0f) atomicAdd(&dtt_s[tb_first], acc_lo);
+              if (acc_hi != 0.0f) atomicAdd(&dtt_s[tb_first + 1], acc_hi);
+            }
+          }
+          if (has_pos) {
+            // diagonal sums of the warp's 32 x 32 block: lane k reads column k, which holds the
+            // diagonals c - r = k (rows r < 32 - k) and c - r = k - 32 (the other rows)
+            __syncwarp();
+            float dpp = 0.0f, dpn = 0.0f;
+#pragma unroll 8
+            for (int rr = 0; rr < 32; rr++) {
+              const float v = xp[rr * 32 + lane];
+              if (rr + lane < 32) dpp += v; else dpn += v;
+            }
+            __syncwarp();
+            // distance of diagonal delta: (q0 + cc) - (k0 + q*32) + delta
+            const int base = q0 + cc - (k0 + q * 32);
+            const int d1 = base + lane, d2 = base + lane - 32;
+            float* dpos_h = prm.dpos + (int64_t)h * P;
+            if (dpp != 0.0f && d1 >= 0) atomicAdd(dpos_h + (d1 < P - 1 ? d1 : P - 1), dpp);
+            if (dpn != 0.0f && d2 >= 0) atomicAdd(dpos_h + (d2 < P - 1 ? d2 : P - 1), dpn);
           }
           // P^T and dS^T into the S^T / dP^T columns this warp has read
           tmem_st16(t_lane + Cfg::S_COL + c0 + ch * 16, pk);
@@ -457,7 +542,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             *reinterpret_cast<uint4*>(dst) = make_uint4(dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]);
           }
         }
-        if (all_clamped && kvalid) atomicAdd(&dpos_s[P - 1], clamped_acc);
         tmem_st_wait();
         tc_fence_before();
         fence_proxy_async_smem();
@@ -510,23 +594,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(dkv_empty);
       // table gradients of this item to global memory
-      if (has_pos || has_time) {
+      if (has_time) {
         if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;
-        if (has_pos) {
-          // distances of this item: 0 .. n - 1 - k0
-          const int64_t top = n - k0;
-          const int lim = top < dcap ? (int)top : dcap;
-          for (int e = tid; e < lim; e += BWD_PW) {
-            const float v = dpos_s[e];
-            if (v != 0.0f) atomicAdd(prm.dpos + (int64_t)h * P + e, v);
-            dpos_s[e] = 0.0f;
-          }
-          if (tid == 0 && dcap == P && lim < P) {   // the clamped bucket when P <= the distances
-            const float v = dpos_s[P - 1];
-            if (v != 0.0f) atomicAdd(prm.dpos + (int64_t)h * P + P - 1, v);
-            dpos_s[P - 1] = 0.0f;
-          }
-        }
         if (has_time)
           for (int e = tid; e < tcap; e += BWD_PW) {
             const float v = dtt_s[e];

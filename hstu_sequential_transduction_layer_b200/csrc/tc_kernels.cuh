@@ -193,6 +193,19 @@ inline size_t attention_bwd_workspace_bytes(int64_t T, int64_t B, int H) {
   return (size_t)(256 + ((16 * B + 255) / 256) * 256 + 8 * attention_bwd_capacity(T, B, H));
 }
 
+template <int BM>
+hstu_status_t launch_attention_bwd_kernel(const CUtensorMap& tm, const CUtensorMap& tdo,
+                                          const BwdParams& prm, const AttnSchedule& sch, int grid,
+                                          cudaStream_t st) {
+  auto kern = attention_bwd_kernel<BM>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg::SMEM) !=
+      cudaSuccess)
+    return HSTU_ERR_CUDA;
+  kern<<<grid, BWD_THREADS, BwdCfg::SMEM, st>>>(tm, tdo, prm, sch);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
 // Backward of Eq. 2 (head dim 64): dq, dpos and dtime are accumulated and must be zero on entry.
 inline hstu_status_t launch_attention_bwd(int64_t T, int64_t B, int H, int64_t max_seq_len,
                                           const bf16* uvqk, const int64_t* off, const int64_t* ts,
@@ -234,13 +247,16 @@ inline hstu_status_t launch_attention_bwd(int64_t T, int64_t B, int H, int64_t m
   prm.dv = dv;
   prm.dpos = dpos;
   prm.dtime = dtime;
-  if (cudaFuncSetAttribute(attention_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           BwdCfg::SMEM) != cudaSuccess)
-    return HSTU_ERR_CUDA;
   const int grid = (int)(capacity < num_sms() ? capacity : num_sms());
-  attention_bwd_kernel<<<grid, BWD_THREADS, BwdCfg::SMEM, st>>>(tm, tdo, prm, sch);
-  count_launch();
-  return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+  const int bm = alibi ? BWD_ALIBI : ((pos ? BWD_POS : 0) | (tim ? BWD_TIME : 0));
+  switch (bm) {
+    case 0: return launch_attention_bwd_kernel<0>(tm, tdo, prm, sch, grid, st);
+    case BWD_POS: return launch_attention_bwd_kernel<BWD_POS>(tm, tdo, prm, sch, grid, st);
+    case BWD_TIME: return launch_attention_bwd_kernel<BWD_TIME>(tm, tdo, prm, sch, grid, st);
+    case BWD_POS | BWD_TIME:
+      return launch_attention_bwd_kernel<BWD_POS | BWD_TIME>(tm, tdo, prm, sch, grid, st);
+    default: return launch_attention_bwd_kernel<BWD_ALIBI>(tm, tdo, prm, sch, grid, st);
+  }
 }
 
 // M-FALCON candidate attention workspace: header (256 B), per-user (candidate start, count,
