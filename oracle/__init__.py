@@ -340,3 +340,57 @@ def f2(g, W2, b2, X) -> np.ndarray:
     Y = np.empty((T, d), np.float64)
     _load().oracle_f2(T, w, d, _p(g), _p(W2), _p(b2), _p(X), _p(Y))
     return Y
+
+
+def layer_bwd(seq_offsets, X, W1, b1, W2, b2, ln_w, ln_b, dY, *, num_heads: int, d_qk: int,
+              d_v: int, timestamps=None, pos_table=None, time_table=None, alibi_slopes=None,
+              scale: float, ln_eps: float = 1e-5, lib=None):
+    """Backward of one layer ("Actions Speak Louder than Words" paper notes, section 3.1, Eqs. 1-3
+    and the residual between layers) for the loss sum(dY * Y): -> dict of dX [T, d], dW1 [d, n1],
+    db1 [n1], dW2 [H*d_v, d], db2 [d], dln_w, dln_b [H*d_v], dpos [H, P], dtime [H, Tb] (or None).
+
+    The chain rule written out step by step in fp64.  The forward is recomputed here (Z = X W1 + b1
+    before the SiLU, the row statistics of the LayerNorm), and the attention's own backward is
+    ``attention_bwd`` above.  ``b2`` only shifts Y, so no gradient flows through it to anything
+    but db2."""
+    X, W1, b1, W2, ln_w, ln_b, dY = (_d(a) for a in (X, W1, b1, W2, ln_w, ln_b, dY))
+    H = int(num_heads)
+    w = H * d_v
+    # Eq. 1, keeping the pre-activation: UVQK = SiLU(Z), SiLU(z) = z * sigmoid(z)
+    Z = X @ W1 + b1
+    sig = 1.0 / (1.0 + np.exp(-Z))
+    uvqk = Z * sig
+    U = uvqk[:, :w]
+    # Eq. 2
+    bias = dict(timestamps=timestamps, pos_table=pos_table, time_table=time_table,
+                alibi_slopes=alibi_slopes, scale=scale)
+    av = attention(seq_offsets, uvqk, num_heads=H, d_qk=d_qk, d_v=d_v, **bias)
+    # Eq. 3: LayerNorm over each row of AV (biased variance, eps under the root), gate by U, f2
+    mean = av.mean(axis=1, keepdims=True)
+    var = ((av - mean) ** 2).mean(axis=1, keepdims=True)
+    rstd = 1.0 / np.sqrt(var + ln_eps)
+    xhat = (av - mean) * rstd
+    ln = xhat * ln_w + ln_b
+    G = ln * U
+    # Y = G W2 + b2 + X
+    dG = dY @ W2.T
+    dW2 = G.T @ dY
+    db2 = dY.sum(axis=0)
+    # G = ln * U
+    dU = dG * ln
+    dln = dG * U
+    dln_w = (dln * xhat).sum(axis=0)
+    dln_b = dln.sum(axis=0)
+    # through the normalisation: d xhat, then the mean and the variance of the row
+    dxhat = dln * ln_w
+    dav = rstd * (dxhat - dxhat.mean(axis=1, keepdims=True)
+                  - xhat * (dxhat * xhat).mean(axis=1, keepdims=True))
+    a = attention_bwd(seq_offsets, uvqk, dav, num_heads=H, d_qk=d_qk, d_v=d_v, lib=lib, **bias)
+    duvqk = np.concatenate([dU, a["dv"], a["dq"], a["dk"]], axis=1)
+    # SiLU'(z) = sigmoid(z) (1 + z (1 - sigmoid(z)))
+    dZ = duvqk * sig * (1.0 + Z * (1.0 - sig))
+    dW1 = X.T @ dZ
+    db1 = dZ.sum(axis=0)
+    dX = dZ @ W1.T + dY
+    return {"dX": dX, "dW1": dW1, "db1": db1, "dW2": dW2, "db2": db2, "dln_w": dln_w,
+            "dln_b": dln_b, "dpos": a["dpos"], "dtime": a["dtime"]}
