@@ -605,6 +605,118 @@ def run_backward(args, rank, world, local_rank):
 
 
 # ------------------------------------------------------------------------------------------------
+# Training step (--train): one step is the layer's forward (its workspace keeps U, V, Q, K, AV and
+# G) followed by the layer's backward for an incoming gradient dY, every parameter gradient and dX.
+# The dominant kernel, the attention backward, is also timed on its own (same inputs, same stream)
+# for the roofline figure.
+# ------------------------------------------------------------------------------------------------
+
+TRAIN_METRIC = "HSTU layer training step throughput (forward + backward: dX and all parameter gradients)"
+
+
+def run_train(args, rank, world, local_rank):
+    import torch
+    import hstu_sequential_transduction_layer_b200 as hstu
+    from workloads.device import to_device, tensor
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = workloads.WORKLOADS[args.workload]
+    if w.head_dim != 64 or w.token_embed or w.dtype != "bf16":
+        raise SystemExit("the layer backward is implemented for bf16, head dim 64 (long_seq, retrieval)")
+    inp = workloads.make_inputs(w)
+    H, hd, d, T = w.num_heads, w.head_dim, w.d_model, inp.T
+    n1, wv = 4 * H * hd, H * hd
+    D = to_device(inp, dev)
+    L = D["layers"][0]
+    max_len = int(inp.lengths.max())
+    shape = hstu.shape_for(D["X"], D["off"], H, hd, hd, max_len, D["pos"], D["tim"], inp.ln_eps)
+    rng = np.random.default_rng(w.index + 600)
+    dY = tensor(rng.standard_normal((T, d), dtype=np.float32), "bf16", dev)
+    Y = torch.empty_like(D["X"])
+    dX = torch.empty_like(D["X"])
+    f32 = lambda *sh: torch.empty(sh, dtype=torch.float32, device=dev)
+    grads = [f32(d, n1), f32(n1), f32(wv, d), f32(d), f32(wv), f32(wv)]
+    dpos = torch.empty_like(D["pos"]) if D["pos"] is not None else None
+    dtim = torch.empty_like(D["tim"]) if D["tim"] is not None else None
+    fws = hstu.alloc_workspace(shape, dev)
+    bws = torch.empty(max(256, hstu.layer_bwd_workspace_size(shape)), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        hstu.hstu_layer_fwd(D["X"], D["off"], D["ts"], L["W1"], L["b1"], L["W2"], L["b2"],
+                            L["ln_w"], L["ln_b"], D["pos"], D["tim"], D["ali"], inp.scale,
+                            num_heads=H, max_seq_len=max_len, ln_eps=inp.ln_eps, out=Y,
+                            workspace=fws, stream=stream)
+        hstu.hstu_layer_bwd(shape, D["X"], D["off"], D["ts"], L["W1"], L["b1"], L["W2"],
+                            L["ln_w"], L["ln_b"], D["pos"], D["tim"], D["ali"], inp.scale, fws, dY,
+                            dX, *grads, dpos, dtim, bws, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if hstu.device_status() != hstu.HSTU_OK:
+        raise SystemExit("device status error during warm-up")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank)
+    torch.cuda.synchronize()
+    sampler.start()
+    launches0 = hstu.launch_count()
+    for k in range(args.steps):
+        flush.zero_()
+        evs[k][0].record(stream)
+        step()
+        evs[k][1].record(stream)
+    torch.cuda.synchronize()
+    launches = hstu.launch_count() - launches0
+    clocks = sampler.stop()
+    total_ms, job_tokens = combine_over_ranks(sum(e[0].elapsed_time(e[1]) for e in evs), T, world, dev)
+    if hstu.device_status() != hstu.HSTU_OK:
+        raise SystemExit("device status error in the timed region")
+    ms = total_ms / args.steps
+    # the attention backward alone, on U, V, Q, K of the layer and a bf16 dAV of the same shape
+    uvqk = torch.empty((T, n1), dtype=torch.bfloat16, device=dev)
+    hstu.hstu_f1_fwd(shape, D["X"], L["W1"], L["b1"], uvqk)
+    dav = tensor(rng.standard_normal((T, wv), dtype=np.float32), "bf16", dev)
+    dq, dk, dv = (f32(T, wv) for _ in range(3))
+    aws = torch.empty(max(256, int(hstu.library().hstu_attention_bwd_workspace_size(shape))),
+                      dtype=torch.uint8, device=dev)
+    a_evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(5)]
+    for k in range(5):
+        flush.zero_()
+        a_evs[k][0].record(stream)
+        hstu.hstu_attention_bwd(shape, uvqk, D["off"], D["ts"], D["pos"], D["tim"], D["ali"],
+                                inp.scale, dav, dq, dk, dv, dpos, dtim, aws, stream)
+        a_evs[k][1].record(stream)
+    torch.cuda.synchronize()
+    a_ms = sum(e[0].elapsed_time(e[1]) for e in a_evs[1:]) / 4
+    peaks, peaks_src = load_peaks()
+    tpk = peaks["bf16_tflops"]
+    pairs = float(np.sum(inp.lengths * (inp.lengths + 1) // 2))
+    a_tf = 2.0 * H * 5 * hd * pairs / a_ms / 1e9
+    # the whole step's tensor work: forward (f1, S and AV, f2) and backward (dG, dW2, S, dP, dV,
+    # dK, dQ, the recomputed f1, dW1, dX): four [T, d] x [d, n1]-sized products, three
+    # [T, wv] x [wv, d]-sized ones, and 2 + 5 products of 2*hd FLOP per causal pair and head
+    step_fl = 8.0 * T * d * n1 + 6.0 * T * wv * d + 2.0 * H * 7 * hd * pairs
+    return {
+        "metric": TRAIN_METRIC, "value": round(job_tokens / (ms * 1e-3), 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded inputs and parameters of the workload, N(0,1) incoming gradient)",
+        "config": {"workload": f"{w.name}: B={len(inp.lengths)}, n={max_len}, d={d}, "
+                               f"H={H}x{hd}, rab P={w.n_pos_buckets}/Tb={w.n_time_buckets}",
+                   "l2": "flushed between timed steps (outside the events)",
+                   "step_tflops": round(step_fl / ms / 1e9, 2)},
+        "roofline": {"bound": "tensor", "kernel": "attention_bwd", "achieved": round(a_tf, 2),
+                     "peak": tpk, "unit": "TFLOP/s", "frac": round(a_tf / tpk, 4), "traffic": None,
+                     "ms_per_launch": round(a_ms, 4),
+                     "peak_source": f"{peaks_src} bf16 burst (MEASURED_PEAKS.json)"},
+        "gpu_launches": int(launches), "clocks": clocks,
+    }
+
+
+# ------------------------------------------------------------------------------------------------
 # Stochastic Length (--stochastic-length ALPHA): a step shortens the workload's batch on the device
 # (cut decisions and new offsets, per-sequence selection) and gathers the shortened batch's X rows
 # and timestamps, the new token count read on the device.
@@ -773,6 +885,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--backward", action="store_true",
                     help="time the attention backward instead")
+    ap.add_argument("--train", action="store_true",
+                    help="time a training step (layer forward + layer backward) instead")
     ap.add_argument("--stochastic-length", type=float, default=0.0,
                     help="time Stochastic Length subsampling with this alpha instead")
     ap.add_argument("--candidates", type=int, default=0,
@@ -798,6 +912,11 @@ def main():
     try:
         if args.backward:
             res = run_backward(args, rank, world, local_rank)
+            if rank == 0:
+                print(json.dumps(res), flush=True)
+            return
+        if args.train:
+            res = run_train(args, rank, world, local_rank)
             if rank == 0:
                 print(json.dumps(res), flush=True)
             return

@@ -33,7 +33,8 @@ EXPORTED = ["hstu_layer_fwd", "hstu_layer_fwd_workspace_size", "hstu_f1_fwd", "h
             "hstu_candidate_workspace_size", "hstu_candidate_attention_fwd",
             "hstu_candidate_layer_workspace_size", "hstu_candidate_layer_fwd",
             "hstu_stochastic_length_workspace_size", "hstu_stochastic_length", "hstu_gather_rows",
-            "hstu_attention_bwd_workspace_size", "hstu_attention_bwd"]
+            "hstu_attention_bwd_workspace_size", "hstu_attention_bwd",
+            "hstu_layer_bwd_workspace_size", "hstu_layer_bwd"]
 
 
 class HstuShape(ctypes.Structure):
@@ -88,6 +89,9 @@ def _load() -> ctypes.CDLL:
         "hstu_attention_bwd": ([SH, P, P, P, P, P, P, F32, P, P, P, P, P, P, P, S, P], ctypes.c_int),
         "hstu_candidate_layer_fwd": ([SH, P, P, P, I64, I64, P, P, P, P, P, P, P, P, P, P, P, P, F32,
                                       P, P, S, P], ctypes.c_int),
+        "hstu_layer_bwd_workspace_size": ([SH], S),
+        "hstu_layer_bwd": ([SH, P, P, P, P, P, P, P, P, P, P, P, F32, P, S, P, P, P, P, P, P, P, P,
+                            P, P, P, S, P], ctypes.c_int),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -296,6 +300,30 @@ def hstu_attention_bwd(shape: HstuShape, uvqk, seq_offsets, timestamps, pos_tabl
                                    _ptr(dtime_table), _ptr(workspace), workspace.numel(),
                                    _stream(stream)), "hstu_attention_bwd")
     return dq, dk, dv
+
+
+def layer_bwd_workspace_size(shape: HstuShape) -> int:
+    return int(_lib.hstu_layer_bwd_workspace_size(ctypes.byref(shape)))
+
+
+def hstu_layer_bwd(shape: HstuShape, X, seq_offsets, timestamps, W1, b1, W2, ln_w, ln_b,
+                   pos_table, time_table, alibi_slopes, scale: float, fwd_workspace, dY, dX, dW1,
+                   db1, dW2, db2, dln_w, dln_b, dpos_table=None, dtime_table=None, workspace=None,
+                   stream=None):
+    """Backward of one layer (see the C header): `fwd_workspace` is the workspace a preceding
+    hstu_layer_fwd call with the same inputs filled; fills dX and every parameter gradient."""
+    if workspace is None:
+        workspace = torch.empty(max(256, layer_bwd_workspace_size(shape)), dtype=torch.uint8,
+                                device=X.device)
+    _check(_lib.hstu_layer_bwd(ctypes.byref(shape), _ptr(X), _ptr(seq_offsets), _ptr(timestamps),
+                               _ptr(W1), _ptr(b1), _ptr(W2), _ptr(ln_w), _ptr(ln_b),
+                               _ptr(pos_table), _ptr(time_table), _ptr(alibi_slopes), float(scale),
+                               _ptr(fwd_workspace), fwd_workspace.numel(), _ptr(dY), _ptr(dX),
+                               _ptr(dW1), _ptr(db1), _ptr(dW2), _ptr(db2), _ptr(dln_w),
+                               _ptr(dln_b), _ptr(dpos_table), _ptr(dtime_table), _ptr(workspace),
+                               workspace.numel(), _stream(stream)), "hstu_layer_bwd")
+    return {"dX": dX, "dW1": dW1, "db1": db1, "dW2": dW2, "db2": db2, "dln_w": dln_w,
+            "dln_b": dln_b, "dpos": dpos_table, "dtime": dtime_table}
 
 
 def hstu_stochastic_length(seq_offsets, max_len: int, alpha: float, u, keys, new_offsets, index,

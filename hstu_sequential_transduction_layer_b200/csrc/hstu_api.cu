@@ -7,6 +7,7 @@
 
 #include "common.cuh"
 #include "hbm_kernels.cuh"
+#include "bwd_kernels.cuh"
 #include "sl_kernels.cuh"
 #include "simt_kernels.cuh"
 #include "tc_kernels.cuh"
@@ -269,6 +270,98 @@ CandWorkspace cand_layout(const hstu_shape_t& s, int64_t Tc, void* base) {
   o += align_up(w.attn_bytes);
   w.total = o;
   return w;
+}
+
+// Widest LayerNorm row the backward handles (its per-block partial sums live in shared memory).
+constexpr int64_t kLnBwdMaxWidth = 8192;
+
+// Arguments of the attention backward that do not depend on the token count.
+hstu_status_t check_attention_bwd(const hstu_shape_t* shape, const int64_t* ts, const float* pos,
+                                  const float* tim, const float* alibi, float scale,
+                                  const float* dpos, const float* dtime) {
+  hstu_status_t rc = check_shape(shape);
+  if (rc != HSTU_OK) return rc;
+  const hstu_shape_t& s = *shape;
+  if (s.dtype != HSTU_BF16 || s.d_qk != 64 || s.d_v != 64) return HSTU_ERR_UNSUPPORTED;
+  if (s.num_seqs * (int64_t)s.num_heads >= (1LL << 31)) return HSTU_ERR_UNSUPPORTED;
+  if ((rc = check_bias(shape, ts, pos, tim, alibi, scale)) != HSTU_OK) return rc;
+  if ((pos && !dpos) || (tim && !dtime)) return HSTU_ERR_INVALID_ARG;
+  return HSTU_OK;
+}
+
+hstu_status_t zero_f32(float* p, int64_t n, cudaStream_t st) {
+  if (!p || n <= 0) return HSTU_OK;
+  zero_f32_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p, n);
+  return launch_status();
+}
+
+// The attention backward once its arguments are checked: zero what the kernel accumulates into
+// (dQ and the tables' gradients), check the offsets, run the kernel.
+hstu_status_t run_attention_bwd(const hstu_shape_t& s, const void* uvqk, const int64_t* off,
+                                const int64_t* ts, const float* pos, const float* tim,
+                                const float* alibi, float scale, const void* dav, float* dq,
+                                float* dk, float* dv, float* dpos, float* dtime, void* ws,
+                                size_t ws_bytes, cudaStream_t st) {
+  hstu_status_t rc;
+  const int64_t T = s.total_tokens, B = s.num_seqs;
+  if (pos && (rc = zero_f32(dpos, (int64_t)s.num_heads * s.n_pos_buckets, st)) != HSTU_OK) return rc;
+  if (tim && (rc = zero_f32(dtime, (int64_t)s.num_heads * s.n_time_buckets, st)) != HSTU_OK)
+    return rc;
+  if (T == 0) return HSTU_OK;
+  if ((rc = zero_f32(dq, T * wv_of(s), st)) != HSTU_OK) return rc;
+  check_offsets_kernel<<<(unsigned)((B + 1 + 255) / 256), 256, 0, st>>>(off, B, T);
+  if (launch_status() != HSTU_OK) return HSTU_ERR_CUDA;
+  return tc::launch_attention_bwd(T, B, s.num_heads, s.max_seq_len, (const bf16*)uvqk, off, ts, pos,
+                                  s.n_pos_buckets, tim, s.n_time_buckets, alibi, scale,
+                                  (const bf16*)dav, dq, dk, dv, dpos, dtime, ws, ws_bytes, st);
+}
+
+struct BwdWorkspace {
+  void *w2t, *w1t, *dg, *dav, *duvqk, *dqkv, *trans, *attn;
+  size_t attn_bytes, total;
+  int64_t t_pad;
+};
+
+BwdWorkspace bwd_layout(const hstu_shape_t& s, void* base) {
+  BwdWorkspace w{};
+  const size_t T = (size_t)s.total_tokens, d = (size_t)s.d_model;
+  const size_t wv = (size_t)wv_of(s), n1 = (size_t)n1_of(s);
+  w.t_pad = (int64_t)((T + 63) / 64 * 64);
+  size_t o = 0;
+  char* b = static_cast<char*>(base);
+  auto take = [&](void*& p, size_t bytes) {
+    p = b ? b + o : nullptr;
+    o += align_up(bytes);
+  };
+  take(w.w2t, d * wv * 2);                      // W2^T [d, H*dv]
+  take(w.w1t, n1 * d * 2);                      // W1^T [n1, d]
+  take(w.dg, T * wv * 4);                       // dG fp32
+  take(w.dav, T * wv * 2);                      // dAV bf16
+  take(w.duvqk, T * n1 * 2);                    // dU|dV|dQ|dK bf16
+  take(w.dqkv, 3 * T * wv * 4);                 // dQ, dK, dV fp32; later dZ bf16 [T, n1]
+  take(w.trans, (wv > d ? wv : d) * (size_t)w.t_pad * 2);   // G^T, later X^T
+  w.attn_bytes = tc::attention_bwd_workspace_bytes(s.total_tokens, s.num_seqs, s.num_heads);
+  take(w.attn, w.attn_bytes);
+  w.total = o;
+  return w;
+}
+
+hstu_status_t run_transpose(int64_t rows, int64_t rows_pad, int cols, int64_t ld, const void* src,
+                            void* dst, cudaStream_t st) {
+  const dim3 grid((unsigned)((rows_pad + 31) / 32), (unsigned)((cols + 31) / 32));
+  bwd::transpose_bf16_kernel<<<grid, dim3(32, 8), 0, st>>>(rows, rows_pad, cols, ld,
+                                                            (const bf16*)src, (bf16*)dst);
+  return launch_status();
+}
+
+hstu_status_t run_colsum(int64_t rows, int cols, const void* src, float* out, cudaStream_t st) {
+  const int64_t want = 4LL * tc::num_sms();
+  int64_t per = (rows + want - 1) / want;
+  if (per < 16) per = 16;
+  const int64_t blocks = (rows + per - 1) / per;
+  bwd::colsum_kernel<bf16><<<(unsigned)blocks, 256, 0, st>>>(rows, cols, cols, per,
+                                                             (const bf16*)src, out);
+  return launch_status();
 }
 
 }  // namespace
@@ -553,43 +646,143 @@ hstu_status_t hstu_attention_bwd(const hstu_shape_t* shape, const void* uvqk,
                                  const float* alibi_slopes, float scale, const void* dav, float* dq,
                                  float* dk, float* dv, float* dpos_table, float* dtime_table,
                                  void* workspace, size_t workspace_bytes, void* stream) {
-  hstu_status_t rc = check_shape(shape);
+  hstu_status_t rc = check_attention_bwd(shape, timestamps, pos_table, time_table, alibi_slopes,
+                                         scale, dpos_table, dtime_table);
   if (rc != HSTU_OK) return rc;
   const hstu_shape_t& s = *shape;
-  if (s.dtype != HSTU_BF16 || s.d_qk != 64 || s.d_v != 64) return HSTU_ERR_UNSUPPORTED;
-  if (s.num_seqs * (int64_t)s.num_heads >= (1LL << 31)) return HSTU_ERR_UNSUPPORTED;
-  if ((rc = check_bias(shape, timestamps, pos_table, time_table, alibi_slopes, scale)) != HSTU_OK)
-    return rc;
-  if ((pos_table && !dpos_table) || (time_table && !dtime_table)) return HSTU_ERR_INVALID_ARG;
   const int64_t T = s.total_tokens, B = s.num_seqs;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  auto zero = [&](float* p, int64_t n) {
-    if (!p || n <= 0) return HSTU_OK;
-    zero_f32_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(p, n);
-    return launch_status();
-  };
-  const int64_t w = (int64_t)s.num_heads * 64;
-  if (pos_table && (rc = zero(dpos_table, (int64_t)s.num_heads * s.n_pos_buckets)) != HSTU_OK) return rc;
-  if (time_table && (rc = zero(dtime_table, (int64_t)s.num_heads * s.n_time_buckets)) != HSTU_OK)
+  if (T > 0) {
+    if (B == 0 || !uvqk || !seq_offsets || !dav || !dq || !dk || !dv || !workspace)
+      return HSTU_ERR_INVALID_ARG;
+    if (!(aligned16(uvqk) && aligned16(dav) && aligned16(dq) && aligned16(dk) && aligned16(dv)))
+      return HSTU_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) return HSTU_ERR_INVALID_ARG;
+    if (workspace_bytes < hstu_attention_bwd_workspace_size(shape)) return HSTU_ERR_INVALID_ARG;
+    const size_t gb = (size_t)T * wv_of(s) * 4;
+    if (overlaps(dq, gb, dk, gb) || overlaps(dq, gb, dv, gb) || overlaps(dk, gb, dv, gb) ||
+        overlaps(dq, gb, workspace, workspace_bytes) ||
+        overlaps(dk, gb, workspace, workspace_bytes) || overlaps(dv, gb, workspace, workspace_bytes))
+      return HSTU_ERR_INVALID_ARG;
+  }
+  return run_attention_bwd(s, uvqk, seq_offsets, timestamps, pos_table, time_table, alibi_slopes,
+                           scale, dav, dq, dk, dv, dpos_table, dtime_table, workspace,
+                           workspace_bytes, st);
+}
+
+// ------------------------------------------------------------------------------------------------
+// Layer backward
+// ------------------------------------------------------------------------------------------------
+
+size_t hstu_layer_bwd_workspace_size(const hstu_shape_t* shape) {
+  if (check_shape(shape) != HSTU_OK) return 0;
+  return bwd_layout(*shape, nullptr).total;
+}
+
+hstu_status_t hstu_layer_bwd(const hstu_shape_t* shape, const void* X, const int64_t* seq_offsets,
+                             const int64_t* timestamps, const void* W1, const void* b1,
+                             const void* W2, const void* ln_w, const void* ln_b,
+                             const float* pos_table, const float* time_table,
+                             const float* alibi_slopes, float scale, const void* fwd_workspace,
+                             size_t fwd_workspace_bytes, const void* dY, void* dX, float* dW1,
+                             float* db1, float* dW2, float* db2, float* dln_w, float* dln_b,
+                             float* dpos_table, float* dtime_table, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  hstu_status_t rc = check_attention_bwd(shape, timestamps, pos_table, time_table, alibi_slopes,
+                                         scale, dpos_table, dtime_table);
+  if (rc != HSTU_OK) return rc;
+  const hstu_shape_t& s = *shape;
+  const int64_t T = s.total_tokens, B = s.num_seqs, wv = wv_of(s), n1 = n1_of(s);
+  const int d = s.d_model;
+  if (wv > kLnBwdMaxWidth) return HSTU_ERR_UNSUPPORTED;
+  if (!W1 || !W2 || !ln_w || !ln_b || !dW1 || !db1 || !dW2 || !db2 || !dln_w || !dln_b)
+    return HSTU_ERR_INVALID_ARG;
+  const void* ptrs16[] = {X, W1, b1, W2, ln_w, ln_b, dY, dX, dW1, db1, dW2, db2, dln_w, dln_b};
+  for (const void* p : ptrs16)
+    if (!aligned16(p)) return HSTU_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  struct Z { float* p; int64_t n; } zeros[] = {{dW1, (int64_t)d * n1}, {db1, n1}, {dW2, wv * d},
+                                               {db2, d}, {dln_w, wv}, {dln_b, wv}};
+  if (T > 0) {
+    if (B == 0 || !X || !seq_offsets || !fwd_workspace || !dY || !dX || !workspace)
+      return HSTU_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) return HSTU_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(fwd_workspace) & (kAlign - 1)) return HSTU_ERR_INVALID_ARG;
+    const Workspace fw = layout(s, const_cast<void*>(fwd_workspace));
+    const BwdWorkspace w = bwd_layout(s, workspace);
+    if (fwd_workspace_bytes < fw.total || workspace_bytes < w.total) return HSTU_ERR_INVALID_ARG;
+    const size_t xb = (size_t)T * d * 2;
+    // dX may not overlap anything it is computed from or any workspace
+    if (overlaps(dX, xb, dY, xb) || overlaps(dX, xb, X, xb) ||
+        overlaps(dX, xb, workspace, w.total) || overlaps(dX, xb, fwd_workspace, fw.total) ||
+        overlaps(workspace, w.total, fwd_workspace, fw.total))
+      return HSTU_ERR_INVALID_ARG;
+  }
+  for (const Z& z : zeros)
+    if ((rc = zero_f32(z.p, z.n, st)) != HSTU_OK) return rc;
+  if (T == 0) return run_attention_bwd(s, nullptr, seq_offsets, timestamps, pos_table, time_table,
+                                       alibi_slopes, scale, nullptr, nullptr, nullptr, nullptr,
+                                       dpos_table, dtime_table, nullptr, 0, st);
+  const Workspace fw = layout(s, const_cast<void*>(fwd_workspace));
+  const BwdWorkspace w = bwd_layout(s, workspace);
+  const bf16* dy = (const bf16*)dY;
+  const int64_t T4 = T * wv;
+  float* dq = (float*)w.dqkv;
+  float* dk = dq + T4;
+  float* dv = dk + T4;
+  bf16* dz = (bf16*)w.dqkv;   // after dQ, dK, dV are packed into dUVQK
+  // f2: Y = G W2 + b2 + X  ->  dG = dY W2^T, dW2 = G^T dY, db2 = column sums of dY
+  if ((rc = run_transpose(wv, wv, d, d, W2, w.w2t, st)) != HSTU_OK) return rc;
+  if ((rc = run_transpose(d, d, (int)n1, n1, W1, w.w1t, st)) != HSTU_OK) return rc;
+  if ((rc = tc::launch_gemm_ext<tc::EPI_F32>(T, (int)wv, d, dy, (const bf16*)w.w2t, nullptr,
+                                             nullptr, nullptr, (float*)w.dg, 1, -1, st)) != HSTU_OK)
     return rc;
-  if (T == 0) return HSTU_OK;
-  if (B == 0 || !uvqk || !seq_offsets || !dav || !dq || !dk || !dv || !workspace)
-    return HSTU_ERR_INVALID_ARG;
-  if (!(aligned16(uvqk) && aligned16(dav) && aligned16(dq) && aligned16(dk) && aligned16(dv)))
-    return HSTU_ERR_INVALID_ARG;
-  if (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) return HSTU_ERR_INVALID_ARG;
-  const size_t gb = (size_t)T * w * 4;
-  if (overlaps(dq, gb, dk, gb) || overlaps(dq, gb, dv, gb) || overlaps(dk, gb, dv, gb) ||
-      overlaps(dq, gb, workspace, workspace_bytes) || overlaps(dk, gb, workspace, workspace_bytes) ||
-      overlaps(dv, gb, workspace, workspace_bytes))
-    return HSTU_ERR_INVALID_ARG;
-  if ((rc = zero(dq, T * w)) != HSTU_OK) return rc;
-  check_offsets_kernel<<<(unsigned)((B + 1 + 255) / 256), 256, 0, st>>>(seq_offsets, B, T);
-  if (launch_status() != HSTU_OK) return HSTU_ERR_CUDA;
-  return tc::launch_attention_bwd(T, B, s.num_heads, s.max_seq_len, (const bf16*)uvqk, seq_offsets,
-                                  timestamps, pos_table, s.n_pos_buckets, time_table,
-                                  s.n_time_buckets, alibi_slopes, scale, (const bf16*)dav, dq, dk,
-                                  dv, dpos_table, dtime_table, workspace, workspace_bytes, st);
+  if ((rc = run_transpose(T, w.t_pad, (int)wv, wv, fw.g, w.trans, st)) != HSTU_OK) return rc;
+  const int kt = (int)w.t_pad;
+  if ((rc = tc::launch_gemm_ext<tc::EPI_RED_F32>(
+           wv, d, kt, (const bf16*)w.trans, dy, nullptr, nullptr, nullptr, dW2,
+           tc::weight_grad_splits(wv, d, kt), T, st)) != HSTU_OK)
+    return rc;
+  if ((rc = run_colsum(T, d, dY, db2, st)) != HSTU_OK) return rc;
+  // G = LayerNorm(AV) * U  ->  dU (block 0 of dUVQK), dAV, dln_w, dln_b
+  {
+    const int64_t blocks = T < 4LL * tc::num_sms() * 8 ? (T + 7) / 8 : 4LL * tc::num_sms();
+    const size_t smem = (size_t)2 * wv * sizeof(float);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(bwd::ln_gate_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return HSTU_ERR_CUDA;
+    bwd::ln_gate_bwd_kernel<<<(unsigned)blocks, 256, smem, st>>>(
+        T, (int)wv, n1, (const float*)fw.av, (const bf16*)fw.uvqk, (const float*)w.dg,
+        (const bf16*)ln_w, (const bf16*)ln_b, s.ln_eps, (bf16*)w.dav, (bf16*)w.duvqk, dln_w,
+        dln_b);
+    if ((rc = launch_status()) != HSTU_OK) return rc;
+  }
+  // Eq. 2  ->  dQ, dK, dV and the bias tables' gradients; then dV|dQ|dK into dUVQK
+  if ((rc = run_attention_bwd(s, fw.uvqk, seq_offsets, timestamps, pos_table, time_table,
+                              alibi_slopes, scale, w.dav, dq, dk, dv, dpos_table, dtime_table,
+                              w.attn, w.attn_bytes, st)) != HSTU_OK)
+    return rc;
+  {
+    const int64_t threads = T * 3 * (wv / 4);
+    bwd::pack_dvqk_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
+        T, (int)wv, n1, dv, dq, dk, (bf16*)w.duvqk);
+    if ((rc = launch_status()) != HSTU_OK) return rc;
+  }
+  // Eq. 1: UVQK = SiLU(X W1 + b1)  ->  dZ = dUVQK * SiLU'(X W1 + b1), dW1 = X^T dZ, db1, dX
+  if ((rc = tc::launch_gemm_ext<tc::EPI_SILU_GRAD>(T, (int)n1, d, (const bf16*)X,
+                                                   (const bf16*)W1, (const bf16*)b1,
+                                                   (const bf16*)w.duvqk, dz, nullptr, 1, -1,
+                                                   st)) != HSTU_OK)
+    return rc;
+  if ((rc = run_colsum(T, (int)n1, dz, db1, st)) != HSTU_OK) return rc;
+  if ((rc = run_transpose(T, w.t_pad, d, d, X, w.trans, st)) != HSTU_OK) return rc;
+  if ((rc = tc::launch_gemm_ext<tc::EPI_RED_F32>(
+           d, (int)n1, kt, (const bf16*)w.trans, dz, nullptr, nullptr, nullptr, dW1,
+           tc::weight_grad_splits(d, (int)n1, kt), T, st)) != HSTU_OK)
+    return rc;
+  return tc::launch_gemm_ext<tc::EPI_BIAS_RESIDUAL>(T, d, (int)n1, dz, (const bf16*)w.w1t,
+                                                    nullptr, dy, (bf16*)dX, nullptr, 1, -1, st);
 }
 
 size_t hstu_stochastic_length_workspace_size(int64_t num_seqs) {

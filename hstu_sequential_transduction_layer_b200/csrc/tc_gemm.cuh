@@ -4,6 +4,12 @@
 //   C[M, N] = epilogue(A[M, K] . B[K, N]),  A row-major (K-major), B row-major (MN-major operand)
 //   EPI_BIAS_SILU:      C = SiLU(acc + bias)              f1: U|V|Q|K = SiLU(X W1 + b1)
 //   EPI_BIAS_RESIDUAL:  C = acc + bias + R                f2: Y = G W2 + b2 + X
+// and for the backward pass:
+//   EPI_F32:            C32 = acc (fp32)                  dG = dY W2^T
+//   EPI_SILU_GRAD:      C = R * SiLU'(acc + bias)         dZ = dUVQK * SiLU'(X W1 + b1)
+//   EPI_RED_F32:        C32 += acc (fp32 reductions)      dW = X^T dZ over a split of K
+// With `splits` > 1 every output tile is computed in that many parts over consecutive ranges of K
+// (split-K, for the weight gradients' short M and N and long K); only EPI_RED_F32 combines parts.
 //
 // One CTA per SM (320 threads):
 //   warp 0      TMA producer: A tile 128x64 and B tile 64xBN per stage into a STAGES-deep ring, both
@@ -24,7 +30,8 @@
 namespace hstu {
 namespace tc {
 
-enum GemmEpilogue { EPI_BIAS_SILU = 0, EPI_BIAS_RESIDUAL = 1 };
+enum GemmEpilogue { EPI_BIAS_SILU = 0, EPI_BIAS_RESIDUAL = 1, EPI_F32 = 2, EPI_SILU_GRAD = 3,
+                    EPI_RED_F32 = 4 };
 
 template <int BN>
 struct GemmCfg {
@@ -55,11 +62,24 @@ __device__ __forceinline__ float silu_tanh(float x) {
   return fmaf(h, sm100::tanh_approx(h), h);
 }
 
-// Bias (+ SiLU | + residual) of 32 consecutive columns n .. n+31 of one row, stored as bf16.
+// The epilogue of 32 consecutive columns n .. n+31 of one row.
 template <int EPI>
 __device__ __forceinline__ void gemm_epilogue_chunk(const uint32_t (&r)[32], const bf16* __restrict__ bias,
                                                     const bf16* __restrict__ R, bf16* __restrict__ C,
-                                                    int64_t row, int64_t M, int N, int n) {
+                                                    float* __restrict__ C32, int64_t row, int64_t M,
+                                                    int N, int n) {
+  if (EPI == EPI_F32 || EPI == EPI_RED_F32) {
+    if (row >= M) return;
+    float* dst = C32 + row * N + n;
+#pragma unroll
+    for (int v = 0; v < 8; v++) {
+      const float a = __uint_as_float(r[4 * v]), b = __uint_as_float(r[4 * v + 1]);
+      const float c = __uint_as_float(r[4 * v + 2]), d = __uint_as_float(r[4 * v + 3]);
+      if (EPI == EPI_F32) reinterpret_cast<float4*>(dst)[v] = make_float4(a, b, c, d);
+      else sm100::red_add_v4(dst + 4 * v, a, b, c, d);
+    }
+    return;
+  }
   uint4 bvec[4];
   if (bias) {
 #pragma unroll
@@ -70,7 +90,7 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const uint32_t (&r)[32], con
   }
   if (row >= M) return;
   uint4 rvec[4] = {};
-  if (EPI == EPI_BIAS_RESIDUAL) {
+  if (EPI == EPI_BIAS_RESIDUAL || EPI == EPI_SILU_GRAD) {
 #pragma unroll
     for (int v = 0; v < 4; v++) rvec[v] = __ldcs(reinterpret_cast<const uint4*>(R + row * N + n) + v);
   }
@@ -87,6 +107,12 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const uint32_t (&r)[32], con
       if (EPI == EPI_BIAS_SILU) {
         lo = silu_tanh(lo);
         hi = silu_tanh(hi);
+      } else if (EPI == EPI_SILU_GRAD) {
+        // SiLU'(z) = s (1 + z (1 - s)), s = sigmoid(z) = 0.5 + 0.5 tanh(z/2)
+        const float sl = fmaf(0.5f, sm100::tanh_approx(0.5f * lo), 0.5f);
+        const float sh = fmaf(0.5f, sm100::tanh_approx(0.5f * hi), 0.5f);
+        lo = bf16_lo(rw[e]) * sl * fmaf(lo, 1.0f - sl, 1.0f);
+        hi = bf16_hi(rw[e]) * sh * fmaf(hi, 1.0f - sh, 1.0f);
       } else {
         lo += bf16_lo(rw[e]);
         hi += bf16_hi(rw[e]);
@@ -104,7 +130,8 @@ template <int BN, int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int64_t M, int N, int K, const bf16* __restrict__ bias,
-                   const bf16* __restrict__ R, bf16* __restrict__ C) {
+                   const bf16* __restrict__ R, bf16* __restrict__ C, float* __restrict__ C32,
+                   int splits) {
   using Cfg = GemmCfg<BN>;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
@@ -121,8 +148,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int tiles_n = N / BN;
   const int64_t tiles_m = (M + Cfg::BM - 1) / Cfg::BM;
-  const int64_t num_tiles = tiles_m * tiles_n;
   const int kblocks = K / Cfg::BK;
+  const int kbps = (kblocks + splits - 1) / splits;   // K blocks per split (every split non-empty)
+  const int64_t num_units = tiles_m * tiles_n * splits;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < Cfg::STAGES; s++) {
@@ -155,12 +183,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t issued_phase[Cfg::STAGES];
       for (int s = 0; s < Cfg::STAGES; s++) issued[s] = false, issued_phase[s] = 0;
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (int64_t u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+        const int64_t t = u / splits;
+        const int kb0 = (int)(u % splits) * kbps, kb1 = min(kb0 + kbps, kblocks);
         int64_t mb;
         int nb;
         gemm_tile_coords(t, tiles_n, tiles_m, mb, nb);
         const int m0 = (int)(mb * Cfg::BM), n0 = nb * BN;
-        for (int kb = 0; kb < kblocks; kb++) {
+        for (int kb = kb0; kb < kb1; kb++) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
           uint8_t* a_s = smem + stage * Cfg::STAGE_BYTES;
           uint8_t* b_s = a_s + Cfg::A_BYTES;
@@ -184,11 +214,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       constexpr uint32_t idesc = idesc_bf16(128, BN, false, true);
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (int64_t u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+        const int kb0 = (int)(u % splits) * kbps, kb1 = min(kb0 + kbps, kblocks);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
-        for (int kb = 0; kb < kblocks; kb++) {
+        for (int kb = kb0; kb < kb1; kb++) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a_addr = smem_u32(smem + stage * Cfg::STAGE_BYTES);
@@ -197,7 +228,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           for (int kk = 0; kk < Cfg::BK / 16; kk++) {
             const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(b_addr + kk * 2048, Cfg::BK * 128, 1024);
-            mma_ss(d_tmem, ad, bd, idesc, (kb | kk) != 0 ? 1u : 0u);
+            mma_ss(d_tmem, ad, bd, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
           }
           mma_commit(&empty[stage]);
           if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
@@ -219,7 +250,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int half = (warp - 2) >> 2;
     constexpr int HALF = BN / 2, CHUNKS = HALF / 32;
     uint32_t acc = 0, acc_phase = 0;
-    for (int64_t t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+    for (int64_t u = blockIdx.x; u < num_units; u += gridDim.x) {
+      const int64_t t = u / splits;
       int64_t mb;
       int nb;
       gemm_tile_coords(t, tiles_n, tiles_m, mb, nb);
@@ -243,7 +275,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[acc]);
         }
-        gemm_epilogue_chunk<EPI>(cur, bias, R, C, row, M, N, n0 + c * 32);
+        gemm_epilogue_chunk<EPI>(cur, bias, R, C, C32, row, M, N, n0 + c * 32);
       }
       acc ^= 1u;
       if (acc == 0) acc_phase ^= 1u;

@@ -50,19 +50,28 @@ inline int num_sms() {
 
 template <int BN, int EPI>
 hstu_status_t launch_gemm_bn(int64_t M, int N, int K, const bf16* A, const bf16* B, const bf16* bias,
-                             const bf16* R, bf16* C, cudaStream_t st) {
+                             const bf16* R, bf16* C, cudaStream_t st, float* C32 = nullptr,
+                             int splits = 1, int64_t b_rows = -1) {
   using Cfg = GemmCfg<BN>;
   CUtensorMap ta, tb;
+  // B may hold fewer than K rows: the tensor map's zero fill stands in for the rest
+  if (b_rows < 0 || b_rows > K) b_rows = K;
   if (!make_map_bf16(&ta, A, K, M, K, 64, 128)) return HSTU_ERR_CUDA;
-  if (!make_map_bf16(&tb, B, N, K, N, 64, 64)) return HSTU_ERR_CUDA;
+  if (!make_map_bf16(&tb, B, N, (uint64_t)b_rows, N, 64, 64)) return HSTU_ERR_CUDA;
   auto kern = gemm_tc_kernel<BN, EPI>;
   // set on every launch: the attribute is per device and the call is cheap
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM) !=
       cudaSuccess)
     return HSTU_ERR_CUDA;
-  const int64_t tiles = ((M + 127) / 128) * (N / BN);
-  const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
-  kern<<<grid, kGemmThreads, Cfg::SMEM, st>>>(ta, tb, M, N, K, bias, R, C);
+  // every split gets at least one K block
+  const int kblocks = K / Cfg::BK;
+  if (splits < 1) splits = 1;
+  if (splits > kblocks) splits = kblocks;
+  const int kbps = (kblocks + splits - 1) / splits;
+  splits = (kblocks + kbps - 1) / kbps;
+  const int64_t units = ((M + 127) / 128) * (N / BN) * splits;
+  const int grid = (int)(units < num_sms() ? units : num_sms());
+  kern<<<grid, kGemmThreads, Cfg::SMEM, st>>>(ta, tb, M, N, K, bias, R, C, C32, splits);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
@@ -80,6 +89,31 @@ hstu_status_t launch_gemm(int64_t M, int N, int K, const bf16* A, const bf16* B,
 inline hstu_status_t launch_gemm_f1(int64_t T, int n1, int d, const bf16* X, const bf16* W1,
                                     const bf16* b1, bf16* uvqk, cudaStream_t st) {
   return launch_gemm<EPI_BIAS_SILU>(T, n1, d, X, W1, b1, nullptr, uvqk, st);
+}
+
+// The backward GEMMs: A [M, K] row-major, B [K, N] row-major of which only the first b_rows rows
+// are read (the rest count as zeros), K % 64 == 0, N % 64 == 0.
+template <int EPI>
+hstu_status_t launch_gemm_ext(int64_t M, int N, int K, const bf16* A, const bf16* B,
+                              const bf16* bias, const bf16* R, bf16* C, float* C32, int splits,
+                              int64_t b_rows, cudaStream_t st) {
+  if (M >= (1LL << 31) || K % 64 != 0 || N % 64 != 0) return HSTU_ERR_UNSUPPORTED;
+  if (N % 256 == 0)
+    return launch_gemm_bn<256, EPI>(M, N, K, A, B, bias, R, C, st, C32, splits, b_rows);
+  if (N % 128 == 0)
+    return launch_gemm_bn<128, EPI>(M, N, K, A, B, bias, R, C, st, C32, splits, b_rows);
+  return launch_gemm_bn<64, EPI>(M, N, K, A, B, bias, R, C, st, C32, splits, b_rows);
+}
+
+// Split count for a weight-gradient GEMM: enough (tile, split) units for two waves over the SMs,
+// and at least 8 K blocks per split.
+inline int weight_grad_splits(int64_t M, int N, int K) {
+  const int bn = N % 256 == 0 ? 256 : (N % 128 == 0 ? 128 : 64);
+  const int64_t tiles = ((M + 127) / 128) * (N / bn);
+  const int64_t want = (2 * (int64_t)num_sms() + tiles - 1) / tiles;
+  const int64_t cap = (K / 64 + 7) / 8;
+  const int64_t s = want < cap ? want : cap;
+  return (int)(s < 1 ? 1 : s);
 }
 
 // Eq. 3 + residual: out[T, d] = G W2 + b2 + X.

@@ -183,6 +183,42 @@ hstu_status_t hstu_attention_bwd(const hstu_shape_t* shape, const void* uvqk,
                                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * hstu_layer_bwd -- backward of one layer ("Actions Speak Louder than Words" paper notes, section
+ * 3.1, Eqs. 1-3 and the residual Y = f2(G) + X), for training: given dY = dL/dY, the gradients of
+ * the loss with respect to X and every parameter of the layer,
+ *   dG = dY W2^T,  dW2 = G^T dY,  db2 = sum_t dY_t,
+ *   dU = dG * LayerNorm(AV),  dln_w, dln_b, dAV through the LayerNorm of each row,
+ *   dQ, dK, dV, dpos, dtime from dAV as hstu_attention_bwd computes them,
+ *   dZ = [dU | dV | dQ | dK] * SiLU'(X W1 + b1),  dW1 = X^T dZ,  db1 = sum_t dZ_t,
+ *   dX = dZ W1^T + dY.
+ * The activations come from the forward: `fwd_workspace` (fwd_workspace_bytes >=
+ * hstu_layer_fwd_workspace_size(shape)) is the workspace that a preceding hstu_layer_fwd call with
+ * the same shape, X, offsets, timestamps, weights and tables filled, not written since; its U, V, Q,
+ * K, AV and G are read, and X W1 + b1 is recomputed.  bf16 with d_qk = d_v = 64 and
+ * H*d_v <= 8192 (else HSTU_ERR_UNSUPPORTED).  Arguments as in hstu_layer_fwd (b2 is not needed),
+ * plus
+ *  dY             [T, d] bf16, the incoming gradient
+ *  dX             [T, d] bf16 output
+ *  dW1 [d, n1], db1 [n1], dW2 [H*d_v, d], db2 [d], dln_w [H*d_v], dln_b [H*d_v]
+ *                 fp32 outputs, 16-byte aligned
+ *  dpos_table, dtime_table   as in hstu_attention_bwd
+ *  workspace      hstu_layer_bwd_workspace_size(shape) bytes, 256-byte aligned
+ * dX may not overlap X, dY or either workspace, nor the two workspaces each other.  All outputs are
+ * overwritten (with T = 0: the parameter gradients are zero).  Bad offsets on the device are
+ * reported through hstu_get_device_status.  Asynchronous on `stream`.
+ */
+size_t hstu_layer_bwd_workspace_size(const hstu_shape_t* shape);
+hstu_status_t hstu_layer_bwd(const hstu_shape_t* shape, const void* X, const int64_t* seq_offsets,
+                             const int64_t* timestamps, const void* W1, const void* b1,
+                             const void* W2, const void* ln_w, const void* ln_b,
+                             const float* pos_table, const float* time_table,
+                             const float* alibi_slopes, float scale, const void* fwd_workspace,
+                             size_t fwd_workspace_bytes, const void* dY, void* dX, float* dW1,
+                             float* db1, float* dW2, float* db2, float* dln_w, float* dln_b,
+                             float* dpos_table, float* dtime_table, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/*
  * M-FALCON candidate scoring ("Actions Speak Louder than Words" paper notes, section 3.6; the
  * efficiency paragraph of "4.4 推荐模型的 Scaling").  A user's m candidates are scored in one pass
  * after its n history tokens: each candidate attends to the whole history and to itself, never to

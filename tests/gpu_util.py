@@ -10,6 +10,11 @@ from workloads import to_bf16_bits, widen_bf16
 F32_MAX_REL = 1e-4
 BF16_MAX_REL = 2e-2
 BF16_MEAN_REL = 2e-3
+# The layer backward's outputs pass through up to six bf16 roundings in a chain (the forward's
+# U|V|Q|K and G, the attention's P and dS operands, dAV, dU|dV|dQ|dK, dZ), each a relative error of
+# rms at most u/sqrt(3) with u = 2^-8 the bf16 unit roundoff.  Independent, they add to a relative
+# rms of at most sqrt(6) u / sqrt(3) = sqrt(2) u, which bounds mean|err| / rms(ref).
+BWD_MEAN_REL = float(np.sqrt(2.0) * 2.0 ** -8)
 
 
 def dev(a, dtype="bf16", device="cuda"):
@@ -50,6 +55,16 @@ def assert_bf16_close(got, ref, what=""):
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
     mx, mn = errors(got, ref)
     assert mx <= BF16_MAX_REL and mn <= BF16_MEAN_REL, \
+        f"{what}: max|err|/max|ref| = {mx:.3e}, mean|err|/rms(ref) = {mn:.3e}"
+    return mx, mn
+
+
+def assert_bwd_close(got, ref, what=""):
+    """The bf16 criteria with the mean bound of the layer backward's chain of roundings."""
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    mx, mn = errors(got, ref)
+    assert mx <= BF16_MAX_REL and mn <= BWD_MEAN_REL, \
         f"{what}: max|err|/max|ref| = {mx:.3e}, mean|err|/rms(ref) = {mn:.3e}"
     return mx, mn
 

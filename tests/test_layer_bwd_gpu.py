@@ -1,0 +1,146 @@
+"""Backward of one layer on the GPU against the fp64 oracle ("Actions Speak Louder than Words"
+paper notes, section 3.1, Eqs. 1-3 and the residual; training).  The activations the backward reads
+(U, V, Q, K, G) are the forward's bf16 values and the intermediate gradients dAV, dU|dV|dQ|dK and dZ
+enter the tensor-core products in bf16: every parameter gradient is held to the bf16 maximum bound
+and to a mean bound for that chain of roundings; dX, whose residual term dY dominates, is checked
+on the part the layer adds (dX - dY)."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from tests.gpu_util import assert_bwd_close, assert_layer_part_close, dev, host, round_bf16
+from workloads import random_case
+
+
+@pytest.fixture(scope="module")
+def hstu():
+    import hstu_sequential_transduction_layer_b200 as m
+    return m
+
+
+def _gpu_bwd(hstu, inp, dY):
+    w, p = inp.workload, inp.layers[0]
+    H, d = w.num_heads, w.d_model
+    n1, wv = 4 * H * 64, H * 64
+    has_t = inp.time_table is not None
+    ts = dev(inp.timestamps) if has_t else None
+    X, off = dev(inp.X), dev(inp.seq_offsets)
+    W1, b1, W2, b2 = dev(p.W1), dev(p.b1), dev(p.W2), dev(p.b2)
+    ln_w, ln_b = dev(p.ln_w), dev(p.ln_b)
+    pos, tim, ali = dev(inp.pos_table, "f32"), dev(inp.time_table, "f32"), dev(inp.alibi_slopes, "f32")
+    max_len = max(1, int(inp.lengths.max(initial=1)))
+    s = hstu.shape_for(X, off, H, 64, 64, max_len, inp.pos_table, inp.time_table, inp.ln_eps)
+    fws = hstu.alloc_workspace(s, "cuda")
+    hstu.hstu_layer_fwd(X, off, ts, W1, b1, W2, b2, ln_w, ln_b, pos, tim, ali, inp.scale,
+                        num_heads=H, max_seq_len=max_len, ln_eps=inp.ln_eps, workspace=fws)
+    nan = lambda *shape: torch.full(shape, float("nan"), dtype=torch.float32, device="cuda")
+    dX = torch.full((inp.T, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    out = hstu.hstu_layer_bwd(s, X, off, ts, W1, b1, W2, ln_w, ln_b, pos, tim, ali, inp.scale, fws,
+                              dev(dY), dX, nan(d, n1), nan(n1), nan(wv, d), nan(d), nan(wv),
+                              nan(wv), nan(*inp.pos_table.shape) if inp.pos_table is not None else None,
+                              nan(*inp.time_table.shape) if has_t else None)
+    torch.cuda.synchronize()
+    assert hstu.device_status() == hstu.HSTU_OK
+    return {k: (host(v) if v is not None else None) for k, v in out.items()}
+
+
+def _oracle_bwd(inp, dY):
+    w, p = inp.workload, inp.layers[0]
+    has_t = inp.time_table is not None
+    return oracle.layer_bwd(inp.seq_offsets, inp.X, p.W1, p.b1, p.W2, p.b2, p.ln_w, p.ln_b, dY,
+                            num_heads=w.num_heads, d_qk=64, d_v=64,
+                            timestamps=inp.timestamps if has_t else None,
+                            pos_table=inp.pos_table, time_table=inp.time_table,
+                            alibi_slopes=inp.alibi_slopes, scale=inp.scale, ln_eps=inp.ln_eps)
+
+
+def _case(seed, lengths, H, bias, P=96, Tb=24):
+    inp = random_case(seed, lengths, H * 64, H, 64, P=P, Tb=Tb, dtype="bf16",
+                      alibi=(bias == "alibi"))
+    if bias in ("pos", "none"):
+        inp.time_table = None
+    if bias == "none":
+        inp.pos_table = None
+    dY = round_bf16(np.random.default_rng(seed + 7).normal(0, 1.0, (inp.T, H * 64)))
+    return inp, dY
+
+
+def _compare(got, ref, dY, what):
+    assert_layer_part_close(got["dX"], ref["dX"], dY, f"dX ({what})")
+    for k in ("dW1", "db1", "dW2", "db2", "dln_w", "dln_b", "dpos", "dtime"):
+        if ref[k] is None:
+            assert got[k] is None
+        else:
+            assert_bwd_close(got[k], ref[k], f"{k} ({what})")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("seed,lengths,H,bias", [
+    (51, [300, 1, 129, 513], 2, "rab"),
+    (52, [256, 0, 1000], 2, "pos"),
+    (53, [700, 31], 2, "alibi"),
+    (54, [128, 255, 257], 1, "none"),
+    (55, [77, 400, 190], 4, "rab"),
+])
+def test_layer_backward_matches_oracle(hstu, seed, lengths, H, bias):
+    inp, dY = _case(seed, lengths, H, bias)
+    _compare(_gpu_bwd(hstu, inp, dY), _oracle_bwd(inp, dY), dY, f"{bias}, H={H}")
+
+
+@pytest.mark.gpu
+def test_layer_backward_longer_sequences(hstu):
+    """Two sequences of ~2k tokens at d = 512: many tiles of every GEMM, several K splits of the
+    weight gradients, and a ragged tail."""
+    inp, dY = _case(56, [2048, 1501], 8, "rab", P=1024, Tb=64)
+    _compare(_gpu_bwd(hstu, inp, dY), _oracle_bwd(inp, dY), dY, "2 x ~2k, d=512")
+
+
+@pytest.mark.gpu
+def test_layer_backward_full_size_properties(hstu):
+    """The long-sequence workload (8 x 8192 tokens, d = 512, 8 heads): db2 is the column sum of dY
+    (computed here in fp64 from the input), every output is finite, and the gradients are linear in
+    dY: doubling dY doubles them up to the order of the fp32 atomic reductions, which may move a
+    bf16 rounding of dQ (and so of dZ and dX) by one unit."""
+    inp = workloads.make_inputs("long_seq")
+    dY = round_bf16(np.random.default_rng(57).normal(0, 1.0, inp.X.shape).astype(np.float32))
+    g1 = _gpu_bwd(hstu, inp, dY)
+    np.testing.assert_allclose(g1["db2"], dY.astype(np.float64).sum(axis=0), rtol=1e-5, atol=1e-3)
+    for k, v in g1.items():
+        assert v is None or np.all(np.isfinite(v)), k
+    g2 = _gpu_bwd(hstu, inp, 2 * dY)
+    for k in ("dX", "dW1", "db1", "dW2", "dln_w", "dln_b", "dpos", "dtime"):
+        tol = 8e-3 if k == "dX" else 1e-3       # two bf16 units; fp32 sums
+        assert np.abs(g2[k] - 2 * g1[k]).max() <= tol * 2 * np.abs(g1[k]).max(), k
+
+
+def test_layer_bwd_host_validation(hstu):
+    lib = hstu.library()
+    fake = ctypes.c_void_p(1 << 20)
+    f = [fake] * 11
+    # head dim 128 is not implemented by the backward
+    s128 = hstu.make_shape(1, 10, 10, 256, 2, 128, 128, hstu.HSTU_BF16, 0, 0)
+    rc = lib.hstu_layer_bwd(ctypes.byref(s128), fake, fake, None, fake, fake, fake, fake, fake, None,
+                            None, None, ctypes.c_float(0.1), fake, 1 << 30, fake, fake, *f[:6],
+                            None, None, fake, 1 << 30, None)
+    assert rc == hstu.HSTU_ERR_UNSUPPORTED
+    s = hstu.make_shape(1, 10, 10, 128, 2, 64, 64, hstu.HSTU_BF16, 16, 0)
+    # a position table without its gradient
+    rc = lib.hstu_layer_bwd(ctypes.byref(s), fake, fake, None, fake, fake, fake, fake, fake, fake,
+                            None, None, ctypes.c_float(0.1), fake, 1 << 30, fake, fake, *f[:6],
+                            None, None, fake, 1 << 30, None)
+    assert rc == hstu.HSTU_ERR_INVALID_ARG
+    # a forward workspace smaller than the forward's
+    rc = lib.hstu_layer_bwd(ctypes.byref(s), fake, fake, None, fake, fake, fake, fake, fake, fake,
+                            None, None, ctypes.c_float(0.1), fake, 16, fake, ctypes.c_void_p(1 << 40),
+                            *f[:6], fake, None, fake, 1 << 30, None)
+    assert rc == hstu.HSTU_ERR_INVALID_ARG
+    # dX overlapping dY
+    rc = lib.hstu_layer_bwd(ctypes.byref(s), fake, fake, None, fake, fake, fake, fake, fake, fake,
+                            None, None, ctypes.c_float(0.1), ctypes.c_void_p(1 << 36), 1 << 30,
+                            fake, fake, *f[:6], fake, None, ctypes.c_void_p(1 << 38), 1 << 30, None)
+    assert rc == hstu.HSTU_ERR_INVALID_ARG
+    assert lib.hstu_layer_bwd_workspace_size(ctypes.byref(s)) > 0
