@@ -13,19 +13,23 @@
 //   dV_j += P^T dAV_i,  dK_j += dS^T Q_i                   (P^T, dS^T read from TMEM)
 //   dQ_i partial = dS K_j                                  (dS from shared memory, MN-major A)
 // and the dQ partial is added to global dQ (fp32) with 16-byte vector reductions.  Table gradients:
-// each pointwise warp writes its 32 x 32 block of dx skewed into shared memory (row r, column
-// (c - r) mod 32), so that every column holds two diagonals, whose sums (one bucket each, all
-// distances along a diagonal being equal) go to the global position gradient with one reduction
-// per diagonal; the time-bucket gradient accumulates per row and chunk in two registers (the
-// chunk's first bucket and the next one), in shared memory per item, then to global memory.
+// each pointwise warp sums the diagonals of its 32 x 32 block of dx systolically (lane l carries
+// the sum of diagonal c - l across the columns c, handing it one lane up per column; the sum
+// leaving lane 31 is complete), and each diagonal's sum (one bucket, all distances along a
+// diagonal being equal) goes to the global position gradient with one reduction; the position
+// bias itself comes from a per-warp window of the table at the block's 63 distances.
+// Time-bucket gradients: where the whole block is in one bucket or two (sorted timestamps), block
+// sums; elsewhere per row and chunk in two registers (the chunk's first bucket and the next one);
+// in shared memory per item, then to global memory.
 // dV and dK are owned by the item and stored directly.
 //
-// Per CTA (320 threads, one per SM): warp 0 producer (TMA of K_j, V_j, and Q_i, dAV_i per query tile
-// into a 2-deep ring; key and query timestamps), warp 1 single-thread MMA issuer, warps 2-9
-// pointwise (two per TMEM lane quadrant, each on 64 of the 128 query columns).
+// Per CTA (640 threads, one per SM): warp 0 producer (TMA of K_j, V_j, and Q_i, dAV_i per query tile
+// into a 2-deep ring; key and query timestamps), warp 1 single-thread MMA issuer, warps 2-3 idle,
+// warps 4-19 pointwise (four per TMEM lane quadrant, each on 32 of the 128 query columns, in two
+// 16-column halves so that 96 registers per thread suffice).
 // TMEM: S^T [0,128) | dP^T [128,256) | dV [256,320) | dK [320,384) | dQ partial [384,448); P^T and
-// dS^T (bf16) overwrite the S^T / dP^T columns each warp has read (a warp's 64 queries pack into 32
-// columns at the start of its own 64).
+// dS^T (bf16) overwrite the S^T / dP^T columns each warp has read (a warp's 32 queries pack into 16
+// columns at the start of its own 32).
 #pragma once
 
 #include <type_traits>
@@ -35,10 +39,9 @@
 namespace hstu {
 namespace tc {
 
-constexpr int BWD_THREADS = 320;
-constexpr int BWD_PW = 256;          // pointwise threads
-constexpr int BWD_PW_WARPS = 8;
-constexpr int BWD_POS_CAP = 8192;    // position buckets staged in shared memory
+constexpr int BWD_THREADS = 640;     // producer, MMA issuer, 2 idle warps, 16 pointwise
+constexpr int BWD_PW = 512;          // pointwise threads
+constexpr int BWD_PW_WARPS = 16;
 constexpr int BWD_TB_CAP = 256;
 
 struct BwdCfg {
@@ -54,9 +57,9 @@ struct BwdCfg {
   static constexpr int OFF_QTS32 = OFF_KTS + 128 * 8;       // [NST][128] int32, relative
   static constexpr int OFF_KTS32 = OFF_QTS32 + NST * 128 * 4;  // [128] int32, relative
   static constexpr int OFF_TFLAG = OFF_KTS32 + 128 * 4;     // [NST] query fits, [NST] key fits
-  static constexpr int OFF_XP = OFF_TFLAG + 64;             // [8 warps][32][32] float: dx blocks
-  static constexpr int OFF_POS = OFF_XP + BWD_PW_WARPS * 32 * 32 * 4;  // [POS_CAP] float pos table
-  static constexpr int OFF_TT = OFF_POS + BWD_POS_CAP * 4;    // [TB_CAP] float time table
+  static constexpr int OFF_PWIN = OFF_TFLAG + 64;           // [16 warps][64] float: table window
+  static constexpr int OFF_CAP = OFF_PWIN + BWD_PW_WARPS * 64 * 4;      // [16 warps][32] float
+  static constexpr int OFF_TT = OFF_CAP + BWD_PW_WARPS * 32 * 4;        // [TB_CAP] float time table
   static constexpr int OFF_DTT = OFF_TT + BWD_TB_CAP * 4;     // [TB_CAP] float its gradient
   static constexpr int OFF_BAR = OFF_DTT + BWD_TB_CAP * 4;
   static constexpr int SMEM = OFF_BAR + 256;
@@ -140,6 +143,20 @@ __device__ __forceinline__ void silu_and_grad(float x, float& silu, float& dsilu
   dsilu = sg * fmaf(x, 1.0f - sg, 1.0f);
 }
 
+// Called by a full warp, lane l holding the 4 consecutive timestamps t[4l .. 4l+3] of a 128-row
+// tile: a 4-bit mask, bit g set when rows 32g .. 32g+31 are in non-decreasing order.
+__device__ __forceinline__ int sorted_groups(const int64_t* t, int lane) {
+  bool srt = t[0] <= t[1] && t[1] <= t[2] && t[2] <= t[3];
+  const long long nxt = __shfl_down_sync(0xffffffffu, (long long)t[0], 1);
+  if ((lane & 7) != 7) srt = srt && t[3] <= nxt;
+  const unsigned b = __ballot_sync(0xffffffffu, srt);
+  int m = 0;
+#pragma unroll
+  for (int g = 0; g < 4; g++)
+    if (((b >> (8 * g)) & 0xffu) == 0xffu) m |= 1 << g;
+  return m;
+}
+
 // Bias modes of the backward kernel (compile-time): position table, time table, ALiBi.
 constexpr int BWD_POS = 1, BWD_TIME = 2, BWD_ALIBI = 4;
 
@@ -158,8 +175,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   int* qts32 = reinterpret_cast<int*>(smem + Cfg::OFF_QTS32);
   int* kts32 = reinterpret_cast<int*>(smem + Cfg::OFF_KTS32);
   int* tflag = reinterpret_cast<int*>(smem + Cfg::OFF_TFLAG);   // [0]: keys fit; [1 + st]: queries
-  float* xp_s = reinterpret_cast<float*>(smem + Cfg::OFF_XP);
-  float* pos_s = reinterpret_cast<float*>(smem + Cfg::OFF_POS);
+  // [0]: bit g set when the key tile's timestamps g*32 .. g*32+31 are non-decreasing;
+  // [1 + st]: the same for the query tile of stage st
+  int* tsort = tflag + 4;
+  float* pwin_s = reinterpret_cast<float*>(smem + Cfg::OFF_PWIN);
+  float* cap_s = reinterpret_cast<float*>(smem + Cfg::OFF_CAP);
   float* tt_s = reinterpret_cast<float*>(smem + Cfg::OFF_TT);
   float* dtt_s = reinterpret_cast<float*>(smem + Cfg::OFF_DTT);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
@@ -250,6 +270,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         }
         fits = __all_sync(0xffffffffu, fits);
         if (lane == 0) tflag[0] = fits ? 1 : 0;
+        const int sm = sorted_groups(kts + 4 * lane, lane);
+        if (lane == 0) tsort[0] = sm;
       }
       __syncwarp();
       if (lane == 0) {
@@ -279,6 +301,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           }
           fits = __all_sync(0xffffffffu, fits);
           if (lane == 0) tflag[1 + st] = fits ? 1 : 0;
+          const int sm = sorted_groups(qts + st * 128 + 4 * lane, lane);
+          if (lane == 0) tsort[1 + st] = sm;
         }
         __syncwarp();
         if (lane == 0) {
@@ -332,18 +356,18 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           if (!mbar_wait(pw_done, t & 1u, abort_flag)) { ok = false; break; }
           if (i == jt && !mbar_wait(dkv_empty, (k & 1u) ^ 1u, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          // dV_j += P^T dAV_i and dK_j += dS^T Q_i (P^T, dS^T from TMEM; the 64 queries of each
-          // pointwise half sit at the start of that half's columns)
+          // dV_j += P^T dAV_i and dK_j += dS^T Q_i (P^T, dS^T from TMEM; the 32 queries of each
+          // pointwise column group sit, packed, at the start of that group's 32 columns)
 #pragma unroll
           for (int kk = 0; kk < 8; kk++) {
-            const uint32_t pc = (kk & 3) * 8 + (kk >> 2) * 64;
+            const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;
             const uint32_t acc = (i > jt || kk > 0) ? 1u : 0u;
             mma_ts(tmem + Cfg::DV_COL, tmem + Cfg::S_COL + pc,
                    sdesc_sw128(do_addr + kk * 2048, Cfg::BOX, 1024), idesc_o, acc);
           }
 #pragma unroll
           for (int kk = 0; kk < 8; kk++) {
-            const uint32_t pc = (kk & 3) * 8 + (kk >> 2) * 64;
+            const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;
             const uint32_t acc = (i > jt || kk > 0) ? 1u : 0u;
             mma_ts(tmem + Cfg::DK_COL, tmem + Cfg::DP_COL + pc,
                    sdesc_sw128(q_addr + kk * 2048, Cfg::BOX, 1024), idesc_o, acc);
@@ -368,19 +392,22 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       mbar_drain(drain, 0);
     }
     __syncwarp();
-  } else if (warp >= 2) {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------------ pointwise warps
-    const int pw = warp - 2;
-    const int half = pw >> 2;            // query columns [64 half, 64 half + 64)
-    const int q = warp & 3;              // TMEM lane quadrant
+    // 16 warps: TMEM lane quadrant q = warp & 3 (keys q*32 .. q*32+31 of the tile), query columns
+    // 32 cg .. 32 cg + 31 (cg = (warp - 4) / 4), each 32 x 32 block in two 16-column halves
+    const int pw = warp - 4;
+    const int cg = pw >> 2;
+    const int q = warp & 3;
     const int r = q * 32 + lane;         // key row of S^T / dP^T, query row of the dQ partial
-    const int tid = threadIdx.x - 64;
-    const int c0 = half * 64;
+    const int tid = threadIdx.x - 128;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const int P = prm.P, Tb = prm.Tb;
-    const int dcap = P < BWD_POS_CAP ? P : BWD_POS_CAP;   // staged / accumulated buckets
     const int tcap = Tb < BWD_TB_CAP ? Tb : BWD_TB_CAP;
     const float scale = prm.scale;
+    const float m0 = lane > 0 ? 1.0f : 0.0f;
+    float* pwin = pwin_s + pw * 64;      // the position table at the block's 63 distances
+    float* cap = cap_s + pw * 32;        // completed diagonals of the systolic sums
     uint32_t k = 0, g = 0, t = 0, pw_cnt = 0;
     int staged_head = -1;
     bool ok = true;
@@ -394,12 +421,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const float* pos_h = has_pos ? prm.pos + (int64_t)h * P : nullptr;
       const float* tim_h = has_time ? prm.tim + (int64_t)h * Tb : nullptr;
       const float slope = alibi ? prm.alibi[h] : 0.0f;
-      if ((has_pos || has_time) && h != staged_head) {
+      if (has_time && h != staged_head) {
         if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;
-        if (has_pos)
-          for (int e = tid; e < dcap; e += BWD_PW) pos_s[e] = __ldg(pos_h + e);
-        if (has_time)
-          for (int e = tid; e < tcap; e += BWD_PW) tt_s[e] = __ldg(tim_h + e);
+        for (int e = tid; e < tcap; e += BWD_PW) tt_s[e] = __ldg(tim_h + e);
         staged_head = h;
         if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;
       }
@@ -407,157 +431,274 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const int j = k0 + r;                       // this thread's key (local index)
       const bool kvalid = j < n;
       const int64_t tj = has_time ? kts[r] : 0;
-      const int tj1 = has_time ? kts32[r] - 1 : 0;   // relative key time minus one
+      const int tk32 = has_time ? kts32[r] : 0;   // relative key time
       const bool keys_rel32 = has_time && tflag[0] != 0;
-      float* xp = xp_s + pw * (32 * 32);          // this warp's 32 x 32 block of dx, skewed
+      const int kq0 = k0 + q * 32;                // the warp's first key
       for (int i = jt; i < nt; i++, g++, t++) {
         const uint32_t st = g % Cfg::NST;
         const int q0 = i * ATT_BM;
-        const int64_t* qt_s = qts + st * 128;
-        const int* qt32 = qts32 + st * 128;
+        const int qc0 = q0 + 32 * cg;             // the warp's first query
+        const int64_t* qt_s = qts + st * 128 + 32 * cg;
+        const int* qt32 = qts32 + st * 128 + 32 * cg;
+        const int dbase = qc0 - kq0;              // distance of (lane 0, e = 0)
+        // the position table at distances dbase - 31 .. dbase + 32 (clamped), loaded before the
+        // MMA wait so that the wait hides the load
+        float wv0 = 0.0f, wv1 = 0.0f;
+        if (has_pos) {
+          const int d0 = dbase - 31 + lane, d1 = dbase + 1 + lane;
+          wv0 = __ldg(pos_h + (d0 < 0 ? 0 : (d0 < P - 1 ? d0 : P - 1)));
+          wv1 = __ldg(pos_h + (d1 < 0 ? 0 : (d1 < P - 1 ? d1 : P - 1)));
+        }
         // the stage's query timestamps are published with its Q/dAV tiles
         if (has_time && !mbar_wait(&q_full[st], (g / Cfg::NST) & 1u, abort_flag)) { ok = false; break; }
         if (!mbar_wait(sp_full, t & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
-#pragma unroll 1
-        for (int ch = 0; ch < 2; ch++) {
-          const int cc = c0 + ch * 32;
-          uint32_t sv[32], dpv[32], pk[16], dk[16];
-          tmem_ld32(t_lane + Cfg::S_COL + cc, sv);
-          tmem_ld32(t_lane + Cfg::DP_COL + cc, dpv);
-          tmem_ld_wait(sv);
-          tmem_ld_wait(dpv);
-          // time-bucket gradient: the chunk's buckets along a row are those of its first query
-          // and the next one up (queries are later in time along the row); others go directly
-          int tb_first = 0;
-          float acc_lo = 0.0f, acc_hi = 0.0f;
-          if (has_time) {
-            const int b = time_bucket(qt_s[cc], tj);
-            tb_first = b < Tb - 1 ? b : Tb - 1;
+        uint32_t sv[16], dpv[16];
+        tmem_ld16(t_lane + Cfg::S_COL + 32 * cg, sv);
+        tmem_ld16(t_lane + Cfg::DP_COL + 32 * cg, dpv);
+        if (has_pos) {
+          pwin[lane] = wv0;
+          pwin[32 + lane] = wv1;
+          __syncwarp();
+        }
+        // Fast path when every score of the block is valid (off the diagonal, inside the
+        // sequence) and the time bucket is the same for the whole block, or takes two values split
+        // by one threshold (sorted timestamps, the extreme corners' buckets equal or adjacent).
+        const bool full = dbase - 31 >= 0 && (int64_t)(qc0 + 31) < n && (int64_t)(kq0 + 31) < n;
+        const bool pos_one = has_pos && full && dbase - 31 >= P - 1;   // all in bucket P - 1
+        int tb_u = -1, tmode = 0;                 // 1: one bucket tb_u; 2: tb_u and tb_u + 1
+        int thr = 0;                              // two buckets: relative dt >= thr is tb_u + 1
+        if (has_time && full && ((tsort[0] >> q) & 1) && ((tsort[1 + st] >> cg) & 1)) {
+          const int b0 = time_bucket(qt_s[0], kts[q * 32 + 31]);
+          const int b1 = time_bucket(qt_s[31], kts[q * 32]);
+          const int c0b = b0 < Tb - 1 ? b0 : Tb - 1, c1b = b1 < Tb - 1 ? b1 : Tb - 1;
+          if (c0b == c1b) {
+            tb_u = c0b;
+            tmode = 1;
+          } else if (c1b == c0b + 1 && keys_rel32 && tflag[1 + st] != 0 && c1b <= 30) {
+            // bucket(dt) >= c1b  <=>  dt + 1 >= 2^c1b (also when c1b is the clamped last one)
+            tb_u = c0b;
+            tmode = 2;
+            thr = (1 << c1b) - 1;
           }
-          // the element loop, with 32-bit time buckets when the tile's timestamps fit
-          auto elements = [&](auto rel_tag) {
+        }
+        const bool fast = full && (!has_time || tmode != 0);
+        const float* pl = pwin + 31 - lane;       // pl[e]: position bias of (lane, e)
+        // time-bucket gradient of the general loop: the block's buckets along a row are those
+        // of its first query and the next one up (queries are later in time along the row);
+        // others go directly
+        int tb_first = 0;
+        if (has_time && !fast) {
+          const int b = time_bucket(qt_s[0], tj);
+          tb_first = b < Tb - 1 ? b : Tb - 1;
+        }
+        const float tlo = (has_time && fast) ? tt_s[tb_u] : 0.0f;
+        const float thi = (has_time && tmode == 2) ? tt_s[tb_u + 1] : 0.0f;
+        const float pone = pos_one ? pl[0] : 0.0f;  // every window entry is the last bucket
+        const float al0 = -slope * (float)(dbase - lane);
+        float acc_u = 0.0f, acc_h = 0.0f, acc_pu = 0.0f, acc_lo = 0.0f, acc_hi = 0.0f;
+        float sacc = 0.0f;                        // systolic diagonal sum (position gradient)
+#pragma unroll 1
+        for (int hf = 0; hf < 2; hf++) {
+          tmem_ld_wait16(sv);
+          tmem_ld_wait16(dpv);
+          uint32_t pk[8], dk[8];
+          const float* plh = pl + 16 * hf;
+          const int* qt32h = qt32 + 16 * hf;
+          const int64_t* qth = qt_s + 16 * hf;
+          float* caph = cap + 16 * hf - 1;        // caph[ee]: diagonal completed at e = 16 hf + ee
+          const float alh = fmaf(-slope, (float)(16 * hf), al0);
+          const int iq0 = qc0 + 16 * hf;
+          // one step of the systolic diagonal sums: lane l holds the sum of diagonal e - l; the
+          // sums move up one lane per column, and lane 31's (complete) is parked in `cap`
+          auto systolic = [&](int ee, float dx) {
+            if (ee == 0 && hf == 0) {
+              sacc = dx;
+            } else {
+              if (lane == 31) caph[ee] = sacc;
+              sacc = fmaf(__shfl_up_sync(0xffffffffu, sacc, 1), m0, dx);
+            }
+          };
+          // the fast element loop: no masks; the time bias one or two constants
+          auto fast16 = [&](auto tm_tag, auto po_tag) {
+            constexpr int TM = decltype(tm_tag)::value;
+            constexpr bool PO = decltype(po_tag)::value;
+#pragma unroll
+            for (int ee = 0; ee < 16; ee += 2) {
+              float a2[2], d2[2];
+#pragma unroll
+              for (int u = 0; u < 2; u++) {
+                float x = __uint_as_float(sv[ee + u]);
+                bool hi = false;
+                if (TM == 2) {
+                  hi = qt32h[ee + u] - tk32 >= thr;
+                  x += hi ? thi : tlo;
+                } else if (TM == 1) {
+                  x += tlo;
+                }
+                if (has_pos) x += PO ? pone : plh[ee + u];
+                if (alibi) x += fmaf(-slope, (float)(ee + u), alh);
+                float sl, dsl;
+                silu_and_grad(x, sl, dsl);
+                const float dx = scale * dsl * __uint_as_float(dpv[ee + u]);
+                a2[u] = scale * sl;
+                d2[u] = dx;
+                if (PO) acc_pu += dx;
+                else if (has_pos) systolic(ee + u, dx);
+                if (TM != 0) acc_u += dx;
+                if (TM == 2) acc_h += hi ? dx : 0.0f;
+              }
+              pk[ee / 2] = pack_bf16x2(a2[0], a2[1]);
+              dk[ee / 2] = pack_bf16x2(d2[0], d2[1]);
+            }
+          };
+          // the general element loop (masks, per-score time buckets), with 32-bit time buckets
+          // when the tile's timestamps fit
+          auto gen16 = [&](auto rel_tag) {
             constexpr bool REL32 = decltype(rel_tag)::value;
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float a2[2], d2[2];
+            for (int ee = 0; ee < 16; ee += 2) {
+              float a2[2], d2[2];
 #pragma unroll
-            for (int u = 0; u < 2; u++) {
-              const int iq = q0 + cc + e + u;        // query (local index)
-              const int dist = iq - j;
-              const bool valid = kvalid && iq < n && dist >= 0;
-              float bias = 0.0f;
-              int tb = 0;
-              if (alibi) bias = -slope * (float)dist;
-              if (has_pos) {
-                const int pb = dist < 0 ? 0 : (dist < P - 1 ? dist : P - 1);
-                bias += pb < BWD_POS_CAP ? pos_s[pb] : __ldg(pos_h + pb);
-              }
-              if (has_time) {
-                if (REL32) {
-                  // floor(log2(1 + max(ti - tj, 0))) = 31 - clz(max(ti - tj, 0) + 1)
-                  const int dd = qt32[cc + e + u] - tj1;
-                  tb = 31 - __clz(dd > 1 ? dd : 1);
-                } else {
-                  tb = time_bucket(qt_s[cc + e + u], tj);
+              for (int u = 0; u < 2; u++) {
+                const int iq = iq0 + ee + u;         // query (local index)
+                const int dist = iq - j;
+                const bool valid = kvalid && iq < n && dist >= 0;
+                float bias = 0.0f;
+                int tb = 0;
+                if (alibi) bias = -slope * (float)dist;
+                if (has_pos) bias += plh[ee + u];
+                if (has_time) {
+                  if (REL32) {
+                    // floor(log2(1 + max(ti - tj, 0))) = 31 - clz(max(ti - tj, 0) + 1)
+                    const int dd = qt32h[ee + u] - tk32 + 1;
+                    tb = 31 - __clz(dd > 1 ? dd : 1);
+                  } else {
+                    tb = time_bucket(qth[ee + u], tj);
+                  }
+                  tb = tb < Tb - 1 ? tb : Tb - 1;
+                  bias += tt_s[tb];
                 }
-                tb = tb < Tb - 1 ? tb : Tb - 1;
-                bias += tt_s[tb];
-              }
-              float sl, dsl;
-              silu_and_grad(__uint_as_float(sv[e + u]) + bias, sl, dsl);
-              const float av = valid ? scale * sl : 0.0f;
-              const float dx = valid ? scale * dsl * __uint_as_float(dpv[e + u]) : 0.0f;
-              a2[u] = av;
-              d2[u] = dx;
-              // row `lane`, column (c - lane) mod 32: diagonal c - lane becomes a column
-              if (has_pos) xp[lane * 32 + ((e + u - lane) & 31)] = dx;
-              if (has_time) {
-                const int db = tb - tb_first;
-                acc_lo += db == 0 ? dx : 0.0f;
-                acc_hi += db == 1 ? dx : 0.0f;
-                // rare (a step of two or more buckets inside a chunk, near the diagonal): a
-                // warp vote keeps the shared-memory atomic off the common path
-                const bool far = valid && (db < 0 || db > 1);
-                if (__any_sync(0xffffffffu, far)) {
-                  if (far) atomicAdd(&dtt_s[tb], dx);
+                float sl, dsl;
+                silu_and_grad(__uint_as_float(sv[ee + u]) + bias, sl, dsl);
+                const float dx = valid ? scale * dsl * __uint_as_float(dpv[ee + u]) : 0.0f;
+                a2[u] = valid ? scale * sl : 0.0f;
+                d2[u] = dx;
+                if (has_pos) systolic(ee + u, dx);
+                if (has_time) {
+                  const int db = tb - tb_first;
+                  acc_lo += db == 0 ? dx : 0.0f;
+                  acc_hi += db == 1 ? dx : 0.0f;
+                  // rare (a step of two or more buckets inside a block, near the diagonal): a
+                  // warp vote keeps the shared-memory atomic off the common path
+                  const bool far = valid && (db < 0 || db > 1);
+                  if (__any_sync(0xffffffffu, far)) {
+                    if (far) atomicAdd(&dtt_s[tb], dx);
+                  }
                 }
               }
+              pk[ee / 2] = pack_bf16x2(a2[0], a2[1]);
+              dk[ee / 2] = pack_bf16x2(d2[0], d2[1]);
             }
-            pk[e / 2] = pack_bf16x2(a2[0], a2[1]);
-            dk[e / 2] = pack_bf16x2(d2[0], d2[1]);
-          }
           };
-          if (has_time && keys_rel32 && tflag[1 + st] != 0) elements(std::true_type{});
-          else elements(std::false_type{});
-          if (has_time) {
-            // one atomic per run of lanes with the same first bucket: the rows of a warp are 32
-            // consecutive keys, so equal first buckets are contiguous; a segmented inclusive scan
-            // leaves each run's sums in its last lane
-            const int prev = __shfl_up_sync(0xffffffffu, tb_first, 1);
-            const unsigned heads = __ballot_sync(0xffffffffu, lane == 0 || prev != tb_first);
-            const int seg0 = 31 - __clz(heads & (0xffffffffu >> (31 - lane)));
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-              const float lo = __shfl_up_sync(0xffffffffu, acc_lo, o);
-              const float hi = __shfl_up_sync(0xffffffffu, acc_hi, o);
-              if (lane - o >= seg0) {
-                acc_lo += lo;
-                acc_hi += hi;
-              }
+          if (fast) {
+            if (tmode == 2) {
+              if (pos_one) fast16(std::integral_constant<int, 2>{}, std::true_type{});
+              else fast16(std::integral_constant<int, 2>{}, std::false_type{});
+            } else if (has_time) {
+              if (pos_one) fast16(std::integral_constant<int, 1>{}, std::true_type{});
+              else fast16(std::integral_constant<int, 1>{}, std::false_type{});
+            } else {
+              if (pos_one) fast16(std::integral_constant<int, 0>{}, std::true_type{});
+              else fast16(std::integral_constant<int, 0>{}, std::false_type{});
             }
-            const bool last = lane == 31 || ((heads >> (lane + 1)) & 1u);
-            if (last) {
-              if (acc_lo != 0.0f) atomicAdd(&dtt_s[tb_first], acc_lo);
-              if (acc_hi != 0.0f) atomicAdd(&dtt_s[tb_first + 1], acc_hi);
-            }
+          } else if (has_time && keys_rel32 && tflag[1 + st] != 0) {
+            gen16(std::true_type{});
+          } else {
+            gen16(std::false_type{});
           }
-          if (has_pos) {
-            // diagonal sums of the warp's 32 x 32 block: lane k reads column k, which holds the
-            // diagonals c - r = k (rows r < 32 - k) and c - r = k - 32 (the other rows)
-            __syncwarp();
-            float dpp = 0.0f, dpn = 0.0f;
-#pragma unroll 8
-            for (int rr = 0; rr < 32; rr++) {
-              const float v = xp[rr * 32 + lane];
-              if (rr + lane < 32) dpp += v; else dpn += v;
-            }
-            __syncwarp();
-            // distance of diagonal delta: (q0 + cc) - (k0 + q*32) + delta
-            const int base = q0 + cc - (k0 + q * 32);
-            const int d1 = base + lane, d2 = base + lane - 32;
-            float* dpos_h = prm.dpos + (int64_t)h * P;
-            if (dpp != 0.0f && d1 >= 0) atomicAdd(dpos_h + (d1 < P - 1 ? d1 : P - 1), dpp);
-            if (dpn != 0.0f && d2 >= 0) atomicAdd(dpos_h + (d2 < P - 1 ? d2 : P - 1), dpn);
+          // P^T and dS^T (bf16 pairs) into the first 8 of the 16 S^T / dP^T columns this half
+          // has read; then the next half's loads
+          tmem_st8(t_lane + Cfg::S_COL + 32 * cg + 8 * hf, pk);
+          tmem_st8(t_lane + Cfg::DP_COL + 32 * cg + 8 * hf, dk);
+          if (hf == 0) {
+            tmem_ld16(t_lane + Cfg::S_COL + 32 * cg + 16, sv);
+            tmem_ld16(t_lane + Cfg::DP_COL + 32 * cg + 16, dpv);
           }
-          // P^T and dS^T into the S^T / dP^T columns this warp has read
-          tmem_st16(t_lane + Cfg::S_COL + c0 + ch * 16, pk);
-          tmem_st16(t_lane + Cfg::DP_COL + c0 + ch * 16, dk);
-          // dS^T into shared memory as the MN-major A operand of dQ = dS K_j: row = key r, 128-byte
-          // swizzled rows of 64 queries per panel; this chunk's 32 queries are 4 16-byte units
+          // dS^T into shared memory as the MN-major A operand of dQ = dS K_j: row = key r,
+          // 128-byte swizzled rows of 64 queries per panel; this half's 16 queries are 2 units
 #pragma unroll
-          for (int v = 0; v < 4; v++) {
-            const int uu = (cc % 64) / 8 + v;
-            uint8_t* dst = ds_s + half * Cfg::BOX + r * 128 + ((uu ^ (r & 7)) * 16);
+          for (int v = 0; v < 2; v++) {
+            const int uu = 4 * (cg & 1) + 2 * hf + v;
+            uint8_t* dst = ds_s + (cg >> 1) * Cfg::BOX + r * 128 + ((uu ^ (r & 7)) * 16);
             *reinterpret_cast<uint4*>(dst) = make_uint4(dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]);
           }
+        }
+        // table gradients of the block
+        if (has_time && fast) {
+          // the block's sums in bucket tb_u (and tb_u + 1)
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            acc_u += __shfl_xor_sync(0xffffffffu, acc_u, o);
+            if (tmode == 2) acc_h += __shfl_xor_sync(0xffffffffu, acc_h, o);
+          }
+          if (lane == 0) {
+            if (acc_u - acc_h != 0.0f) atomicAdd(&dtt_s[tb_u], acc_u - acc_h);
+            if (acc_h != 0.0f) atomicAdd(&dtt_s[tb_u + 1], acc_h);
+          }
+        } else if (has_time) {
+          // one atomic per run of lanes with the same first bucket: the rows of a warp are 32
+          // consecutive keys, so equal first buckets are contiguous; a segmented inclusive scan
+          // leaves each run's sums in its last lane
+          const int prev = __shfl_up_sync(0xffffffffu, tb_first, 1);
+          const unsigned heads = __ballot_sync(0xffffffffu, lane == 0 || prev != tb_first);
+          const int seg0 = 31 - __clz(heads & (0xffffffffu >> (31 - lane)));
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const float lo = __shfl_up_sync(0xffffffffu, acc_lo, o);
+            const float hi = __shfl_up_sync(0xffffffffu, acc_hi, o);
+            if (lane - o >= seg0) {
+              acc_lo += lo;
+              acc_hi += hi;
+            }
+          }
+          const bool last = lane == 31 || ((heads >> (lane + 1)) & 1u);
+          if (last) {
+            if (acc_lo != 0.0f) atomicAdd(&dtt_s[tb_first], acc_lo);
+            if (acc_hi != 0.0f) atomicAdd(&dtt_s[tb_first + 1], acc_hi);
+          }
+        }
+        if (pos_one && fast) {
+          // every distance of the block is clamped to the last bucket
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) acc_pu += __shfl_xor_sync(0xffffffffu, acc_pu, o);
+          if (lane == 0 && acc_pu != 0.0f) atomicAdd(prm.dpos + (int64_t)h * P + (P - 1), acc_pu);
+        } else if (has_pos) {
+          // lane l: diagonal 31 - l in the systolic sum, diagonal l - 31 parked in cap[l]
+          __syncwarp();
+          const float parked = lane < 31 ? cap[lane] : 0.0f;
+          __syncwarp();
+          const int da = dbase + 31 - lane, db = dbase + lane - 31;
+          float* dpos_h = prm.dpos + (int64_t)h * P;
+          if (sacc != 0.0f && da >= 0) atomicAdd(dpos_h + (da < P - 1 ? da : P - 1), sacc);
+          if (parked != 0.0f && db >= 0) atomicAdd(dpos_h + (db < P - 1 ? db : P - 1), parked);
         }
         tmem_st_wait();
         tc_fence_before();
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(pw_done);
-        // the dQ partial of query tile i: TMEM lane = query row; this warp's 32 of the 64 columns
+        // the dQ partial of query tile i: TMEM lane = query row; this warp's 16 of the 64 columns
         if (!mbar_wait(dq_full, t & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         {
-          uint32_t ov[32];
-          tmem_ld32(t_lane + Cfg::DQ_COL + half * 32, ov);
-          tmem_ld_wait(ov);
+          uint32_t ov[16];
+          tmem_ld16(t_lane + Cfg::DQ_COL + 16 * cg, ov);
+          tmem_ld_wait16(ov);
           if (q0 + r < n) {
-            float* dst = prm.dq + (row0 + q0 + r) * (int64_t)(H * 64) + h * 64 + half * 32;
+            float* dst = prm.dq + (row0 + q0 + r) * (int64_t)(H * 64) + h * 64 + 16 * cg;
 #pragma unroll
-            for (int v = 0; v < 8; v++)
+            for (int v = 0; v < 4; v++)
               red_add_v4(dst + 4 * v, __uint_as_float(ov[4 * v]), __uint_as_float(ov[4 * v + 1]),
                          __uint_as_float(ov[4 * v + 2]), __uint_as_float(ov[4 * v + 3]));
           }
@@ -567,20 +708,20 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         if (lane == 0) mbar_arrive(dq_empty);
       }
       if (!ok) break;
-      // dV_j and dK_j of this item: TMEM lane = key row
+      // dV_j and dK_j of this item: TMEM lane = key row; this warp's 16 of the 64 columns
       if (!mbar_wait(dkv_full, k & 1u, abort_flag)) break;
       tc_fence_after();
       {
-        uint32_t vv[32], kv[32];
-        tmem_ld32(t_lane + Cfg::DV_COL + half * 32, vv);
-        tmem_ld32(t_lane + Cfg::DK_COL + half * 32, kv);
-        tmem_ld_wait(vv);
-        tmem_ld_wait(kv);
+        uint32_t vv[16], kv[16];
+        tmem_ld16(t_lane + Cfg::DV_COL + 16 * cg, vv);
+        tmem_ld16(t_lane + Cfg::DK_COL + 16 * cg, kv);
+        tmem_ld_wait16(vv);
+        tmem_ld_wait16(kv);
         if (kvalid) {
-          float* dvr = prm.dv + (row0 + j) * (int64_t)(H * 64) + h * 64 + half * 32;
-          float* dkr = prm.dk + (row0 + j) * (int64_t)(H * 64) + h * 64 + half * 32;
+          float* dvr = prm.dv + (row0 + j) * (int64_t)(H * 64) + h * 64 + 16 * cg;
+          float* dkr = prm.dk + (row0 + j) * (int64_t)(H * 64) + h * 64 + 16 * cg;
 #pragma unroll
-          for (int v = 0; v < 8; v++) {
+          for (int v = 0; v < 4; v++) {
             reinterpret_cast<float4*>(dvr)[v] =
                 make_float4(__uint_as_float(vv[4 * v]), __uint_as_float(vv[4 * v + 1]),
                             __uint_as_float(vv[4 * v + 2]), __uint_as_float(vv[4 * v + 3]));
@@ -596,12 +737,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       // table gradients of this item to global memory
       if (has_time) {
         if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;
-        if (has_time)
-          for (int e = tid; e < tcap; e += BWD_PW) {
-            const float v = dtt_s[e];
-            if (v != 0.0f) atomicAdd(prm.dtime + (int64_t)h * Tb + e, v);
-            dtt_s[e] = 0.0f;
-          }
+        for (int e = tid; e < tcap; e += BWD_PW) {
+          const float v = dtt_s[e];
+          if (v != 0.0f) atomicAdd(prm.dtime + (int64_t)h * Tb + e, v);
+          dtt_s[e] = 0.0f;
+        }
         if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;
       }
     }
