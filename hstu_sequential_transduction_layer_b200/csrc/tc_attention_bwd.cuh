@@ -12,7 +12,7 @@
 //   pointwise: P^T = scale*SiLU(S^T + bias^T), dS^T = scale*SiLU'(.) * dP^T, masked to j <= i
 //   dV_j += P^T dAV_i,  dK_j += dS^T Q_i                   (P^T, dS^T read from TMEM)
 //   dQ_i partial = dS K_j                                  (dS from shared memory, MN-major A)
-// and the dQ partial is added to global dQ (fp32) with 16-byte vector reductions.  Table gradients:
+// and the dQ partial, staged in shared memory, is added to global dQ (fp32) with TMA reductions.  Table gradients:
 // each pointwise warp sums the diagonals of its 32 x 32 block of dx systolically (lane l carries
 // the sum of diagonal c - l across the columns c, handing it one lane up per column; the sum
 // leaving lane 31 is complete), and each diagonal's sum (one bucket, all distances along a
@@ -24,7 +24,8 @@
 // dV and dK are owned by the item and stored directly.
 //
 // Per CTA (640 threads, one per SM): warp 0 producer (TMA of K_j, V_j, and Q_i, dAV_i per query tile
-// into a 2-deep ring; key and query timestamps), warp 1 single-thread MMA issuer, warps 2-3 idle,
+// into a 2-deep ring; key and query timestamps), warp 1 single-thread MMA issuer, warp 2 the dQ
+// TMA reductions, warp 3 idle,
 // warps 4-19 pointwise (four per TMEM lane quadrant, each on 32 of the 128 query columns, in two
 // 16-column halves so that 96 registers per thread suffice).
 // TMEM: S^T [0,128) | dP^T [128,256) | dV [256,320) | dK [320,384) | dQ partial [384,448); P^T and
@@ -52,7 +53,9 @@ struct BwdCfg {
   static constexpr int OFF_Q = OFF_V + BOX;                 // [NST] Q tiles
   static constexpr int OFF_DO = OFF_Q + NST * BOX;          // [NST] dAV tiles
   static constexpr int OFF_DS = OFF_DO + NST * BOX;         // dS^T, two 16 KB panels (MN-major A)
-  static constexpr int OFF_QTS = OFF_DS + 2 * BOX;          // [NST][128] int64 query timestamps
+  static constexpr int OFF_STG = OFF_DS + 2 * BOX;          // [2] dQ partial, fp32, 2 swizzled boxes
+  static constexpr int STG_BYTES = 128 * 64 * 4;            //     of 32 columns x 128 rows
+  static constexpr int OFF_QTS = OFF_STG + 2 * STG_BYTES;   // [NST][128] int64 query timestamps
   static constexpr int OFF_KTS = OFF_QTS + NST * 128 * 8;   // [128] int64 key timestamps
   static constexpr int OFF_QTS32 = OFF_KTS + 128 * 8;       // [NST][128] int32, relative
   static constexpr int OFF_KTS32 = OFF_QTS32 + NST * 128 * 4;  // [128] int32, relative
@@ -163,7 +166,7 @@ constexpr int BWD_POS = 1, BWD_TIME = 2, BWD_ALIBI = 4;
 template <int BM>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     attention_bwd_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tdo,
-                         BwdParams prm, AttnSchedule sch) {
+                         const __grid_constant__ CUtensorMap tdq, BwdParams prm, AttnSchedule sch) {
   using Cfg = BwdCfg;
   using namespace sm100;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -180,6 +183,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   int* tsort = tflag + 4;
   float* pwin_s = reinterpret_cast<float*>(smem + Cfg::OFF_PWIN);
   float* cap_s = reinterpret_cast<float*>(smem + Cfg::OFF_CAP);
+  uint8_t* stg_s = smem + Cfg::OFF_STG;
   float* tt_s = reinterpret_cast<float*>(smem + Cfg::OFF_TT);
   float* dtt_s = reinterpret_cast<float*>(smem + Cfg::OFF_DTT);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
@@ -195,7 +199,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   uint64_t* dkv_empty = bars + 11;
   uint64_t* pw_bar = bars + 12;
   uint64_t* drain = bars + 13;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* stg_full = bars + 14;     // [2] dQ partial staged (16 pointwise warps)
+  uint64_t* stg_empty = bars + 16;    // [2] staged dQ partial read by the TMA reduce
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -223,10 +229,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     mbar_init(dkv_empty, BWD_PW_WARPS);
     mbar_init(pw_bar, BWD_PW);
     mbar_init(drain, 1);
+    for (int b = 0; b < 2; b++) {
+      mbar_init(&stg_full[b], BWD_PW_WARPS);
+      mbar_init(&stg_empty[b], 1);
+    }
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tm);
     prefetch_tensormap(&tdo);
+    prefetch_tensormap(&tdq);
   }
   for (int e = threadIdx.x; e < BWD_TB_CAP; e += BWD_THREADS) dtt_s[e] = 0.0f;
   if (warp == 1) {
@@ -390,6 +401,35 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       }
       mma_commit(drain);
       mbar_drain(drain, 0);
+    }
+    __syncwarp();
+  } else if (warp == 2) {
+    // ------------------------------------------------------------------ dQ reducer
+    // Adds each query tile's dQ partial, staged by the pointwise warps, to global dQ with two TMA
+    // reductions; rows past the sequence hold zeros (their dS is masked), so the tile can run
+    // into the next sequence, and rows past T are not written.
+    if (lane == 0) {
+      uint32_t t = 0;
+      bool ok = true;
+      for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const int64_t item = sch.items[it];
+        const int64_t seq = item & 0xffffffffLL;
+        const int jt = (int)((item >> 32) & 0xffff), h = (int)(item >> 48);
+        const int64_t row0 = sch.seqinfo[2 * seq], n = sch.seqinfo[2 * seq + 1];
+        const int nt = (int)((n + ATT_BN - 1) / ATT_BN);
+        for (int i = jt; i < nt; i++, t++) {
+          const uint32_t sb = t & 1u;
+          if (!mbar_wait(&stg_full[sb], (t >> 1) & 1u, abort_flag)) { ok = false; break; }
+          const uint8_t* src = stg_s + sb * Cfg::STG_BYTES;
+          const int y = (int)row0 + i * ATT_BM;
+          tma_reduce_add_2d(&tdq, src, h * 64, y);
+          tma_reduce_add_2d(&tdq, src + 128 * 128, h * 64 + 32, y);
+          bulk_commit();
+          bulk_wait_read_all();
+          mbar_arrive(&stg_empty[sb]);
+        }
+      }
+      bulk_wait_all();
     }
     __syncwarp();
   } else if (warp >= 4) {
@@ -668,26 +708,39 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             if (acc_hi != 0.0f) atomicAdd(&dtt_s[tb_first + 1], acc_hi);
           }
         }
+        // the position gradient's two sums per lane (the global reductions are issued after the
+        // arrive below: an arrive releases this warp's earlier writes, so reductions still in
+        // flight would hold it back)
+        float pg0 = 0.0f, pg1 = 0.0f;
+        int pd0 = -1, pd1 = -1;
         if (pos_one && fast) {
           // every distance of the block is clamped to the last bucket
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) acc_pu += __shfl_xor_sync(0xffffffffu, acc_pu, o);
-          if (lane == 0 && acc_pu != 0.0f) atomicAdd(prm.dpos + (int64_t)h * P + (P - 1), acc_pu);
+          if (lane == 0) {
+            pg0 = acc_pu;
+            pd0 = P - 1;
+          }
         } else if (has_pos) {
           // lane l: diagonal 31 - l in the systolic sum, diagonal l - 31 parked in cap[l]
           __syncwarp();
-          const float parked = lane < 31 ? cap[lane] : 0.0f;
+          pg1 = lane < 31 ? cap[lane] : 0.0f;
           __syncwarp();
           const int da = dbase + 31 - lane, db = dbase + lane - 31;
-          float* dpos_h = prm.dpos + (int64_t)h * P;
-          if (sacc != 0.0f && da >= 0) atomicAdd(dpos_h + (da < P - 1 ? da : P - 1), sacc);
-          if (parked != 0.0f && db >= 0) atomicAdd(dpos_h + (db < P - 1 ? db : P - 1), parked);
+          pg0 = sacc;
+          pd0 = da < 0 ? -1 : (da < P - 1 ? da : P - 1);
+          pd1 = db < 0 ? -1 : (db < P - 1 ? db : P - 1);
         }
         tmem_st_wait();
         tc_fence_before();
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(pw_done);
+        if (has_pos) {
+          float* dpos_h = prm.dpos + (int64_t)h * P;
+          if (pg0 != 0.0f && pd0 >= 0) atomicAdd(dpos_h + pd0, pg0);
+          if (pg1 != 0.0f && pd1 >= 0) atomicAdd(dpos_h + pd1, pg1);
+        }
         // the dQ partial of query tile i: TMEM lane = query row; this warp's 16 of the 64 columns
         if (!mbar_wait(dq_full, t & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -695,17 +748,24 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           uint32_t ov[16];
           tmem_ld16(t_lane + Cfg::DQ_COL + 16 * cg, ov);
           tmem_ld_wait16(ov);
-          if (q0 + r < n) {
-            float* dst = prm.dq + (row0 + q0 + r) * (int64_t)(H * 64) + h * 64 + 16 * cg;
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(dq_empty);
+          // into the staging buffer of this tile's parity, from which warp 2 adds it to global dQ
+          // with TMA reductions: row = query r, two 128-byte-swizzled boxes of 32 columns
+          const uint32_t sb = t & 1u;
+          if (!mbar_wait(&stg_empty[sb], ((t >> 1) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* box = stg_s + sb * Cfg::STG_BYTES + (cg >> 1) * (128 * 128) + r * 128;
 #pragma unroll
-            for (int v = 0; v < 4; v++)
-              red_add_v4(dst + 4 * v, __uint_as_float(ov[4 * v]), __uint_as_float(ov[4 * v + 1]),
-                         __uint_as_float(ov[4 * v + 2]), __uint_as_float(ov[4 * v + 3]));
+          for (int v = 0; v < 4; v++) {
+            const int ch = 4 * (cg & 1) + v;
+            *reinterpret_cast<uint4*>(box + ((ch ^ (r & 7)) * 16)) =
+                make_uint4(ov[4 * v], ov[4 * v + 1], ov[4 * v + 2], ov[4 * v + 3]);
           }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&stg_full[sb]);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(dq_empty);
       }
       if (!ok) break;
       // dV_j and dK_j of this item: TMEM lane = key row; this warp's 16 of the 64 columns
@@ -717,6 +777,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         tmem_ld16(t_lane + Cfg::DK_COL + 16 * cg, kv);
         tmem_ld_wait16(vv);
         tmem_ld_wait16(kv);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(dkv_empty);
         if (kvalid) {
           float* dvr = prm.dv + (row0 + j) * (int64_t)(H * 64) + h * 64 + 16 * cg;
           float* dkr = prm.dk + (row0 + j) * (int64_t)(H * 64) + h * 64 + 16 * cg;
@@ -731,9 +794,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(dkv_empty);
       // table gradients of this item to global memory
       if (has_time) {
         if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;

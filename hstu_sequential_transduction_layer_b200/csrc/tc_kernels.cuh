@@ -41,6 +41,20 @@ inline bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t inner, ui
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same for an fp32 matrix (box_inner * 4 must be 128).
+inline bool make_map_f32(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                         uint64_t ld, uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 4};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline int num_sms() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -229,13 +243,13 @@ inline size_t attention_bwd_workspace_bytes(int64_t T, int64_t B, int H) {
 
 template <int BM>
 hstu_status_t launch_attention_bwd_kernel(const CUtensorMap& tm, const CUtensorMap& tdo,
-                                          const BwdParams& prm, const AttnSchedule& sch, int grid,
-                                          cudaStream_t st) {
+                                          const CUtensorMap& tdq, const BwdParams& prm,
+                                          const AttnSchedule& sch, int grid, cudaStream_t st) {
   auto kern = attention_bwd_kernel<BM>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg::SMEM) !=
       cudaSuccess)
     return HSTU_ERR_CUDA;
-  kern<<<grid, BWD_THREADS, BwdCfg::SMEM, st>>>(tm, tdo, prm, sch);
+  kern<<<grid, BWD_THREADS, BwdCfg::SMEM, st>>>(tm, tdo, tdq, prm, sch);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
@@ -263,9 +277,10 @@ inline hstu_status_t launch_attention_bwd(int64_t T, int64_t B, int H, int64_t m
   count_launch();
   if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
   const int n1 = 4 * H * 64;
-  CUtensorMap tm, tdo;
+  CUtensorMap tm, tdo, tdq;
   if (!make_map_bf16(&tm, uvqk, n1, T, n1, 64, 128)) return HSTU_ERR_CUDA;
   if (!make_map_bf16(&tdo, dav, (uint64_t)H * 64, T, (uint64_t)H * 64, 64, 128)) return HSTU_ERR_CUDA;
+  if (!make_map_f32(&tdq, dq, (uint64_t)H * 64, T, (uint64_t)H * 64, 32, 128)) return HSTU_ERR_CUDA;
   BwdParams prm;
   prm.ts = ts;
   prm.pos = pos;
@@ -284,12 +299,12 @@ inline hstu_status_t launch_attention_bwd(int64_t T, int64_t B, int H, int64_t m
   const int grid = (int)(capacity < num_sms() ? capacity : num_sms());
   const int bm = alibi ? BWD_ALIBI : ((pos ? BWD_POS : 0) | (tim ? BWD_TIME : 0));
   switch (bm) {
-    case 0: return launch_attention_bwd_kernel<0>(tm, tdo, prm, sch, grid, st);
-    case BWD_POS: return launch_attention_bwd_kernel<BWD_POS>(tm, tdo, prm, sch, grid, st);
-    case BWD_TIME: return launch_attention_bwd_kernel<BWD_TIME>(tm, tdo, prm, sch, grid, st);
+    case 0: return launch_attention_bwd_kernel<0>(tm, tdo, tdq, prm, sch, grid, st);
+    case BWD_POS: return launch_attention_bwd_kernel<BWD_POS>(tm, tdo, tdq, prm, sch, grid, st);
+    case BWD_TIME: return launch_attention_bwd_kernel<BWD_TIME>(tm, tdo, tdq, prm, sch, grid, st);
     case BWD_POS | BWD_TIME:
-      return launch_attention_bwd_kernel<BWD_POS | BWD_TIME>(tm, tdo, prm, sch, grid, st);
-    default: return launch_attention_bwd_kernel<BWD_ALIBI>(tm, tdo, prm, sch, grid, st);
+      return launch_attention_bwd_kernel<BWD_POS | BWD_TIME>(tm, tdo, tdq, prm, sch, grid, st);
+    default: return launch_attention_bwd_kernel<BWD_ALIBI>(tm, tdo, tdq, prm, sch, grid, st);
   }
 }
 
