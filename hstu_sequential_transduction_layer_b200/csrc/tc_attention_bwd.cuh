@@ -52,10 +52,10 @@ struct BwdCfg {
   static constexpr int OFF_V = OFF_K + BOX;
   static constexpr int OFF_Q = OFF_V + BOX;                 // [NST] Q tiles
   static constexpr int OFF_DO = OFF_Q + NST * BOX;          // [NST] dAV tiles
-  static constexpr int OFF_DS = OFF_DO + NST * BOX;         // dS^T, two 16 KB panels (MN-major A)
-  static constexpr int OFF_STG = OFF_DS + 2 * BOX;          // [2] dQ partial, fp32, 2 swizzled boxes
-  static constexpr int STG_BYTES = 128 * 64 * 4;            //     of 32 columns x 128 rows
-  static constexpr int OFF_QTS = OFF_STG + 2 * STG_BYTES;   // [NST][128] int64 query timestamps
+  static constexpr int OFF_DS = OFF_DO + NST * BOX;         // [2] dS^T, two 16 KB panels (MN-major A)
+  static constexpr int OFF_STG = OFF_DS + 4 * BOX;          // dQ partial, fp32, 2 swizzled boxes
+  static constexpr int STG_BYTES = 128 * 64 * 4;            // of 32 columns x 128 rows
+  static constexpr int OFF_QTS = OFF_STG + STG_BYTES;       // [NST][128] int64 query timestamps
   static constexpr int OFF_KTS = OFF_QTS + NST * 128 * 8;   // [128] int64 key timestamps
   static constexpr int OFF_QTS32 = OFF_KTS + 128 * 8;       // [NST][128] int32, relative
   static constexpr int OFF_KTS32 = OFF_QTS32 + NST * 128 * 4;  // [128] int32, relative
@@ -191,16 +191,18 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   uint64_t* kv_empty = bars + 1;
   uint64_t* q_full = bars + 2;        // [NST]
   uint64_t* q_empty = bars + 4;       // [NST]
-  uint64_t* sp_full = bars + 6;
-  uint64_t* pw_done = bars + 7;
+  uint64_t* sa_full = bars + 6;       // S^T, dP^T of the tile's first 64 queries
+  uint64_t* pwa_done = bars + 7;      // their P^T, dS^T written (16 pointwise warps)
   uint64_t* dq_full = bars + 8;
   uint64_t* dq_empty = bars + 9;
   uint64_t* dkv_full = bars + 10;
   uint64_t* dkv_empty = bars + 11;
   uint64_t* pw_bar = bars + 12;
   uint64_t* drain = bars + 13;
-  uint64_t* stg_full = bars + 14;     // [2] dQ partial staged (16 pointwise warps)
-  uint64_t* stg_empty = bars + 16;    // [2] staged dQ partial read by the TMA reduce
+  uint64_t* sb_full = bars + 14;      // the same for the last 64 queries
+  uint64_t* pwb_done = bars + 15;
+  uint64_t* stg_full = bars + 16;     // dQ partial staged (16 pointwise warps)
+  uint64_t* stg_empty = bars + 17;    // staged dQ partial read by the TMA reduce
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -221,18 +223,18 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
     }
-    mbar_init(sp_full, 1);
-    mbar_init(pw_done, BWD_PW_WARPS);
+    mbar_init(sa_full, 1);
+    mbar_init(sb_full, 1);
+    mbar_init(pwa_done, BWD_PW_WARPS);
+    mbar_init(pwb_done, BWD_PW_WARPS);
     mbar_init(dq_full, 1);
     mbar_init(dq_empty, BWD_PW_WARPS);
     mbar_init(dkv_full, 1);
     mbar_init(dkv_empty, BWD_PW_WARPS);
     mbar_init(pw_bar, BWD_PW);
     mbar_init(drain, 1);
-    for (int b = 0; b < 2; b++) {
-      mbar_init(&stg_full[b], BWD_PW_WARPS);
-      mbar_init(&stg_empty[b], 1);
-    }
+    mbar_init(stg_full, BWD_PW_WARPS);
+    mbar_init(stg_empty, 1);
     *abort_flag = 0;
     fence_mbar_init();
     prefetch_tensormap(&tm);
@@ -334,13 +336,47 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
+    // Per query tile, two 64-query halves A and B: S^T and dP^T of a half are ready for the
+    // pointwise warps while the other half is being computed, and the next tile's half A is
+    // issued as soon as this tile's half A has been consumed, so that the tensor cores run while
+    // the pointwise warps work.
     if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t idesc_s = idesc_bf16(128, 64, false, false);
       constexpr uint32_t idesc_o = idesc_bf16(128, 64, false, true);
       constexpr uint32_t idesc_q = idesc_bf16(128, 64, true, true);
-      const uint32_t k_addr = smem_u32(k_s), v_addr = smem_u32(v_s), ds_addr = smem_u32(ds_s);
+      const uint32_t k_addr = smem_u32(k_s), v_addr = smem_u32(v_s);
       uint32_t k = 0, g = 0, t = 0;
       bool ok = true;
+      // S^T / dP^T of half ht of the query tile in stage st
+      auto issue_s = [&](uint32_t st, int ht) {
+        const uint32_t q_addr = smem_u32(smem + Cfg::OFF_Q + st * Cfg::BOX) + ht * 8192;
+        const uint32_t do_addr = smem_u32(smem + Cfg::OFF_DO + st * Cfg::BOX) + ht * 8192;
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)
+          mma_ss(tmem + Cfg::S_COL + 64 * ht, sdesc_sw128(k_addr + kk * 32, 16, 1024),
+                 sdesc_sw128(q_addr + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)
+          mma_ss(tmem + Cfg::DP_COL + 64 * ht, sdesc_sw128(v_addr + kk * 32, 16, 1024),
+                 sdesc_sw128(do_addr + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        mma_commit(ht == 0 ? sa_full : sb_full);
+      };
+      // dV_j += P^T dAV and dK_j += dS^T Q over half ht's 64 queries (P^T, dS^T from TMEM: the
+      // 16 queries of pointwise column group cg sit, packed, at the start of its 16 columns)
+      auto issue_dkv = [&](uint32_t st, int ht, bool first) {
+        const uint32_t q_addr = smem_u32(smem + Cfg::OFF_Q + st * Cfg::BOX);
+        const uint32_t do_addr = smem_u32(smem + Cfg::OFF_DO + st * Cfg::BOX);
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)
+          mma_ts(tmem + Cfg::DV_COL, tmem + Cfg::S_COL + 64 * ht + 16 * kk,
+                 sdesc_sw128(do_addr + (4 * ht + kk) * 2048, Cfg::BOX, 1024), idesc_o,
+                 (first && kk == 0) ? 0u : 1u);
+#pragma unroll
+        for (int kk = 0; kk < 4; kk++)
+          mma_ts(tmem + Cfg::DK_COL, tmem + Cfg::DP_COL + 64 * ht + 16 * kk,
+                 sdesc_sw128(q_addr + (4 * ht + kk) * 2048, Cfg::BOX, 1024), idesc_o,
+                 (first && kk == 0) ? 0u : 1u);
+      };
       for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x, k++) {
         const int64_t item = sch.items[it];
         const int64_t seq = item & 0xffffffffLL;
@@ -348,44 +384,30 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         const int64_t n = sch.seqinfo[2 * seq + 1];
         const int nt = (int)((n + ATT_BN - 1) / ATT_BN);
         if (!mbar_wait(kv_full, k & 1u, abort_flag)) break;
+        if (!mbar_wait(&q_full[g % Cfg::NST], (g / Cfg::NST) & 1u, abort_flag)) break;
+        tc_fence_after();
+        issue_s(g % Cfg::NST, 0);
+        issue_s(g % Cfg::NST, 1);
         for (int i = jt; i < nt; i++, g++, t++) {
-          const uint32_t st = g % Cfg::NST, ph = (g / Cfg::NST) & 1u;
-          if (!mbar_wait(&q_full[st], ph, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t q_addr = smem_u32(smem + Cfg::OFF_Q + st * Cfg::BOX);
-          const uint32_t do_addr = smem_u32(smem + Cfg::OFF_DO + st * Cfg::BOX);
-          // S^T = K_j Q_i^T and dP^T = V_j dAV_i^T
-#pragma unroll
-          for (int kk = 0; kk < 4; kk++)
-            mma_ss(tmem + Cfg::S_COL, sdesc_sw128(k_addr + kk * 32, 16, 1024),
-                   sdesc_sw128(q_addr + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < 4; kk++)
-            mma_ss(tmem + Cfg::DP_COL, sdesc_sw128(v_addr + kk * 32, 16, 1024),
-                   sdesc_sw128(do_addr + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-          mma_commit(sp_full);
-          if (!mbar_wait(pw_done, t & 1u, abort_flag)) { ok = false; break; }
+          const uint32_t st = g % Cfg::NST;
+          if (!mbar_wait(pwa_done, t & 1u, abort_flag)) { ok = false; break; }
           if (i == jt && !mbar_wait(dkv_empty, (k & 1u) ^ 1u, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          // dV_j += P^T dAV_i and dK_j += dS^T Q_i (P^T, dS^T from TMEM; the 32 queries of each
-          // pointwise column group sit, packed, at the start of that group's 32 columns)
-#pragma unroll
-          for (int kk = 0; kk < 8; kk++) {
-            const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;
-            const uint32_t acc = (i > jt || kk > 0) ? 1u : 0u;
-            mma_ts(tmem + Cfg::DV_COL, tmem + Cfg::S_COL + pc,
-                   sdesc_sw128(do_addr + kk * 2048, Cfg::BOX, 1024), idesc_o, acc);
+          issue_dkv(st, 0, i == jt);
+          if (i + 1 < nt) {
+            const uint32_t g1 = g + 1;
+            if (!mbar_wait(&q_full[g1 % Cfg::NST], (g1 / Cfg::NST) & 1u, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            issue_s(g1 % Cfg::NST, 0);
           }
-#pragma unroll
-          for (int kk = 0; kk < 8; kk++) {
-            const uint32_t pc = (kk >> 1) * 32 + (kk & 1) * 8;
-            const uint32_t acc = (i > jt || kk > 0) ? 1u : 0u;
-            mma_ts(tmem + Cfg::DK_COL, tmem + Cfg::DP_COL + pc,
-                   sdesc_sw128(q_addr + kk * 2048, Cfg::BOX, 1024), idesc_o, acc);
-          }
-          // dQ_i partial = dS K_j: dS from shared memory (MN-major: rows = keys), K_j as MN-major B
+          if (!mbar_wait(pwb_done, t & 1u, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_dkv(st, 1, false);
+          // dQ_i partial = dS K_j: dS from shared memory (MN-major: rows = keys; the buffer of this
+          // tile's parity), K_j as MN-major B
           if (t > 0 && !mbar_wait(dq_empty, (t - 1) & 1u, abort_flag)) { ok = false; break; }
           tc_fence_after();
+          const uint32_t ds_addr = smem_u32(ds_s + (t & 1u) * (2 * Cfg::BOX));
 #pragma unroll
           for (int kk = 0; kk < 8; kk++)
             mma_ss(tmem + Cfg::DQ_COL, sdesc_sw128(ds_addr + kk * 2048, Cfg::BOX, 1024),
@@ -395,6 +417,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           if (i == nt - 1) {
             mma_commit(dkv_full);
             mma_commit(kv_empty);
+          } else {
+            issue_s((g + 1) % Cfg::NST, 1);
           }
         }
         if (!ok) break;
@@ -418,15 +442,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         const int64_t row0 = sch.seqinfo[2 * seq], n = sch.seqinfo[2 * seq + 1];
         const int nt = (int)((n + ATT_BN - 1) / ATT_BN);
         for (int i = jt; i < nt; i++, t++) {
-          const uint32_t sb = t & 1u;
-          if (!mbar_wait(&stg_full[sb], (t >> 1) & 1u, abort_flag)) { ok = false; break; }
-          const uint8_t* src = stg_s + sb * Cfg::STG_BYTES;
+          if (!mbar_wait(stg_full, t & 1u, abort_flag)) { ok = false; break; }
           const int y = (int)row0 + i * ATT_BM;
-          tma_reduce_add_2d(&tdq, src, h * 64, y);
-          tma_reduce_add_2d(&tdq, src + 128 * 128, h * 64 + 32, y);
+          tma_reduce_add_2d(&tdq, stg_s, h * 64, y);
+          tma_reduce_add_2d(&tdq, stg_s + 128 * 128, h * 64 + 32, y);
           bulk_commit();
           bulk_wait_read_all();
-          mbar_arrive(&stg_empty[sb]);
+          mbar_arrive(stg_empty);
         }
       }
       bulk_wait_all();
@@ -434,8 +456,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ pointwise warps
-    // 16 warps: TMEM lane quadrant q = warp & 3 (keys q*32 .. q*32+31 of the tile), query columns
-    // 32 cg .. 32 cg + 31 (cg = (warp - 4) / 4), each 32 x 32 block in two 16-column halves
+    // 16 warps: TMEM lane quadrant q = warp & 3 (keys q*32 .. q*32+31 of the tile); column group
+    // cg = (warp - 4) / 4 takes queries 16 cg .. 16 cg + 15 of each 64-query half of the tile
     const int pw = warp - 4;
     const int cg = pw >> 2;
     const int q = warp & 3;
@@ -446,11 +468,36 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const int tcap = Tb < BWD_TB_CAP ? Tb : BWD_TB_CAP;
     const float scale = prm.scale;
     const float m0 = lane > 0 ? 1.0f : 0.0f;
-    float* pwin = pwin_s + pw * 64;      // the position table at the block's 63 distances
+    float* pwin = pwin_s + pw * 64;      // the position table at the block's 47 distances
     float* cap = cap_s + pw * 32;        // completed diagonals of the systolic sums
     uint32_t k = 0, g = 0, t = 0, pw_cnt = 0;
     int staged_head = -1;
     bool ok = true;
+    // The dQ partial of tile tt (TMEM lane = query row; this warp's 16 of the 64 columns) into the
+    // staging buffer, from which warp 2 adds it to global dQ with TMA reductions: row = query r,
+    // two 128-byte-swizzled boxes of 32 columns.
+    auto dq_readout = [&](uint32_t tt) -> bool {
+      if (!mbar_wait(dq_full, tt & 1u, abort_flag)) return false;
+      tc_fence_after();
+      uint32_t ov[16];
+      tmem_ld16(t_lane + Cfg::DQ_COL + 16 * cg, ov);
+      tmem_ld_wait16(ov);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(dq_empty);
+      if (!mbar_wait(stg_empty, (tt & 1u) ^ 1u, abort_flag)) return false;
+      uint8_t* box = stg_s + (cg >> 1) * (128 * 128) + r * 128;
+#pragma unroll
+      for (int v = 0; v < 4; v++) {
+        const int ch = 4 * (cg & 1) + v;
+        *reinterpret_cast<uint4*>(box + ((ch ^ (r & 7)) * 16)) =
+            make_uint4(ov[4 * v], ov[4 * v + 1], ov[4 * v + 2], ov[4 * v + 3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(stg_full);
+      return true;
+    };
     for (int64_t it = blockIdx.x; it < n_items && ok; it += gridDim.x, k++) {
       const int64_t item = sch.items[it];
       const int64_t seq = item & 0xffffffffLL;
@@ -474,12 +521,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const int tk32 = has_time ? kts32[r] : 0;   // relative key time
       const bool keys_rel32 = has_time && tflag[0] != 0;
       const int kq0 = k0 + q * 32;                // the warp's first key
-      for (int i = jt; i < nt; i++, g++, t++) {
+      for (int i = jt; i < nt && ok; i++, g++, t++) {
         const uint32_t st = g % Cfg::NST;
         const int q0 = i * ATT_BM;
-        const int qc0 = q0 + 32 * cg;             // the warp's first query
-        const int64_t* qt_s = qts + st * 128 + 32 * cg;
-        const int* qt32 = qts32 + st * 128 + 32 * cg;
+#pragma unroll 1
+        for (int ht = 0; ht < 2; ht++) {
+        const int qb = 64 * ht + 16 * cg;         // the block's first query within the tile
+        const int qc0 = q0 + qb;
+        const int64_t* qt_s = qts + st * 128 + qb;
+        const int* qt32 = qts32 + st * 128 + qb;
         const int dbase = qc0 - kq0;              // distance of (lane 0, e = 0)
         // the position table at distances dbase - 31 .. dbase + 32 (clamped), loaded before the
         // MMA wait so that the wait hides the load
@@ -490,27 +540,29 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           wv1 = __ldg(pos_h + (d1 < 0 ? 0 : (d1 < P - 1 ? d1 : P - 1)));
         }
         // the stage's query timestamps are published with its Q/dAV tiles
-        if (has_time && !mbar_wait(&q_full[st], (g / Cfg::NST) & 1u, abort_flag)) { ok = false; break; }
-        if (!mbar_wait(sp_full, t & 1u, abort_flag)) { ok = false; break; }
+        if (ht == 0 && has_time &&
+            !mbar_wait(&q_full[st], (g / Cfg::NST) & 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(ht == 0 ? sa_full : sb_full, t & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         uint32_t sv[16], dpv[16];
-        tmem_ld16(t_lane + Cfg::S_COL + 32 * cg, sv);
-        tmem_ld16(t_lane + Cfg::DP_COL + 32 * cg, dpv);
+        tmem_ld16(t_lane + Cfg::S_COL + qb, sv);
+        tmem_ld16(t_lane + Cfg::DP_COL + qb, dpv);
         if (has_pos) {
           pwin[lane] = wv0;
           pwin[32 + lane] = wv1;
           __syncwarp();
         }
-        // Fast path when every score of the block is valid (off the diagonal, inside the
-        // sequence) and the time bucket is the same for the whole block, or takes two values split
-        // by one threshold (sorted timestamps, the extreme corners' buckets equal or adjacent).
-        const bool full = dbase - 31 >= 0 && (int64_t)(qc0 + 31) < n && (int64_t)(kq0 + 31) < n;
+        // Fast path when every score of the 32 x 16 block is valid (off the diagonal, inside the
+        // sequence) and the time bucket is the same for the whole block, or takes two values
+        // split by one threshold (sorted timestamps, the extreme corners' buckets equal or
+        // adjacent).
+        const bool full = dbase - 31 >= 0 && (int64_t)(qc0 + 15) < n && (int64_t)(kq0 + 31) < n;
         const bool pos_one = has_pos && full && dbase - 31 >= P - 1;   // all in bucket P - 1
         int tb_u = -1, tmode = 0;                 // 1: one bucket tb_u; 2: tb_u and tb_u + 1
         int thr = 0;                              // two buckets: relative dt >= thr is tb_u + 1
-        if (has_time && full && ((tsort[0] >> q) & 1) && ((tsort[1 + st] >> cg) & 1)) {
+        if (has_time && full && ((tsort[0] >> q) & 1) && ((tsort[1 + st] >> (qb >> 5)) & 1)) {
           const int b0 = time_bucket(qt_s[0], kts[q * 32 + 31]);
-          const int b1 = time_bucket(qt_s[31], kts[q * 32]);
+          const int b1 = time_bucket(qt_s[15], kts[q * 32]);
           const int c0b = b0 < Tb - 1 ? b0 : Tb - 1, c1b = b1 < Tb - 1 ? b1 : Tb - 1;
           if (c0b == c1b) {
             tb_u = c0b;
@@ -538,141 +590,130 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         const float al0 = -slope * (float)(dbase - lane);
         float acc_u = 0.0f, acc_h = 0.0f, acc_pu = 0.0f, acc_lo = 0.0f, acc_hi = 0.0f;
         float sacc = 0.0f;                        // systolic diagonal sum (position gradient)
-#pragma unroll 1
-        for (int hf = 0; hf < 2; hf++) {
-          tmem_ld_wait16(sv);
-          tmem_ld_wait16(dpv);
-          uint32_t pk[8], dk[8];
-          const float* plh = pl + 16 * hf;
-          const int* qt32h = qt32 + 16 * hf;
-          const int64_t* qth = qt_s + 16 * hf;
-          float* caph = cap + 16 * hf - 1;        // caph[ee]: diagonal completed at e = 16 hf + ee
-          const float alh = fmaf(-slope, (float)(16 * hf), al0);
-          const int iq0 = qc0 + 16 * hf;
-          // one step of the systolic diagonal sums: lane l holds the sum of diagonal e - l; the
-          // sums move up one lane per column, and lane 31's (complete) is parked in `cap`
-          auto systolic = [&](int ee, float dx) {
-            if (ee == 0 && hf == 0) {
-              sacc = dx;
-            } else {
-              if (lane == 31) caph[ee] = sacc;
-              sacc = fmaf(__shfl_up_sync(0xffffffffu, sacc, 1), m0, dx);
-            }
-          };
-          // the fast element loop: no masks; the time bias one or two constants
-          auto fast16 = [&](auto tm_tag, auto po_tag) {
-            constexpr int TM = decltype(tm_tag)::value;
-            constexpr bool PO = decltype(po_tag)::value;
-#pragma unroll
-            for (int ee = 0; ee < 16; ee += 2) {
-              float a2[2], d2[2];
-#pragma unroll
-              for (int u = 0; u < 2; u++) {
-                float x = __uint_as_float(sv[ee + u]);
-                bool hi = false;
-                if (TM == 2) {
-                  hi = qt32h[ee + u] - tk32 >= thr;
-                  x += hi ? thi : tlo;
-                } else if (TM == 1) {
-                  x += tlo;
-                }
-                if (has_pos) x += PO ? pone : plh[ee + u];
-                if (alibi) x += fmaf(-slope, (float)(ee + u), alh);
-                float sl, dsl;
-                silu_and_grad(x, sl, dsl);
-                const float dx = scale * dsl * __uint_as_float(dpv[ee + u]);
-                a2[u] = scale * sl;
-                d2[u] = dx;
-                if (PO) acc_pu += dx;
-                else if (has_pos) systolic(ee + u, dx);
-                if (TM != 0) acc_u += dx;
-                if (TM == 2) acc_h += hi ? dx : 0.0f;
-              }
-              pk[ee / 2] = pack_bf16x2(a2[0], a2[1]);
-              dk[ee / 2] = pack_bf16x2(d2[0], d2[1]);
-            }
-          };
-          // the general element loop (masks, per-score time buckets), with 32-bit time buckets
-          // when the tile's timestamps fit
-          auto gen16 = [&](auto rel_tag) {
-            constexpr bool REL32 = decltype(rel_tag)::value;
-#pragma unroll
-            for (int ee = 0; ee < 16; ee += 2) {
-              float a2[2], d2[2];
-#pragma unroll
-              for (int u = 0; u < 2; u++) {
-                const int iq = iq0 + ee + u;         // query (local index)
-                const int dist = iq - j;
-                const bool valid = kvalid && iq < n && dist >= 0;
-                float bias = 0.0f;
-                int tb = 0;
-                if (alibi) bias = -slope * (float)dist;
-                if (has_pos) bias += plh[ee + u];
-                if (has_time) {
-                  if (REL32) {
-                    // floor(log2(1 + max(ti - tj, 0))) = 31 - clz(max(ti - tj, 0) + 1)
-                    const int dd = qt32h[ee + u] - tk32 + 1;
-                    tb = 31 - __clz(dd > 1 ? dd : 1);
-                  } else {
-                    tb = time_bucket(qth[ee + u], tj);
-                  }
-                  tb = tb < Tb - 1 ? tb : Tb - 1;
-                  bias += tt_s[tb];
-                }
-                float sl, dsl;
-                silu_and_grad(__uint_as_float(sv[ee + u]) + bias, sl, dsl);
-                const float dx = valid ? scale * dsl * __uint_as_float(dpv[ee + u]) : 0.0f;
-                a2[u] = valid ? scale * sl : 0.0f;
-                d2[u] = dx;
-                if (has_pos) systolic(ee + u, dx);
-                if (has_time) {
-                  const int db = tb - tb_first;
-                  acc_lo += db == 0 ? dx : 0.0f;
-                  acc_hi += db == 1 ? dx : 0.0f;
-                  // rare (a step of two or more buckets inside a block, near the diagonal): a
-                  // warp vote keeps the shared-memory atomic off the common path
-                  const bool far = valid && (db < 0 || db > 1);
-                  if (__any_sync(0xffffffffu, far)) {
-                    if (far) atomicAdd(&dtt_s[tb], dx);
-                  }
-                }
-              }
-              pk[ee / 2] = pack_bf16x2(a2[0], a2[1]);
-              dk[ee / 2] = pack_bf16x2(d2[0], d2[1]);
-            }
-          };
-          if (fast) {
-            if (tmode == 2) {
-              if (pos_one) fast16(std::integral_constant<int, 2>{}, std::true_type{});
-              else fast16(std::integral_constant<int, 2>{}, std::false_type{});
-            } else if (has_time) {
-              if (pos_one) fast16(std::integral_constant<int, 1>{}, std::true_type{});
-              else fast16(std::integral_constant<int, 1>{}, std::false_type{});
-            } else {
-              if (pos_one) fast16(std::integral_constant<int, 0>{}, std::true_type{});
-              else fast16(std::integral_constant<int, 0>{}, std::false_type{});
-            }
-          } else if (has_time && keys_rel32 && tflag[1 + st] != 0) {
-            gen16(std::true_type{});
+        float* caph = cap - 1;                    // caph[ee]: diagonal completed at column ee
+        tmem_ld_wait16(sv);
+        tmem_ld_wait16(dpv);
+        uint32_t pk[8], dk[8];
+        // one step of the systolic diagonal sums: lane l holds the sum of diagonal e - l; the
+        // sums move up one lane per column, and lane 31's (complete) is parked in `cap`
+        auto systolic = [&](int ee, float dx) {
+          if (ee == 0) {
+            sacc = dx;
           } else {
-            gen16(std::false_type{});
+            if (lane == 31) caph[ee] = sacc;
+            sacc = fmaf(__shfl_up_sync(0xffffffffu, sacc, 1), m0, dx);
           }
-          // P^T and dS^T (bf16 pairs) into the first 8 of the 16 S^T / dP^T columns this half
-          // has read; then the next half's loads
-          tmem_st8(t_lane + Cfg::S_COL + 32 * cg + 8 * hf, pk);
-          tmem_st8(t_lane + Cfg::DP_COL + 32 * cg + 8 * hf, dk);
-          if (hf == 0) {
-            tmem_ld16(t_lane + Cfg::S_COL + 32 * cg + 16, sv);
-            tmem_ld16(t_lane + Cfg::DP_COL + 32 * cg + 16, dpv);
-          }
-          // dS^T into shared memory as the MN-major A operand of dQ = dS K_j: row = key r,
-          // 128-byte swizzled rows of 64 queries per panel; this half's 16 queries are 2 units
+        };
+        // the fast element loop: no masks; the time bias one or two constants
+        auto fast16 = [&](auto tm_tag, auto po_tag) {
+          constexpr int TM = decltype(tm_tag)::value;
+          constexpr bool PO = decltype(po_tag)::value;
 #pragma unroll
-          for (int v = 0; v < 2; v++) {
-            const int uu = 4 * (cg & 1) + 2 * hf + v;
-            uint8_t* dst = ds_s + (cg >> 1) * Cfg::BOX + r * 128 + ((uu ^ (r & 7)) * 16);
-            *reinterpret_cast<uint4*>(dst) = make_uint4(dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]);
+          for (int ee = 0; ee < 16; ee += 2) {
+            float a2[2], d2[2];
+#pragma unroll
+            for (int u = 0; u < 2; u++) {
+              float x = __uint_as_float(sv[ee + u]);
+              bool hi = false;
+              if (TM == 2) {
+                hi = qt32[ee + u] - tk32 >= thr;
+                x += hi ? thi : tlo;
+              } else if (TM == 1) {
+                x += tlo;
+              }
+              if (has_pos) x += PO ? pone : pl[ee + u];
+              if (alibi) x += fmaf(-slope, (float)(ee + u), al0);
+              float sl, dsl;
+              silu_and_grad(x, sl, dsl);
+              const float dx = scale * dsl * __uint_as_float(dpv[ee + u]);
+              a2[u] = scale * sl;
+              d2[u] = dx;
+              if (PO) acc_pu += dx;
+              else if (has_pos) systolic(ee + u, dx);
+              if (TM != 0) acc_u += dx;
+              if (TM == 2) acc_h += hi ? dx : 0.0f;
+            }
+            pk[ee / 2] = pack_bf16x2(a2[0], a2[1]);
+            dk[ee / 2] = pack_bf16x2(d2[0], d2[1]);
           }
+        };
+        // the general element loop (masks, per-score time buckets), with 32-bit time buckets
+        // when the tile's timestamps fit
+        auto gen16 = [&](auto rel_tag) {
+          constexpr bool REL32 = decltype(rel_tag)::value;
+#pragma unroll
+          for (int ee = 0; ee < 16; ee += 2) {
+            float a2[2], d2[2];
+#pragma unroll
+            for (int u = 0; u < 2; u++) {
+              const int iq = qc0 + ee + u;           // query (local index)
+              const int dist = iq - j;
+              const bool valid = kvalid && iq < n && dist >= 0;
+              float bias = 0.0f;
+              int tb = 0;
+              if (alibi) bias = -slope * (float)dist;
+              if (has_pos) bias += pl[ee + u];
+              if (has_time) {
+                if (REL32) {
+                  // floor(log2(1 + max(ti - tj, 0))) = 31 - clz(max(ti - tj, 0) + 1)
+                  const int dd = qt32[ee + u] - tk32 + 1;
+                  tb = 31 - __clz(dd > 1 ? dd : 1);
+                } else {
+                  tb = time_bucket(qt_s[ee + u], tj);
+                }
+                tb = tb < Tb - 1 ? tb : Tb - 1;
+                bias += tt_s[tb];
+              }
+              float sl, dsl;
+              silu_and_grad(__uint_as_float(sv[ee + u]) + bias, sl, dsl);
+              const float dx = valid ? scale * dsl * __uint_as_float(dpv[ee + u]) : 0.0f;
+              a2[u] = valid ? scale * sl : 0.0f;
+              d2[u] = dx;
+              if (has_pos) systolic(ee + u, dx);
+              if (has_time) {
+                const int db = tb - tb_first;
+                acc_lo += db == 0 ? dx : 0.0f;
+                acc_hi += db == 1 ? dx : 0.0f;
+                // rare (a step of two or more buckets inside a block, near the diagonal): a
+                // warp vote keeps the shared-memory atomic off the common path
+                const bool far = valid && (db < 0 || db > 1);
+                if (__any_sync(0xffffffffu, far)) {
+                  if (far) atomicAdd(&dtt_s[tb], dx);
+                }
+              }
+            }
+            pk[ee / 2] = pack_bf16x2(a2[0], a2[1]);
+            dk[ee / 2] = pack_bf16x2(d2[0], d2[1]);
+          }
+        };
+        if (fast) {
+          if (tmode == 2) {
+            if (pos_one) fast16(std::integral_constant<int, 2>{}, std::true_type{});
+            else fast16(std::integral_constant<int, 2>{}, std::false_type{});
+          } else if (has_time) {
+            if (pos_one) fast16(std::integral_constant<int, 1>{}, std::true_type{});
+            else fast16(std::integral_constant<int, 1>{}, std::false_type{});
+          } else {
+            if (pos_one) fast16(std::integral_constant<int, 0>{}, std::true_type{});
+            else fast16(std::integral_constant<int, 0>{}, std::false_type{});
+          }
+        } else if (has_time && keys_rel32 && tflag[1 + st] != 0) {
+          gen16(std::true_type{});
+        } else {
+          gen16(std::false_type{});
+        }
+        // P^T and dS^T (bf16 pairs) into the first 8 of the 16 S^T / dP^T columns just read
+        tmem_st8(t_lane + Cfg::S_COL + qb, pk);
+        tmem_st8(t_lane + Cfg::DP_COL + qb, dk);
+        // dS^T into shared memory (the buffer of this tile's parity) as the MN-major A operand of
+        // dQ = dS K_j: row = key r, 128-byte swizzled rows of 64 queries per panel (one panel per
+        // half); this block's 16 queries are 2 units
+#pragma unroll
+        for (int v = 0; v < 2; v++) {
+          const int uu = 2 * cg + v;
+          uint8_t* dst = ds_s + (t & 1u) * (2 * Cfg::BOX) + ht * Cfg::BOX + r * 128 +
+                         ((uu ^ (r & 7)) * 16);
+          *reinterpret_cast<uint4*>(dst) = make_uint4(dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]);
         }
         // table gradients of the block
         if (has_time && fast) {
@@ -722,11 +763,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             pd0 = P - 1;
           }
         } else if (has_pos) {
-          // lane l: diagonal 31 - l in the systolic sum, diagonal l - 31 parked in cap[l]
+          // lane l: diagonal 15 - l in the systolic sum; lanes 0..14: diagonal l - 31 parked in
+          // cap[l]
           __syncwarp();
-          pg1 = lane < 31 ? cap[lane] : 0.0f;
+          pg1 = lane < 15 ? cap[lane] : 0.0f;
           __syncwarp();
-          const int da = dbase + 31 - lane, db = dbase + lane - 31;
+          const int da = dbase + 15 - lane, db = dbase + lane - 31;
           pg0 = sacc;
           pd0 = da < 0 ? -1 : (da < P - 1 ? da : P - 1);
           pd1 = db < 0 ? -1 : (db < P - 1 ? db : P - 1);
@@ -735,39 +777,19 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         tc_fence_before();
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(pw_done);
+        if (lane == 0) mbar_arrive(ht == 0 ? pwa_done : pwb_done);
         if (has_pos) {
           float* dpos_h = prm.dpos + (int64_t)h * P;
           if (pg0 != 0.0f && pd0 >= 0) atomicAdd(dpos_h + pd0, pg0);
           if (pg1 != 0.0f && pd1 >= 0) atomicAdd(dpos_h + pd1, pg1);
         }
-        // the dQ partial of query tile i: TMEM lane = query row; this warp's 16 of the 64 columns
-        if (!mbar_wait(dq_full, t & 1u, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        {
-          uint32_t ov[16];
-          tmem_ld16(t_lane + Cfg::DQ_COL + 16 * cg, ov);
-          tmem_ld_wait16(ov);
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(dq_empty);
-          // into the staging buffer of this tile's parity, from which warp 2 adds it to global dQ
-          // with TMA reductions: row = query r, two 128-byte-swizzled boxes of 32 columns
-          const uint32_t sb = t & 1u;
-          if (!mbar_wait(&stg_empty[sb], ((t >> 1) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
-          uint8_t* box = stg_s + sb * Cfg::STG_BYTES + (cg >> 1) * (128 * 128) + r * 128;
-#pragma unroll
-          for (int v = 0; v < 4; v++) {
-            const int ch = 4 * (cg & 1) + v;
-            *reinterpret_cast<uint4*>(box + ((ch ^ (r & 7)) * 16)) =
-                make_uint4(ov[4 * v], ov[4 * v + 1], ov[4 * v + 2], ov[4 * v + 3]);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&stg_full[sb]);
+        // the previous tile's dQ partial, while the tensor cores work on this tile
+        if (ht == 0 && i > jt && !dq_readout(t - 1)) { ok = false; break; }
         }
       }
       if (!ok) break;
+      // the item's last dQ partial
+      if (!dq_readout(t - 1)) break;
       // dV_j and dK_j of this item: TMEM lane = key row; this warp's 16 of the 64 columns
       if (!mbar_wait(dkv_full, k & 1u, abort_flag)) break;
       tc_fence_after();
