@@ -521,6 +521,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const int tk32 = has_time ? kts32[r] : 0;   // relative key time
       const bool keys_rel32 = has_time && tflag[0] != 0;
       const int kq0 = k0 + q * 32;                // the warp's first key
+      // pending time-gradient sums of the fast blocks (per lane, buckets pend_b and pend_b + 1)
+      // and of the blocks entirely in the last position bucket
+      int pend_b = -2;
+      float pend_lo = 0.0f, pend_hi = 0.0f, pend_p = 0.0f;
+      auto flush_time = [&](int b, float v) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0 && b >= 0 && v != 0.0f) atomicAdd(&dtt_s[b], v);
+      };
       for (int i = jt; i < nt && ok; i++, g++, t++) {
         const uint32_t st = g % Cfg::NST;
         const int q0 = i * ATT_BM;
@@ -561,8 +570,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         int tb_u = -1, tmode = 0;                 // 1: one bucket tb_u; 2: tb_u and tb_u + 1
         int thr = 0;                              // two buckets: relative dt >= thr is tb_u + 1
         if (has_time && full && ((tsort[0] >> q) & 1) && ((tsort[1 + st] >> (qb >> 5)) & 1)) {
-          const int b0 = time_bucket(qt_s[0], kts[q * 32 + 31]);
-          const int b1 = time_bucket(qt_s[15], kts[q * 32]);
+          int b0, b1;
+          if (keys_rel32 && tflag[1 + st] != 0) {
+            // 32-bit: floor(log2(1 + max(dt, 0))) = 31 - clz(max(dt, 0) + 1)
+            const int e0 = qt32[0] - kts32[q * 32 + 31], e1 = qt32[15] - kts32[q * 32];
+            b0 = 31 - __clz((e0 > 0 ? e0 : 0) + 1);
+            b1 = 31 - __clz((e1 > 0 ? e1 : 0) + 1);
+          } else {
+            b0 = time_bucket(qt_s[0], kts[q * 32 + 31]);
+            b1 = time_bucket(qt_s[15], kts[q * 32]);
+          }
           const int c0b = b0 < Tb - 1 ? b0 : Tb - 1, c1b = b1 < Tb - 1 ? b1 : Tb - 1;
           if (c0b == c1b) {
             tb_u = c0b;
@@ -717,15 +734,23 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         }
         // table gradients of the block
         if (has_time && fast) {
-          // the block's sums in bucket tb_u (and tb_u + 1)
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            acc_u += __shfl_xor_sync(0xffffffffu, acc_u, o);
-            if (tmode == 2) acc_h += __shfl_xor_sync(0xffffffffu, acc_h, o);
-          }
-          if (lane == 0) {
-            if (acc_u - acc_h != 0.0f) atomicAdd(&dtt_s[tb_u], acc_u - acc_h);
-            if (acc_h != 0.0f) atomicAdd(&dtt_s[tb_u + 1], acc_h);
+          // the block's sums in buckets tb_u and tb_u + 1 join the pending pair (flushed when the
+          // buckets move on: along a warp's blocks the queries only get later)
+          const float lo = acc_u - acc_h, hi = acc_h;
+          if (tb_u == pend_b) {
+            pend_lo += lo;
+            pend_hi += hi;
+          } else if (tb_u == pend_b + 1) {
+            flush_time(pend_b, pend_lo);
+            pend_b = tb_u;
+            pend_lo = pend_hi + lo;
+            pend_hi = hi;
+          } else {
+            flush_time(pend_b, pend_lo);
+            flush_time(pend_b + 1, pend_hi);
+            pend_b = tb_u;
+            pend_lo = lo;
+            pend_hi = hi;
           }
         } else if (has_time) {
           // one atomic per run of lanes with the same first bucket: the rows of a warp are 32
@@ -755,13 +780,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         float pg0 = 0.0f, pg1 = 0.0f;
         int pd0 = -1, pd1 = -1;
         if (pos_one && fast) {
-          // every distance of the block is clamped to the last bucket
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) acc_pu += __shfl_xor_sync(0xffffffffu, acc_pu, o);
-          if (lane == 0) {
-            pg0 = acc_pu;
-            pd0 = P - 1;
-          }
+          // every distance of the block is clamped to the last bucket: summed per lane over the
+          // item, sent at its end
+          pend_p += acc_pu;
         } else if (has_pos) {
           // lane l: diagonal 15 - l in the systolic sum; lanes 0..14: diagonal l - 31 parked in
           // cap[l]
@@ -790,6 +811,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       if (!ok) break;
       // the item's last dQ partial
       if (!dq_readout(t - 1)) break;
+      // the pending table-gradient sums
+      if (has_time) {
+        flush_time(pend_b, pend_lo);
+        flush_time(pend_b + 1, pend_hi);
+      }
+      if (has_pos) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) pend_p += __shfl_xor_sync(0xffffffffu, pend_p, o);
+        if (lane == 0 && pend_p != 0.0f) atomicAdd(prm.dpos + (int64_t)h * P + (P - 1), pend_p);
+      }
       // dV_j and dK_j of this item: TMEM lane = key row; this warp's 16 of the 64 columns
       if (!mbar_wait(dkv_full, k & 1u, abort_flag)) break;
       tc_fence_after();
