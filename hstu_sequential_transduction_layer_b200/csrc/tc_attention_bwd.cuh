@@ -139,13 +139,6 @@ __global__ void __launch_bounds__(1024) bwd_schedule_kernel(const int64_t* __res
   }
 }
 
-// SiLU and its derivative from one MUFU tanh: s = sigmoid(x) = 0.5 + 0.5 tanh(x/2).
-__device__ __forceinline__ void silu_and_grad(float x, float& silu, float& dsilu) {
-  const float sg = fmaf(0.5f, sm100::tanh_approx(0.5f * x), 0.5f);
-  silu = x * sg;
-  dsilu = sg * fmaf(x, 1.0f - sg, 1.0f);
-}
-
 // Called by a full warp, lane l holding the 4 consecutive timestamps t[4l .. 4l+3] of a 128-row
 // tile: a 4-bit mask, bit g set when rows 32g .. 32g+31 are in non-decreasing order.
 __device__ __forceinline__ int sorted_groups(const int64_t* t, int lane) {
@@ -212,6 +205,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   constexpr bool has_time = (BM & BWD_TIME) != 0;
   constexpr bool has_pos = (BM & BWD_POS) != 0;
   constexpr bool alibi = (BM & BWD_ALIBI) != 0;
+  constexpr bool WIN = has_pos || alibi;   // a per-block window of the distance bias
   const bool aligned = (smem_u32(smem) & 1023u) == 0;
   const int64_t n_items = aligned ? sch.header[0] : 0;
 
@@ -510,7 +504,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const float slope = alibi ? prm.alibi[h] : 0.0f;
       if (has_time && h != staged_head) {
         if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;
-        for (int e = tid; e < tcap; e += BWD_PW) tt_s[e] = __ldg(tim_h + e);
+        for (int e = tid; e < tcap; e += BWD_PW) tt_s[e] = 0.5f * __ldg(tim_h + e);
         staged_head = h;
         if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;
       }
@@ -556,11 +550,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         uint32_t sv[16], dpv[16];
         tmem_ld16(t_lane + Cfg::S_COL + qb, sv);
         tmem_ld16(t_lane + Cfg::DP_COL + qb, dpv);
-        if (has_pos) {
-          pwin[lane] = wv0;
-          pwin[32 + lane] = wv1;
-          __syncwarp();
-        }
         // Fast path when every score of the 32 x 16 block is valid (off the diagonal, inside the
         // sequence) and the time bucket is the same for the whole block, or takes two values
         // split by one threshold (sorted timestamps, the extreme corners' buckets equal or
@@ -592,19 +581,34 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           }
         }
         const bool fast = full && (!has_time || tmode != 0);
-        const float* pl = pwin + 31 - lane;       // pl[e]: position bias of (lane, e)
-        // time-bucket gradient of the general loop: the block's buckets along a row are those
-        // of its first query and the next one up (queries are later in time along the row);
+        // time-gradient bucket of the general loop's rows: the block's buckets along a row are
+        // those of its first query and the next one up (queries are later in time along the row);
         // others go directly
         int tb_first = 0;
         if (has_time && !fast) {
           const int b = time_bucket(qt_s[0], tj);
           tb_first = b < Tb - 1 ? b : Tb - 1;
         }
-        const float tlo = (has_time && fast) ? tt_s[tb_u] : 0.0f;
-        const float thi = (has_time && tmode == 2) ? tt_s[tb_u + 1] : 0.0f;
-        const float pone = pos_one ? pl[0] : 0.0f;  // every window entry is the last bucket
-        const float al0 = -slope * (float)(dbase - lane);
+        // Everything below works on h = x / 2 (the table holds half the time biases, the window
+        // half the position or ALiBi biases): sigmoid(x) = (1 + tanh(h)) / 2.
+        const float htlo = (has_time && fast) ? tt_s[tb_u] : 0.0f;
+        const float hthi = (has_time && tmode == 2) ? tt_s[tb_u + 1] : 0.0f;
+        // the window: half the bias at distances dbase - 31 + x, with a fast block's one time
+        // bucket folded in
+        if (WIN) {
+          const float add = tmode == 1 ? htlo : 0.0f;
+          float w0 = 0.5f * wv0, w1 = 0.5f * wv1;
+          if (alibi) {
+            w0 = -0.5f * slope * (float)(dbase - 31 + lane);
+            w1 = -0.5f * slope * (float)(dbase + 1 + lane);
+          }
+          pwin[lane] = w0 + add;
+          pwin[32 + lane] = w1 + add;
+          __syncwarp();
+        }
+        const float* pl = pwin + 31 - lane;       // pl[e]: half bias of (lane, e)
+        // the constant half bias of a fast block without a per-element lookup
+        const float hconst = pos_one ? pl[0] : (tmode == 1 ? htlo : 0.0f);
         float acc_u = 0.0f, acc_h = 0.0f, acc_pu = 0.0f, acc_lo = 0.0f, acc_hi = 0.0f;
         float sacc = 0.0f;                        // systolic diagonal sum (position gradient)
         float* caph = cap - 1;                    // caph[ee]: diagonal completed at column ee
@@ -621,7 +625,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             sacc = fmaf(__shfl_up_sync(0xffffffffu, sacc, 1), m0, dx);
           }
         };
-        // the fast element loop: no masks; the time bias one or two constants
+        // P = scale SiLU(x) = h c2 and dS = scale SiLU'(x) dP = c2 (1/2 + h (1 - sigmoid)) dP,
+        // with c2 = 2 scale sigmoid(x) = scale (1 + tanh(h))
+        // the fast element loop: no masks; the half bias a window entry or a constant (TM = 2:
+        // plus one of two time biases split by a threshold)
         auto fast16 = [&](auto tm_tag, auto po_tag) {
           constexpr int TM = decltype(tm_tag)::value;
           constexpr bool PO = decltype(po_tag)::value;
@@ -630,24 +637,22 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             float a2[2], d2[2];
 #pragma unroll
             for (int u = 0; u < 2; u++) {
-              float x = __uint_as_float(sv[ee + u]);
+              float hb = (WIN && !PO) ? pl[ee + u] : hconst;
               bool hi = false;
               if (TM == 2) {
                 hi = qt32[ee + u] - tk32 >= thr;
-                x += hi ? thi : tlo;
-              } else if (TM == 1) {
-                x += tlo;
+                hb += hi ? hthi : htlo;
               }
-              if (has_pos) x += PO ? pone : pl[ee + u];
-              if (alibi) x += fmaf(-slope, (float)(ee + u), al0);
-              float sl, dsl;
-              silu_and_grad(x, sl, dsl);
-              const float dx = scale * dsl * __uint_as_float(dpv[ee + u]);
-              a2[u] = scale * sl;
+              const float hh = fmaf(__uint_as_float(sv[ee + u]), 0.5f, hb);
+              const float th = tanh_approx(hh);
+              const float c2 = fmaf(scale, th, scale);
+              const float om = fmaf(-0.5f, th, 0.5f);
+              const float dx = c2 * fmaf(hh, om, 0.5f) * __uint_as_float(dpv[ee + u]);
+              a2[u] = hh * c2;
               d2[u] = dx;
               if (PO) acc_pu += dx;
               else if (has_pos) systolic(ee + u, dx);
-              if (TM != 0) acc_u += dx;
+              if (has_time && !has_pos) acc_u += dx;
               if (TM == 2) acc_h += hi ? dx : 0.0f;
             }
             pk[ee / 2] = pack_bf16x2(a2[0], a2[1]);
@@ -664,12 +669,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 #pragma unroll
             for (int u = 0; u < 2; u++) {
               const int iq = qc0 + ee + u;           // query (local index)
-              const int dist = iq - j;
-              const bool valid = kvalid && iq < n && dist >= 0;
-              float bias = 0.0f;
+              const bool valid = kvalid && iq < n && iq >= j;
+              float hb = WIN ? pl[ee + u] : 0.0f;
               int tb = 0;
-              if (alibi) bias = -slope * (float)dist;
-              if (has_pos) bias += pl[ee + u];
               if (has_time) {
                 if (REL32) {
                   // floor(log2(1 + max(ti - tj, 0))) = 31 - clz(max(ti - tj, 0) + 1)
@@ -679,12 +681,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                   tb = time_bucket(qt_s[ee + u], tj);
                 }
                 tb = tb < Tb - 1 ? tb : Tb - 1;
-                bias += tt_s[tb];
+                hb += tt_s[tb];
               }
-              float sl, dsl;
-              silu_and_grad(__uint_as_float(sv[ee + u]) + bias, sl, dsl);
-              const float dx = valid ? scale * dsl * __uint_as_float(dpv[ee + u]) : 0.0f;
-              a2[u] = valid ? scale * sl : 0.0f;
+              const float hh = fmaf(__uint_as_float(sv[ee + u]), 0.5f, hb);
+              const float th = tanh_approx(hh);
+              const float c2 = fmaf(scale, th, scale);
+              const float om = fmaf(-0.5f, th, 0.5f);
+              const float dx = valid ? c2 * fmaf(hh, om, 0.5f) * __uint_as_float(dpv[ee + u]) : 0.0f;
+              a2[u] = valid ? hh * c2 : 0.0f;
               d2[u] = dx;
               if (has_pos) systolic(ee + u, dx);
               if (has_time) {
@@ -732,11 +736,32 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                          ((uu ^ (r & 7)) * 16);
           *reinterpret_cast<uint4*>(dst) = make_uint4(dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]);
         }
-        // table gradients of the block
+        // position gradient of the block: its diagonal sums, two per lane (the global reductions
+        // are issued after the arrive below: an arrive releases this warp's earlier writes, so
+        // reductions still in flight would hold it back); a block entirely in the last bucket
+        // adds its total to a per-lane sum sent at the item's end
+        float pg0 = 0.0f, pg1 = 0.0f;
+        int pd0 = -1, pd1 = -1;
+        if (pos_one && fast) {
+          pend_p += acc_pu;
+        } else if (has_pos) {
+          // lane l: diagonal 15 - l in the systolic sum; lanes 0..14: diagonal l - 31 parked in
+          // cap[l]
+          __syncwarp();
+          pg1 = lane < 15 ? cap[lane] : 0.0f;
+          __syncwarp();
+          const int da = dbase + 15 - lane, db = dbase + lane - 31;
+          pg0 = sacc;
+          pd0 = da < 0 ? -1 : (da < P - 1 ? da : P - 1);
+          pd1 = db < 0 ? -1 : (db < P - 1 ? db : P - 1);
+        }
+        // time gradient of the block
         if (has_time && fast) {
-          // the block's sums in buckets tb_u and tb_u + 1 join the pending pair (flushed when the
-          // buckets move on: along a warp's blocks the queries only get later)
-          const float lo = acc_u - acc_h, hi = acc_h;
+          // per-lane part of the block's sum (every diagonal sum sits in one lane), split into
+          // buckets tb_u and tb_u + 1; it joins the pending pair, flushed when the buckets move
+          // on (along a warp's blocks the queries only get later)
+          const float tot = has_pos ? (pos_one ? acc_pu : pg0 + pg1) : acc_u;
+          const float lo = tot - acc_h, hi = acc_h;
           if (tb_u == pend_b) {
             pend_lo += lo;
             pend_hi += hi;
@@ -773,26 +798,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             if (acc_lo != 0.0f) atomicAdd(&dtt_s[tb_first], acc_lo);
             if (acc_hi != 0.0f) atomicAdd(&dtt_s[tb_first + 1], acc_hi);
           }
-        }
-        // the position gradient's two sums per lane (the global reductions are issued after the
-        // arrive below: an arrive releases this warp's earlier writes, so reductions still in
-        // flight would hold it back)
-        float pg0 = 0.0f, pg1 = 0.0f;
-        int pd0 = -1, pd1 = -1;
-        if (pos_one && fast) {
-          // every distance of the block is clamped to the last bucket: summed per lane over the
-          // item, sent at its end
-          pend_p += acc_pu;
-        } else if (has_pos) {
-          // lane l: diagonal 15 - l in the systolic sum; lanes 0..14: diagonal l - 31 parked in
-          // cap[l]
-          __syncwarp();
-          pg1 = lane < 15 ? cap[lane] : 0.0f;
-          __syncwarp();
-          const int da = dbase + 15 - lane, db = dbase + lane - 31;
-          pg0 = sacc;
-          pd0 = da < 0 ? -1 : (da < P - 1 ? da : P - 1);
-          pd1 = db < 0 ? -1 : (db < P - 1 ? db : P - 1);
         }
         tmem_st_wait();
         tc_fence_before();
