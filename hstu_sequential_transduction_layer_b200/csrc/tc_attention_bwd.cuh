@@ -257,21 +257,33 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const int64_t row0 = sch.seqinfo[2 * seq], n = sch.seqinfo[2 * seq + 1];
       const int nt = (int)((n + ATT_BN - 1) / ATT_BN);
       const int k0 = jt * ATT_BN;
+      // the key tile's timestamps, loaded before the stage is free
+      int64_t tv[4] = {0, 0, 0, 0};
+      int64_t t0 = 0;
+      if (has_time) {
+        t0 = prm.ts[row0];
+#pragma unroll
+        for (int e = 0; e < 4; e++) {
+          const int64_t jj = k0 + 4 * lane + e;
+          tv[e] = prm.ts[row0 + (jj < n ? jj : n - 1)];
+        }
+      }
       if (lane == 0) ok = mbar_wait(kv_empty, (k & 1u) ^ 1u, abort_flag);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
+      if (lane == 0) {
+        mbar_expect_tx(kv_full, 2 * Cfg::BOX);
+        tma_load_2d(k_s, &tm, kv_full, col_k + h * 64, (int)row0 + k0);
+        tma_load_2d(v_s, &tm, kv_full, col_v + h * 64, (int)row0 + k0);
+        kv_par = (int)(k & 1u);
+      }
       if (has_time) {
-#pragma unroll
-        for (int e = 0; e < 4; e++) {
-          const int64_t j = k0 + 4 * lane + e;
-          kts[4 * lane + e] = prm.ts[row0 + (j < n ? j : n - 1)];
-        }
-        // the same relative to the sequence's first timestamp, as int32 when every one fits
-        const int64_t t0 = prm.ts[row0];
+        // also relative to the sequence's first timestamp, as int32 when every one fits
         bool fits = true;
 #pragma unroll
         for (int e = 0; e < 4; e++) {
-          const int64_t rel = kts[4 * lane + e] - t0;
+          kts[4 * lane + e] = tv[e];
+          const int64_t rel = tv[e] - t0;
           fits = fits && rel > -(1LL << 30) && rel < (1LL << 30);
           kts32[4 * lane + e] = (int)rel;
         }
@@ -281,28 +293,34 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         if (lane == 0) tsort[0] = sm;
       }
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_expect_tx(kv_full, 2 * Cfg::BOX);
-        tma_load_2d(k_s, &tm, kv_full, col_k + h * 64, (int)row0 + k0);
-        tma_load_2d(v_s, &tm, kv_full, col_v + h * 64, (int)row0 + k0);
-        kv_par = (int)(k & 1u);
-      }
+      if (lane == 0) mbar_arrive(kv_full);
       for (int i = jt; i < nt && ok; i++, g++) {
         const uint32_t st = g % Cfg::NST, ph = (g / Cfg::NST) & 1u;
-        if (lane == 0) ok = mbar_wait(&q_empty[st], ph ^ 1u, abort_flag);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
+        // the query tile's timestamps, loaded before the stage is free
         if (has_time) {
 #pragma unroll
           for (int e = 0; e < 4; e++) {
             const int64_t qi = (int64_t)i * ATT_BM + 4 * lane + e;
-            qts[st * 128 + 4 * lane + e] = prm.ts[row0 + (qi < n ? qi : n - 1)];
+            tv[e] = prm.ts[row0 + (qi < n ? qi : n - 1)];
           }
-          const int64_t t0 = prm.ts[row0];
+        }
+        if (lane == 0) ok = mbar_wait(&q_empty[st], ph ^ 1u, abort_flag);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        if (lane == 0) {
+          mbar_expect_tx(&q_full[st], 2 * Cfg::BOX);
+          tma_load_2d(smem + Cfg::OFF_Q + st * Cfg::BOX, &tm, &q_full[st], col_q + h * 64,
+                      (int)row0 + i * ATT_BM);
+          tma_load_2d(smem + Cfg::OFF_DO + st * Cfg::BOX, &tdo, &q_full[st], h * 64,
+                      (int)row0 + i * ATT_BM);
+          q_par[st] = (int)ph;
+        }
+        if (has_time) {
           bool fits = true;
 #pragma unroll
           for (int e = 0; e < 4; e++) {
-            const int64_t rel = qts[st * 128 + 4 * lane + e] - t0;
+            qts[st * 128 + 4 * lane + e] = tv[e];
+            const int64_t rel = tv[e] - t0;
             fits = fits && rel > -(1LL << 30) && rel < (1LL << 30);
             qts32[st * 128 + 4 * lane + e] = (int)rel;
           }
@@ -311,15 +329,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           const int sm = sorted_groups(qts + st * 128 + 4 * lane, lane);
           if (lane == 0) tsort[1 + st] = sm;
         }
+        // the timestamps are published with the tiles: the arrival completes the phase
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&q_full[st], 2 * Cfg::BOX);
-          tma_load_2d(smem + Cfg::OFF_Q + st * Cfg::BOX, &tm, &q_full[st], col_q + h * 64,
-                      (int)row0 + i * ATT_BM);
-          tma_load_2d(smem + Cfg::OFF_DO + st * Cfg::BOX, &tdo, &q_full[st], h * 64,
-                      (int)row0 + i * ATT_BM);
-          q_par[st] = (int)ph;
-        }
+        if (lane == 0) mbar_arrive(&q_full[st]);
       }
     }
     if (!ok && lane == 0) {
