@@ -43,7 +43,10 @@ namespace tc {
 constexpr int BWD_THREADS = 640;     // producer, MMA issuer, 2 idle warps, 16 pointwise
 constexpr int BWD_PW = 512;          // pointwise threads
 constexpr int BWD_PW_WARPS = 16;
-constexpr int BWD_TB_CAP = 256;
+// Time buckets floor(log2(1 + dt)) never exceed 63, so at most 64 entries of a time table are
+// used; the tables of all heads are staged at once when H * min(Tb, 64) entries fit.
+constexpr int BWD_TB_USED = 64;
+constexpr int BWD_TT_ALL = 2048;
 
 struct BwdCfg {
   static constexpr int BOX = 128 * 64 * 2;                  // 128 rows x 64 bf16
@@ -62,9 +65,9 @@ struct BwdCfg {
   static constexpr int OFF_TFLAG = OFF_KTS32 + 128 * 4;     // [NST] query fits, [NST] key fits
   static constexpr int OFF_PWIN = OFF_TFLAG + 64;           // [16 warps][64] float: table window
   static constexpr int OFF_CAP = OFF_PWIN + BWD_PW_WARPS * 64 * 4;      // [16 warps][32] float
-  static constexpr int OFF_TT = OFF_CAP + BWD_PW_WARPS * 32 * 4;        // [TB_CAP] float time table
-  static constexpr int OFF_DTT = OFF_TT + BWD_TB_CAP * 4;     // [TB_CAP] float its gradient
-  static constexpr int OFF_BAR = OFF_DTT + BWD_TB_CAP * 4;
+  static constexpr int OFF_TT = OFF_CAP + BWD_PW_WARPS * 32 * 4;        // [TT_ALL] half time tables
+  static constexpr int OFF_DTT = OFF_TT + BWD_TT_ALL * 4;     // [TT_ALL] float their gradients
+  static constexpr int OFF_BAR = OFF_DTT + BWD_TT_ALL * 4;
   static constexpr int SMEM = OFF_BAR + 256;
   static constexpr int TMEM_COLS = 512;
   static constexpr int S_COL = 0, DP_COL = 128, DV_COL = 256, DK_COL = 320, DQ_COL = 384;
@@ -235,7 +238,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     prefetch_tensormap(&tdo);
     prefetch_tensormap(&tdq);
   }
-  for (int e = threadIdx.x; e < BWD_TB_CAP; e += BWD_THREADS) dtt_s[e] = 0.0f;
+  for (int e = threadIdx.x; e < BWD_TT_ALL; e += BWD_THREADS) dtt_s[e] = 0.0f;
   if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tmem_relinquish();
@@ -471,7 +474,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const int tid = threadIdx.x - 128;
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const int P = prm.P, Tb = prm.Tb;
-    const int tcap = Tb < BWD_TB_CAP ? Tb : BWD_TB_CAP;
+    const int tcap = Tb < BWD_TB_USED ? Tb : BWD_TB_USED;          // entries in use per head
+    const bool all_heads = has_time && H * tcap <= BWD_TT_ALL;     // every head staged at once
     const float scale = prm.scale;
     const float m0 = lane > 0 ? 1.0f : 0.0f;
     float* pwin = pwin_s + pw * 64;      // the position table at the block's 47 distances
@@ -479,6 +483,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     uint32_t k = 0, g = 0, t = 0, pw_cnt = 0;
     int staged_head = -1;
     bool ok = true;
+    if (all_heads) {
+      for (int e = tid; e < H * tcap; e += BWD_PW) {
+        const int hh = e / tcap, b = e - hh * tcap;
+        tt_s[e] = 0.5f * __ldg(prm.tim + (int64_t)hh * Tb + b);
+      }
+      ok = group_sync(pw_bar, pw_cnt, abort_flag);
+    }
     // The dQ partial of tile tt (TMEM lane = query row; this warp's 16 of the 64 columns) into the
     // staging buffer, from which warp 2 adds it to global dQ with TMA reductions: row = query r,
     // two 128-byte-swizzled boxes of 32 columns.
@@ -514,12 +525,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       const float* pos_h = has_pos ? prm.pos + (int64_t)h * P : nullptr;
       const float* tim_h = has_time ? prm.tim + (int64_t)h * Tb : nullptr;
       const float slope = alibi ? prm.alibi[h] : 0.0f;
-      if (has_time && h != staged_head) {
+      if (has_time && !all_heads && h != staged_head) {
         if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;
         for (int e = tid; e < tcap; e += BWD_PW) tt_s[e] = 0.5f * __ldg(tim_h + e);
         staged_head = h;
         if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;
       }
+      // this head's half time table and its gradient in shared memory
+      const float* tt_h = tt_s + (all_heads ? h * tcap : 0);
+      float* dtt_h = dtt_s + (all_heads ? h * tcap : 0);
       if (!mbar_wait(kv_full, k & 1u, abort_flag)) break;
       const int j = k0 + r;                       // this thread's key (local index)
       const bool kvalid = j < n;
@@ -534,7 +548,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       auto flush_time = [&](int b, float v) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0 && b >= 0 && v != 0.0f) atomicAdd(&dtt_s[b], v);
+        if (lane == 0 && b >= 0 && v != 0.0f) atomicAdd(&dtt_h[b], v);
       };
       for (int i = jt; i < nt && ok; i++, g++, t++) {
         const uint32_t st = g % Cfg::NST;
@@ -603,8 +617,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         }
         // Everything below works on h = x / 2 (the table holds half the time biases, the window
         // half the position or ALiBi biases): sigmoid(x) = (1 + tanh(h)) / 2.
-        const float htlo = (has_time && fast) ? tt_s[tb_u] : 0.0f;
-        const float hthi = (has_time && tmode == 2) ? tt_s[tb_u + 1] : 0.0f;
+        const float htlo = (has_time && fast) ? tt_h[tb_u] : 0.0f;
+        const float hthi = (has_time && tmode == 2) ? tt_h[tb_u + 1] : 0.0f;
         // the window: half the bias at distances dbase - 31 + x, with a fast block's one time
         // bucket folded in
         if (WIN) {
@@ -693,7 +707,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                   tb = time_bucket(qt_s[ee + u], tj);
                 }
                 tb = tb < Tb - 1 ? tb : Tb - 1;
-                hb += tt_s[tb];
+                hb += tt_h[tb];
               }
               const float hh = fmaf(__uint_as_float(sv[ee + u]), 0.5f, hb);
               const float th = tanh_approx(hh);
@@ -711,7 +725,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                 // warp vote keeps the shared-memory atomic off the common path
                 const bool far = valid && (db < 0 || db > 1);
                 if (__any_sync(0xffffffffu, far)) {
-                  if (far) atomicAdd(&dtt_s[tb], dx);
+                  if (far) atomicAdd(&dtt_h[tb], dx);
                 }
               }
             }
@@ -807,8 +821,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           }
           const bool last = lane == 31 || ((heads >> (lane + 1)) & 1u);
           if (last) {
-            if (acc_lo != 0.0f) atomicAdd(&dtt_s[tb_first], acc_lo);
-            if (acc_hi != 0.0f) atomicAdd(&dtt_s[tb_first + 1], acc_hi);
+            if (acc_lo != 0.0f) atomicAdd(&dtt_h[tb_first], acc_lo);
+            if (acc_hi != 0.0f) atomicAdd(&dtt_h[tb_first + 1], acc_hi);
           }
         }
         tmem_st_wait();
@@ -864,8 +878,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           }
         }
       }
-      // table gradients of this item to global memory
-      if (has_time) {
+      // the time-table gradient of this item to global memory (one head staged at a time)
+      if (has_time && !all_heads) {
         if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;
         for (int e = tid; e < tcap; e += BWD_PW) {
           const float v = dtt_s[e];
@@ -873,6 +887,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           dtt_s[e] = 0.0f;
         }
         if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;
+      }
+    }
+    // every head's time-table gradient, once, after the last item
+    if (all_heads && ok && group_sync(pw_bar, pw_cnt, abort_flag)) {
+      for (int e = tid; e < H * tcap; e += BWD_PW) {
+        const float v = dtt_s[e];
+        const int hh = e / tcap, b = e - hh * tcap;
+        if (v != 0.0f) atomicAdd(prm.dtime + (int64_t)hh * Tb + b, v);
       }
     }
   }
