@@ -46,11 +46,11 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per attention launch from the committed ncu summary, if it was captured on this
+def profiled_traffic(workload: str, kernel: str = "attention_tc_kernel"):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if it was captured on this
     workload from the kernel source as it is now (else None)."""
     import hashlib
-    path = os.path.join(ROOT, "profiles", f"attention_tc_kernel_{workload}.md")
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(path):
         return None
     fields = {}
@@ -598,7 +598,8 @@ def run_backward(args, rank, world, local_rank):
                                f"H={H}x{hd}, rab P={w.n_pos_buckets}/Tb={w.n_time_buckets}",
                    "l2": "flushed between timed steps (outside the events)"},
         "roofline": {"bound": "tensor", "kernel": "attention_bwd", "achieved": round(tf, 2),
-                     "peak": tpk, "unit": "TFLOP/s", "frac": round(tf / tpk, 4), "traffic": None,
+                     "peak": tpk, "unit": "TFLOP/s", "frac": round(tf / tpk, 4),
+                     "traffic": profiled_traffic(w.name, "attention_bwd_kernel"),
                      "peak_source": f"{peaks_src} bf16 burst (MEASURED_PEAKS.json)"},
         "gpu_launches": int(launches), "clocks": clocks,
     }
@@ -709,7 +710,8 @@ def run_train(args, rank, world, local_rank):
                    "l2": "flushed between timed steps (outside the events)",
                    "step_tflops": round(step_fl / ms / 1e9, 2)},
         "roofline": {"bound": "tensor", "kernel": "attention_bwd", "achieved": round(a_tf, 2),
-                     "peak": tpk, "unit": "TFLOP/s", "frac": round(a_tf / tpk, 4), "traffic": None,
+                     "peak": tpk, "unit": "TFLOP/s", "frac": round(a_tf / tpk, 4),
+                     "traffic": profiled_traffic(w.name, "attention_bwd_kernel"),
                      "ms_per_launch": round(a_ms, 4),
                      "peak_source": f"{peaks_src} bf16 burst (MEASURED_PEAKS.json)"},
         "gpu_launches": int(launches), "clocks": clocks,
