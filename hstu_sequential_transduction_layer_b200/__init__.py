@@ -34,7 +34,10 @@ EXPORTED = ["hstu_layer_fwd", "hstu_layer_fwd_workspace_size", "hstu_f1_fwd", "h
             "hstu_candidate_layer_workspace_size", "hstu_candidate_layer_fwd",
             "hstu_stochastic_length_workspace_size", "hstu_stochastic_length", "hstu_gather_rows",
             "hstu_attention_bwd_workspace_size", "hstu_attention_bwd",
-            "hstu_layer_bwd_workspace_size", "hstu_layer_bwd"]
+            "hstu_layer_bwd_workspace_size", "hstu_layer_bwd", "hstu_layer_pipeline_create",
+            "hstu_layer_pipeline_submit", "hstu_layer_pipeline_sync",
+            "hstu_layer_pipeline_timing_begin", "hstu_layer_pipeline_timing_end",
+            "hstu_layer_pipeline_destroy"]
 
 
 class HstuShape(ctypes.Structure):
@@ -90,6 +93,13 @@ def _load() -> ctypes.CDLL:
         "hstu_candidate_layer_fwd": ([SH, P, P, P, I64, I64, P, P, P, P, P, P, P, P, P, P, P, P, F32,
                                       P, P, S, P], ctypes.c_int),
         "hstu_layer_bwd_workspace_size": ([SH], S),
+        "hstu_layer_pipeline_create": ([SH, I32, ctypes.POINTER(ctypes.c_void_p)], ctypes.c_int),
+        "hstu_layer_pipeline_submit": ([P, SH, P, P, P, P, P, P, P, P, P, P, P, P, F32, P],
+                                       ctypes.c_int),
+        "hstu_layer_pipeline_sync": ([P], ctypes.c_int),
+        "hstu_layer_pipeline_timing_begin": ([P], ctypes.c_int),
+        "hstu_layer_pipeline_timing_end": ([P, ctypes.POINTER(ctypes.c_float)], ctypes.c_int),
+        "hstu_layer_pipeline_destroy": ([P], None),
         "hstu_layer_bwd": ([SH, P, P, P, P, P, P, P, P, P, P, P, F32, P, S, P, P, P, P, P, P, P, P,
                             P, P, P, S, P], ctypes.c_int),
     }
@@ -324,6 +334,48 @@ def hstu_layer_bwd(shape: HstuShape, X, seq_offsets, timestamps, W1, b1, W2, ln_
                                workspace.numel(), _stream(stream)), "hstu_layer_bwd")
     return {"dX": dX, "dW1": dW1, "db1": db1, "dW2": dW2, "db2": db2, "dln_w": dln_w,
             "dln_b": dln_b, "dpos": dpos_table, "dtime": dtime_table}
+
+
+class LayerPipeline:
+    """hstu_layer_fwd over batches in host memory, the copies in and out overlapped with the
+    layers of neighbouring batches (see the C header).  Host tensors should be pinned."""
+
+    def __init__(self, capacity: HstuShape, depth: int = 2):
+        self._p = ctypes.c_void_p()
+        _check(_lib.hstu_layer_pipeline_create(ctypes.byref(capacity), int(depth),
+                                               ctypes.byref(self._p)), "hstu_layer_pipeline_create")
+
+    def submit(self, shape: HstuShape, X_host, seq_offsets_host, timestamps_host, W1, b1, W2, b2,
+               ln_w, ln_b, pos_table, time_table, alibi_slopes, scale: float, out_host):
+        _check(_lib.hstu_layer_pipeline_submit(
+            self._p, ctypes.byref(shape), _ptr(X_host), _ptr(seq_offsets_host),
+            _ptr(timestamps_host), _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), _ptr(ln_w), _ptr(ln_b),
+            _ptr(pos_table), _ptr(time_table), _ptr(alibi_slopes), float(scale), _ptr(out_host)),
+            "hstu_layer_pipeline_submit")
+        return out_host
+
+    def sync(self) -> None:
+        _check(_lib.hstu_layer_pipeline_sync(self._p), "hstu_layer_pipeline_sync")
+
+    def timing_begin(self) -> None:
+        _check(_lib.hstu_layer_pipeline_timing_begin(self._p), "hstu_layer_pipeline_timing_begin")
+
+    def timing_end(self) -> float:
+        ms = ctypes.c_float()
+        _check(_lib.hstu_layer_pipeline_timing_end(self._p, ctypes.byref(ms)),
+               "hstu_layer_pipeline_timing_end")
+        return float(ms.value)
+
+    def close(self) -> None:
+        if self._p:
+            _lib.hstu_layer_pipeline_destroy(self._p)
+            self._p = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def hstu_stochastic_length(seq_offsets, max_len: int, alpha: float, u, keys, new_offsets, index,

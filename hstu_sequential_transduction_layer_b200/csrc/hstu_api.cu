@@ -4,6 +4,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "common.cuh"
 #include "hbm_kernels.cuh"
@@ -844,5 +845,180 @@ hstu_status_t hstu_selftest_bounded_wait(uint64_t limit_ns, long long* result, v
   selftest_bounded_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, result);
   return launch_status();
 }
+
+}  // extern "C"
+
+// ------------------------------------------------------------------------------------------------
+// Host-to-host layer pipeline
+// ------------------------------------------------------------------------------------------------
+
+struct hstu_layer_pipeline {
+  hstu_shape_t cap;
+  int depth = 0;
+  uint64_t count = 0;
+  cudaStream_t s_in = nullptr, s_comp = nullptr, s_out = nullptr;
+  std::vector<void*> X, out;
+  std::vector<int64_t*> off, ts;
+  std::vector<cudaEvent_t> in_done, comp_done, out_done;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  cudaEvent_t t0 = nullptr, t1 = nullptr;
+  bool timing = false;
+};
+
+namespace {
+
+void pipeline_free(hstu_layer_pipeline* p) {
+  if (!p) return;
+  for (cudaStream_t s : {p->s_in, p->s_comp, p->s_out})
+    if (s) cudaStreamSynchronize(s);
+  for (void* b : p->X) cudaFree(b);
+  for (void* b : p->out) cudaFree(b);
+  for (int64_t* b : p->off) cudaFree(b);
+  for (int64_t* b : p->ts) cudaFree(b);
+  for (auto* v : {&p->in_done, &p->comp_done, &p->out_done})
+    for (cudaEvent_t e : *v) cudaEventDestroy(e);
+  if (p->t0) cudaEventDestroy(p->t0);
+  if (p->t1) cudaEventDestroy(p->t1);
+  cudaFree(p->ws);
+  for (cudaStream_t s : {p->s_in, p->s_comp, p->s_out})
+    if (s) cudaStreamDestroy(s);
+  delete p;
+}
+
+bool same_model(const hstu_shape_t& a, const hstu_shape_t& b) {
+  return a.d_model == b.d_model && a.num_heads == b.num_heads && a.d_qk == b.d_qk &&
+         a.d_v == b.d_v && a.n_pos_buckets == b.n_pos_buckets &&
+         a.n_time_buckets == b.n_time_buckets && a.dtype == b.dtype && a.ln_eps == b.ln_eps;
+}
+
+}  // namespace
+
+extern "C" {
+
+hstu_status_t hstu_layer_pipeline_create(const hstu_shape_t* capacity, int32_t depth,
+                                         hstu_layer_pipeline_t** out) {
+  if (!out) return HSTU_ERR_INVALID_ARG;
+  *out = nullptr;
+  hstu_status_t rc = check_shape(capacity);
+  if (rc != HSTU_OK) return rc;
+  if (depth < 2 || depth > 8 || capacity->total_tokens <= 0 || capacity->num_seqs <= 0)
+    return HSTU_ERR_INVALID_ARG;
+  auto* p = new hstu_layer_pipeline();
+  p->cap = *capacity;
+  p->depth = depth;
+  const size_t T = (size_t)capacity->total_tokens, B = (size_t)capacity->num_seqs;
+  const size_t xb = T * (size_t)capacity->d_model * esize(*capacity);
+  bool okc = cudaStreamCreateWithFlags(&p->s_in, cudaStreamNonBlocking) == cudaSuccess &&
+             cudaStreamCreateWithFlags(&p->s_comp, cudaStreamNonBlocking) == cudaSuccess &&
+             cudaStreamCreateWithFlags(&p->s_out, cudaStreamNonBlocking) == cudaSuccess &&
+             cudaEventCreate(&p->t0) == cudaSuccess && cudaEventCreate(&p->t1) == cudaSuccess;
+  for (int i = 0; okc && i < depth; i++) {
+    void *x = nullptr, *o = nullptr;
+    int64_t *f = nullptr, *tt = nullptr;
+    cudaEvent_t e[3] = {nullptr, nullptr, nullptr};
+    okc = cudaMalloc(&x, xb) == cudaSuccess && cudaMalloc(&o, xb) == cudaSuccess &&
+          cudaMalloc(&f, (B + 1) * sizeof(int64_t)) == cudaSuccess &&
+          cudaMalloc(&tt, T * sizeof(int64_t)) == cudaSuccess;
+    for (int k = 0; okc && k < 3; k++)
+      okc = cudaEventCreateWithFlags(&e[k], cudaEventDisableTiming) == cudaSuccess;
+    p->X.push_back(x);
+    p->out.push_back(o);
+    p->off.push_back(f);
+    p->ts.push_back(tt);
+    if (e[0]) p->in_done.push_back(e[0]);
+    if (e[1]) p->comp_done.push_back(e[1]);
+    if (e[2]) p->out_done.push_back(e[2]);
+  }
+  if (okc) {
+    p->ws_bytes = hstu_layer_fwd_workspace_size(capacity);
+    okc = p->ws_bytes > 0 && cudaMalloc(&p->ws, p->ws_bytes) == cudaSuccess;
+  }
+  if (!okc) {
+    cudaGetLastError();
+    pipeline_free(p);
+    return HSTU_ERR_CUDA;
+  }
+  *out = p;
+  return HSTU_OK;
+}
+
+hstu_status_t hstu_layer_pipeline_submit(hstu_layer_pipeline_t* p, const hstu_shape_t* shape,
+                                         const void* X_host, const int64_t* seq_offsets_host,
+                                         const int64_t* timestamps_host, const void* W1,
+                                         const void* b1, const void* W2, const void* b2,
+                                         const void* ln_w, const void* ln_b,
+                                         const float* pos_table, const float* time_table,
+                                         const float* alibi_slopes, float scale, void* out_host) {
+  if (!p) return HSTU_ERR_INVALID_ARG;
+  hstu_status_t rc = check_shape(shape);
+  if (rc != HSTU_OK) return rc;
+  const hstu_shape_t& s = *shape;
+  if (!same_model(s, p->cap) || s.total_tokens > p->cap.total_tokens ||
+      s.num_seqs > p->cap.num_seqs || s.max_seq_len > p->cap.max_seq_len)
+    return HSTU_ERR_INVALID_ARG;
+  if (s.total_tokens == 0) return HSTU_OK;
+  if (!X_host || !seq_offsets_host || !out_host || (time_table && !timestamps_host))
+    return HSTU_ERR_INVALID_ARG;
+  // the layer's own checks of the device arguments, before anything is enqueued
+  if ((rc = check_bias(shape, time_table ? p->ts[0] : nullptr, pos_table, time_table,
+                       alibi_slopes, scale)) != HSTU_OK)
+    return rc;
+  if (s.num_seqs == 0 || !W1 || !W2 || !ln_w || !ln_b) return HSTU_ERR_INVALID_ARG;
+  if (s.dtype == HSTU_BF16 && !(aligned16(W1) && aligned16(b1) && aligned16(W2) && aligned16(b2) &&
+                                aligned16(ln_w) && aligned16(ln_b)))
+    return HSTU_ERR_INVALID_ARG;
+  const int slot = (int)(p->count % (uint64_t)p->depth);
+  const size_t xb = (size_t)s.total_tokens * s.d_model * esize(s);
+  const bool reuse = p->count >= (uint64_t)p->depth;
+  bool okc = true;
+  // copy in: the slot's inputs are free once the layer that last read them has finished
+  if (reuse) okc = cudaStreamWaitEvent(p->s_in, p->comp_done[slot], 0) == cudaSuccess;
+  okc = okc && cudaMemcpyAsync(p->X[slot], X_host, xb, cudaMemcpyHostToDevice, p->s_in) == cudaSuccess;
+  okc = okc && cudaMemcpyAsync(p->off[slot], seq_offsets_host, (size_t)(s.num_seqs + 1) * sizeof(int64_t),
+                               cudaMemcpyHostToDevice, p->s_in) == cudaSuccess;
+  if (time_table)
+    okc = okc && cudaMemcpyAsync(p->ts[slot], timestamps_host, (size_t)s.total_tokens * sizeof(int64_t),
+                                 cudaMemcpyHostToDevice, p->s_in) == cudaSuccess;
+  okc = okc && cudaEventRecord(p->in_done[slot], p->s_in) == cudaSuccess;
+  // compute: after the copy in, and after the slot's previous output has been read back
+  okc = okc && cudaStreamWaitEvent(p->s_comp, p->in_done[slot], 0) == cudaSuccess;
+  if (reuse) okc = okc && cudaStreamWaitEvent(p->s_comp, p->out_done[slot], 0) == cudaSuccess;
+  if (!okc) return HSTU_ERR_CUDA;
+  rc = hstu_layer_fwd(shape, p->X[slot], p->off[slot], time_table ? p->ts[slot] : nullptr, W1, b1,
+                      W2, b2, ln_w, ln_b, pos_table, time_table, alibi_slopes, scale,
+                      p->out[slot], p->ws, p->ws_bytes, p->s_comp);
+  if (rc != HSTU_OK) return rc;
+  okc = cudaEventRecord(p->comp_done[slot], p->s_comp) == cudaSuccess &&
+        cudaStreamWaitEvent(p->s_out, p->comp_done[slot], 0) == cudaSuccess &&
+        cudaMemcpyAsync(out_host, p->out[slot], xb, cudaMemcpyDeviceToHost, p->s_out) == cudaSuccess &&
+        cudaEventRecord(p->out_done[slot], p->s_out) == cudaSuccess;
+  if (!okc) return HSTU_ERR_CUDA;
+  p->count++;
+  return HSTU_OK;
+}
+
+hstu_status_t hstu_layer_pipeline_sync(hstu_layer_pipeline_t* p) {
+  if (!p) return HSTU_ERR_INVALID_ARG;
+  for (cudaStream_t s : {p->s_in, p->s_comp, p->s_out})
+    if (cudaStreamSynchronize(s) != cudaSuccess) return HSTU_ERR_CUDA;
+  return HSTU_OK;
+}
+
+hstu_status_t hstu_layer_pipeline_timing_begin(hstu_layer_pipeline_t* p) {
+  if (!p) return HSTU_ERR_INVALID_ARG;
+  p->timing = true;
+  return cudaEventRecord(p->t0, p->s_in) == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+hstu_status_t hstu_layer_pipeline_timing_end(hstu_layer_pipeline_t* p, float* ms) {
+  if (!p || !ms || !p->timing) return HSTU_ERR_INVALID_ARG;
+  p->timing = false;
+  if (cudaEventRecord(p->t1, p->s_out) != cudaSuccess || hstu_layer_pipeline_sync(p) != HSTU_OK)
+    return HSTU_ERR_CUDA;
+  return cudaEventElapsedTime(ms, p->t0, p->t1) == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+void hstu_layer_pipeline_destroy(hstu_layer_pipeline_t* p) { pipeline_free(p); }
 
 }  // extern "C"

@@ -183,6 +183,43 @@ hstu_status_t hstu_attention_bwd(const hstu_shape_t* shape, const void* uvqk,
                                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * hstu_layer_pipeline_* -- hstu_layer_fwd over batches that live in host memory, with each batch's
+ * host-to-device copy, the previous batch's layer and the read-back of the one before overlapped
+ * on three CUDA streams (copy in, compute, copy out) and `depth` sets of device buffers.  A
+ * runtime convenience around hstu_layer_fwd (the pages describe no host pipeline).
+ *
+ *  create      capacity: the model dimensions of every batch (d, H, d_qk, d_v, P, Tb, dtype, eps)
+ *              and upper bounds on its token count, sequence count and longest sequence; depth
+ *              >= 2 buffer sets.  Allocates the device buffers and the workspace (cudaMalloc) and
+ *              the streams and events on the current device.  *out receives the pipeline.
+ *  submit      one batch: `shape` within the capacity (same model dimensions), X_host [T, d],
+ *              seq_offsets_host [B + 1], timestamps_host [T] (or NULL when time_table is NULL)
+ *              and out_host [T, d] in host memory (page-locked memory lets the copies overlap;
+ *              pageable memory works but serialises them); the weights and bias tables on the
+ *              device, as in hstu_layer_fwd.  Returns once the work is enqueued; the host buffers
+ *              must stay untouched until a later hstu_layer_pipeline_sync.  Argument errors are
+ *              returned before anything is enqueued.
+ *  sync        waits for every submitted batch; out_host then holds each batch's Y.
+ *  timing_begin / timing_end   device time from the start of the next submitted copy to the end
+ *              of the last read-back before timing_end (which synchronises), in milliseconds.
+ *  destroy     synchronises, then frees everything the pipeline owns.
+ */
+typedef struct hstu_layer_pipeline hstu_layer_pipeline_t;
+hstu_status_t hstu_layer_pipeline_create(const hstu_shape_t* capacity, int32_t depth,
+                                         hstu_layer_pipeline_t** out);
+hstu_status_t hstu_layer_pipeline_submit(hstu_layer_pipeline_t* p, const hstu_shape_t* shape,
+                                         const void* X_host, const int64_t* seq_offsets_host,
+                                         const int64_t* timestamps_host, const void* W1,
+                                         const void* b1, const void* W2, const void* b2,
+                                         const void* ln_w, const void* ln_b,
+                                         const float* pos_table, const float* time_table,
+                                         const float* alibi_slopes, float scale, void* out_host);
+hstu_status_t hstu_layer_pipeline_sync(hstu_layer_pipeline_t* p);
+hstu_status_t hstu_layer_pipeline_timing_begin(hstu_layer_pipeline_t* p);
+hstu_status_t hstu_layer_pipeline_timing_end(hstu_layer_pipeline_t* p, float* ms);
+void hstu_layer_pipeline_destroy(hstu_layer_pipeline_t* p);
+
+/*
  * hstu_layer_bwd -- backward of one layer ("Actions Speak Louder than Words" paper notes, section
  * 3.1, Eqs. 1-3 and the residual Y = f2(G) + X), for training: given dY = dL/dY, the gradients of
  * the loss with respect to X and every parameter of the layer,
