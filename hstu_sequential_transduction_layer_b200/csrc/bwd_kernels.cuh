@@ -49,6 +49,110 @@ __global__ void __launch_bounds__(256) colsum_kernel(int64_t rows, int cols, int
   }
 }
 
+// Column sums of a bf16 matrix [rows, cols] (cols % 8 == 0, cols <= 8 * blockDim.x): thread t
+// sums columns 8t .. 8t+7 over a range of rows with 16-byte loads, then adds its 8 sums to `out`.
+__global__ void __launch_bounds__(256) colsum8_bf16_kernel(int64_t rows, int cols,
+                                                           int64_t rows_per_block,
+                                                           const bf16* __restrict__ src,
+                                                           float* __restrict__ out) {
+  const int c = threadIdx.x * 8;
+  if (c >= cols) return;
+  const int64_t r0 = (int64_t)blockIdx.x * rows_per_block;
+  const int64_t r1 = r0 + rows_per_block < rows ? r0 + rows_per_block : rows;
+  float acc[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+  for (int64_t r = r0; r < r1; r++) {
+    const uint4 v = __ldcs(reinterpret_cast<const uint4*>(src + r * cols + c));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; k++) {
+      acc[2 * k] += bf16_lo(w[k]);
+      acc[2 * k + 1] += bf16_hi(w[k]);
+    }
+  }
+  if (r1 > r0) {
+#pragma unroll
+    for (int k = 0; k < 8; k++) atomicAdd(out + c + k, acc[k]);
+  }
+}
+
+// The LayerNorm*U backward below with each row held in registers (NC = W / 32 columns per lane,
+// columns lane + 32 k) and the parameter gradients summed per lane over the warp's rows.
+template <int NC>
+__global__ void __launch_bounds__(256) ln_gate_bwd_reg_kernel(int64_t T, int64_t ldu,
+                                                              const float* __restrict__ av,
+                                                              const bf16* __restrict__ u,
+                                                              const float* __restrict__ dg,
+                                                              const bf16* __restrict__ ln_w,
+                                                              const bf16* __restrict__ ln_b,
+                                                              float eps, bf16* __restrict__ dav,
+                                                              bf16* __restrict__ du,
+                                                              float* __restrict__ dln_w,
+                                                              float* __restrict__ dln_b) {
+  constexpr int W = NC * 32;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  float w[NC], b[NC], sw[NC], sb[NC];
+#pragma unroll
+  for (int k = 0; k < NC; k++) {
+    w[k] = __bfloat162float(ln_w[lane + 32 * k]);
+    b[k] = __bfloat162float(ln_b[lane + 32 * k]);
+    sw[k] = 0.0f;
+    sb[k] = 0.0f;
+  }
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x / 32);
+  for (int64_t row = (int64_t)blockIdx.x * (blockDim.x / 32) + warp; row < T; row += warps) {
+    float x[NC], g[NC], uu[NC];
+    float s = 0.0f;
+#pragma unroll
+    for (int k = 0; k < NC; k++) {
+      x[k] = __ldcs(av + row * W + lane + 32 * k);
+      g[k] = __ldcs(dg + row * W + lane + 32 * k);
+      uu[k] = __bfloat162float(u[row * ldu + lane + 32 * k]);
+      s += x[k];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const float mean = s / (float)W;
+    float var = 0.0f;
+#pragma unroll
+    for (int k = 0; k < NC; k++) {
+      x[k] -= mean;
+      var = fmaf(x[k], x[k], var);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) var += __shfl_xor_sync(0xffffffffu, var, o);
+    const float rstd = rsqrtf(var / (float)W + eps);
+    float m1 = 0.0f, m2 = 0.0f;   // sums of dy*w and dy*w*xhat
+#pragma unroll
+    for (int k = 0; k < NC; k++) {
+      const float xh = x[k] * rstd;
+      const float dy = g[k] * uu[k];
+      du[row * ldu + lane + 32 * k] = __float2bfloat16_rn(g[k] * fmaf(xh, w[k], b[k]));
+      sw[k] = fmaf(dy, xh, sw[k]);
+      sb[k] += dy;
+      const float dyw = dy * w[k];
+      m1 += dyw;
+      m2 = fmaf(dyw, xh, m2);
+      x[k] = xh;
+      g[k] = dyw;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      m1 += __shfl_xor_sync(0xffffffffu, m1, o);
+      m2 += __shfl_xor_sync(0xffffffffu, m2, o);
+    }
+    m1 /= (float)W;
+    m2 /= (float)W;
+#pragma unroll
+    for (int k = 0; k < NC; k++)
+      dav[row * W + lane + 32 * k] = __float2bfloat16_rn(rstd * (g[k] - m1 - x[k] * m2));
+  }
+#pragma unroll
+  for (int k = 0; k < NC; k++) {
+    atomicAdd(dln_w + lane + 32 * k, sw[k]);
+    atomicAdd(dln_b + lane + 32 * k, sb[k]);
+  }
+}
+
 // Backward of G = LayerNorm(AV) * U (Eq. 3, first half), one warp per row, W = H*d_v columns:
 //   y = xhat * w + b,  xhat = (x - mean) * rstd
 //   dU = dG * y,  dy = dG * U,  dln_w += dy * xhat,  dln_b += dy

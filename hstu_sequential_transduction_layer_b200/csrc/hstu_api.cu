@@ -4,6 +4,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 #include <vector>
 
 #include "common.cuh"
@@ -360,8 +361,13 @@ hstu_status_t run_colsum(int64_t rows, int cols, const void* src, float* out, cu
   int64_t per = (rows + want - 1) / want;
   if (per < 16) per = 16;
   const int64_t blocks = (rows + per - 1) / per;
-  bwd::colsum_kernel<bf16><<<(unsigned)blocks, 256, 0, st>>>(rows, cols, cols, per,
-                                                             (const bf16*)src, out);
+  if (cols % 8 == 0 && cols <= 8 * 256 && aligned16(src)) {
+    bwd::colsum8_bf16_kernel<<<(unsigned)blocks, 256, 0, st>>>(rows, cols, per, (const bf16*)src,
+                                                               out);
+  } else {
+    bwd::colsum_kernel<bf16><<<(unsigned)blocks, 256, 0, st>>>(rows, cols, cols, per,
+                                                               (const bf16*)src, out);
+  }
   return launch_status();
 }
 
@@ -746,7 +752,30 @@ hstu_status_t hstu_layer_bwd(const hstu_shape_t* shape, const void* X, const int
     return rc;
   if ((rc = run_colsum(T, d, dY, db2, st)) != HSTU_OK) return rc;
   // G = LayerNorm(AV) * U  ->  dU (block 0 of dUVQK), dAV, dln_w, dln_b
-  {
+  if (wv == 64 || wv == 128 || wv == 256 || wv == 512 || wv == 1024) {
+    // rows in registers, parameter gradients summed per lane
+    auto go = [&](auto nc) {
+      auto kern = bwd::ln_gate_bwd_reg_kernel<decltype(nc)::value>;
+      int per_sm = 1;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0) != cudaSuccess ||
+          per_sm < 1)
+        per_sm = 1;
+      const int64_t full = (int64_t)per_sm * tc::num_sms();   // one wave of resident blocks
+      const int64_t blocks = T < full * 8 ? (T + 7) / 8 : full;
+      kern<<<(unsigned)blocks, 256, 0, st>>>(
+          T, n1, (const float*)fw.av, (const bf16*)fw.uvqk, (const float*)w.dg,
+          (const bf16*)ln_w, (const bf16*)ln_b, s.ln_eps, (bf16*)w.dav, (bf16*)w.duvqk, dln_w,
+          dln_b);
+    };
+    switch (wv) {
+      case 64: go(std::integral_constant<int, 2>{}); break;
+      case 128: go(std::integral_constant<int, 4>{}); break;
+      case 256: go(std::integral_constant<int, 8>{}); break;
+      case 512: go(std::integral_constant<int, 16>{}); break;
+      default: go(std::integral_constant<int, 32>{}); break;
+    }
+    if ((rc = launch_status()) != HSTU_OK) return rc;
+  } else {
     const int64_t blocks = T < 4LL * tc::num_sms() * 8 ? (T + 7) / 8 : 4LL * tc::num_sms();
     const size_t smem = (size_t)2 * wv * sizeof(float);
     if (smem > 48 * 1024 &&

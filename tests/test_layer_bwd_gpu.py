@@ -85,6 +85,7 @@ def _compare(got, ref, dY, what):
     (53, [700, 31], 2, "alibi"),
     (54, [128, 255, 257], 1, "none"),
     (55, [77, 400, 190], 4, "rab"),
+    (58, [150, 129], 16, "rab"),
 ])
 def test_layer_backward_matches_oracle(hstu, seed, lengths, H, bias):
     inp, dY = _case(seed, lengths, H, bias)
