@@ -1,7 +1,7 @@
 // HBM-bound kernels of the layer backward ("Actions Speak Louder than Words" paper notes, section
 // 3.1, Eqs. 1-3, differentiated): transposes that feed the weight-gradient GEMMs, column sums for
-// the bias gradients, the LayerNorm*U backward, and the packing of the attention gradients into the
-// dU|dV|dQ|dK layout of f1's output.
+// the bias gradients, the LayerNorm*U backward, and the packing of dQ into the dU|dV|dQ|dK layout
+// of f1's output.
 #pragma once
 
 #include "common.cuh"
@@ -235,25 +235,21 @@ __global__ void __launch_bounds__(256) ln_gate_bwd_kernel(int64_t T, int W, int6
   }
 }
 
-// dUVQK blocks 1..3 (V, Q, K; block 0, dU, is written by the LayerNorm backward): bf16 from the
-// attention backward's fp32 dV, dQ, dK [T, W]; one thread per 4 columns.
-__global__ void __launch_bounds__(256) pack_dvqk_kernel(int64_t T, int W, int64_t ldu,
-                                                        const float* __restrict__ dv,
-                                                        const float* __restrict__ dq,
-                                                        const float* __restrict__ dk,
-                                                        bf16* __restrict__ duvqk) {
+// dst[r][c] = bf16(src[r][c]) for a [T, W] fp32 matrix into rows of stride ldu (e.g. the dQ block
+// of dUVQK); one thread per 4 columns.
+__global__ void __launch_bounds__(256) pack_rows_bf16_kernel(int64_t T, int W, int64_t ldu,
+                                                             const float* __restrict__ src,
+                                                             bf16* __restrict__ dst) {
   const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int per_row = W / 4;
-  if (t >= T * 3 * per_row) return;
-  const int64_t row = t / (3 * per_row);
-  const int rem = (int)(t - row * 3 * per_row);
-  const int blk = rem / per_row, c = (rem - blk * per_row) * 4;
-  const float* src = blk == 0 ? dv : (blk == 1 ? dq : dk);
-  const float4 v = *reinterpret_cast<const float4*>(src + row * W + c);
+  if (t >= T * per_row) return;
+  const int64_t row = t / per_row;
+  const int c = (int)(t - row * per_row) * 4;
+  const float4 v = __ldcs(reinterpret_cast<const float4*>(src + row * W + c));
   uint2 o;
   o.x = pack_bf16x2(v.x, v.y);
   o.y = pack_bf16x2(v.z, v.w);
-  *reinterpret_cast<uint2*>(duvqk + row * ldu + (int64_t)(blk + 1) * W + c) = o;
+  *reinterpret_cast<uint2*>(dst + row * ldu + c) = o;
 }
 
 }  // namespace bwd

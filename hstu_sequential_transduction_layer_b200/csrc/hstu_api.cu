@@ -303,7 +303,7 @@ hstu_status_t run_attention_bwd(const hstu_shape_t& s, const void* uvqk, const i
                                 const int64_t* ts, const float* pos, const float* tim,
                                 const float* alibi, float scale, const void* dav, float* dq,
                                 float* dk, float* dv, float* dpos, float* dtime, void* ws,
-                                size_t ws_bytes, cudaStream_t st) {
+                                size_t ws_bytes, cudaStream_t st, void* duvqk = nullptr) {
   hstu_status_t rc;
   const int64_t T = s.total_tokens, B = s.num_seqs;
   if (pos && (rc = zero_f32(dpos, (int64_t)s.num_heads * s.n_pos_buckets, st)) != HSTU_OK) return rc;
@@ -315,7 +315,8 @@ hstu_status_t run_attention_bwd(const hstu_shape_t& s, const void* uvqk, const i
   if (launch_status() != HSTU_OK) return HSTU_ERR_CUDA;
   return tc::launch_attention_bwd(T, B, s.num_heads, s.max_seq_len, (const bf16*)uvqk, off, ts, pos,
                                   s.n_pos_buckets, tim, s.n_time_buckets, alibi, scale,
-                                  (const bf16*)dav, dq, dk, dv, dpos, dtime, ws, ws_bytes, st);
+                                  (const bf16*)dav, dq, dk, dv, dpos, dtime, ws, ws_bytes, st,
+                                  (bf16*)duvqk);
 }
 
 struct BwdWorkspace {
@@ -340,7 +341,7 @@ BwdWorkspace bwd_layout(const hstu_shape_t& s, void* base) {
   take(w.dg, T * wv * 4);                       // dG fp32
   take(w.dav, T * wv * 2);                      // dAV bf16
   take(w.duvqk, T * n1 * 2);                    // dU|dV|dQ|dK bf16
-  take(w.dqkv, 3 * T * wv * 4);                 // dQ, dK, dV fp32; later dZ bf16 [T, n1]
+  take(w.dqkv, 2 * T * wv * 4);                 // dQ fp32; later dZ bf16 [T, n1]
   take(w.trans, (wv > d ? wv : d) * (size_t)w.t_pad * 2);   // G^T, later X^T
   w.attn_bytes = tc::attention_bwd_workspace_bytes(s.total_tokens, s.num_seqs, s.num_heads);
   take(w.attn, w.attn_bytes);
@@ -733,11 +734,10 @@ hstu_status_t hstu_layer_bwd(const hstu_shape_t* shape, const void* X, const int
   const Workspace fw = layout(s, const_cast<void*>(fwd_workspace));
   const BwdWorkspace w = bwd_layout(s, workspace);
   const bf16* dy = (const bf16*)dY;
-  const int64_t T4 = T * wv;
   float* dq = (float*)w.dqkv;
-  float* dk = dq + T4;
-  float* dv = dk + T4;
-  bf16* dz = (bf16*)w.dqkv;   // after dQ, dK, dV are packed into dUVQK
+  float* dk = nullptr;        // dV and dK are written as bf16 into dUVQK by the kernel
+  float* dv = nullptr;
+  bf16* dz = (bf16*)w.dqkv;   // after dQ is packed into dUVQK
   // f2: Y = G W2 + b2 + X  ->  dG = dY W2^T, dW2 = G^T dY, db2 = column sums of dY
   if ((rc = run_transpose(wv, wv, d, d, W2, w.w2t, st)) != HSTU_OK) return rc;
   if ((rc = run_transpose(d, d, (int)n1, n1, W1, w.w1t, st)) != HSTU_OK) return rc;
@@ -791,12 +791,13 @@ hstu_status_t hstu_layer_bwd(const hstu_shape_t* shape, const void* X, const int
   // Eq. 2  ->  dQ, dK, dV and the bias tables' gradients; then dV|dQ|dK into dUVQK
   if ((rc = run_attention_bwd(s, fw.uvqk, seq_offsets, timestamps, pos_table, time_table,
                               alibi_slopes, scale, w.dav, dq, dk, dv, dpos_table, dtime_table,
-                              w.attn, w.attn_bytes, st)) != HSTU_OK)
+                              w.attn, w.attn_bytes, st, w.duvqk)) != HSTU_OK)
     return rc;
   {
-    const int64_t threads = T * 3 * (wv / 4);
-    bwd::pack_dvqk_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
-        T, (int)wv, n1, dv, dq, dk, (bf16*)w.duvqk);
+    // dV and dK went to dUVQK as bf16 from the kernel; dQ (reduced in fp32) joins them
+    const int64_t threads = T * (wv / 4);
+    bwd::pack_rows_bf16_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
+        T, (int)wv, n1, dq, (bf16*)w.duvqk + 2 * wv);
     if ((rc = launch_status()) != HSTU_OK) return rc;
   }
   // Eq. 1: UVQK = SiLU(X W1 + b1)  ->  dZ = dUVQK * SiLU'(X W1 + b1), dW1 = X^T dZ, db1, dX

@@ -82,8 +82,9 @@ struct BwdParams {
   int P, Tb, H, n1;
   float scale;
   float* dq;             // [T, H*64] fp32, accumulated (zeroed by the caller)
-  float* dk;             // [T, H*64] fp32
-  float* dv;             // [T, H*64] fp32
+  float* dk;             // [T, H*64] fp32 (unused when duvqk is set)
+  float* dv;             // [T, H*64] fp32 (unused when duvqk is set)
+  bf16* duvqk;           // or null: dV and dK as bf16 into blocks 1 and 3 of [T, 4*H*64]
   float* dpos;           // [H, P] fp32, accumulated, or null
   float* dtime;          // [H, Tb] fp32, accumulated, or null
 };
@@ -864,7 +865,22 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(dkv_empty);
-        if (kvalid) {
+        if (kvalid && prm.duvqk) {
+          // bf16 into the V and K blocks of a [T, 4 H 64] gradient of U|V|Q|K
+          bf16* base = prm.duvqk + (row0 + j) * (int64_t)(4 * H * 64) + h * 64 + 16 * cg;
+          uint32_t pv[8], pk2[8];
+#pragma unroll
+          for (int v = 0; v < 8; v++) {
+            pv[v] = pack_bf16x2(__uint_as_float(vv[2 * v]), __uint_as_float(vv[2 * v + 1]));
+            pk2[v] = pack_bf16x2(__uint_as_float(kv[2 * v]), __uint_as_float(kv[2 * v + 1]));
+          }
+          uint4* dvb = reinterpret_cast<uint4*>(base + H * 64);
+          uint4* dkb = reinterpret_cast<uint4*>(base + 3 * H * 64);
+          dvb[0] = make_uint4(pv[0], pv[1], pv[2], pv[3]);
+          dvb[1] = make_uint4(pv[4], pv[5], pv[6], pv[7]);
+          dkb[0] = make_uint4(pk2[0], pk2[1], pk2[2], pk2[3]);
+          dkb[1] = make_uint4(pk2[4], pk2[5], pk2[6], pk2[7]);
+        } else if (kvalid) {
           float* dvr = prm.dv + (row0 + j) * (int64_t)(H * 64) + h * 64 + 16 * cg;
           float* dkr = prm.dk + (row0 + j) * (int64_t)(H * 64) + h * 64 + 16 * cg;
 #pragma unroll

@@ -260,7 +260,8 @@ inline hstu_status_t launch_attention_bwd(int64_t T, int64_t B, int H, int64_t m
                                           const float* pos, int P, const float* tim, int Tb,
                                           const float* alibi, float scale, const bf16* dav, float* dq,
                                           float* dk, float* dv, float* dpos, float* dtime, void* ws,
-                                          size_t ws_bytes, cudaStream_t st) {
+                                          size_t ws_bytes, cudaStream_t st,
+                                          bf16* duvqk = nullptr) {
   if (T >= (1LL << 31) || H >= (1 << 15)) return HSTU_ERR_UNSUPPORTED;
   if (ws_bytes < attention_bwd_workspace_bytes(T, B, H)) return HSTU_ERR_INVALID_ARG;
   const int64_t max_tiles64 = ((max_seq_len > 0 ? max_seq_len : T) + ATT_BN - 1) / ATT_BN;
@@ -294,6 +295,7 @@ inline hstu_status_t launch_attention_bwd(int64_t T, int64_t B, int H, int64_t m
   prm.dq = dq;
   prm.dk = dk;
   prm.dv = dv;
+  prm.duvqk = duvqk;
   prm.dpos = dpos;
   prm.dtime = dtime;
   const int grid = (int)(capacity < num_sms() ? capacity : num_sms());
