@@ -63,7 +63,8 @@ struct BwdCfg {
   static constexpr int OFF_QTS32 = OFF_KTS + 128 * 8;       // [NST][128] int32, relative
   static constexpr int OFF_KTS32 = OFF_QTS32 + NST * 128 * 4;  // [128] int32, relative
   static constexpr int OFF_TFLAG = OFF_KTS32 + 128 * 4;     // [NST] query fits, [NST] key fits
-  static constexpr int OFF_PWIN = OFF_TFLAG + 64;           // [16 warps][64] float: table window
+  static constexpr int OFF_CLS = OFF_TFLAG + 64;            // [NST][32] int2: time mode of each block
+  static constexpr int OFF_PWIN = OFF_CLS + NST * 32 * 8;   // [16 warps][64] float: table window
   static constexpr int OFF_CAP = OFF_PWIN + BWD_PW_WARPS * 64 * 4;      // [16 warps][32] float
   static constexpr int OFF_TT = OFF_CAP + BWD_PW_WARPS * 32 * 4;        // [TT_ALL] half time tables
   static constexpr int OFF_DTT = OFF_TT + BWD_TT_ALL * 4;     // [TT_ALL] float their gradients
@@ -178,6 +179,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   // [0]: bit g set when the key tile's timestamps g*32 .. g*32+31 are non-decreasing;
   // [1 + st]: the same for the query tile of stage st
   int* tsort = tflag + 4;
+  // [st][q * 8 + g]: the time-bias mode of the block of key quadrant q and queries 16 g .. 16 g + 15
+  // of the stage's tile: x = mode (0 general, 1 one bucket, 2 two buckets) | bucket << 8, y = the
+  // two-bucket threshold on the relative time difference
+  int2* cls_s = reinterpret_cast<int2*>(smem + Cfg::OFF_CLS);
   float* pwin_s = reinterpret_cast<float*>(smem + Cfg::OFF_PWIN);
   float* cap_s = reinterpret_cast<float*>(smem + Cfg::OFF_CAP);
   uint8_t* stg_s = smem + Cfg::OFF_STG;
@@ -300,12 +305,51 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       if (lane == 0) mbar_arrive(kv_full);
       for (int i = jt; i < nt && ok; i++, g++) {
         const uint32_t st = g % Cfg::NST, ph = (g / Cfg::NST) & 1u;
-        // the query tile's timestamps, loaded before the stage is free
+        // the query tile's timestamps, loaded, checked and classified before the stage is free
+        int rel4[4] = {0, 0, 0, 0};
+        bool fits = true;
+        int sm = 0;
+        int2 cls = make_int2(0, 0);
         if (has_time) {
 #pragma unroll
           for (int e = 0; e < 4; e++) {
             const int64_t qi = (int64_t)i * ATT_BM + 4 * lane + e;
             tv[e] = prm.ts[row0 + (qi < n ? qi : n - 1)];
+            const int64_t rel = tv[e] - t0;
+            fits = fits && rel > -(1LL << 30) && rel < (1LL << 30);
+            rel4[e] = (int)rel;
+          }
+          fits = __all_sync(0xffffffffu, fits);
+          sm = sorted_groups(tv, lane);
+          // the time-bias mode of the tile's 32 blocks (lane = q * 8 + g: keys of quadrant q,
+          // queries 16 g .. 16 g + 15): with both sides sorted, the buckets at the block's
+          // extreme corners bound all of its buckets
+          const int cq = lane >> 3, cgp = lane & 7;
+          const long long qf = __shfl_sync(0xffffffffu, (long long)tv[0], 4 * cgp);
+          const long long ql = __shfl_sync(0xffffffffu, (long long)tv[3], 4 * cgp + 3);
+          const int qf32 = __shfl_sync(0xffffffffu, rel4[0], 4 * cgp);
+          const int ql32 = __shfl_sync(0xffffffffu, rel4[3], 4 * cgp + 3);
+          if (((tsort[0] >> cq) & 1) && ((sm >> (cgp >> 1)) & 1)) {
+            const bool r32 = tflag[0] != 0 && fits;
+            int b0, b1;
+            if (r32) {
+              // 32-bit: floor(log2(1 + max(dt, 0))) = 31 - clz(max(dt, 0) + 1)
+              const int e0 = qf32 - kts32[cq * 32 + 31], e1 = ql32 - kts32[cq * 32];
+              b0 = 31 - __clz((e0 > 0 ? e0 : 0) + 1);
+              b1 = 31 - __clz((e1 > 0 ? e1 : 0) + 1);
+            } else {
+              b0 = time_bucket(qf, kts[cq * 32 + 31]);
+              b1 = time_bucket(ql, kts[cq * 32]);
+            }
+            const int c0b = b0 < prm.Tb - 1 ? b0 : prm.Tb - 1;
+            const int c1b = b1 < prm.Tb - 1 ? b1 : prm.Tb - 1;
+            if (c0b == c1b) {
+              cls.x = 1 | (c0b << 8);
+            } else if (c1b == c0b + 1 && r32 && c1b <= 30) {
+              // bucket(dt) >= c1b  <=>  dt + 1 >= 2^c1b (also when c1b is the clamped last one)
+              cls.x = 2 | (c0b << 8);
+              cls.y = (1 << c1b) - 1;
+            }
           }
         }
         if (lane == 0) ok = mbar_wait(&q_empty[st], ph ^ 1u, abort_flag);
@@ -320,18 +364,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           q_par[st] = (int)ph;
         }
         if (has_time) {
-          bool fits = true;
 #pragma unroll
           for (int e = 0; e < 4; e++) {
             qts[st * 128 + 4 * lane + e] = tv[e];
-            const int64_t rel = tv[e] - t0;
-            fits = fits && rel > -(1LL << 30) && rel < (1LL << 30);
-            qts32[st * 128 + 4 * lane + e] = (int)rel;
+            qts32[st * 128 + 4 * lane + e] = rel4[e];
           }
-          fits = __all_sync(0xffffffffu, fits);
-          if (lane == 0) tflag[1 + st] = fits ? 1 : 0;
-          const int sm = sorted_groups(qts + st * 128 + 4 * lane, lane);
-          if (lane == 0) tsort[1 + st] = sm;
+          if (lane == 0) {
+            tflag[1 + st] = fits ? 1 : 0;
+            tsort[1 + st] = sm;
+          }
+          cls_s[st * 32 + lane] = cls;
         }
         // the timestamps are published with the tiles: the arrival completes the phase
         __syncwarp();
@@ -583,29 +625,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         // adjacent).
         const bool full = dbase - 31 >= 0 && (int64_t)(qc0 + 15) < n && (int64_t)(kq0 + 31) < n;
         const bool pos_one = has_pos && full && dbase - 31 >= P - 1;   // all in bucket P - 1
+        // the block's time mode, classified by the producer
         int tb_u = -1, tmode = 0;                 // 1: one bucket tb_u; 2: tb_u and tb_u + 1
         int thr = 0;                              // two buckets: relative dt >= thr is tb_u + 1
-        if (has_time && full && ((tsort[0] >> q) & 1) && ((tsort[1 + st] >> (qb >> 5)) & 1)) {
-          int b0, b1;
-          if (keys_rel32 && tflag[1 + st] != 0) {
-            // 32-bit: floor(log2(1 + max(dt, 0))) = 31 - clz(max(dt, 0) + 1)
-            const int e0 = qt32[0] - kts32[q * 32 + 31], e1 = qt32[15] - kts32[q * 32];
-            b0 = 31 - __clz((e0 > 0 ? e0 : 0) + 1);
-            b1 = 31 - __clz((e1 > 0 ? e1 : 0) + 1);
-          } else {
-            b0 = time_bucket(qt_s[0], kts[q * 32 + 31]);
-            b1 = time_bucket(qt_s[15], kts[q * 32]);
-          }
-          const int c0b = b0 < Tb - 1 ? b0 : Tb - 1, c1b = b1 < Tb - 1 ? b1 : Tb - 1;
-          if (c0b == c1b) {
-            tb_u = c0b;
-            tmode = 1;
-          } else if (c1b == c0b + 1 && keys_rel32 && tflag[1 + st] != 0 && c1b <= 30) {
-            // bucket(dt) >= c1b  <=>  dt + 1 >= 2^c1b (also when c1b is the clamped last one)
-            tb_u = c0b;
-            tmode = 2;
-            thr = (1 << c1b) - 1;
-          }
+        if (has_time && full) {
+          const int2 c = cls_s[st * 32 + q * 8 + (qb >> 4)];
+          tmode = c.x & 3;
+          tb_u = c.x >> 8;
+          thr = c.y;
         }
         const bool fast = full && (!has_time || tmode != 0);
         // time-gradient bucket of the general loop's rows: the block's buckets along a row are
