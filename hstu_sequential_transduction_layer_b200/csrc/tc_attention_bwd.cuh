@@ -6,31 +6,33 @@
 //   dQ_i = sum_j dx_ij k_j,    dK_j = sum_i dx_ij q_i,   dpos / dtime = sums of dx_ij per bucket
 //
 // Work item = (sequence, 128-key tile j, head), key-stationary: K_j and V_j stay in shared memory
-// while the item walks the query tiles i = j, j+1, ... of the sequence.  Per query tile, with the
-// keys as the MMA's M dimension (TMEM lane = key row):
-//   S^T  = K_j Q_i^T,  dP^T = V_j dAV_i^T                 (M=128 keys, N=128 queries, K=64)
+// while the item walks the query tiles i = j, j+1, ... of the sequence.  Per query tile, in two
+// halves of 64 queries, with the keys as the MMA's M dimension (TMEM lane = key row):
+//   S^T  = K_j Q_i^T,  dP^T = V_j dAV_i^T                 (M=128 keys, N=64 queries, K=64)
 //   pointwise: P^T = scale*SiLU(S^T + bias^T), dS^T = scale*SiLU'(.) * dP^T, masked to j <= i
 //   dV_j += P^T dAV_i,  dK_j += dS^T Q_i                   (P^T, dS^T read from TMEM)
+// and once per tile
 //   dQ_i partial = dS K_j                                  (dS from shared memory, MN-major A)
-// and the dQ partial, staged in shared memory, is added to global dQ (fp32) with TMA reductions.  Table gradients:
-// each pointwise warp sums the diagonals of its 32 x 32 block of dx systolically (lane l carries
-// the sum of diagonal c - l across the columns c, handing it one lane up per column; the sum
-// leaving lane 31 is complete), and each diagonal's sum (one bucket, all distances along a
-// diagonal being equal) goes to the global position gradient with one reduction; the position
-// bias itself comes from a per-warp window of the table at the block's 63 distances.
-// Time-bucket gradients: where the whole block is in one bucket or two (sorted timestamps), block
-// sums; elsewhere per row and chunk in two registers (the chunk's first bucket and the next one);
-// in shared memory per item, then to global memory.
-// dV and dK are owned by the item and stored directly.
+// which, staged in shared memory, is added to global dQ (fp32) with TMA reductions.  The tensor
+// cores compute one half (and the next tile's first half) while the pointwise warps work on the
+// other.  Table gradients: each pointwise warp sums the diagonals of its 32 x 16 block of dx
+// systolically (lane l carries the sum of diagonal c - l across the columns c, handing it one lane
+// up per column; the sum leaving lane 31 is complete), and each diagonal's sum (one bucket, all
+// distances along a diagonal being equal) goes to the global position gradient with one reduction;
+// the position (or ALiBi) bias itself comes from a per-warp window of half biases at the block's 47
+// distances.  Time-bucket gradients: blocks that sit in one bucket or two (sorted timestamps) add
+// block sums to per-lane pending sums; other blocks use per-row registers for the row's first
+// bucket and the next one; all gathered in shared memory, then sent to global memory.  dV and dK
+// are owned by the item and stored directly (fp32, or bf16 into a dU|dV|dQ|dK gradient).
 //
 // Per CTA (640 threads, one per SM): warp 0 producer (TMA of K_j, V_j, and Q_i, dAV_i per query tile
-// into a 2-deep ring; key and query timestamps), warp 1 single-thread MMA issuer, warp 2 the dQ
-// TMA reductions, warp 3 idle,
-// warps 4-19 pointwise (four per TMEM lane quadrant, each on 32 of the 128 query columns, in two
-// 16-column halves so that 96 registers per thread suffice).
-// TMEM: S^T [0,128) | dP^T [128,256) | dV [256,320) | dK [320,384) | dQ partial [384,448); P^T and
-// dS^T (bf16) overwrite the S^T / dP^T columns each warp has read (a warp's 32 queries pack into 16
-// columns at the start of its own 32).
+// into a 2-deep ring; key and query timestamps and each block's time-bias mode), warp 1
+// single-thread MMA issuer, warp 2 the dQ TMA reductions, warp 3 idle, warps 4-19 pointwise (four
+// per TMEM lane quadrant; column group cg takes queries 16 cg .. 16 cg + 15 of each half, so that
+// 96 registers per thread suffice).
+// TMEM: S^T [0,128) | dP^T [128,256) (each: half A in the first 64 columns, half B in the next) |
+// dV [256,320) | dK [320,384) | dQ partial [384,448); P^T and dS^T (bf16) overwrite the S^T / dP^T
+// columns each warp has read (a warp's 16 queries pack into the first 8 of its 16 columns).
 #pragma once
 
 #include <type_traits>
