@@ -1,5 +1,7 @@
 /*
- * hstu.h -- C ABI of the B200 (sm_100a) HSTU layer forward library, libhstu_b200.so.
+ * hstu.h -- C ABI of the B200 (sm_100a) HSTU layer library, libhstu_b200.so: the layer forward,
+ * its steps one at a time, M-FALCON candidate scoring, Stochastic Length subsampling, the attention
+ * and layer backward passes (training), and a host-to-host forward pipeline.
  *
  * The layer (one "HSTU" block of "Actions Speak Louder than Words", paper notes, section 3.1,
  * Eqs. 1-3; also the HSTU-layer section of "4.4 推荐模型的 Scaling") over a jagged batch of
@@ -21,9 +23,11 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- *  - All tensor pointers are DEVICE pointers (cudaMalloc'd or equivalent), owned by the caller.
- *    The library allocates, frees and retains no memory; intermediates live in the caller's
- *    workspace.  Every matrix is row-major and densely packed.
+ *  - All tensor pointers are DEVICE pointers (cudaMalloc'd or equivalent), owned by the caller,
+ *    except the host buffers of the hstu_layer_pipeline_* calls.  The library allocates, frees
+ *    and retains no memory (intermediates live in the caller's workspace), except the pipeline
+ *    object, which owns its device buffers and streams, and the fixed schedule array of
+ *    hstu_attention_fwd_noalloc.  Every matrix is row-major and densely packed.
  *  - `stream` is a cudaStream_t passed as void*; NULL means the legacy default stream.  Calls are
  *    asynchronous: they only enqueue kernels and return.  They never synchronise.
  *  - Errors checkable on the host (NULL pointers, bad dimensions, misalignment, aliasing) are
