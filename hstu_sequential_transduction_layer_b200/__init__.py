@@ -30,6 +30,7 @@ EXPORTED = ["hstu_layer_fwd", "hstu_layer_fwd_workspace_size", "hstu_f1_fwd", "h
             "hstu_attention_workspace_size", "hstu_ln_gate_fwd", "hstu_f2_fwd",
             "hstu_token_embed_fwd", "hstu_status_string", "hstu_get_device_status", "hstu_version",
             "hstu_launch_count", "hstu_attention_fwd_noalloc", "hstu_selftest_bounded_wait",
+            "hstu_selftest_scratch_cache",
             "hstu_candidate_workspace_size", "hstu_candidate_attention_fwd",
             "hstu_candidate_layer_workspace_size", "hstu_candidate_layer_fwd",
             "hstu_stochastic_length_workspace_size", "hstu_stochastic_length", "hstu_gather_rows",
@@ -80,6 +81,7 @@ def _load() -> ctypes.CDLL:
         "hstu_version": ([], ctypes.c_char_p),
         "hstu_launch_count": ([], ctypes.c_uint64),
         "hstu_selftest_bounded_wait": ([ctypes.c_uint64, P, P], ctypes.c_int),
+        "hstu_selftest_scratch_cache": ([], ctypes.c_int32),
         "hstu_candidate_workspace_size": ([SH, I64], S),
         "hstu_candidate_attention_fwd": ([SH, P, P, P, I64, I64, P, P, P, P, P, P, F32, P, P, S, P],
                                          ctypes.c_int),

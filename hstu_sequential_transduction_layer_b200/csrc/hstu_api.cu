@@ -25,21 +25,75 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 namespace {
 
 constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mutex;
-void* g_noalloc_addr[kMaxDevices] = {};
 
-// Device address of g_noalloc_scratch on the current device (looked up once per device).
+// The device address of g_noalloc_scratch belongs to the CUDA context the module was loaded in:
+// when that context is destroyed (cudaDeviceReset, or the primary context released and made
+// again) the module is loaded anew and the array may sit elsewhere.  So a looked-up address is
+// cached together with the context it was looked up in, and reused only in that same context.
+struct ScratchAddr {
+  const void* ctx;   // the context current at the lookup (null: unknown, never reused)
+  void* addr;
+};
+
+// The cached address when `ctx` is the context of the cached lookup; otherwise runs `lookup`
+// (with `ctx` current), caches its result under `ctx` and returns it.  A failed lookup leaves the
+// cache as it was.
+template <class Lookup>
+hstu_status_t scratch_addr_for(ScratchAddr& e, const void* ctx, Lookup lookup, void** out) {
+  if (ctx && e.addr && e.ctx == ctx) {
+    *out = e.addr;
+    return HSTU_OK;
+  }
+  void* p = nullptr;
+  const hstu_status_t rc = lookup(&p);
+  if (rc != HSTU_OK) return rc;
+  e.ctx = ctx;
+  e.addr = p;
+  *out = p;
+  return HSTU_OK;
+}
+
+// The driver's cuCtxGetCurrent, reached through the runtime (the library does not link libcuda).
+typedef int (*CtxGetCurrentFn)(void**);
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<CtxGetCurrentFn>(p);
+    return static_cast<CtxGetCurrentFn>(nullptr);
+  }();
+  return fn;
+}
+
+const void* current_context() {
+  void* ctx = nullptr;
+  CtxGetCurrentFn fn = ctx_get_current_fn();
+  if (!fn || fn(&ctx) != 0) return nullptr;
+  return ctx;
+}
+
+std::mutex g_noalloc_mutex;
+ScratchAddr g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch in the current device's current context.  The lookup runs
+// once per device and context (the first call there, and again after the context was replaced).
 hstu_status_t noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return HSTU_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (!g_noalloc_addr[dev]) {
+  auto lookup = [](void** p) {
+    return cudaGetSymbolAddress(p, g_noalloc_scratch) == cudaSuccess && *p ? HSTU_OK
+                                                                           : HSTU_ERR_CUDA;
+  };
+  const void* ctx = current_context();
+  if (!ctx) {  // nothing current yet: a runtime call makes the device's primary context current
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return HSTU_ERR_CUDA;
-    g_noalloc_addr[dev] = p;
+    if (lookup(&p) != HSTU_OK) return HSTU_ERR_CUDA;
+    ctx = current_context();
   }
-  *out = g_noalloc_addr[dev];
-  return HSTU_OK;
+  return scratch_addr_for(g_noalloc_addr[dev], ctx, lookup, out);
 }
 
 constexpr size_t kAlign = 256;
@@ -874,6 +928,42 @@ hstu_status_t hstu_selftest_bounded_wait(uint64_t limit_ns, long long* result, v
   if (limit_ns == 0 || limit_ns > kSelftestMaxWaitNs || !result) return HSTU_ERR_INVALID_ARG;
   selftest_bounded_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, result);
   return launch_status();
+}
+
+int32_t hstu_selftest_scratch_cache(void) {
+  // host-only: fake contexts and a fake lookup that counts its calls and returns its own address
+  int calls = 0;
+  void* next = nullptr;
+  bool fail = false;
+  auto lookup = [&](void** p) {
+    calls++;
+    if (fail) return HSTU_ERR_CUDA;
+    *p = next;
+    return HSTU_OK;
+  };
+  char a_ctx, b_ctx, a_mem, b_mem, c_mem;
+  ScratchAddr e{nullptr, nullptr};
+  void* got = nullptr;
+  next = &a_mem;
+  if (scratch_addr_for(e, &a_ctx, lookup, &got) != HSTU_OK || got != &a_mem || calls != 1) return 1;
+  next = &c_mem;   // same context: the cached address, no lookup
+  if (scratch_addr_for(e, &a_ctx, lookup, &got) != HSTU_OK || got != &a_mem || calls != 1) return 2;
+  next = &b_mem;   // another context (e.g. after a device reset): looked up again
+  if (scratch_addr_for(e, &b_ctx, lookup, &got) != HSTU_OK || got != &b_mem || calls != 2) return 3;
+  next = &a_mem;   // and back: the cache holds the latest context only
+  if (scratch_addr_for(e, &a_ctx, lookup, &got) != HSTU_OK || got != &a_mem || calls != 3) return 4;
+  next = &c_mem;   // an unknown (null) context never reuses the cache
+  if (scratch_addr_for(e, nullptr, lookup, &got) != HSTU_OK || got != &c_mem || calls != 4) return 5;
+  if (scratch_addr_for(e, nullptr, lookup, &got) != HSTU_OK || calls != 5) return 6;
+  fail = true;     // a failed lookup reports the error and keeps the cache
+  got = nullptr;
+  if (scratch_addr_for(e, &b_ctx, lookup, &got) != HSTU_ERR_CUDA || got != nullptr || calls != 6)
+    return 7;
+  fail = false;
+  next = &b_mem;
+  if (scratch_addr_for(e, &b_ctx, lookup, &got) != HSTU_OK || got != &b_mem || calls != 7) return 8;
+  if (scratch_addr_for(e, &b_ctx, lookup, &got) != HSTU_OK || got != &b_mem || calls != 7) return 9;
+  return 0;
 }
 
 }  // extern "C"

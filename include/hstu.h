@@ -148,7 +148,9 @@ size_t hstu_attention_workspace_size(const hstu_shape_t* shape);
  * The attention tile schedule lives instead in a fixed 8 MiB device array inside this library,
  * which every GPU that loads the library keeps until the process exits.  The first call on a device
  * looks the array's address up (cudaGetSymbolAddress); make that first call before any stream
- * capture.  Shapes whose schedule needs more than 8 MiB (hstu_attention_workspace_size(shape) >
+ * capture.  The address is remembered together with the CUDA context it was looked up in and is
+ * looked up again when the device's current context has changed (after cudaDeviceReset, for
+ * instance, the library's device code is loaded anew and the array may move).  Shapes whose schedule needs more than 8 MiB (hstu_attention_workspace_size(shape) >
  * 8 MiB) are rejected with HSTU_ERR_UNSUPPORTED before anything is enqueued.  All calls share the
  * one array and each call rewrites the part it uses, so calls whose executions overlap on the GPU
  * (different streams, or different host threads, on the same device) race: serialise them.
@@ -369,6 +371,17 @@ hstu_status_t hstu_gather_rows(int64_t max_rows, const int64_t* row_count, int64
  *           barrier completed, 0 = gave up), then the nanoseconds each wait took.
  */
 hstu_status_t hstu_selftest_bounded_wait(uint64_t limit_ns, long long* result, void* stream);
+
+/*
+ * hstu_selftest_scratch_cache -- host-only check of how hstu_attention_fwd_noalloc remembers the
+ * device address of its scratch array: reused in the context it was looked up in, looked up again
+ * in any other context (or when the context is unknown), and left unchanged by a failed lookup.
+ *
+ * The paper has no counterpart: it is a diagnostic of this library.  It runs the cache logic with
+ * fake contexts and a fake lookup; it touches no GPU and needs none.  Returns 0 when every check
+ * passes, else the number of the first check that failed.
+ */
+int32_t hstu_selftest_scratch_cache(void);
 
 /*
  * hstu_token_embed_fwd -- action-oriented token assembly of the GenRank blog ("item-action

@@ -124,6 +124,44 @@ def test_attention_kernel(hstu, case):
     assert_bf16_close(host(av), ref, "attention")
 
 
+# The kernel stages the halved position table in shared memory for distances below 7168 at head
+# dim 128 (8192 at 64); tiles reaching farther take the exact path, which reads the table from
+# global memory and clamps at P-1.  Sequences long enough to reach both, every row compared.
+FAR_CASES = [
+    dict(seed=37, lengths=[7500, 8300], d=128, hd=128, P=8192, Tb=128),
+    dict(seed=38, lengths=[8500, 300], d=64, hd=64, P=16384, Tb=128),
+    dict(seed=39, lengths=[7400], d=128, hd=128, P=2048, Tb=128),
+]
+
+
+@pytest.mark.parametrize("case", FAR_CASES, ids=lambda c: f"seed{c['seed']}-hd{c['hd']}-P{c['P']}")
+def test_attention_far_distances(hstu, case):
+    hd, d = case["hd"], case["d"]
+    inp, uvqk = _attention_inputs(case["seed"], case["lengths"], d, hd, P=case["P"], Tb=case["Tb"])
+    inp.scale = 1.0 / 8192
+    H = inp.workload.num_heads
+    ref = oracle.attention(inp.seq_offsets, uvqk, num_heads=H, d_qk=hd, d_v=hd,
+                           timestamps=inp.timestamps, pos_table=inp.pos_table,
+                           time_table=inp.time_table, scale=inp.scale)
+    T = inp.T
+    s = hstu.make_shape(len(inp.lengths), T, int(inp.lengths.max()), d, H, hd, hd, hstu.HSTU_BF16,
+                        inp.pos_table.shape[1], inp.time_table.shape[1])
+    av = torch.empty((T, H * hd), dtype=torch.float32, device="cuda")
+    hstu.hstu_attention_fwd(s, dev(uvqk), dev(inp.seq_offsets), dev(inp.timestamps),
+                            dev(inp.pos_table, "f32"), dev(inp.time_table, "f32"), None,
+                            inp.scale, av)
+    assert hstu.device_status() == hstu.HSTU_OK
+    got = host(av)
+    assert_bf16_close(got, ref, "attention, far distances")
+    # the rows whose keys reach past the staged distances, on their own
+    far = 7168 if hd == 128 else 8192
+    for b, n in enumerate(inp.lengths):
+        if n > far:
+            a = int(inp.seq_offsets[b])
+            assert_bf16_close(got[a + far - 128:a + n], ref[a + far - 128:a + n],
+                              f"attention, rows reaching past {far} in sequence {b}")
+
+
 @pytest.mark.parametrize("T,wv", [(1, 256), (300, 512), (77, 1024), (40, 4096), (90, 192)])
 def test_ln_gate_kernel(hstu, T, wv):
     rng = np.random.default_rng(T + wv)
@@ -272,8 +310,11 @@ def test_layer_full_size_sampled(hstu, name):
         seqs, local = [int(order[0]), int(order[1])], [0, 127, 128, 255, -1]
     rows = _sample_rows(inp, seqs, local)
     if name == "large":
-        a = int(inp.seq_offsets[order[-1]])
-        rows += [a, a + 129, a + 700]
+        # early rows of the longest sequence, and the rows whose keys reach past the 7168 position
+        # buckets the hd=128 kernel stages in shared memory (exact path, table read from global)
+        a, n = int(inp.seq_offsets[order[-1]]), int(inp.lengths[order[-1]])
+        assert n > 7169
+        rows += [a, a + 129, a + 700, a + 7167, a + 7168, a + 7169, a + n - 1]
     ref, av_ref = oracle.layer_rows_inputs(inp, rows)
     got = _gpu_layer(hstu, inp)[rows]
     assert_bf16_close(got, ref, name)
