@@ -160,6 +160,39 @@ def combine_over_ranks(local_ms: float, local_tokens: int, world: int, device):
 # Our arm
 # ------------------------------------------------------------------------------------------------
 
+def workload_text(w, max_len):
+    bias = ("ALiBi slopes 2^(-8h/H)" if w.alibi
+            else f"rab P={w.n_pos_buckets}/Tb={w.n_time_buckets}")
+    tokens = ", X = item + action embeddings" if w.token_embed else ""
+    layers = f"{w.num_layers} layers" if w.num_layers > 1 else "1 layer"
+    return (f"{w.name}: B={w.num_seqs} jagged (max n={max_len}), d={w.d_model}, "
+            f"H={w.num_heads}x{w.head_dim}, {bias}{tokens}, {layers}")
+
+
+def assemble_tokens(hstu, torch, inp, dev, stream, reps=20):
+    """Action-oriented token assembly (row a0) on the device, outside the layer's timed region:
+    X = bf16(item_table[id] + action_table[a]).  Returns X and the gather's timing."""
+    from workloads.device import tensor
+    ii, ai = tensor(inp.item_ids, "bf16", dev), tensor(inp.action_ids, "bf16", dev)
+    itab, atab = tensor(inp.item_table_bits, "bf16", dev), tensor(inp.action_table_bits, "bf16", dev)
+    X = hstu.hstu_token_embed_fwd(ii, ai, itab, atab, stream=stream)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        hstu.hstu_token_embed_fwd(ii, ai, itab, atab, out=X, stream=stream)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    if hstu.device_status() != hstu.HSTU_OK:
+        raise SystemExit("device status error in the token assembly")
+    ms = float(np.mean([e0.elapsed_time(e1) for e0, e1 in evs]))
+    T, d = X.shape
+    byts = 6.0 * d * T          # two bf16 rows read, one written, per token
+    return X, {"ms": round(ms, 4), "GB/s": round(byts / ms / 1e6, 1), "bytes": int(byts)}
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import hstu_sequential_transduction_layer_b200 as hstu
@@ -169,43 +202,57 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     w = workloads.WORKLOADS[args.workload]
     inp = workloads.make_inputs(w)
-    if w.token_embed:
-        raise SystemExit("bench.py times the layer on workloads with explicit X; "
-                         "use long_seq, retrieval or large")
     H, hd, d = w.num_heads, w.head_dim, w.d_model
     T = inp.T
     D = to_device(inp, dev)
-    L = D["layers"][0]
+    stream = torch.cuda.current_stream()
+    gather = None
+    if w.token_embed:
+        D["X"], gather = assemble_tokens(hstu, torch, inp, dev, stream)
     max_len = int(inp.lengths.max())
     shape = hstu.shape_for(D["X"], D["off"], H, hd, hd, max_len, D["pos"], D["tim"], inp.ln_eps)
     n1 = 4 * d
     wv = H * hd
+    nl = w.num_layers
     uvqk = torch.empty((T, n1), dtype=torch.bfloat16, device=dev)
     av = torch.empty((T, wv), dtype=torch.float32, device=dev)     # fp32 LayerNorm input
     g = torch.empty((T, wv), dtype=torch.bfloat16, device=dev)
     attn_ws = torch.empty(max(256, hstu.attention_workspace_size(shape)), dtype=torch.uint8,
                           device=dev)
-    out = torch.empty_like(D["X"])
+    outs = [torch.empty_like(D["X"]) for _ in range(nl)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream()
+    # hstu_layer_fwd runs LayerNorm*U and f2 as one kernel where it can (H*d_v == d in 128/256/512)
+    fused = wv == d and d in (128, 256, 512)
 
     def step(evs=None):
-        # the four entry points hstu_layer_fwd chains, with events between them
-        if evs:
-            evs[0].record(stream)
-        hstu.hstu_f1_fwd(shape, D["X"], L["W1"], L["b1"], uvqk, stream)
-        if evs:
-            evs[1].record(stream)
-        hstu.hstu_attention_fwd(shape, uvqk, D["off"], D["ts"], D["pos"], D["tim"], D["ali"],
-                                inp.scale, av, attn_ws, stream)
-        if evs:
-            evs[2].record(stream)
-        hstu.hstu_ln_gate_fwd(shape, av, uvqk, L["ln_w"], L["ln_b"], g, stream)
-        if evs:
-            evs[3].record(stream)
-        hstu.hstu_f2_fwd(shape, g, L["W2"], L["b2"], D["X"], out, stream)
-        if evs:
-            evs[4].record(stream)
+        # every layer through the entry points hstu_layer_fwd chains, events between them
+        x = D["X"]
+        for l in range(nl):
+            L = D["layers"][l]
+            e = evs[l] if evs else None
+            if e:
+                e[0].record(stream)
+            hstu.hstu_f1_fwd(shape, x, L["W1"], L["b1"], uvqk, stream)
+            if e:
+                e[1].record(stream)
+            hstu.hstu_attention_fwd(shape, uvqk, D["off"], D["ts"], D["pos"], D["tim"], D["ali"],
+                                    inp.scale, av, attn_ws, stream)
+            if e:
+                e[2].record(stream)
+            if fused:
+                hstu.hstu_ln_f2_fwd(shape, av, uvqk, L["ln_w"], L["ln_b"], L["W2"], L["b2"], x,
+                                    outs[l], stream)
+                if e:
+                    e[3].record(stream)
+                    e[4].record(stream)
+            else:
+                hstu.hstu_ln_gate_fwd(shape, av, uvqk, L["ln_w"], L["ln_b"], g, stream)
+                if e:
+                    e[3].record(stream)
+                hstu.hstu_f2_fwd(shape, g, L["W2"], L["b2"], x, outs[l], stream)
+                if e:
+                    e[4].record(stream)
+            x = outs[l]
 
     for _ in range(args.warmup):
         step()
@@ -213,7 +260,8 @@ def run_ours(args, rank, world, local_rank):
     if hstu.device_status() != hstu.HSTU_OK:
         raise SystemExit("device status error during warm-up")
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(nl)]
+           for _ in range(args.steps)]
     sampler = ClockSampler(local_rank)
     if world > 1:
         torch.distributed.barrier()
@@ -228,8 +276,10 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop()
-    per_kernel = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in evs])  # ms
-    step_ms = per_kernel.sum(axis=1)
+    # [step, layer, kernel] milliseconds
+    per_kernel = np.array([[[e[i].elapsed_time(e[i + 1]) for i in range(4)] for e in ev]
+                           for ev in evs])
+    step_ms = per_kernel.sum(axis=(1, 2))
     total_ms = float(step_ms.sum())
     total_ms, job_tokens = combine_over_ranks(total_ms, T, world, dev)
     if hstu.device_status() != hstu.HSTU_OK:
@@ -237,7 +287,7 @@ def run_ours(args, rank, world, local_rank):
 
     ms_per_step = total_ms / args.steps
     tokens_per_s = job_tokens / (ms_per_step * 1e-3)
-    kern_ms = per_kernel.mean(axis=0)
+    kern_ms = per_kernel.mean(axis=(0, 1))       # per layer
     peaks, peaks_src = load_peaks()
     attn_fl = attention_flops(inp.lengths, H, hd, hd)
     f1_fl, f2_fl = gemm_flops(T, d, n1, wv)
@@ -246,16 +296,25 @@ def run_ours(args, rank, world, local_rank):
     kernels = {
         "f1_gemm": {"ms": kern_ms[0], "TFLOP/s": f1_fl / kern_ms[0] / 1e9},
         "attention": {"ms": kern_ms[1], "TFLOP/s": attn_fl / kern_ms[1] / 1e9},
-        "ln_gate": {"ms": kern_ms[2], "GB/s": ln_bytes / kern_ms[2] / 1e6},
-        "f2_gemm": {"ms": kern_ms[3], "TFLOP/s": f2_fl / kern_ms[3] / 1e9},
     }
+    if fused:
+        # HBM bytes of the fused kernel: AV (fp32) and U read, X read, Y written, W2 once
+        lnf2_bytes = (4.0 * wv + 2.0 * wv + 2.0 * d + 2.0 * d) * T + 2.0 * wv * d
+        kernels["ln_f2_fused"] = {"ms": kern_ms[2], "GB/s": lnf2_bytes / kern_ms[2] / 1e6,
+                                  "TFLOP/s (f2 part)": f2_fl / kern_ms[2] / 1e9}
+    else:
+        kernels["ln_gate"] = {"ms": kern_ms[2], "GB/s": ln_bytes / kern_ms[2] / 1e6}
+        kernels["f2_gemm"] = {"ms": kern_ms[3], "TFLOP/s": f2_fl / kern_ms[3] / 1e9}
     for k, v in kernels.items():
-        if "TFLOP/s" in v:
-            v["frac_of_bf16_peak"] = v["TFLOP/s"] / tpk
-        else:
+        if "GB/s" in v:
             v["frac_of_hbm"] = v["GB/s"] / peaks["hbm_gbs"]
+        else:
+            v["frac_of_bf16_peak"] = v["TFLOP/s"] / tpk
         for kk in list(v):
             v[kk] = round(float(v[kk]), 4)
+    if gather is not None:
+        gather["frac_of_hbm"] = round(gather["GB/s"] / peaks["hbm_gbs"], 4)
+        kernels["token_gather (outside the step)"] = gather
     attn_tflops = attn_fl / kern_ms[1] / 1e9
 
     e2e = run_e2e(args, hstu, torch, inp, D, shape, dev, stream, world)
@@ -264,9 +323,8 @@ def run_ours(args, rank, world, local_rank):
         "metric": METRIC, "value": round(tokens_per_s, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded; shapes of the pages' long-sequence encoder benchmark)",
-        "config": {"workload": f"{w.name}: B={w.num_seqs} x n={max_len} jagged, d={d}, "
-                               f"H={H}x{hd}, rab P={w.n_pos_buckets}/Tb={w.n_time_buckets}, 1 layer",
+        "data": "synthetic (seeded; shapes of the pages' workloads)",
+        "config": {"workload": workload_text(w, max_len),
                    "global_batch_tokens": job_tokens, "seq_len": max_len,
                    "parallelism": f"replicas over sequences x{world} (no collective)",
                    "l2": "flushed between timed steps (256 MB write, outside the events)"},
@@ -282,6 +340,8 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": int(launches),
         "clocks": clocks,
     }
+    if nl > 1:
+        result["config"]["layers_per_step"] = nl
     return result
 
 
@@ -292,6 +352,8 @@ def run_e2e(args, hstu, torch, inp, D, shape, dev, stream, world):
     runs from the first step's copy in to the last step's read-back, so it includes filling and
     draining the pipeline once; up to 100 steps keep that share small, as in steady serving."""
     steps = max(3, min(args.steps, 100))
+    if inp.workload.num_layers > 1:
+        return run_e2e_stack(args, hstu, torch, inp, D, dev, stream, world, steps)
     X_h = D["X"].cpu().pin_memory()
     off_h = D["off"].cpu().pin_memory()
     ts_h = D["ts"].cpu().pin_memory() if D["ts"] is not None else None
@@ -322,6 +384,59 @@ def run_e2e(args, hstu, torch, inp, D, shape, dev, stream, world):
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "ms_per_step": round(ms, 4), "steps": steps,
             "path": "hstu_layer_pipeline (copy-in, layer, copy-out streams; 2 buffer sets)"}
+
+
+def run_e2e_stack(args, hstu, torch, inp, D, dev, stream, world, steps):
+    """End to end for a stack of layers: every step copies X, the offsets and the timestamps in
+    from pinned host memory, runs each layer through hstu_layer_fwd (the next layer reads the
+    previous one's output on the device) and reads the last output back, all on one stream."""
+    w = inp.workload
+    X_h = D["X"].cpu().pin_memory()
+    off_h = D["off"].cpu().pin_memory()
+    ts_h = D["ts"].cpu().pin_memory() if D["ts"] is not None else None
+    y_h = torch.empty_like(X_h).pin_memory()
+    X_d, off_d = torch.empty_like(D["X"]), torch.empty_like(D["off"])
+    ts_d = torch.empty_like(D["ts"]) if ts_h is not None else None
+    max_len = int(inp.lengths.max())
+    shape = hstu.shape_for(X_d, off_d, w.num_heads, w.head_dim, w.head_dim, max_len, D["pos"],
+                           D["tim"], inp.ln_eps)
+    ws = hstu.alloc_workspace(shape, dev)
+    ys = [torch.empty_like(X_d) for _ in range(w.num_layers)]
+
+    def one():
+        X_d.copy_(X_h, non_blocking=True)
+        off_d.copy_(off_h, non_blocking=True)
+        if ts_h is not None:
+            ts_d.copy_(ts_h, non_blocking=True)
+        x = X_d
+        for l in range(w.num_layers):
+            L = D["layers"][l]
+            x = hstu.hstu_layer_fwd(x, off_d, ts_d, L["W1"], L["b1"], L["W2"], L["b2"], L["ln_w"],
+                                    L["ln_b"], D["pos"], D["tim"], D["ali"], inp.scale,
+                                    num_heads=w.num_heads, max_seq_len=max_len,
+                                    ln_eps=inp.ln_eps, out=ys[l], workspace=ws, stream=stream)
+        y_h.copy_(x, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if hstu.device_status() != hstu.HSTU_OK:
+        raise SystemExit("device status error in the end-to-end run")
+    ms, job_tokens = combine_over_ranks(e0.elapsed_time(e1) / steps, inp.T, world, dev)
+    h2d = X_h.numel() * X_h.element_size() + off_h.numel() * 8 + (ts_h.numel() * 8 if ts_h is not None else 0)
+    d2h = y_h.numel() * y_h.element_size()
+    return {"value": round(job_tokens / (ms * 1e-3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": round(ms, 4), "steps": steps,
+            "path": f"pinned host copies + hstu_layer_fwd x{w.num_layers} + read-back, one stream"}
 
 
 # ------------------------------------------------------------------------------------------------
@@ -814,13 +929,27 @@ def run_stochastic_length(args, rank, world, local_rank):
 # The oracle on the host cores (cpu_baseline of our arm, and the whole reference arm)
 # ------------------------------------------------------------------------------------------------
 
-def oracle_sample_time(inp, seq: int, L: int):
+def oracle_inputs_X(inp):
+    """The layer input X as the oracle sees it: the workload's X, or for action-oriented tokens the
+    oracle's own token assembly (item + action embedding, rounded to bf16)."""
+    if inp.X is not None:
+        return inp.X
+    import oracle
+    from workloads import widen_bf16
+    ids = np.unique(inp.item_ids)
+    return oracle.token_embed(np.searchsorted(ids, inp.item_ids), inp.action_ids,
+                              widen_bf16(inp.item_table_bits[ids], np.float64),
+                              widen_bf16(inp.action_table_bits, np.float64))
+
+
+def oracle_sample_time(inp, seq: int, L: int, X=None):
     import oracle
     a = int(inp.seq_offsets[seq])
     p = inp.layers[0]
     w = inp.workload
+    X = inp.X if X is None else X
     t0 = time.perf_counter()
-    oracle.layer_fwd(np.array([0, L]), inp.X[a:a + L], p.W1, p.b1, p.W2, p.b2, p.ln_w, p.ln_b,
+    oracle.layer_fwd(np.array([0, L]), X[a:a + L], p.W1, p.b1, p.W2, p.b2, p.ln_w, p.ln_b,
                      num_heads=w.num_heads, d_qk=w.head_dim, d_v=w.head_dim,
                      timestamps=None if inp.timestamps is None else inp.timestamps[a:a + L],
                      pos_table=inp.pos_table, time_table=inp.time_table,
@@ -828,15 +957,27 @@ def oracle_sample_time(inp, seq: int, L: int):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(inp):
+def cpu_baseline(inp, budget_s: float = 20.0):
+    """The oracle on a bounded sample of the workload: one layer over the longest causal prefix of
+    its longest sequence that fits about `budget_s` seconds (the whole sequence when it fits)."""
     import oracle
     oracle.build()
-    L = int(inp.lengths[0])
-    dt = oracle_sample_time(inp, 0, L)
+    X = oracle_inputs_X(inp)
+    s = int(np.argmax(inp.lengths))
+    n = int(inp.lengths[s])
+    L = min(n, 256)
+    dt = oracle_sample_time(inp, s, L, X)
+    while L < n:
+        # f1/f2 grow with L, attention with L^2: estimate the next size's time from this one
+        nxt = min(n, 2 * L)
+        if dt * (nxt / L) ** 2 > budget_s:
+            break
+        L = nxt
+        dt = oracle_sample_time(inp, s, L, X)
     return {"value": round(L / dt, 2), "unit": "tokens/s", "cores": oracle.num_threads(),
             "kind": "oracle",
-            "sample": f"one whole sequence ({L} tokens, all rows, 1 layer) of the workload; "
-                      f"{dt:.1f} s; C fp64 loops, OpenMP, -O2",
+            "sample": f"the first {L} of {n} tokens of the longest sequence (a whole causal "
+                      f"prefix), 1 layer; {dt:.1f} s; C fp64 loops, OpenMP, -O2",
             "host_cpus": len(os.sched_getaffinity(0))}
 
 
@@ -848,15 +989,16 @@ def run_reference(args, rank, world):
     w = workloads.WORKLOADS[args.workload]
     inp = workloads.make_inputs(w)
     # size each step so the whole warm-up + timed run stays within about three minutes
-    n = int(inp.lengths[0])
+    X = oracle_inputs_X(inp)
+    n = int(inp.lengths.min())
     budget = 180.0 / max(1, args.steps + args.warmup)
     L = n
-    t_probe = oracle_sample_time(inp, 0, min(n, 1024))
+    t_probe = oracle_sample_time(inp, 0, min(n, 1024), X)
     while L > 256 and t_probe * (L / min(n, 1024)) ** 2 > budget:
         L //= 2
     for k in range(args.warmup):
-        oracle_sample_time(inp, k % len(inp.lengths), L)
-    times = [oracle_sample_time(inp, k % len(inp.lengths), L) for k in range(args.steps)]
+        oracle_sample_time(inp, k % len(inp.lengths), L, X)
+    times = [oracle_sample_time(inp, k % len(inp.lengths), L, X) for k in range(args.steps)]
     ms = 1e3 * sum(times) / len(times)
     value = L / (ms * 1e-3)
     sample = (f"per step: the first {L} tokens of one sequence (a whole causal prefix) of "

@@ -30,7 +30,7 @@ EXPORTED = ["hstu_layer_fwd", "hstu_layer_fwd_workspace_size", "hstu_f1_fwd", "h
             "hstu_attention_workspace_size", "hstu_ln_gate_fwd", "hstu_f2_fwd",
             "hstu_token_embed_fwd", "hstu_status_string", "hstu_get_device_status", "hstu_version",
             "hstu_launch_count", "hstu_attention_fwd_noalloc", "hstu_selftest_bounded_wait",
-            "hstu_selftest_scratch_cache",
+            "hstu_selftest_scratch_cache", "hstu_ln_f2_fwd",
             "hstu_candidate_workspace_size", "hstu_candidate_attention_fwd",
             "hstu_candidate_layer_workspace_size", "hstu_candidate_layer_fwd",
             "hstu_stochastic_length_workspace_size", "hstu_stochastic_length", "hstu_gather_rows",
@@ -75,6 +75,7 @@ def _load() -> ctypes.CDLL:
         "hstu_attention_fwd_noalloc": ([SH, P, P, P, P, P, P, F32, P, P], ctypes.c_int),
         "hstu_ln_gate_fwd": ([SH, P, P, P, P, P, P], ctypes.c_int),
         "hstu_f2_fwd": ([SH, P, P, P, P, P, P], ctypes.c_int),
+        "hstu_ln_f2_fwd": ([SH, P, P, P, P, P, P, P, P, P], ctypes.c_int),
         "hstu_token_embed_fwd": ([I64, I32, P, P, P, I64, P, I64, P, P], ctypes.c_int),
         "hstu_status_string": ([ctypes.c_int], ctypes.c_char_p),
         "hstu_get_device_status": ([P], ctypes.c_int),
@@ -413,6 +414,14 @@ def hstu_ln_gate_fwd(shape: HstuShape, av, uvqk, ln_w, ln_b, g, stream=None):
 def hstu_f2_fwd(shape: HstuShape, g, W2, b2, X, out, stream=None):
     _check(_lib.hstu_f2_fwd(ctypes.byref(shape), _ptr(g), _ptr(W2), _ptr(b2), _ptr(X), _ptr(out),
                             _stream(stream)), "hstu_f2_fwd")
+    return out
+
+
+def hstu_ln_f2_fwd(shape: HstuShape, av, uvqk, ln_w, ln_b, W2, b2, X, out, stream=None):
+    """out = (LayerNorm(av) * U) W2 + b2 + X in one kernel (bf16, H*d_v == d in {128, 256, 512})."""
+    _check(_lib.hstu_ln_f2_fwd(ctypes.byref(shape), _ptr(av), _ptr(uvqk), _ptr(ln_w), _ptr(ln_b),
+                               _ptr(W2), _ptr(b2), _ptr(X), _ptr(out), _stream(stream)),
+           "hstu_ln_f2_fwd")
     return out
 
 

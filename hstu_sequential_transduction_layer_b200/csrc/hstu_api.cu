@@ -229,6 +229,20 @@ hstu_status_t run_f2(const hstu_shape_t& s, const void* g, const void* W2, const
   return launch_status();
 }
 
+// LayerNorm * U and f2 in one kernel, for the shapes it covers (bf16, LayerNorm width = d = 128,
+// 256 or 512); the caller checks ln_f2_fused() first.
+bool ln_f2_fused(const hstu_shape_t& s) {
+  return s.dtype == HSTU_BF16 && tc::ln_f2_supported(s.total_tokens, s.d_model, wv_of(s));
+}
+
+hstu_status_t run_ln_f2(const hstu_shape_t& s, const void* av, const void* uvqk, const void* ln_w,
+                        const void* ln_b, const void* W2, const void* b2, const void* X, void* out,
+                        cudaStream_t st) {
+  return tc::launch_ln_f2(s.total_tokens, s.d_model, (int)n1_of(s), (const float*)av,
+                          (const bf16*)uvqk, (const bf16*)ln_w, (const bf16*)ln_b, s.ln_eps,
+                          (const bf16*)W2, (const bf16*)b2, (const bf16*)X, (bf16*)out, st);
+}
+
 size_t attention_ws_bytes(const hstu_shape_t& s) {
   return s.dtype == HSTU_BF16 ? tc::attention_workspace_bytes(s.total_tokens, s.num_seqs,
                                                                s.num_heads)
@@ -601,8 +615,29 @@ hstu_status_t hstu_layer_fwd(const hstu_shape_t* shape, const void* X, const int
   if ((rc = run_attention(s, w.uvqk, seq_offsets, timestamps, pos_table, time_table, alibi_slopes,
                           scale, w.av, w.attn, w.attn_bytes, st)) != HSTU_OK)
     return rc;
+  if (ln_f2_fused(s)) return run_ln_f2(s, w.av, w.uvqk, ln_w, ln_b, W2, b2, X, out, st);
   if ((rc = run_ln_gate(s, w.av, w.uvqk, ln_w, ln_b, w.g, st)) != HSTU_OK) return rc;
   return run_f2(s, w.g, W2, b2, X, out, st);
+}
+
+hstu_status_t hstu_ln_f2_fwd(const hstu_shape_t* shape, const void* av, const void* uvqk,
+                             const void* ln_w, const void* ln_b, const void* W2, const void* b2,
+                             const void* X, void* out, void* stream) {
+  hstu_status_t rc = check_shape(shape);
+  if (rc != HSTU_OK) return rc;
+  const hstu_shape_t& s = *shape;
+  if (s.total_tokens == 0) return HSTU_OK;
+  if (!ln_f2_fused(s)) return HSTU_ERR_UNSUPPORTED;
+  if (!av || !uvqk || !ln_w || !ln_b || !W2 || !X || !out) return HSTU_ERR_INVALID_ARG;
+  const void* ptrs16[] = {av, uvqk, ln_w, ln_b, W2, b2, X, out};
+  for (const void* p : ptrs16)
+    if (!aligned16(p)) return HSTU_ERR_INVALID_ARG;
+  const size_t xbytes = (size_t)s.total_tokens * s.d_model * 2;
+  if (overlaps(out, xbytes, X, xbytes) ||
+      overlaps(out, xbytes, uvqk, (size_t)s.total_tokens * n1_of(s) * 2) ||
+      overlaps(out, xbytes, av, (size_t)s.total_tokens * wv_of(s) * 4))
+    return HSTU_ERR_INVALID_ARG;
+  return run_ln_f2(s, av, uvqk, ln_w, ln_b, W2, b2, X, out, static_cast<cudaStream_t>(stream));
 }
 
 hstu_status_t hstu_token_embed_fwd(int64_t T, int32_t d, const int64_t* item_ids,
@@ -798,7 +833,10 @@ hstu_status_t hstu_layer_bwd(const hstu_shape_t* shape, const void* X, const int
   if ((rc = tc::launch_gemm_ext<tc::EPI_F32>(T, (int)wv, d, dy, (const bf16*)w.w2t, nullptr,
                                              nullptr, nullptr, (float*)w.dg, 1, -1, st)) != HSTU_OK)
     return rc;
-  if ((rc = run_transpose(T, w.t_pad, (int)wv, wv, fw.g, w.trans, st)) != HSTU_OK) return rc;
+  // G = LayerNorm(AV) * U again from the forward's AV and U (the forward may have formed it only in
+  // shared memory), into the dAV buffer, which the LayerNorm backward fills only later
+  if ((rc = run_ln_gate(s, fw.av, fw.uvqk, ln_w, ln_b, w.dav, st)) != HSTU_OK) return rc;
+  if ((rc = run_transpose(T, w.t_pad, (int)wv, wv, w.dav, w.trans, st)) != HSTU_OK) return rc;
   const int kt = (int)w.t_pad;
   if ((rc = tc::launch_gemm_ext<tc::EPI_RED_F32>(
            wv, d, kt, (const bf16*)w.trans, dy, nullptr, nullptr, nullptr, dW2,

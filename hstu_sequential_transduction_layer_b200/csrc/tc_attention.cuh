@@ -14,24 +14,41 @@
 // sequences is small against L2, the list is one batch and CTA b takes items b, b + grid, ...;
 // otherwise each CTA's producer claims the next item from a global counter whenever it starts one,
 // and hands it to the CTA's other warps through a small ring in shared memory, so that the CTAs
-// running at the same time stay inside one or two batches whose K/V fit in L2.  Sequences are never padded: tiles that
-// straddle a sequence end read the next rows (or TMA zero fill past T) and the causal mask, which
-// coincides with the length mask for valid rows, removes them; rows past the end are not stored.
+// running at the same time stay inside one or two batches whose K/V fit in L2.  Sequences are never
+// padded: tiles that straddle a sequence end read the next rows (or TMA zero fill past T) and the
+// causal mask, which coincides with the length mask for valid rows, removes them; rows past the end
+// are not stored.
 //
-// Per CTA (384 threads, one CTA per SM), TMEM = S_A | S_B | O_A | O_B (128 columns each):
+// Per CTA (640 threads = 20 warps, one CTA per SM):
 //   warp 0      producer: Q_A and Q_B once per item, then K/V tiles into an NST-deep ring by TMA.  Its
-//               32 lanes also copy the tile's key timestamps into the ring stage and flag whether
-//               they are sorted; the stage's mbarrier publishes both.
-//   warps 1, 2  one single-thread MMA issuer per query tile X (warp 1 also owns TMEM).  Per key tile:
-//                 S_X(j) = Q_X K_j^T   (M=128, N=128, K=hd) into S_X
-//                 O_X   += P_X(j) V_j  (M=128, N=hd, K=128), P_X read from TMEM (aliased into S_X)
-//               tcgen05.mma issue blocks until the tensor pipe takes the instruction, so each query
-//               tile has its own issuer: neither waits behind the other's MMAs, and the tensor core
-//               works for one query tile while the other's pointwise warps compute P.
-//   warp 3      idle.
-//   warps 4-7   pointwise warpgroup A, warps 8-11 warpgroup B: one TMEM lane quadrant (32 query rows)
-//               per warp.  tcgen05.ld S, add the bias, SiLU, causal mask, pack to bf16 and tcgen05.st
-//               P over the S columns already read; at the end of the item, scale * O -> AV (fp32).
+//               lanes also copy the tile's key timestamps into the ring stage (as int64 and as int32
+//               relative to the sequence's first) and flag whether they are sorted and fit in int32;
+//               the stage's mbarrier publishes them with the tile.
+//   warp 1      S issuer (and TMEM owner): S_X(j) = Q_X K_j^T (M=128, N=128, K=hd) for both query
+//               tiles, in slot order, each into the next free S buffer.
+//   warps 2, 3  PV issuers of query tile A and B: O_X += P_X(j) V_j (M=128, N=hd, K=128), P_X read
+//               from TMEM, as soon as the pointwise warps have written it.  tcgen05.mma issue blocks
+//               until the tensor pipe takes the instruction, so S products for later tiles and the
+//               PV products of either query tile each have their own thread and none waits behind
+//               the others.  One elected lane of each of these warps issues.
+//   warps 4-19  16 pointwise warps: for query tile x = (warp-4)/8, two warps per TMEM lane quadrant
+//               (32 query rows), each on 64 of the tile's 128 keys.  tcgen05.ld S, add the bias,
+//               SiLU, causal mask, pack to bf16 and tcgen05.st P; at the end of the item,
+//               scale * O -> AV (fp32).
+// TMEM: NSB buffers of S (128 columns each; hd = 64: three, hd = 128: two) that rotate over the
+// (query tile, key tile) slots, then O_A | O_B (hd columns each).  Each warp writes its P over the
+// first 32 of its 64 S columns once it has read them; with three buffers the S of the next slots
+// is computed while the pointwise warps work on the current one.
+//
+// The pointwise stage works on pairs of scores with the sm_100 packed f32x2 instructions: per pair,
+// two 32-bit shared loads of the two halved position biases, one
+// packed add of the row's halved time bias, one packed FMA for h = S/2 + bias/2, two MUFU tanh and
+// one packed FMA for SiLU(2h) = h + h tanh(h), and one bf16x2 conversion.  The position (or ALiBi)
+// bias is staged per head as a reversed table of halved values, so the 32 keys of a chunk read it
+// at increasing addresses.  The time bias of a row is constant across a
+// half tile, or steps once (sorted keys) at a column found by binary search, applied through a
+// small table of 0/1 pairs.  Diagonal tiles, tiles whose time bucket steps more than once and tiles
+// beyond the staged distances take an exact per-element path.
 #pragma once
 
 #include "sm100.cuh"
@@ -45,11 +62,11 @@ constexpr int ATT_BM = 128;       // query rows per query tile
 constexpr int ATT_BN = 128;       // keys per key tile
 constexpr int ATT_ITEM_ROWS = 2 * ATT_BM;  // query rows per work item (a pair of query tiles)
 constexpr int ATT_TB_CAP = 256;   // time buckets staged in shared memory (more: read from global)
-constexpr int ATT_THREADS = 640;  // producer, 2 MMA issuers, idle warp, 4 pointwise warpgroups
+constexpr int ATT_THREADS = 640;  // producer, 3 MMA issuers, 4 pointwise warpgroups
 constexpr int ATT_PW = 512;       // pointwise threads
 constexpr int ATT_PW_WARPS = 8;   // pointwise warps per query tile
 constexpr int ATT_ITEM_RING = 4;  // work items handed from the producer to the other roles
-constexpr int ATT_ITEM_READERS = 2 + 2 * ATT_PW_WARPS;  // MMA issuers and pointwise warps
+constexpr int ATT_ITEM_READERS = 3 + 2 * ATT_PW_WARPS;  // MMA issuers and pointwise warps
 
 template <int HD>
 struct AttnCfg {
@@ -58,23 +75,32 @@ struct AttnCfg {
   static constexpr int KV_TILE = HD / 64 * BOX;             // K or V tile
   static constexpr int NST = HD == 64 ? 4 : 2;              // K/V ring depth
   static constexpr int STAGE_BYTES = 2 * KV_TILE;
-  static constexpr int POS_CAP = HD == 64 ? 8192 : 7168;    // position buckets staged (half values)
+  // Position (or ALiBi) bias of distances below POS_CAP, halved and reversed: tab[POS_CAP-1-d]
+  // holds the bias at distance d, followed by 128 zeros for the masked distances -128 < d < 0.
+  // (A copy shifted by one element, so that every pair of elements is one aligned 8-byte load,
+  // measured slower on long sequences than two 4-byte loads: PAIRED stays off.)
+  static constexpr int POS_CAP = HD == 64 ? 8192 : 7168;
+  static constexpr bool PAIRED = false;
+  static constexpr int TAB_N = POS_CAP + 128;
   static constexpr int OFF_KV = 2 * Q_BYTES;
   static constexpr int OFF_TS = OFF_KV + NST * STAGE_BYTES;          // [NST][128] int64
   static constexpr int OFF_TS32 = OFF_TS + NST * ATT_BN * 8;         // [NST][128] int32, relative
   static constexpr int OFF_FLAG = OFF_TS32 + NST * ATT_BN * 4;       // [NST] int
-  static constexpr int OFF_POS = OFF_FLAG + 64;                      // [POS_CAP] float
-  static constexpr int OFF_TT = OFF_POS + POS_CAP * 4;               // [TB_CAP] float
+  static constexpr int OFF_TAB = OFF_FLAG + 64;                      // [TAB_N] float
+  static constexpr int OFF_TAB2 = OFF_TAB + TAB_N * 4;               // [TAB_N] float (PAIRED)
+  static constexpr int OFF_TT = OFF_TAB2 + (PAIRED ? TAB_N * 4 : 0); // [TB_CAP] float
   static constexpr int OFF_CLZ = OFF_TT + ATT_TB_CAP * 4;            // [32] float
-  static constexpr int OFF_BAR = OFF_CLZ + 32 * 4;
+  static constexpr int OFF_STEP = OFF_CLZ + 32 * 4;                  // [64] float2
+  static constexpr int OFF_BAR = OFF_STEP + 64 * 8;
   static constexpr int SMEM = OFF_BAR + 512;
   static constexpr int TMEM_COLS = 512;
-  // TMEM columns.  hd = 64: S_A | S_B | O_A | O_B | P_A | P_B (128, 128, 64, 64, 64, 64), P apart
-  // from S so that S(j+1) can be computed while P(j) still waits for its PV product.  hd = 128:
-  // S_A | S_B | O_A | O_B (128 each) and P written over the S columns already read.
-  static constexpr bool SEP_P = HD == 64;
-  static constexpr int O_COL = 256, O_STRIDE = SEP_P ? 64 : 128, P_COL = 384;
+  // TMEM: NSB buffers of S (128 columns each, P written over the columns its warp has read) that
+  // rotate over the (query tile x, key tile g) slots, slot -> buffer (2g + x) % NSB, then O_A, O_B
+  static constexpr int NSB = HD == 64 ? 3 : 2;
+  static constexpr int O_COL = NSB * 128, O_STRIDE = HD;
+  static_assert(O_COL + 2 * O_STRIDE <= TMEM_COLS, "tensor memory budget");
   static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(OFF_TAB % 8 == 0 && OFF_TAB2 % 8 == 0 && OFF_STEP % 8 == 0, "8-byte pair loads");
 };
 
 // Header of the attention workspace: [0] item count, [1] next item to hand out (the persistent CTAs
@@ -360,6 +386,17 @@ __device__ __forceinline__ float silu_from_half(float h) {
   return fmaf(h, sm100::tanh_approx(h), h);
 }
 
+// The same for a pair of halves h2 = (h0, h1), packed to bf16x2 (low half = h0's): two MUFU
+// operations and one packed f32x2 FMA.
+__device__ __forceinline__ uint32_t silu_pair_bf16(uint64_t h2) {
+  float h0, h1;
+  sm100::f2_unpack(h2, h0, h1);
+  const uint64_t t2 = sm100::f2_pack(sm100::tanh_approx(h0), sm100::tanh_approx(h1));
+  float p0, p1;
+  sm100::f2_unpack(sm100::f2_fma(h2, t2, h2), p0, p1);
+  return pack_bf16x2(p0, p1);
+}
+
 // All 256 pointwise threads arrive and wait (bounded) on a group barrier.
 __device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& count, volatile int* abort_flag) {
   sm100::mbar_arrive(bar);
@@ -368,170 +405,169 @@ __device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& count, volat
   return ok;
 }
 
-// How a pointwise warp forms the bias of its 32 rows x 128 keys of one tile.
-enum TileMode { TILE_GENERAL = 0, TILE_FAST = 1, TILE_GEN32 = 2 };
-
 // Key-tile flags written by the producer next to the staged timestamps.
 constexpr int KEYS_SORTED = 1;   // non-decreasing along the tile
 constexpr int KEYS_REL32 = 2;    // every key's timestamp is within +-2^30 of the sequence's first
 
-// Fast path over 32 columns (col0 + e, e = 0..31): h = S/2 + hb, P = SiLU(2h).
-//   BIAS_RAB:   hb = hpos_ext[i - key] + (SPLIT && col >= cstar ? hb1 : hb0), where hpos_ext holds
-//               half the position table extended with its clamped last entry, and hb0/hb1 are the
-//               halved time biases before/after the one bucket change inside the tile
-//               (prow = hpos_ext + i - key0 - col0 for this chunk, cst = cstar - col0)
-//   BIAS_ALIBI: hb = hb0 + e * m/2                (hb0 = -(m/2) (i - key0 - col0) for this chunk)
-//   BIAS_NONE:  hb = 0
-template <int BIAS, bool SPLIT>
-__device__ __forceinline__ void fast_chunk(const uint32_t (&sv)[32], float hb0, float hb1, int cst,
-                                           const float* prow, float half_slope,
-                                           uint32_t (&pk)[16]) {
+// Fast path over 32 keys (columns c0 + e, e = 0..31) none of which is masked and whose distances
+// are all staged: h = S/2 + b, P = SiLU(2h), with b the halved bias
+//   b(e) = tab[e] (+ hb0, or with SPLIT hb0 + dhb * [e >= cst]),
+// where `tab` points at the reversed table's entry of this row's distance to key c0 (so key c0 + e
+// reads tab[e]), 8-byte aligned when PAIRED; hb0x2 = (hb0, hb0) is the row's halved time bias;
+// `step` points at a table of 0/1 pairs such that step[e] = ([e >= cst], [e + 1 >= cst]).
+template <bool PAIRED, bool TIME, bool SPLIT>
+__device__ __forceinline__ void fast_chunk(const uint32_t (&sv)[32], const float* tab, uint64_t hb0x2,
+                                           uint64_t dhb2, const float2* step, uint32_t (&pk)[16]) {
+  const uint64_t half2 = sm100::f2_pack(0.5f, 0.5f);
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
-    float p2[2];
-#pragma unroll
-    for (int u = 0; u < 2; u++) {
-      float hb;
-      if (BIAS == BIAS_RAB) {
-        hb = ((SPLIT && e + u >= cst) ? hb1 : hb0) + prow[-(e + u)];
-      } else if (BIAS == BIAS_ALIBI) {
-        hb = fmaf((float)(e + u), half_slope, hb0);
-      } else {
-        hb = 0.0f;
-      }
-      p2[u] = silu_from_half(fmaf(__uint_as_float(sv[e + u]), 0.5f, hb));
+    uint64_t b2;
+    if (PAIRED) {
+      const float2 t = *reinterpret_cast<const float2*>(tab + e);
+      b2 = sm100::f2_pack(t.x, t.y);
+    } else {
+      b2 = sm100::f2_pack(tab[e], tab[e + 1]);
     }
-    pk[e / 2] = pack_bf16x2(p2[0], p2[1]);
+    if (TIME) {
+      uint64_t tb2 = hb0x2;
+      if (SPLIT) {
+        const float2 st = step[e];
+        tb2 = sm100::f2_fma(sm100::f2_pack(st.x, st.y), dhb2, hb0x2);
+      }
+      b2 = sm100::f2_add(b2, tb2);
+    }
+    pk[e / 2] = silu_pair_bf16(sm100::f2_fma(sm100::f2_pack_bits(sv[e], sv[e + 1]), half2, b2));
   }
 }
 
-// Exact path over 32 columns: clamped position bucket, per-element time bucket, mask.
-// dist0 = i - (key0 + col0) with i the row's position; keys at distance < dmin are masked (0: the
-// causal mask j <= i; 1: a candidate sees history keys j < n_hist only); tsk points at this chunk's
-// staged key timestamps.
-template <int BIAS>
-__device__ __forceinline__ void general_chunk(const uint32_t (&sv)[32], int dist0, int dmin, int P, int Tb,
-                                              int staged_n, int64_t ti, const int64_t* tsk,
-                                              const float* hpos, const float* htt,
-                                              const float* pos_h, const float* tim_h,
-                                              float half_slope, uint32_t (&pk)[16]) {
+// No bias: h = S/2.
+__device__ __forceinline__ void nobias_chunk(const uint32_t (&sv)[32], uint32_t (&pk)[16]) {
+  const uint64_t half2 = sm100::f2_pack(0.5f, 0.5f);
 #pragma unroll
-  for (int e = 0; e < 32; e += 2) {
-    float p2[2];
-#pragma unroll
-    for (int u = 0; u < 2; u++) {
-      const int dist = dist0 - (e + u);
-      float hb = 0.0f;
-      if (BIAS == BIAS_RAB) {
-        if (pos_h) {
-          const int pi = dist < 0 ? 0 : dist;   // the staged table already clamps to P-1
-          hb += pi < staged_n ? hpos[pi] : 0.5f * __ldg(pos_h + (pi < P - 1 ? pi : P - 1));
-        }
-        if (tim_h) {
-          int b = time_bucket(ti, tsk[e + u]);
-          b = b < Tb - 1 ? b : Tb - 1;
-          hb += b < ATT_TB_CAP ? htt[b] : 0.5f * __ldg(tim_h + b);
-        }
-      } else if (BIAS == BIAS_ALIBI) {
-        hb = -half_slope * (float)dist;
-      }
-      const float h = fmaf(__uint_as_float(sv[e + u]), 0.5f, hb);
-      p2[u] = dist < dmin ? 0.0f : silu_from_half(h);
-    }
-    pk[e / 2] = pack_bf16x2(p2[0], p2[1]);
-  }
+  for (int e = 0; e < 32; e += 2)
+    pk[e / 2] = silu_pair_bf16(sm100::f2_mul(sm100::f2_pack_bits(sv[e], sv[e + 1]), half2));
 }
 
-// Exact path with 32-bit timestamps relative to the sequence's first one: the time bucket
-// floor(log2(1 + max(ti - tj, 0))) is 31 - clz(max(ti1 - tj, 1)) with ti1 = ti + 1, and hclz[c]
-// holds the halved time bias of bucket min(31 - c, Tb - 1).  Mask as in general_chunk.
-__device__ __forceinline__ void general32_chunk(const uint32_t (&sv)[32], int dist0, int dmin, int P,
-                                                int staged_n, int ti1, const int* tsk32,
-                                                const float* hpos, const float* hclz,
-                                                const float* pos_h, uint32_t (&pk)[16]) {
-#pragma unroll
-  for (int e = 0; e < 32; e += 2) {
-    float p2[2];
-#pragma unroll
-    for (int u = 0; u < 2; u++) {
-      const int dist = dist0 - (e + u);
-      float hb = 0.0f;
-      if (pos_h) {
-        const int pi = dist < 0 ? 0 : dist;   // the staged table already clamps to P-1
-        hb = pi < staged_n ? hpos[pi] : 0.5f * __ldg(pos_h + (pi < P - 1 ? pi : P - 1));
-      }
-      const int d1 = max(ti1 - tsk32[e + u], 1);
-      hb += hclz[__clz(d1)];
-      const float h = fmaf(__uint_as_float(sv[e + u]), 0.5f, hb);
-      p2[u] = dist < dmin ? 0.0f : silu_from_half(h);
-    }
-    pk[e / 2] = pack_bf16x2(p2[0], p2[1]);
-  }
-}
-
-// Per-tile state of one pointwise thread.
-struct TileArgs {
-  int i, key0, P, Tb, staged_n, cstar, ti1, dmin;
+// Per-tile state of one pointwise thread for the exact path.
+struct ExactArgs {
+  int P, Tb, ti1, dmin;
   int64_t ti;
-  const int64_t* tsk;       // staged timestamps of the tile's 128 keys
+  const int64_t* tsk;       // staged timestamps of the chunk's 32 keys
   const int* tsk32;         // the same, relative to the sequence's first timestamp
-  const float *hpos, *htt, *hclz, *pos_h, *tim_h;
-  float hb0, hb1, half_slope;
+  const float* tab0;        // the reversed table's distance-0 entry: distance d at tab0[-d]
+  const float *htt, *hclz, *pos_h, *tim_h;
+  float half_slope;
 };
 
-template <int BIAS, int MODE, bool SPLIT>
-__device__ __forceinline__ void do_chunk(const uint32_t (&sv)[32], int col0, const TileArgs& a,
-                                         uint32_t (&pk)[16]) {
-  if (MODE == TILE_GENERAL) {
-    general_chunk<BIAS>(sv, a.i - a.key0 - col0, a.dmin, a.P, a.Tb, a.staged_n, a.ti, a.tsk + col0, a.hpos,
-                        a.htt, a.pos_h, a.tim_h, a.half_slope, pk);
-  } else if (MODE == TILE_GEN32) {
-    general32_chunk(sv, a.i - a.key0 - col0, a.dmin, a.P, a.staged_n, a.ti1, a.tsk32 + col0, a.hpos, a.hclz,
-                    a.pos_h, pk);
-  } else if (BIAS == BIAS_ALIBI) {
-    fast_chunk<BIAS, false>(sv, fmaf((float)col0, a.half_slope, a.hb0), 0.0f, 0, nullptr,
-                            a.half_slope, pk);
-  } else {
-    fast_chunk<BIAS, SPLIT>(sv, a.hb0, a.hb1, a.cstar - col0, a.hpos + (a.i - a.key0 - col0), 0.0f,
-                            pk);
+// Exact path over 32 keys: per-element distance dist0 - e and position bias from the staged table
+// (FAR: distances beyond the staged ones read the table from global memory, clamped to P-1),
+// per-element time bucket (TMODE 1: int64 timestamps; 2: int32 relative ones, where
+// floor(log2(1 + max(ti - tj, 0))) is 31 - clz(max(ti1 - tj, 1)) with ti1 = ti + 1 and hclz[c]
+// holds the halved time bias of bucket min(31 - c, Tb - 1)); with MASK, keys at distance < dmin
+// get P = 0 (0: the causal mask j <= i; 1: a candidate sees history keys j < n_hist only).
+template <int BIAS, bool MASK, int TMODE, bool FAR>
+__device__ __forceinline__ void exact_chunk(const uint32_t (&sv)[32], int dist0, int staged_n,
+                                            const ExactArgs& a, uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int e4 = 0; e4 < 32; e4 += 4) {
+    int t4[4] = {0, 0, 0, 0};
+    if (TMODE == 2) {   // four keys' timestamps in one 16-byte load (broadcast to the warp)
+      const int4 q = reinterpret_cast<const int4*>(a.tsk32)[e4 / 4];
+      t4[0] = q.x, t4[1] = q.y, t4[2] = q.z, t4[3] = q.w;
+    }
+#pragma unroll
+    for (int e = e4; e < e4 + 4; e += 2) {
+      float p2[2];
+#pragma unroll
+      for (int u = 0; u < 2; u++) {
+        const int dist = dist0 - (e + u);
+        float hb = 0.0f;
+        if (BIAS == BIAS_RAB) {
+          if (a.pos_h) {  // distances below 0 read the table's zero padding (masked anyway)
+            if (FAR)
+              hb = dist < staged_n ? a.tab0[-dist]
+                                   : 0.5f * __ldg(a.pos_h + (dist < a.P - 1 ? dist : a.P - 1));
+            else
+              hb = a.tab0[-dist];
+          }
+          if (TMODE == 1) {
+            int b = time_bucket(a.ti, a.tsk[e + u]);
+            b = b < a.Tb - 1 ? b : a.Tb - 1;
+            hb += b < ATT_TB_CAP ? a.htt[b] : 0.5f * __ldg(a.tim_h + b);
+          } else if (TMODE == 2) {
+            hb += a.hclz[__clz(max(a.ti1 - t4[e + u - e4], 1))];
+          }
+        } else if (BIAS == BIAS_ALIBI) {
+          hb = -a.half_slope * (float)dist;
+        }
+        const float h = fmaf(__uint_as_float(sv[e + u]), 0.5f, hb);
+        p2[u] = (MASK && dist < a.dmin) ? 0.0f : silu_from_half(h);
+      }
+      pk[e / 2] = pack_bf16x2(p2[0], p2[1]);
+    }
   }
 }
 
-// One warp's 32 rows x 64 keys (columns col0 .. col0+63 of the S tile), as two 32-column chunks.
-// P (bf16 pairs) of the 64 keys overwrites the first 32 of these S columns, which this thread has
-// already read.  The next chunk's TMEM load is issued before the current chunk's P is stored.
-template <int BIAS, int MODE, bool SPLIT>
-__device__ __forceinline__ void pointwise_tile(uint32_t s_col, int col0, const TileArgs& a) {
-  uint32_t sv[32], pk[16];
-  sm100::tmem_ld32(s_col, sv);
-  sm100::tmem_ld_wait(sv);
-  do_chunk<BIAS, MODE, SPLIT>(sv, col0, a, pk);
-  sm100::tmem_ld32(s_col + 32, sv);
-  sm100::tmem_st16(s_col, pk);
-  sm100::tmem_ld_wait(sv);
-  do_chunk<BIAS, MODE, SPLIT>(sv, col0 + 32, a, pk);
-  sm100::tmem_st16(s_col + 16, pk);
+// Time-bias set-up of one pointwise thread for one key tile: the buckets of its first and last key
+// (k = 0 and 63 of the warp's 64), and, when they differ by one (sorted keys step down once), the
+// first key of the lower bucket, found by a branch-free binary search.
+struct TimeSetup {
+  bool fast, split, rel32;
+  int cst;          // first of the warp's 64 keys in the lower bucket (64: none)
+  float hb0, hb1;   // halved time bias before and after it
+};
+
+template <bool CAND>
+__device__ __forceinline__ TimeSetup time_setup(bool fast_in, int flags, bool row_rel32, int ti1,
+                                                int64_t ti, const int* tsk32, const int64_t* tsk,
+                                                const float* htt, const float* tim_h, int Tb) {
+  constexpr unsigned FULL = 0xffffffffu;
+  TimeSetup ts;
+  ts.rel32 = __all_sync(FULL, (flags & KEYS_REL32) && row_rel32);
+  ts.split = false;
+  ts.cst = 64;
+  ts.hb0 = ts.hb1 = 0.0f;
+  ts.fast = fast_in;
+  if (!fast_in) return ts;
+  int bf, bl;
+  if (ts.rel32) {
+    bf = 31 - __clz(max(ti1 - tsk32[0], 1));
+    bl = 31 - __clz(max(ti1 - tsk32[63], 1));
+  } else {
+    bf = time_bucket(ti, tsk[0]);
+    bl = time_bucket(ti, tsk[63]);
+  }
+  ts.fast = __all_sync(FULL, (flags & KEYS_SORTED) && bf - bl <= 1 && bf < 62);
+  if (!ts.fast) return ts;
+  ts.split = __any_sync(FULL, bf != bl);
+  if (ts.split) {
+    // the largest k with t_k <= ti + 1 - 2^bf (k = 0 qualifies: its bucket is bf); keys after it
+    // are in bucket bf - 1 when bf != bl, and none is when bf == bl (then k ends at 63)
+    int base = 0;
+    if (ts.rel32) {
+      const int thr = ti1 - (1 << bf);
+#pragma unroll
+      for (int step = 32; step >= 1; step >>= 1) base += tsk32[base + step] <= thr ? step : 0;
+    } else {
+      const int64_t thr = ti + 1 - (1LL << bf);
+#pragma unroll
+      for (int step = 32; step >= 1; step >>= 1) base += tsk[base + step] <= thr ? step : 0;
+    }
+    ts.cst = bf != bl ? base + 1 : 64;
+  }
+  const int b0 = bf < Tb - 1 ? bf : Tb - 1, b1 = bl < Tb - 1 ? bl : Tb - 1;
+  ts.hb0 = b0 < ATT_TB_CAP ? htt[b0] : 0.5f * __ldg(tim_h + b0);
+  ts.hb1 = b1 < ATT_TB_CAP ? htt[b1] : 0.5f * __ldg(tim_h + b1);
+  return ts;
 }
 
-// Separate-P form (hd = 64): P goes to its own TMEM columns.  `s_consumed()` is called as soon as
-// the warp's S columns are in registers, so that the next S can be computed while P is; `p_free()`
-// is called before the first P store: the previous tile's PV must have read the P columns.
-template <int BIAS, int MODE, bool SPLIT, class PFree, class SConsumed>
-__device__ __forceinline__ void pointwise_tile_sep(uint32_t s_col, uint32_t p_col, int col0,
-                                                   const TileArgs& a, PFree p_free,
-                                                   SConsumed s_consumed) {
-  uint32_t sv[32], pk[16];
-  sm100::tmem_ld32(s_col, sv);
-  sm100::tmem_ld_wait(sv);
-  do_chunk<BIAS, MODE, SPLIT>(sv, col0, a, pk);
-  sm100::tmem_ld32(s_col + 32, sv);
-  p_free();
-  sm100::tmem_st16(p_col, pk);
-  sm100::tmem_ld_wait(sv);
-  s_consumed();
-  do_chunk<BIAS, MODE, SPLIT>(sv, col0 + 32, a, pk);
-  sm100::tmem_st16(p_col + 16, pk);
-}
+// How a pointwise warp forms the bias of one 32-key chunk.
+enum ChunkMode {
+  CH_FAST = 0,        // staged bias table + one or two time-bias constants
+  CH_EXACT = 1,       // per-element buckets, no mask
+  CH_EXACT_MASK = 2,  // per-element buckets and the mask
+  CH_ZERO = 3         // every key masked: P = 0
+};
 
 // Producer side (one thread): claims the next unhandled entry of the item list (or -1 past its end)
 // and hands it over as item k in ring slot k % ATT_ITEM_RING, once every reader has taken the slot's
@@ -580,22 +616,29 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   int* ts32_ring = reinterpret_cast<int*>(smem + Cfg::OFF_TS32);
   float* hclz_s = reinterpret_cast<float*>(smem + Cfg::OFF_CLZ);
   int* flag_ring = reinterpret_cast<int*>(smem + Cfg::OFF_FLAG);
-  float* hpos_s = reinterpret_cast<float*>(smem + Cfg::OFF_POS);  // 0.5 * pos[h][.]
-  float* htt_s = reinterpret_cast<float*>(smem + Cfg::OFF_TT);    // 0.5 * tim[h][.]
+  float* tab_s = reinterpret_cast<float*>(smem + Cfg::OFF_TAB);    // reversed halved bias table
+  float* tab2_s = reinterpret_cast<float*>(smem + Cfg::OFF_TAB2);  // the same, shifted by one
+  float* htt_s = reinterpret_cast<float*>(smem + Cfg::OFF_TT);     // 0.5 * tim[h][.]
+  float2* step_s = reinterpret_cast<float2*>(smem + Cfg::OFF_STEP);  // 0/1 pairs
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
   uint64_t* kv_full = bars;                  // [NST]
   uint64_t* kv_empty = kv_full + Cfg::NST;   // [NST]
-  uint64_t* s_full = kv_empty + Cfg::NST;    // [2] per query tile
-  uint64_t* p_full = s_full + 2;             // [2]
-  uint64_t* o_full = p_full + 2;             // [2]
+  // [NSB][2]: S of query tile x's next computed slot in buffer b is ready (one phase per slot x
+  // computes) / x's slot in buffer b is done (one phase per slot, computed or passed through).
+  // Each barrier advances with one query tile's uses of one buffer, and no party is ever two phases
+  // ahead of a waiter, so a parity wait always refers to the phase meant.
+  uint64_t* s_full = kv_empty + Cfg::NST;
+  uint64_t* buf_free = s_full + 2 * Cfg::NSB;
+  // [2][2]: query tile x's P of its t-th computed tile is in TMEM, on barrier [x][t & 1]: with
+  // three S buffers the pointwise warps can be two tiles ahead of the PV products
+  uint64_t* p_full = buf_free + 2 * Cfg::NSB;
+  uint64_t* o_full = p_full + 4;             // [2]
   uint64_t* o_empty = o_full + 2;            // [2]
-  uint64_t* s_free = o_empty + 2;            // [2] S read into registers (separate-P form)
-  uint64_t* p_free = s_free + 2;             // [2] previous PV has read P (separate-P form)
-  uint64_t* q_full = p_free + 2;
+  uint64_t* q_full = o_empty + 2;
   uint64_t* q_empty = q_full + 1;
   uint64_t* pw_bar = q_empty + 1;
-  uint64_t* drain = pw_bar + 1;             // [2]
-  uint64_t* item_full = drain + 2;          // [ATT_ITEM_RING] the producer published an item
+  uint64_t* drain = pw_bar + 1;             // [3] one per MMA-issuing warp
+  uint64_t* item_full = drain + 3;          // [ATT_ITEM_RING] the producer published an item
   uint64_t* item_empty = item_full + ATT_ITEM_RING;  // [ATT_ITEM_RING] every consumer has read it
   int64_t* item_ring = reinterpret_cast<int64_t*>(item_empty + ATT_ITEM_RING);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(item_ring + ATT_ITEM_RING);
@@ -613,21 +656,24 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     if (!aligned) report(HSTU_ERR_CUDA);
     for (int s = 0; s < Cfg::NST; s++) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 2);   // one arrival per MMA issuer
+      mbar_init(&kv_empty[s], 2);   // one arrival per PV issuer
     }
     for (int x = 0; x < 2; x++) {
-      mbar_init(&s_full[x], 1);
-      mbar_init(&p_full[x], ATT_PW_WARPS);
+      mbar_init(&p_full[2 * x], ATT_PW_WARPS);
+      mbar_init(&p_full[2 * x + 1], ATT_PW_WARPS);
       mbar_init(&o_full[x], 1);
       mbar_init(&o_empty[x], ATT_PW_WARPS);
-      mbar_init(&s_free[x], ATT_PW_WARPS);
-      mbar_init(&p_free[x], 1);
+    }
+    for (int b = 0; b < 2 * Cfg::NSB; b++) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&buf_free[b], 1);
     }
     mbar_init(q_full, 1);
     mbar_init(q_empty, 2);
     mbar_init(pw_bar, ATT_PW);
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
+    mbar_init(&drain[2], 1);
     for (int r = 0; r < ATT_ITEM_RING; r++) {
       mbar_init(&item_full[r], 1);
       mbar_init(&item_empty[r], ATT_ITEM_READERS);
@@ -734,123 +780,171 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         if (kv_par[s] >= 0) mbar_drain(&kv_full[s], (uint32_t)kv_par[s]);
     }
     __syncwarp();
-  } else if (warp == 1 || warp == 2) {
-    // ------------------------------------------------------------------ MMA issuer of query tile x
-    const int x = warp - 1;
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16(128, ATT_BN, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16(128, HD, false, true);
-      uint32_t g = 0, k = 0, kx = 0, gx = 0;   // tiles, items, items with tile x, P tiles consumed
-      bool ok = true;
-      auto wait_kv = [&](uint32_t gg) {
-        return mbar_wait(&kv_full[gg % Cfg::NST], (gg / Cfg::NST) & 1u, abort_flag);
-      };
-      const uint32_t q_addr = smem_u32(q_s + x * Cfg::Q_BYTES);
-      const uint32_t s_tmem = tmem + x * 128, o_tmem = tmem + Cfg::O_COL + x * Cfg::O_STRIDE;
-      const uint32_t p_tmem = Cfg::SEP_P ? tmem + Cfg::P_COL + x * 64 : s_tmem;
-      auto issue_s = [&](uint32_t gg) {
-        const uint32_t k_addr = smem_u32(kv_s + (gg % Cfg::NST) * Cfg::STAGE_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; kk++) {
-          const uint32_t off = (kk / 4) * Cfg::BOX + (kk % 4) * 32;
-          mma_ss(s_tmem, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024),
-                 idesc_s, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(&s_full[x]);
-      };
-      auto issue_pv = [&](uint32_t gg, bool accumulate) {
-        const uint32_t v_addr = smem_u32(kv_s + (gg % Cfg::NST) * Cfg::STAGE_BYTES + Cfg::KV_TILE);
-#pragma unroll
-        for (int kk = 0; kk < ATT_BN / 16; kk++) {
-          // P of keys 16kk .. 16kk+15: 8 columns; with P aliased into S, the P of keys 64..127 sits
-          // at S column 64 (the first S column the second half's warps read)
-          const uint32_t pc = Cfg::SEP_P ? kk * 8 : (kk & 3) * 8 + (kk >> 2) * 64;
-          mma_ts(o_tmem, p_tmem + pc, sdesc_sw128(v_addr + kk * 2048, Cfg::BOX, 1024), idesc_o,
-                 (accumulate || kk > 0) ? 1u : 0u);
-        }
-      };
-      for (; ok; k++) {
-        const int64_t item = prm.dynamic
-                                 ? read_item(k, item_full, item_empty, item_ring, abort_flag)
-                                 : static_item(k, sch, n_items);
-        if (item < 0) break;
-        const ItemGeom ig = item_geom<CAND>(item, sch);
-        const int m = ig.m, nk = ig.nk;
-        const bool has_b = ig.has_b;
-        // this query tile's last key tile: the diagonal one, or the history's last
-        const int last = CAND ? nk - 1 : 2 * m + x;
-        // a candidate item without history has no key tile: its query tiles take no MMA
-        const bool mine = (x == 0 || has_b) && nk > 0;
-        if (!mbar_wait(q_full, k & 1u, abort_flag)) break;
-        int j = 0;
-        if (mine) {
-          if (!wait_kv(g)) break;
-          tc_fence_after();
-          issue_s(g);
-          if (last == 0) mma_commit(q_empty);
-          for (; j <= last; j++) {
-            const uint32_t gj = g + j;
-            if (Cfg::SEP_P) {
-              // S(j) is in the pointwise warps' registers: compute S(j+1) right away
-              if (!mbar_wait(&s_free[x], gx & 1u, abort_flag)) { ok = false; break; }
-              if (j < last) {
-                if (!wait_kv(gj + 1)) { ok = false; break; }
-                tc_fence_after();
-                issue_s(gj + 1);
-                if (j + 1 == last) mma_commit(q_empty);
-              }
-            }
-            if (!mbar_wait(&p_full[x], gx & 1u, abort_flag)) { ok = false; break; }
-            gx++;
-            if (j == 0 && !mbar_wait(&o_empty[x], (kx & 1u) ^ 1u, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            issue_pv(gj, j > 0);
-            if (Cfg::SEP_P) {
-              mma_commit(&p_free[x]);
-            } else if (j < last) {
-              if (!wait_kv(gj + 1)) { ok = false; break; }
-              tc_fence_after();
-              issue_s(gj + 1);
-              if (j + 1 == last) mma_commit(q_empty);
-            }
-            if (j == last) mma_commit(&o_full[x]);
-            mma_commit(&kv_empty[gj % Cfg::NST]);
-          }
-          if (!ok) break;
-          kx++;
-        } else {
-          mbar_arrive(q_empty);                       // Q of this item was loaded; nothing to read
-        }
-        // key tiles of the item this query tile does not read: release them once they are filled
-        for (; j < nk; j++) {
-          if (!wait_kv(g + j)) { ok = false; break; }
-          mbar_arrive(&kv_empty[(g + j) % Cfg::NST]);
-        }
-        g += nk;
-      }
-      mma_commit(&drain[x]);
-      mbar_drain(&drain[x], 0);
-    }
-    __syncwarp();
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------------ pointwise warpgroups
-    const int x = (warp - 4) >> 3;        // 0: query tile A, 1: query tile B
-    const int half = (warp >> 2) & 1;     // key columns [64 half, 64 half + 64) of each S tile
-    const int q = warp & 3;               // TMEM lane quadrant
-    const int tid = threadIdx.x - 128;    // 0..511 over the four warpgroups
-    const int r = q * 32 + lane;          // query row inside the tile
-    const int col0 = half * 64;
-    const uint32_t t_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    const uint32_t s_col = t_lane + x * 128 + col0;
-    const bool has_pos = BIAS == BIAS_RAB && prm.pos != nullptr;
-    const int P = prm.P, Tb = prm.Tb;
-    uint32_t g = 0, kx = 0, gx = 0, pw_cnt = 0;
-    int staged_head = -1, staged_n = 0;  // what hpos_s / htt_s hold
-    for (uint32_t k = 0;; k++) {
+  } else if (warp >= 1 && warp <= 3) {
+    uint32_t pv_count = 0, o_count = 0;   // P tiles consumed, items with PV products (warps 2, 3)
+    // ------------------------------------------------------------------ MMA issuers
+    // Warp 1 issues every S product, warps 2 and 3 the PV products of query tile A and B.  The
+    // whole warp runs the control flow (waits, item geometry, descriptor arithmetic: warp-uniform
+    // values) and one elected lane issues each group of MMAs and its commit.  Slot (x, g) of key
+    // tile g (counted over the CTA's items) owns S buffer b = (2g + x) % NSB; its S waits until
+    // the buffer's previous slot, 2g + x - NSB, is done (its PV has run), and a slot that its
+    // query tile does not read is passed through unused.  Query tile x uses a buffer every
+    // NSB / gcd(2, NSB) key tiles: its k-th use is at key tile g with k = g / 3 (three buffers) or
+    // k = g (two).  With S and PV in separate threads, the S of later slots is issued as soon as a
+    // buffer is free, while the PV products follow the pointwise warps.
+    constexpr unsigned FULL = 0xffffffffu;
+    constexpr uint32_t idesc_s = idesc_bf16(128, ATT_BN, false, false);
+    constexpr uint32_t idesc_o = idesc_bf16(128, HD, false, true);
+    auto wait_kv = [&](uint32_t gg) {
+      return __all_sync(FULL, mbar_wait(&kv_full[gg % Cfg::NST], (gg / Cfg::NST) & 1u, abort_flag));
+    };
+    auto commit = [&](uint64_t* bar) {
+      if (elect_one()) mma_commit(bar);
+      __syncwarp();
+    };
+    auto arrive1 = [&](uint64_t* bar) {
+      if (lane == 0) mbar_arrive(bar);
+      __syncwarp();
+    };
+    // shared-memory descriptors of Q_A and of ring stage 0's K and V; a byte offset `o` below 2^18
+    // moves a descriptor by adding o >> 4 to its start-address field
+    const uint64_t q_desc0 = sdesc_sw128(smem_u32(q_s), 16, 1024);
+    const uint64_t k_desc0 = sdesc_sw128(smem_u32(kv_s), 16, 1024);
+    const uint64_t v_desc0 = sdesc_sw128(smem_u32(kv_s + Cfg::KV_TILE), Cfg::BOX, 1024);
+    uint32_t g = 0;
+    bool ok = true;
+    for (uint32_t k = 0; ok; k++) {
       int64_t item = -1;
       if (prm.dynamic) {
         if (lane == 0) item = read_item(k, item_full, item_empty, item_ring, abort_flag);
-        item = __shfl_sync(0xffffffffu, item, 0);
+        item = __shfl_sync(FULL, item, 0);
+      } else {
+        item = static_item(k, sch, n_items);
+      }
+      if (item < 0) break;
+      const ItemGeom ig = item_geom<CAND>(item, sch);
+      const int m = ig.m, nk = ig.nk;
+      const bool has_b = ig.has_b;
+      // query tile x's last key tile (the diagonal one, or the history's last); a candidate item
+      // without history has no key tile, and its query tiles take no MMA
+      auto last_of = [&](int x) { return CAND ? nk - 1 : 2 * m + x; };
+      auto mine_of = [&](int x) { return (x == 0 || has_b) && nk > 0; };
+      if (warp == 1) {
+        // ---------------------------------------------------------- S products, slot order
+        if (!__all_sync(FULL, mbar_wait(q_full, k & 1u, abort_flag))) break;
+        for (int x = 0; x < 2; x++)
+          if (!mine_of(x)) arrive1(q_empty);      // Q of this item was loaded; nothing to read
+        for (int j = 0; j < nk && ok; j++) {
+          const uint32_t gj = g + j;
+          if (!wait_kv(gj)) { ok = false; break; }
+          const uint64_t kd = k_desc0 + (uint64_t)(((gj % Cfg::NST) * Cfg::STAGE_BYTES) >> 4);
+          for (int x = 0; x < 2; x++) {
+            const uint32_t sl = 2 * gj + x, b = sl % Cfg::NSB;
+            if (sl >= Cfg::NSB) {   // the buffer's previous slot (query tile xp, key tile gp) is done
+              const uint32_t pl = sl - Cfg::NSB, xp = pl & 1u, gp = pl >> 1;
+              const uint32_t use = Cfg::NSB == 3 ? gp / 3 : gp;
+              if (!__all_sync(FULL, mbar_wait(&buf_free[2 * b + xp], use & 1u, abort_flag))) {
+                ok = false;
+                break;
+              }
+            }
+            if (mine_of(x) && j <= last_of(x)) {
+              tc_fence_after();
+              const uint64_t qd = q_desc0 + (uint64_t)((x * Cfg::Q_BYTES) >> 4);
+              if (elect_one()) {
+#pragma unroll
+                for (int kk = 0; kk < HD / 16; kk++) {
+                  const uint64_t off = (uint64_t)((kk / 4) * Cfg::BOX + (kk % 4) * 32) >> 4;
+                  mma_ss(tmem + b * 128, qd + off, kd + off, idesc_s, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&s_full[2 * b + x]);
+              }
+              __syncwarp();
+              if (j == last_of(x)) commit(q_empty);
+            } else {
+              arrive1(&buf_free[2 * b + x]);      // the slot passes through unused
+            }
+          }
+        }
+      } else {
+        // ---------------------------------------------------------- PV products of query tile x
+        const int x = warp - 2;
+        const int last = last_of(x);
+        const bool mine = mine_of(x);
+        const uint32_t o_tmem = tmem + Cfg::O_COL + x * Cfg::O_STRIDE;
+        for (int j = 0; j < nk && ok; j++) {
+          const uint32_t gj = g + j;
+          if (mine && j <= last) {
+            if (!__all_sync(FULL, mbar_wait(&p_full[2 * x + (pv_count & 1u)], (pv_count >> 1) & 1u,
+                                            abort_flag))) {
+              ok = false;
+              break;
+            }
+            pv_count++;
+            if (j == 0 &&
+                !__all_sync(FULL, mbar_wait(&o_empty[x], (o_count & 1u) ^ 1u, abort_flag))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            // O_x (+)= P V of key tile gj: P of keys 16kk .. 16kk+15 sits in 8 columns of the
+            // slot's S buffer, keys 0..63 at columns 0..31 and keys 64..127 at columns 64..95
+            const uint32_t b = (2 * gj + x) % Cfg::NSB;
+            const uint64_t vd = v_desc0 + (uint64_t)(((gj % Cfg::NST) * Cfg::STAGE_BYTES) >> 4);
+            if (elect_one()) {
+#pragma unroll
+              for (int kk = 0; kk < ATT_BN / 16; kk++)
+                mma_ts(o_tmem, tmem + b * 128 + (kk & 3) * 8 + (kk >> 2) * 64,
+                       vd + (uint64_t)((kk * 2048) >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+              mma_commit(&buf_free[2 * b + x]);
+              if (j == last) mma_commit(&o_full[x]);
+              mma_commit(&kv_empty[gj % Cfg::NST]);
+            }
+            __syncwarp();
+          } else {
+            // a key tile this query tile does not read: release it once it is filled
+            if (!wait_kv(gj)) { ok = false; break; }
+            arrive1(&kv_empty[gj % Cfg::NST]);
+          }
+        }
+        if (mine) o_count++;
+      }
+      if (!ok) break;
+      g += nk;
+    }
+    commit(&drain[warp - 1]);
+    if (lane == 0) mbar_drain(&drain[warp - 1], 0);
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ pointwise warps
+    const int x = (warp - 4) >> 3;        // 0: query tile A, 1: query tile B
+    const int half = (warp >> 2) & 1;     // key columns [64 half, 64 half + 64) of each S tile
+    const int q = warp & 3;               // TMEM lane quadrant
+    const int tid = threadIdx.x - 128;    // 0..511 over the pointwise warps
+    const int r = q * 32 + lane;          // query row inside the tile
+    const int col0 = half * 64;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    constexpr int M = Cfg::POS_CAP - 1;   // tab_s[M - d] holds the halved bias at distance d
+    constexpr unsigned FULL = 0xffffffffu;
+    const bool has_pos = BIAS == BIAS_RAB && prm.pos != nullptr;
+    const int P = prm.P, Tb = prm.Tb;
+    uint32_t g = 0, kx = 0, pw_cnt = 0, tcount = 0;   // tcount: tiles this warp computed
+    uint32_t s_uses[Cfg::NSB];                        // computed slots per S buffer
+    for (int b = 0; b < Cfg::NSB; b++) s_uses[b] = 0;
+    int staged_head = -1, staged_n = 0;  // what tab_s / htt_s hold
+    // once: the tables' zero padding (masked distances) and the 0/1 step pairs
+    for (int e = tid; e < 129; e += ATT_PW) {
+      if (e < 128) tab_s[M + 1 + e] = 0.0f;
+      if (Cfg::PAIRED) tab2_s[M + e] = 0.0f;
+    }
+    for (int e = tid; e < 64; e += ATT_PW)
+      step_s[e] = make_float2(e >= 32 ? 1.0f : 0.0f, e >= 31 ? 1.0f : 0.0f);
+    bool run = group_sync(pw_bar, pw_cnt, abort_flag);
+    for (uint32_t k = 0; run; k++) {
+      int64_t item = -1;
+      if (prm.dynamic) {
+        if (lane == 0) item = read_item(k, item_full, item_empty, item_ring, abort_flag);
+        item = __shfl_sync(FULL, item, 0);
       } else {
         item = static_item(k, sch, n_items);
       }
@@ -861,15 +955,20 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
       const bool has_b = ig.has_b;
       const float* pos_h = has_pos ? prm.pos + (int64_t)h * P : nullptr;
       const float* tim_h = has_time ? prm.tim + (int64_t)h * Tb : nullptr;
-      // stage the halved bias tables of this head: the first 128*nk position buckets suffice, or
-      // n_hist + 1 for candidates (distances 0 .. n_hist)
+      const float half_slope = BIAS == BIAS_ALIBI ? 0.5f * prm.alibi[h] : 0.0f;
+      // stage this head's halved position (or ALiBi) bias for the distances the item reaches:
+      // 128*nk, or n_hist + 1 for candidates (distances 0 .. n_hist)
       const int need = CAND ? (int)(n + 1 < Cfg::POS_CAP ? n + 1 : Cfg::POS_CAP)
                             : min(nk * ATT_BN, Cfg::POS_CAP);
-      if (BIAS == BIAS_RAB && (h != staged_head || need > staged_n)) {
+      if (BIAS != BIAS_NONE && (h != staged_head || need > staged_n)) {
         if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;   // earlier items are done reading
-        // hpos_s[d] = pos[h][min(d, P-1)] / 2 for every distance d < need (zeros without a table)
-        for (int e = tid; e < need; e += ATT_PW)
-          hpos_s[e] = has_pos ? 0.5f * __ldg(pos_h + (e < P - 1 ? e : P - 1)) : 0.0f;
+        for (int d = tid; d < need; d += ATT_PW) {
+          const float v = BIAS == BIAS_ALIBI
+                              ? -half_slope * (float)d
+                              : (has_pos ? 0.5f * __ldg(pos_h + (d < P - 1 ? d : P - 1)) : 0.0f);
+          tab_s[M - d] = v;
+          if (Cfg::PAIRED && d < M) tab2_s[M - 1 - d] = v;
+        }
         if (has_time) {
           for (int e = tid; e < Tb && e < ATT_TB_CAP; e += ATT_PW) htt_s[e] = 0.5f * __ldg(tim_h + e);
           if (tid < 32) hclz_s[tid] = 0.5f * __ldg(tim_h + (31 - tid < Tb - 1 ? 31 - tid : Tb - 1));
@@ -878,7 +977,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         staged_n = need;
         if (!group_sync(pw_bar, pw_cnt, abort_flag)) break;   // tables visible to all
       }
-      const int qt = 2 * m + x;                    // this warpgroup's query tile
+      const int qt = 2 * m + x;                    // this warp's query tile
       if (x == 1 && !has_b) {                      // no B tile in this item
         g += nk;
         continue;
@@ -891,132 +990,140 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         ti = CAND ? prm.cts[ig.qrow0 + (i < ig.nq ? i : ig.nq - 1)] : prm.ts[row0 + (i < n ? i : n - 1)];
       const int64_t ti_rel = has_time && n > 0 ? ti - prm.ts[row0] : 0;
       const bool row_rel32 = ti_rel > -(1LL << 30) && ti_rel < (1LL << 30);
-      const int ti1 = (int)ti_rel + 1;
-      const float half_slope = BIAS == BIAS_ALIBI ? 0.5f * prm.alibi[h] : 0.0f;
+      ExactArgs ea;
+      ea.P = P;
+      ea.Tb = Tb;
+      ea.ti = ti;
+      ea.ti1 = (int)ti_rel + 1;
+      ea.dmin = CAND ? 1 : 0;
+      ea.tab0 = tab_s + M;
+      ea.htt = htt_s;
+      ea.hclz = hclz_s;
+      ea.pos_h = pos_h;
+      ea.tim_h = tim_h;
+      ea.half_slope = half_slope;
+      // the warp's largest distance in tile j is (this query tile's last row) - key0
+      const int dmax0 = CAND ? ipos : q0 + ATT_BM - 1;
       bool ok = true;
       const int last = CAND ? nk - 1 : qt;
+      // tiles that need the per-element mask: the diagonal one, or the history's last when it is
+      // partial; the fast path also needs every distance of the tile staged
+      auto is_diag = [&](int jj) {
+        return CAND ? (jj == nk - 1 && (n % ATT_BN) != 0) : (jj == qt);
+      };
+      auto fast_in = [&](int jj) {
+        return !is_diag(jj) && (BIAS == BIAS_NONE || dmax0 - jj * ATT_BN < staged_n);
+      };
+      auto setup = [&](int jj, uint32_t stj) {
+        return time_setup<CAND>(fast_in(jj), flag_ring[stj], row_rel32, ea.ti1, ti,
+                                ts32_ring + stj * ATT_BN + col0, ts_ring + stj * ATT_BN + col0,
+                                htt_s, tim_h, Tb);
+      };
+      TimeSetup nxt;
+      bool have_nxt = false;
       for (int j = 0; j <= last; j++) {
         const uint32_t gj = g + j;
+        const uint32_t st = gj % Cfg::NST;
         const int key0 = j * ATT_BN;
-        // tiles that need the per-element mask: the diagonal one, or the history's last when it
-        // is partial
-        const bool diag = CAND ? (j == nk - 1 && (n % ATT_BN) != 0) : (j == qt);
-        const int64_t* tsk = ts_ring + (gj % Cfg::NST) * ATT_BN;
-        const int* tsk32 = ts32_ring + (gj % Cfg::NST) * ATT_BN;
-        bool rel32 = false;
-        // ---- per-tile bias set-up (overlaps the tensor core's work on S)
-        bool split = false;
-        float hb0 = 0.0f, hb1 = 0.0f;
-        int cstar = ATT_BN;
-        bool time_fast = true;
+        const bool diag = is_diag(j);
+        const bool far = BIAS == BIAS_RAB && dmax0 - key0 >= staged_n;
+        const int64_t* tsk = ts_ring + st * ATT_BN + col0;
+        const int* tsk32 = ts32_ring + st * ATT_BN + col0;
+        // ---- per-tile bias set-up (computed during the previous tile when it could be)
+        TimeSetup ts;
         if (has_time) {
-          // the tile's timestamps arrived with its K/V stage
-          if (!mbar_wait(&kv_full[gj % Cfg::NST], (gj / Cfg::NST) & 1u, abort_flag)) { ok = false; break; }
-          const int flags = flag_ring[gj % Cfg::NST];
-          const bool sorted = (flags & KEYS_SORTED) != 0;
-          rel32 = __all_sync(0xffffffffu, (flags & KEYS_REL32) && row_rel32);
-          int bf, bl;
-          if (rel32) {
-            bf = 31 - __clz(max(ti1 - tsk32[0], 1));
-            bl = 31 - __clz(max(ti1 - tsk32[ATT_BN - 1], 1));
+          if (have_nxt) {
+            ts = nxt;
           } else {
-            bf = time_bucket(ti, tsk[0]);
-            bl = time_bucket(ti, tsk[ATT_BN - 1]);
+            // the tile's timestamps arrived with its K/V stage
+            if (!mbar_wait(&kv_full[st], (gj / Cfg::NST) & 1u, abort_flag)) { ok = false; break; }
+            ts = setup(j, st);
           }
-          time_fast = __all_sync(0xffffffffu, sorted && bf - bl <= 1 && bf < 62);
-          if (time_fast) {
-            if (bf != bl) {
-              // the keys are sorted, so the bucket steps down once: find the first key in the lower one
-              int lo = 1, hi = ATT_BN - 1;
-              if (rel32) {
-                const int thr = ti1 - (1 << bf);
-                while (lo < hi) {
-                  const int mid = (lo + hi) >> 1;
-                  if (tsk32[mid] > thr) hi = mid; else lo = mid + 1;
+        } else {
+          ts.fast = fast_in(j);
+          ts.split = ts.rel32 = false;
+          ts.cst = 64;
+          ts.hb0 = ts.hb1 = 0.0f;
+        }
+        have_nxt = false;
+        const int tmode = has_time ? (ts.rel32 ? 2 : 1) : 0;
+        // this slot's S buffer (see the MMA issuer); P goes over the columns already read
+        const uint32_t sb = (2 * gj + x) % Cfg::NSB;
+        const uint32_t s_col = t_lane + sb * 128 + col0;
+        uint32_t use = s_uses[0];
+#pragma unroll
+        for (int b = 1; b < Cfg::NSB; b++) use = sb == (uint32_t)b ? s_uses[b] : use;
+#pragma unroll
+        for (int b = 0; b < Cfg::NSB; b++) s_uses[b] += sb == (uint32_t)b ? 1u : 0u;
+        if (!mbar_wait(&s_full[2 * sb + x], use & 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 2; c++) {
+          uint32_t sv[32], pk[16];
+          tmem_ld32_sync(s_col + 32 * c, sv);
+          const int dist0 = ipos - key0 - col0 - 32 * c;   // this row's distance to the chunk's key 0
+          int mode = ts.fast ? CH_FAST : CH_EXACT;
+          if (diag) {
+            const int idx = (col0 >> 5) + c;   // causal: chunks right of the warp's rows are masked
+            mode = CAND ? CH_EXACT_MASK : (idx > q ? CH_ZERO : (idx == q ? CH_EXACT_MASK : CH_EXACT));
+          }
+          if (mode == CH_FAST) {
+            if (BIAS == BIAS_NONE) {
+              nobias_chunk(sv, pk);
+            } else {
+              const int y0 = M - dist0;
+              const float* tb = (Cfg::PAIRED && (y0 & 1)) ? tab2_s + (y0 - 1) : tab_s + y0;
+              if (BIAS == BIAS_RAB && has_time) {
+                const uint64_t hb0x2 = f2_pack(ts.hb0, ts.hb0);
+                if (ts.split) {
+                  int cc = ts.cst - 32 * c;
+                  cc = cc < 0 ? 0 : (cc > 32 ? 32 : cc);
+                  const float dh = ts.hb1 - ts.hb0;
+                  fast_chunk<Cfg::PAIRED, true, true>(sv, tb, hb0x2, f2_pack(dh, dh),
+                                                      step_s + (32 - cc), pk);
+                } else {
+                  fast_chunk<Cfg::PAIRED, true, false>(sv, tb, hb0x2, 0ull, nullptr, pk);
                 }
               } else {
-                const int64_t thr = ti + 1 - (1LL << bf);
-                while (lo < hi) {
-                  const int mid = (lo + hi) >> 1;
-                  if (tsk[mid] > thr) hi = mid; else lo = mid + 1;
-                }
+                fast_chunk<Cfg::PAIRED, false, false>(sv, tb, 0ull, 0ull, nullptr, pk);
               }
-              cstar = lo;
             }
-            split = __any_sync(0xffffffffu, bf != bl);
-            const int b0 = bf < Tb - 1 ? bf : Tb - 1, b1 = bl < Tb - 1 ? bl : Tb - 1;
-            hb0 = b0 < ATT_TB_CAP ? htt_s[b0] : 0.5f * __ldg(tim_h + b0);
-            hb1 = b1 < ATT_TB_CAP ? htt_s[b1] : 0.5f * __ldg(tim_h + b1);
-          }
-        }
-        int mode = TILE_GENERAL;
-        if (!diag && time_fast) {
-          if (BIAS == BIAS_ALIBI) {
-            mode = TILE_FAST;
-            hb0 = -half_slope * (float)(ipos - key0);
-          } else if (BIAS == BIAS_NONE) {
-            mode = TILE_FAST;
-          } else if ((CAND ? ipos : q0 + ATT_BM - 1) - key0 < staged_n) {  // all distances staged
-            mode = TILE_FAST;
-          }
-        }
-        if (mode == TILE_GENERAL && has_time && rel32) mode = TILE_GEN32;
-        TileArgs ta;
-        ta.i = ipos;
-        ta.dmin = CAND ? 1 : 0;
-        ta.key0 = key0;
-        ta.P = P;
-        ta.Tb = Tb;
-        ta.staged_n = staged_n;
-        ta.cstar = cstar;
-        ta.ti = ti;
-        ta.ti1 = ti1;
-        ta.tsk = tsk;
-        ta.tsk32 = tsk32;
-        ta.hclz = hclz_s;
-        ta.hpos = hpos_s;
-        ta.htt = htt_s;
-        ta.pos_h = pos_h;
-        ta.tim_h = tim_h;
-        ta.hb0 = hb0;
-        ta.hb1 = hb1;
-        ta.half_slope = half_slope;
-        if (!mbar_wait(&s_full[x], gx & 1u, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        if (Cfg::SEP_P) {
-          bool pf_ok = true;
-          auto wait_pf = [&]() {
-            if (gx > 0 && !mbar_wait(&p_free[x], (gx - 1) & 1u, abort_flag)) pf_ok = false;
-            tc_fence_after();
-          };
-          auto consumed = [&]() {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&s_free[x]);
-          };
-          const uint32_t p_col = t_lane + Cfg::P_COL + x * 64 + half * 32;
-          if (mode == TILE_FAST) {
-            if (split) pointwise_tile_sep<BIAS, TILE_FAST, true>(s_col, p_col, col0, ta, wait_pf, consumed);
-            else pointwise_tile_sep<BIAS, TILE_FAST, false>(s_col, p_col, col0, ta, wait_pf, consumed);
-          } else if (BIAS == BIAS_RAB && mode == TILE_GEN32) {
-            pointwise_tile_sep<BIAS, TILE_GEN32, false>(s_col, p_col, col0, ta, wait_pf, consumed);
+          } else if (mode == CH_ZERO) {
+#pragma unroll
+            for (int e = 0; e < 16; e++) pk[e] = 0u;
           } else {
-            pointwise_tile_sep<BIAS, TILE_GENERAL, false>(s_col, p_col, col0, ta, wait_pf, consumed);
+            ea.tsk = tsk + 32 * c;
+            ea.tsk32 = tsk32 + 32 * c;
+            if (mode == CH_EXACT_MASK) {   // diagonal distances are all staged
+              if (tmode == 2) exact_chunk<BIAS, true, 2, false>(sv, dist0, staged_n, ea, pk);
+              else if (tmode == 1) exact_chunk<BIAS, true, 1, false>(sv, dist0, staged_n, ea, pk);
+              else exact_chunk<BIAS, true, 0, false>(sv, dist0, staged_n, ea, pk);
+            } else if (far) {
+              if (tmode == 2) exact_chunk<BIAS, false, 2, true>(sv, dist0, staged_n, ea, pk);
+              else if (tmode == 1) exact_chunk<BIAS, false, 1, true>(sv, dist0, staged_n, ea, pk);
+              else exact_chunk<BIAS, false, 0, true>(sv, dist0, staged_n, ea, pk);
+            } else {
+              if (tmode == 2) exact_chunk<BIAS, false, 2, false>(sv, dist0, staged_n, ea, pk);
+              else if (tmode == 1) exact_chunk<BIAS, false, 1, false>(sv, dist0, staged_n, ea, pk);
+              else exact_chunk<BIAS, false, 0, false>(sv, dist0, staged_n, ea, pk);
+            }
           }
-          if (!pf_ok) { ok = false; break; }
-        } else if (mode == TILE_FAST) {
-          if (split) pointwise_tile<BIAS, TILE_FAST, true>(s_col, col0, ta);
-          else pointwise_tile<BIAS, TILE_FAST, false>(s_col, col0, ta);
-        } else if (BIAS == BIAS_RAB && mode == TILE_GEN32) {
-          pointwise_tile<BIAS, TILE_GEN32, false>(s_col, col0, ta);
-        } else {
-          pointwise_tile<BIAS, TILE_GENERAL, false>(s_col, col0, ta);
+          tmem_st16(s_col + 16 * c, pk);
+        }
+        if (!ok) break;
+        // the next tile's time-bias set-up while the P stores drain (its stage is filled by now,
+        // or soon: it depends only on PV products that were issued before this tile's)
+        if (has_time && j < last) {
+          const uint32_t gn = gj + 1, stn = gn % Cfg::NST;
+          if (!mbar_wait(&kv_full[stn], (gn / Cfg::NST) & 1u, abort_flag)) { ok = false; break; }
+          nxt = setup(j + 1, stn);
+          have_nxt = true;
         }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[x]);
-        gx++;
+        if (lane == 0) mbar_arrive(&p_full[2 * x + (tcount & 1u)]);
+        tcount++;
       }
       if (!ok) break;
       g += nk;
@@ -1049,7 +1156,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         }
         // the staged tables hold half values; distance 0 and time bucket 0
         const float bias0 =
-            BIAS == BIAS_RAB ? 2.0f * (hpos_s[0] + (has_time ? htt_s[0] : 0.0f)) : 0.0f;
+            BIAS == BIAS_RAB ? 2.0f * (tab_s[M] + (has_time ? htt_s[0] : 0.0f)) : 0.0f;
         const float xs = sdot + bias0;
         self_p = prm.scale * __fdividef(xs, 1.0f + __expf(-xs));
         v_self = crow + col_v + h * HD + half * (HD / 2);

@@ -9,6 +9,7 @@
 #include "tc_attention.cuh"
 #include "tc_attention_bwd.cuh"
 #include "tc_gemm.cuh"
+#include "tc_ln_f2.cuh"
 
 namespace hstu {
 namespace tc {
@@ -88,6 +89,41 @@ hstu_status_t launch_gemm_bn(int64_t M, int N, int K, const bf16* A, const bf16*
   kern<<<grid, kGemmThreads, Cfg::SMEM, st>>>(ta, tb, M, N, K, bias, R, C, C32, splits);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+// LayerNorm(AV) * U followed by f2 and the residual, as one kernel (tc_ln_f2.cuh).  Shapes: the
+// LayerNorm width equals d, and d is 128, 256 or 512 (the whole output row in one TMEM accumulator).
+inline bool ln_f2_supported(int64_t M, int d, int64_t wv) {
+  return M > 0 && M < (1LL << 31) && wv == d && (d == 128 || d == 256 || d == 512);
+}
+
+template <int N>
+hstu_status_t launch_ln_f2_n(int64_t M, int n1, const float* av, const bf16* uvqk,
+                             const bf16* ln_w, const bf16* ln_b, float eps, const bf16* W2,
+                             const bf16* b2, const bf16* X, bf16* Y, cudaStream_t st) {
+  using Cfg = LnF2Cfg<N>;
+  CUtensorMap tb;
+  if (!make_map_bf16(&tb, W2, N, N, N, 64, 64)) return HSTU_ERR_CUDA;
+  auto kern = ln_f2_kernel<N, N>;
+  constexpr int smem = Cfg::SMEM + 1024;   // + alignment slack
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return HSTU_ERR_CUDA;
+  const int64_t blocks = (M + Cfg::BM - 1) / Cfg::BM;
+  const int grid = (int)(blocks < num_sms() ? blocks : num_sms());
+  kern<<<grid, LNF2_THREADS, smem, st>>>(tb, M, n1, av, uvqk, ln_w, ln_b, eps, b2, X, Y);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+}
+
+inline hstu_status_t launch_ln_f2(int64_t M, int d, int n1, const float* av, const bf16* uvqk,
+                                  const bf16* ln_w, const bf16* ln_b, float eps, const bf16* W2,
+                                  const bf16* b2, const bf16* X, bf16* Y, cudaStream_t st) {
+  switch (d) {
+    case 128: return launch_ln_f2_n<128>(M, n1, av, uvqk, ln_w, ln_b, eps, W2, b2, X, Y, st);
+    case 256: return launch_ln_f2_n<256>(M, n1, av, uvqk, ln_w, ln_b, eps, W2, b2, X, Y, st);
+    case 512: return launch_ln_f2_n<512>(M, n1, av, uvqk, ln_w, ln_b, eps, W2, b2, X, Y, st);
+  }
+  return HSTU_ERR_UNSUPPORTED;
 }
 
 template <int EPI>

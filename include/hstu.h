@@ -167,6 +167,26 @@ hstu_status_t hstu_f2_fwd(const hstu_shape_t* shape, const void* g, const void* 
                           const void* X, void* out, void* stream);
 
 /*
+ * hstu_ln_f2_fwd -- Eq. 3 and the residual in one kernel: out[T, d] = (LayerNorm(av) * U) W2 + b2 + X,
+ * the result of hstu_ln_gate_fwd followed by hstu_f2_fwd, without G ever reaching global memory
+ * ("Actions Speak Louder than Words" paper notes, section 3.5: the normalisation and the output
+ * projection fused into one operator).  The tensor core's A operand is formed in shared memory
+ * from AV and U; the LayerNorm statistics are computed in fp32 per row as hstu_ln_gate_fwd does,
+ * and G is rounded to bf16 before the product, as in the two-step path.
+ *
+ *  av     [T, H*d_v] fp32     uvqk [T, n1] bf16 (U = block 0)
+ *  ln_w, ln_b [H*d_v] bf16    W2 [H*d_v, d] bf16    b2 [d] bf16 (nullable: zero)
+ *  X      [T, d] bf16         out [T, d] bf16 (may not overlap X, av or uvqk)
+ * Shapes: bf16 with H*d_v == d and d in {128, 256, 512} (the whole output row fits one tensor-
+ * memory accumulator); others return HSTU_ERR_UNSUPPORTED before any launch, and hstu_layer_fwd
+ * then uses the two steps.  All pointers 16-byte aligned device memory, caller-owned; the call is
+ * asynchronous on `stream` and allocates nothing.
+ */
+hstu_status_t hstu_ln_f2_fwd(const hstu_shape_t* shape, const void* av, const void* uvqk,
+                             const void* ln_w, const void* ln_b, const void* W2, const void* b2,
+                             const void* X, void* out, void* stream);
+
+/*
  * hstu_attention_bwd -- backward of Eq. 2 (training): given dAV = dL/dAV, the gradients of the
  * loss with respect to Q, K, V and the rab tables.  With x_ij = q_i . k_j + bias(i, j),
  *   dv_j = sum_{i>=j} scale*SiLU(x_ij) dAV_i,   dx_ij = scale*SiLU'(x_ij) (dAV_i . v_j),
@@ -237,7 +257,7 @@ void hstu_layer_pipeline_destroy(hstu_layer_pipeline_t* p);
  * The activations come from the forward: `fwd_workspace` (fwd_workspace_bytes >=
  * hstu_layer_fwd_workspace_size(shape)) is the workspace that a preceding hstu_layer_fwd call with
  * the same shape, X, offsets, timestamps, weights and tables filled, not written since; its U, V, Q,
- * K, AV and G are read, and X W1 + b1 is recomputed.  bf16 with d_qk = d_v = 64 and
+ * K and AV are read, and X W1 + b1 and G = LayerNorm(AV) * U are recomputed.  bf16 with d_qk = d_v = 64 and
  * H*d_v <= 8192 (else HSTU_ERR_UNSUPPORTED).  Arguments as in hstu_layer_fwd (b2 is not needed),
  * plus
  *  dY             [T, d] bf16, the incoming gradient

@@ -104,3 +104,21 @@ def test_host_validation_rejects_bad_arguments(hstu):
     lib = hstu.library()
     assert lib.hstu_token_embed_fwd(10, 12, None, None, None, 5, None, 5, None, None) == E  # d % 8
     assert lib.hstu_token_embed_fwd(0, 16, None, None, None, 5, None, 5, None, None) == hstu.HSTU_OK
+
+
+def test_ln_f2_host_validation(hstu):
+    # the fused LayerNorm * U -> f2 entry point covers bf16 with H*d_v == d in {128, 256, 512}
+    lib = hstu.library()
+    E, U = hstu.HSTU_ERR_INVALID_ARG, hstu.HSTU_ERR_UNSUPPORTED
+    P = [ctypes.c_void_p(FAKE + 4096 * i) for i in range(8)]
+
+    def call(shape, ptrs=P):
+        return lib.hstu_ln_f2_fwd(ctypes.byref(shape), *ptrs, None)
+
+    assert call(_shape(hstu, d_model=192, num_heads=3)) == U            # d not 128/256/512
+    assert call(_shape(hstu, d_model=256, num_heads=2)) == U            # H*d_v != d
+    assert call(_shape(hstu, dtype=hstu.HSTU_F32, d_qk=32, d_v=32, d_model=64)) == U
+    assert call(_shape(hstu), [None] + P[1:]) == E                      # no AV
+    assert call(_shape(hstu), P[:7] + [ctypes.c_void_p(FAKE + 2)]) == E  # misaligned out
+    assert call(_shape(hstu), P[:7] + [P[6]]) == E                      # out aliases X
+    assert call(_shape(hstu, num_seqs=0, total_tokens=0)) == hstu.HSTU_OK

@@ -179,6 +179,39 @@ def test_ln_gate_kernel(hstu, T, wv):
     assert_bf16_close(host(g), ref, "ln_gate")
 
 
+@pytest.mark.parametrize("T,d", [(1, 128), (300, 128), (129, 256), (1000, 256), (517, 512),
+                                 (4097, 512)])
+def test_ln_f2_fused_kernel(hstu, T, d):
+    # LayerNorm(AV) * U, then f2 and the residual, in one kernel: against the oracle's two steps
+    rng = np.random.default_rng(T + 7 * d)
+    hd = 64
+    H = d // hd
+    n1 = 4 * d
+    av = (rng.standard_normal((T, d)) * 1e-3 + 2e-4).astype(np.float32).astype(np.float64)
+    uvqk = round_bf16(rng.standard_normal((T, n1)))
+    ln_w = round_bf16(rng.uniform(0.5, 1.5, d))
+    ln_b = round_bf16(rng.normal(0, 0.5, d))
+    W2 = round_bf16(rng.uniform(-1, 1, (d, d)) * np.sqrt(3 / d))
+    b2 = round_bf16(rng.normal(0, 0.1, d))
+    X = round_bf16(rng.standard_normal((T, d)))
+    g = oracle.ln_gate(av, uvqk, ln_w, ln_b, num_heads=H, d_qk=hd, d_v=hd)
+    ref = oracle.f2(round_bf16(g), W2, b2, X)   # G is stored as bf16 in both GPU paths
+    s = hstu.make_shape(1, T, T, d, H, hd, hd, hstu.HSTU_BF16)
+    out = torch.full((T, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    hstu.hstu_ln_f2_fwd(s, dev(av, "f32"), dev(uvqk), dev(ln_w), dev(ln_b), dev(W2), dev(b2),
+                        dev(X), out)
+    assert hstu.device_status() == hstu.HSTU_OK
+    got = host(out)
+    assert_bf16_close(got, ref, "ln_f2")
+    assert_layer_part_close(got, ref, X, "ln_f2 without residual")
+    # and the two-step path on the same inputs
+    g_d = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    hstu.hstu_ln_gate_fwd(s, dev(av, "f32"), dev(uvqk), dev(ln_w), dev(ln_b), g_d)
+    two = torch.empty((T, d), dtype=torch.bfloat16, device="cuda")
+    hstu.hstu_f2_fwd(s, g_d, dev(W2), dev(b2), dev(X), two)
+    assert_layer_part_close(got, host(two), X, "ln_f2 vs the two steps")
+
+
 def test_token_embed_bit_exact(hstu):
     rng = np.random.default_rng(5)
     itab = rng.standard_normal((1000, 1024)).astype(np.float32)
