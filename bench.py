@@ -160,6 +160,20 @@ def combine_over_ranks(local_ms: float, local_tokens: int, world: int, device):
 # Our arm
 # ------------------------------------------------------------------------------------------------
 
+def first_sequences(inp, max_tokens: int):
+    """The workload restricted to its first sequences, as many as fit in `max_tokens` tokens (at
+    least one): a smaller case of the same kernels for profiler captures (--max-tokens)."""
+    import dataclasses
+    if max_tokens <= 0 or inp.T <= max_tokens:
+        return inp
+    b = max(1, int(np.searchsorted(inp.seq_offsets[1:], max_tokens, side="right")))
+    T = int(inp.seq_offsets[b])
+    cut = lambda a: None if a is None else a[:T]
+    return dataclasses.replace(inp, lengths=inp.lengths[:b], seq_offsets=inp.seq_offsets[:b + 1],
+                               X=cut(inp.X), timestamps=cut(inp.timestamps),
+                               item_ids=cut(inp.item_ids), action_ids=cut(inp.action_ids))
+
+
 def workload_text(w, max_len):
     bias = ("ALiBi slopes 2^(-8h/H)" if w.alibi
             else f"rab P={w.n_pos_buckets}/Tb={w.n_time_buckets}")
@@ -201,7 +215,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = workloads.WORKLOADS[args.workload]
-    inp = workloads.make_inputs(w)
+    inp = first_sequences(workloads.make_inputs(w), args.max_tokens)
     H, hd, d = w.num_heads, w.head_dim, w.d_model
     T = inp.T
     D = to_device(inp, dev)
@@ -342,6 +356,8 @@ def run_ours(args, rank, world, local_rank):
     }
     if nl > 1:
         result["config"]["layers_per_step"] = nl
+    if args.max_tokens > 0:
+        result["config"]["sequences"] = f"the first {len(inp.lengths)} (--max-tokens {args.max_tokens})"
     return result
 
 
@@ -1022,6 +1038,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long_seq", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--max-tokens", type=int, default=0,
+                    help="only the workload's first sequences, up to this many tokens (profiler "
+                         "captures of a smaller case); the bench line then names the cut")
     ap.add_argument("--backward", action="store_true",
                     help="time the attention backward instead")
     ap.add_argument("--train", action="store_true",

@@ -261,6 +261,18 @@ __device__ __forceinline__ float tanh_approx(float x) {
   return y;
 }
 
+// Per-warpgroup register budgets: the warpgroup (four consecutive warps, all of them executing)
+// gives up registers down to, or takes them up to, N per thread.  The block's total stays within
+// what it was launched with: the caller keeps sum(threads x N) <= threads x launch registers.
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // One lane of the (fully active) warp is elected, the same one every time: the lowest.
 __device__ __forceinline__ bool elect_one() {
   uint32_t e;

@@ -66,6 +66,8 @@ constexpr int ATT_THREADS = 640;  // producer, 3 MMA issuers, 4 pointwise warpgr
 constexpr int ATT_PW = 512;       // pointwise threads
 constexpr int ATT_PW_WARPS = 8;   // pointwise warps per query tile
 constexpr int ATT_ITEM_RING = 4;  // work items handed from the producer to the other roles
+constexpr int ATT_REGS_SERVICE = 64;  // hd = 64: registers per thread of warpgroup 0 (producer, MMA issuers)
+constexpr int ATT_REGS_PW = 104;      // hd = 64: registers per thread of the pointwise warpgroups
 constexpr int ATT_ITEM_READERS = 3 + 2 * ATT_PW_WARPS;  // MMA issuers and pointwise warps
 
 template <int HD>
@@ -691,6 +693,14 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // registers at hd = 64: the producer and the MMA issuers (warpgroup 0) need few, the pointwise
+  // warps many; launched with 96 per thread (640 x 96 = 61440): 128 x 64 + 512 x 104 = 61440 fits.
+  // (At hd = 128 warpgroup 0 itself needs more than 64, and the even split stays.)
+  static_assert(128 * ATT_REGS_SERVICE + ATT_PW * ATT_REGS_PW <= ATT_THREADS * 96, "register split");
+  if (HD == 64) {
+    if (warp < 4) regs_dec<ATT_REGS_SERVICE>();
+    else regs_inc<ATT_REGS_PW>();
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer warp
@@ -990,18 +1000,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         ti = CAND ? prm.cts[ig.qrow0 + (i < ig.nq ? i : ig.nq - 1)] : prm.ts[row0 + (i < n ? i : n - 1)];
       const int64_t ti_rel = has_time && n > 0 ? ti - prm.ts[row0] : 0;
       const bool row_rel32 = ti_rel > -(1LL << 30) && ti_rel < (1LL << 30);
-      ExactArgs ea;
-      ea.P = P;
-      ea.Tb = Tb;
-      ea.ti = ti;
-      ea.ti1 = (int)ti_rel + 1;
-      ea.dmin = CAND ? 1 : 0;
-      ea.tab0 = tab_s + M;
-      ea.htt = htt_s;
-      ea.hclz = hclz_s;
-      ea.pos_h = pos_h;
-      ea.tim_h = tim_h;
-      ea.half_slope = half_slope;
+      const int ti1 = (int)ti_rel + 1;
       // the warp's largest distance in tile j is (this query tile's last row) - key0
       const int dmax0 = CAND ? ipos : q0 + ATT_BM - 1;
       bool ok = true;
@@ -1015,7 +1014,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         return !is_diag(jj) && (BIAS == BIAS_NONE || dmax0 - jj * ATT_BN < staged_n);
       };
       auto setup = [&](int jj, uint32_t stj) {
-        return time_setup<CAND>(fast_in(jj), flag_ring[stj], row_rel32, ea.ti1, ti,
+        return time_setup<CAND>(fast_in(jj), flag_ring[stj], row_rel32, ti1, ti,
                                 ts32_ring + stj * ATT_BN + col0, ts_ring + stj * ATT_BN + col0,
                                 htt_s, tim_h, Tb);
       };
@@ -1092,6 +1091,19 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
 #pragma unroll
             for (int e = 0; e < 16; e++) pk[e] = 0u;
           } else {
+            // the exact path's arguments, formed here rather than kept live across the tile loop
+            ExactArgs ea;
+            ea.P = P;
+            ea.Tb = Tb;
+            ea.ti = ti;
+            ea.ti1 = ti1;
+            ea.dmin = CAND ? 1 : 0;
+            ea.tab0 = tab_s + M;
+            ea.htt = htt_s;
+            ea.hclz = hclz_s;
+            ea.pos_h = has_pos ? prm.pos + (int64_t)h * P : nullptr;
+            ea.tim_h = has_time ? prm.tim + (int64_t)h * Tb : nullptr;
+            ea.half_slope = half_slope;
             ea.tsk = tsk + 32 * c;
             ea.tsk32 = tsk32 + 32 * c;
             if (mode == CH_EXACT_MASK) {   // diagonal distances are all staged
