@@ -174,9 +174,13 @@ def first_sequences(inp, max_tokens: int):
                                item_ids=cut(inp.item_ids), action_ids=cut(inp.action_ids))
 
 
-def workload_text(w, max_len):
-    bias = ("ALiBi slopes 2^(-8h/H)" if w.alibi
+def bias_text(w):
+    return ("ALiBi slopes 2^(-8h/H)" if w.alibi
             else f"rab P={w.n_pos_buckets}/Tb={w.n_time_buckets}")
+
+
+def workload_text(w, max_len):
+    bias = bias_text(w)
     tokens = ", X = item + action embeddings" if w.token_embed else ""
     layers = f"{w.num_layers} layers" if w.num_layers > 1 else "1 layer"
     return (f"{w.name}: B={w.num_seqs} jagged (max n={max_len}), d={w.d_model}, "
@@ -663,11 +667,13 @@ def run_backward(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = workloads.WORKLOADS[args.workload]
-    if w.head_dim != 64 or w.token_embed:
-        raise SystemExit("the attention backward is implemented for head dim 64 (long_seq, retrieval)")
-    inp = workloads.make_inputs(w)
+    if w.head_dim not in (64, 128) or w.dtype != "bf16":
+        raise SystemExit("the attention backward is implemented for bf16, head dims 64 and 128")
+    inp = first_sequences(workloads.make_inputs(w), args.max_tokens)
     H, hd, d, T = w.num_heads, w.head_dim, w.d_model, inp.T
     D = to_device(inp, dev)
+    if w.token_embed:
+        D["X"], _ = assemble_tokens(hstu, torch, inp, dev, torch.cuda.current_stream(), reps=1)
     L = D["layers"][0]
     shape = hstu.shape_for(D["X"], D["off"], H, hd, hd, int(inp.lengths.max()), D["pos"], D["tim"],
                            inp.ln_eps)
@@ -721,7 +727,7 @@ def run_backward(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded inputs of the workload, N(0,1) incoming gradient)",
         "config": {"workload": f"{w.name}: B={len(inp.lengths)}, n={int(inp.lengths.max())}, "
-                               f"H={H}x{hd}, rab P={w.n_pos_buckets}/Tb={w.n_time_buckets}",
+                               f"H={H}x{hd}, {bias_text(w)}",
                    "l2": "flushed between timed steps (outside the events)"},
         "roofline": {"bound": "tensor", "kernel": "attention_bwd", "achieved": round(tf, 2),
                      "peak": tpk, "unit": "TFLOP/s", "frac": round(tf / tpk, 4),
@@ -749,12 +755,14 @@ def run_train(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     w = workloads.WORKLOADS[args.workload]
-    if w.head_dim != 64 or w.token_embed or w.dtype != "bf16":
-        raise SystemExit("the layer backward is implemented for bf16, head dim 64 (long_seq, retrieval)")
-    inp = workloads.make_inputs(w)
+    if w.head_dim not in (64, 128) or w.dtype != "bf16":
+        raise SystemExit("the layer backward is implemented for bf16, head dims 64 and 128")
+    inp = first_sequences(workloads.make_inputs(w), args.max_tokens)
     H, hd, d, T = w.num_heads, w.head_dim, w.d_model, inp.T
     n1, wv = 4 * H * hd, H * hd
     D = to_device(inp, dev)
+    if w.token_embed:
+        D["X"], _ = assemble_tokens(hstu, torch, inp, dev, torch.cuda.current_stream(), reps=1)
     L = D["layers"][0]
     max_len = int(inp.lengths.max())
     shape = hstu.shape_for(D["X"], D["off"], H, hd, hd, max_len, D["pos"], D["tim"], inp.ln_eps)
@@ -832,7 +840,7 @@ def run_train(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded inputs and parameters of the workload, N(0,1) incoming gradient)",
         "config": {"workload": f"{w.name}: B={len(inp.lengths)}, n={max_len}, d={d}, "
-                               f"H={H}x{hd}, rab P={w.n_pos_buckets}/Tb={w.n_time_buckets}",
+                               f"H={H}x{hd}, {bias_text(w)}",
                    "l2": "flushed between timed steps (outside the events)",
                    "step_tflops": round(step_fl / ms / 1e9, 2)},
         "roofline": {"bound": "tensor", "kernel": "attention_bwd", "achieved": round(a_tf, 2),

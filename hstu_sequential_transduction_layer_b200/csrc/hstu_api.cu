@@ -352,7 +352,8 @@ hstu_status_t check_attention_bwd(const hstu_shape_t* shape, const int64_t* ts, 
   hstu_status_t rc = check_shape(shape);
   if (rc != HSTU_OK) return rc;
   const hstu_shape_t& s = *shape;
-  if (s.dtype != HSTU_BF16 || s.d_qk != 64 || s.d_v != 64) return HSTU_ERR_UNSUPPORTED;
+  if (s.dtype != HSTU_BF16 || s.d_qk != s.d_v || (s.d_qk != 64 && s.d_qk != 128))
+    return HSTU_ERR_UNSUPPORTED;
   if (s.num_seqs * (int64_t)s.num_heads >= (1LL << 31)) return HSTU_ERR_UNSUPPORTED;
   if ((rc = check_bias(shape, ts, pos, tim, alibi, scale)) != HSTU_OK) return rc;
   if ((pos && !dpos) || (tim && !dtime)) return HSTU_ERR_INVALID_ARG;
@@ -365,8 +366,8 @@ hstu_status_t zero_f32(float* p, int64_t n, cudaStream_t st) {
   return launch_status();
 }
 
-// The attention backward once its arguments are checked: zero what the kernel accumulates into
-// (dQ and the tables' gradients), check the offsets, run the kernel.
+// The attention backward once its arguments are checked: zero what the kernels accumulate into
+// (the tables' gradients, and dQ unless it goes to dUVQK), check the offsets, run the kernels.
 hstu_status_t run_attention_bwd(const hstu_shape_t& s, const void* uvqk, const int64_t* off,
                                 const int64_t* ts, const float* pos, const float* tim,
                                 const float* alibi, float scale, const void* dav, float* dq,
@@ -378,10 +379,10 @@ hstu_status_t run_attention_bwd(const hstu_shape_t& s, const void* uvqk, const i
   if (tim && (rc = zero_f32(dtime, (int64_t)s.num_heads * s.n_time_buckets, st)) != HSTU_OK)
     return rc;
   if (T == 0) return HSTU_OK;
-  if ((rc = zero_f32(dq, T * wv_of(s), st)) != HSTU_OK) return rc;
+  if (!(duvqk && s.d_qk == 128) && (rc = zero_f32(dq, T * wv_of(s), st)) != HSTU_OK) return rc;
   check_offsets_kernel<<<(unsigned)((B + 1 + 255) / 256), 256, 0, st>>>(off, B, T);
   if (launch_status() != HSTU_OK) return HSTU_ERR_CUDA;
-  return tc::launch_attention_bwd(T, B, s.num_heads, s.max_seq_len, (const bf16*)uvqk, off, ts, pos,
+  return tc::launch_attention_bwd(T, B, s.num_heads, s.d_qk, s.max_seq_len, (const bf16*)uvqk, off, ts, pos,
                                   s.n_pos_buckets, tim, s.n_time_buckets, alibi, scale,
                                   (const bf16*)dav, dq, dk, dv, dpos, dtime, ws, ws_bytes, st,
                                   (bf16*)duvqk);
@@ -885,8 +886,9 @@ hstu_status_t hstu_layer_bwd(const hstu_shape_t* shape, const void* X, const int
                               alibi_slopes, scale, w.dav, dq, dk, dv, dpos_table, dtime_table,
                               w.attn, w.attn_bytes, st, w.duvqk)) != HSTU_OK)
     return rc;
-  {
-    // dV and dK went to dUVQK as bf16 from the kernel; dQ (reduced in fp32) joins them
+  if (s.d_qk == 64) {
+    // dV and dK went to dUVQK as bf16 from the kernel; dQ (reduced in fp32) joins them (at head
+    // dim 128 the dQ kernel wrote it there)
     const int64_t threads = T * (wv / 4);
     bwd::pack_rows_bf16_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(
         T, (int)wv, n1, dq, (bf16*)w.duvqk + 2 * wv);

@@ -1,5 +1,5 @@
 // Backward of the jagged causal pointwise-SiLU attention (Eq. 2 of "Actions Speak Louder than
-// Words" paper notes, section 3.1; training) on tcgen05 tensor cores, head dim 64:
+// Words" paper notes, section 3.1; training) on tcgen05 tensor cores, head dims 64 and 128:
 //
 //   x_ij = q_i . k_j + bias(i, j),  a_ij = scale * SiLU(x_ij)          (j <= i, same sequence)
 //   dV_j = sum_i a_ij dAV_i,   dx_ij = scale * SiLU'(x_ij) (dAV_i . v_j)
@@ -31,8 +31,12 @@
 // per TMEM lane quadrant; column group cg takes queries 16 cg .. 16 cg + 15 of each half, so that
 // 96 registers per thread suffice).
 // TMEM: S^T [0,128) | dP^T [128,256) (each: half A in the first 64 columns, half B in the next) |
-// dV [256,320) | dK [320,384) | dQ partial [384,448); P^T and dS^T (bf16) overwrite the S^T / dP^T
-// columns each warp has read (a warp's 16 queries pack into the first 8 of its 16 columns).
+// dV [256,256+hd) | dK [256+hd,256+2hd) | at hd = 64 the dQ partial [384,448); P^T and dS^T (bf16)
+// overwrite the S^T / dP^T columns each warp has read (a warp's 16 queries pack into the first 8
+// of its 16 columns).  At head dim 128 dV and dK fill the rest of TMEM and the tiles take 192 KB of
+// shared memory, so this kernel forms dK, dV and the table gradients only (no dS^T panels, no dQ
+// staging, warp 2 idle) and attention_bwd_dq_kernel forms dQ query-stationary, on the same
+// schedule.
 #pragma once
 
 #include <type_traits>
@@ -50,16 +54,21 @@ constexpr int BWD_PW_WARPS = 16;
 constexpr int BWD_TB_USED = 64;
 constexpr int BWD_TT_ALL = 2048;
 
+template <int HD>
 struct BwdCfg {
+  // head dim 64: the dQ partials are formed here too; head dim 128: TMEM holds only S^T, dP^T, dV
+  // and dK, and dQ comes from the query-stationary kernel
+  static constexpr bool DQ = HD == 64;
   static constexpr int BOX = 128 * 64 * 2;                  // 128 rows x 64 bf16
+  static constexpr int TILE = HD / 64 * BOX;                // 128 rows x HD bf16
   static constexpr int NST = 2;                             // query-tile ring depth
   static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = OFF_K + BOX;
-  static constexpr int OFF_Q = OFF_V + BOX;                 // [NST] Q tiles
-  static constexpr int OFF_DO = OFF_Q + NST * BOX;          // [NST] dAV tiles
-  static constexpr int OFF_DS = OFF_DO + NST * BOX;         // [2] dS^T, two 16 KB panels (MN-major A)
-  static constexpr int OFF_STG = OFF_DS + 4 * BOX;          // dQ partial, fp32, 2 swizzled boxes
-  static constexpr int STG_BYTES = 128 * 64 * 4;            // of 32 columns x 128 rows
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int OFF_Q = OFF_V + TILE;                // [NST] Q tiles
+  static constexpr int OFF_DO = OFF_Q + NST * TILE;         // [NST] dAV tiles
+  static constexpr int OFF_DS = OFF_DO + NST * TILE;        // [2] dS^T, two 16 KB panels (MN-major A)
+  static constexpr int OFF_STG = OFF_DS + (DQ ? 4 * BOX : 0);  // dQ partial, fp32, 2 swizzled boxes
+  static constexpr int STG_BYTES = DQ ? 128 * 64 * 4 : 0;   // of 32 columns x 128 rows
   static constexpr int OFF_QTS = OFF_STG + STG_BYTES;       // [NST][128] int64 query timestamps
   static constexpr int OFF_KTS = OFF_QTS + NST * 128 * 8;   // [128] int64 key timestamps
   static constexpr int OFF_QTS32 = OFF_KTS + 128 * 8;       // [NST][128] int32, relative
@@ -73,8 +82,11 @@ struct BwdCfg {
   static constexpr int OFF_BAR = OFF_DTT + BWD_TT_ALL * 4;
   static constexpr int SMEM = OFF_BAR + 256;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int S_COL = 0, DP_COL = 128, DV_COL = 256, DK_COL = 320, DQ_COL = 384;
+  static constexpr int S_COL = 0, DP_COL = 128, DV_COL = 256, DK_COL = 256 + HD,
+                       DQ_COL = 256 + 2 * HD;
   static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert(!DQ || DQ_COL + HD <= TMEM_COLS, "TMEM budget");
+  static_assert(DK_COL + HD <= TMEM_COLS, "TMEM budget");
 };
 
 struct BwdParams {
@@ -84,10 +96,11 @@ struct BwdParams {
   const float* alibi;    // [H] or null
   int P, Tb, H, n1;
   float scale;
-  float* dq;             // [T, H*64] fp32, accumulated (zeroed by the caller)
-  float* dk;             // [T, H*64] fp32 (unused when duvqk is set)
-  float* dv;             // [T, H*64] fp32 (unused when duvqk is set)
-  bf16* duvqk;           // or null: dV and dK as bf16 into blocks 1 and 3 of [T, 4*H*64]
+  float* dq;             // [T, H*hd] fp32: accumulated (zeroed by the caller) at head dim 64,
+                         // written by the query-stationary kernel at head dim 128
+  float* dk;             // [T, H*hd] fp32 (unused when duvqk is set)
+  float* dv;             // [T, H*hd] fp32 (unused when duvqk is set)
+  bf16* duvqk;           // or null: dV and dK as bf16 into blocks 1 and 3 of [T, 4*H*hd]
   float* dpos;           // [H, P] fp32, accumulated, or null
   float* dtime;          // [H, Tb] fp32, accumulated, or null
 };
@@ -163,11 +176,12 @@ __device__ __forceinline__ int sorted_groups(const int64_t* t, int lane) {
 // Bias modes of the backward kernel (compile-time): position table, time table, ALiBi.
 constexpr int BWD_POS = 1, BWD_TIME = 2, BWD_ALIBI = 4;
 
-template <int BM>
+template <int BM, int HD>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     attention_bwd_kernel(const __grid_constant__ CUtensorMap tm, const __grid_constant__ CUtensorMap tdo,
                          const __grid_constant__ CUtensorMap tdq, BwdParams prm, AttnSchedule sch) {
-  using Cfg = BwdCfg;
+  using Cfg = BwdCfg<HD>;
+  constexpr int NP = HD / 64;         // 64-column panels of a tile
   using namespace sm100;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint8_t* k_s = smem + Cfg::OFF_K;
@@ -212,7 +226,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int H = prm.H;
-  const int col_v = H * 64, col_q = 2 * H * 64, col_k = 3 * H * 64;
+  const int col_v = H * HD, col_q = 2 * H * HD, col_k = 3 * H * HD;
   constexpr bool has_time = (BM & BWD_TIME) != 0;
   constexpr bool has_pos = (BM & BWD_POS) != 0;
   constexpr bool alibi = (BM & BWD_ALIBI) != 0;
@@ -244,7 +258,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     fence_mbar_init();
     prefetch_tensormap(&tm);
     prefetch_tensormap(&tdo);
-    prefetch_tensormap(&tdq);
+    if (Cfg::DQ) prefetch_tensormap(&tdq);
   }
   for (int e = threadIdx.x; e < BWD_TT_ALL; e += BWD_THREADS) dtt_s[e] = 0.0f;
   if (warp == 1) {
@@ -283,9 +297,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       if (lane == 0) {
-        mbar_expect_tx(kv_full, 2 * Cfg::BOX);
-        tma_load_2d(k_s, &tm, kv_full, col_k + h * 64, (int)row0 + k0);
-        tma_load_2d(v_s, &tm, kv_full, col_v + h * 64, (int)row0 + k0);
+        mbar_expect_tx(kv_full, 2 * Cfg::TILE);
+#pragma unroll
+        for (int p = 0; p < NP; p++) {
+          tma_load_2d(k_s + p * Cfg::BOX, &tm, kv_full, col_k + h * HD + 64 * p, (int)row0 + k0);
+          tma_load_2d(v_s + p * Cfg::BOX, &tm, kv_full, col_v + h * HD + 64 * p, (int)row0 + k0);
+        }
         kv_par = (int)(k & 1u);
       }
       if (has_time) {
@@ -358,11 +375,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         if (lane == 0) {
-          mbar_expect_tx(&q_full[st], 2 * Cfg::BOX);
-          tma_load_2d(smem + Cfg::OFF_Q + st * Cfg::BOX, &tm, &q_full[st], col_q + h * 64,
-                      (int)row0 + i * ATT_BM);
-          tma_load_2d(smem + Cfg::OFF_DO + st * Cfg::BOX, &tdo, &q_full[st], h * 64,
-                      (int)row0 + i * ATT_BM);
+          mbar_expect_tx(&q_full[st], 2 * Cfg::TILE);
+#pragma unroll
+          for (int p = 0; p < NP; p++) {
+            tma_load_2d(smem + Cfg::OFF_Q + st * Cfg::TILE + p * Cfg::BOX, &tm, &q_full[st],
+                        col_q + h * HD + 64 * p, (int)row0 + i * ATT_BM);
+            tma_load_2d(smem + Cfg::OFF_DO + st * Cfg::TILE + p * Cfg::BOX, &tdo, &q_full[st],
+                        h * HD + 64 * p, (int)row0 + i * ATT_BM);
+          }
           q_par[st] = (int)ph;
         }
         if (has_time) {
@@ -396,30 +416,36 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     // the pointwise warps work.
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(128, 64, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16(128, 64, false, true);
+      constexpr uint32_t idesc_o = idesc_bf16(128, HD, false, true);
       constexpr uint32_t idesc_q = idesc_bf16(128, 64, true, true);
       const uint32_t k_addr = smem_u32(k_s), v_addr = smem_u32(v_s);
       uint32_t k = 0, g = 0, t = 0;
       bool ok = true;
       // S^T / dP^T of half ht of the query tile in stage st
       auto issue_s = [&](uint32_t st, int ht) {
-        const uint32_t q_addr = smem_u32(smem + Cfg::OFF_Q + st * Cfg::BOX) + ht * 8192;
-        const uint32_t do_addr = smem_u32(smem + Cfg::OFF_DO + st * Cfg::BOX) + ht * 8192;
+        const uint32_t q_addr = smem_u32(smem + Cfg::OFF_Q + st * Cfg::TILE) + ht * 8192;
+        const uint32_t do_addr = smem_u32(smem + Cfg::OFF_DO + st * Cfg::TILE) + ht * 8192;
+        // the reduction over the head dim runs through the tiles' 64-column panels
 #pragma unroll
-        for (int kk = 0; kk < 4; kk++)
-          mma_ss(tmem + Cfg::S_COL + 64 * ht, sdesc_sw128(k_addr + kk * 32, 16, 1024),
-                 sdesc_sw128(q_addr + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < HD / 16; kk++) {
+          const uint32_t off = (kk / 4) * Cfg::BOX + (kk % 4) * 32;
+          mma_ss(tmem + Cfg::S_COL + 64 * ht, sdesc_sw128(k_addr + off, 16, 1024),
+                 sdesc_sw128(q_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        }
 #pragma unroll
-        for (int kk = 0; kk < 4; kk++)
-          mma_ss(tmem + Cfg::DP_COL + 64 * ht, sdesc_sw128(v_addr + kk * 32, 16, 1024),
-                 sdesc_sw128(do_addr + kk * 32, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < HD / 16; kk++) {
+          const uint32_t off = (kk / 4) * Cfg::BOX + (kk % 4) * 32;
+          mma_ss(tmem + Cfg::DP_COL + 64 * ht, sdesc_sw128(v_addr + off, 16, 1024),
+                 sdesc_sw128(do_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+        }
         mma_commit(ht == 0 ? sa_full : sb_full);
       };
       // dV_j += P^T dAV and dK_j += dS^T Q over half ht's 64 queries (P^T, dS^T from TMEM: the
-      // 16 queries of pointwise column group cg sit, packed, at the start of its 16 columns)
+      // 16 queries of pointwise column group cg sit, packed, at the start of its 16 columns); the
+      // MN-major B operand's head-dim panels lie Cfg::BOX apart
       auto issue_dkv = [&](uint32_t st, int ht, bool first) {
-        const uint32_t q_addr = smem_u32(smem + Cfg::OFF_Q + st * Cfg::BOX);
-        const uint32_t do_addr = smem_u32(smem + Cfg::OFF_DO + st * Cfg::BOX);
+        const uint32_t q_addr = smem_u32(smem + Cfg::OFF_Q + st * Cfg::TILE);
+        const uint32_t do_addr = smem_u32(smem + Cfg::OFF_DO + st * Cfg::TILE);
 #pragma unroll
         for (int kk = 0; kk < 4; kk++)
           mma_ts(tmem + Cfg::DV_COL, tmem + Cfg::S_COL + 64 * ht + 16 * kk,
@@ -457,16 +483,18 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           if (!mbar_wait(pwb_done, t & 1u, abort_flag)) { ok = false; break; }
           tc_fence_after();
           issue_dkv(st, 1, false);
-          // dQ_i partial = dS K_j: dS from shared memory (MN-major: rows = keys; the buffer of this
-          // tile's parity), K_j as MN-major B
-          if (t > 0 && !mbar_wait(dq_empty, (t - 1) & 1u, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t ds_addr = smem_u32(ds_s + (t & 1u) * (2 * Cfg::BOX));
+          if constexpr (Cfg::DQ) {
+            // dQ_i partial = dS K_j: dS from shared memory (MN-major: rows = keys; the buffer of
+            // this tile's parity), K_j as MN-major B
+            if (t > 0 && !mbar_wait(dq_empty, (t - 1) & 1u, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t ds_addr = smem_u32(ds_s + (t & 1u) * (2 * Cfg::BOX));
 #pragma unroll
-          for (int kk = 0; kk < 8; kk++)
-            mma_ss(tmem + Cfg::DQ_COL, sdesc_sw128(ds_addr + kk * 2048, Cfg::BOX, 1024),
-                   sdesc_sw128(k_addr + kk * 2048, Cfg::BOX, 1024), idesc_q, kk > 0 ? 1u : 0u);
-          mma_commit(dq_full);
+            for (int kk = 0; kk < 8; kk++)
+              mma_ss(tmem + Cfg::DQ_COL, sdesc_sw128(ds_addr + kk * 2048, Cfg::BOX, 1024),
+                     sdesc_sw128(k_addr + kk * 2048, Cfg::BOX, 1024), idesc_q, kk > 0 ? 1u : 0u);
+            mma_commit(dq_full);
+          }
           mma_commit(&q_empty[st]);
           if (i == nt - 1) {
             mma_commit(dkv_full);
@@ -481,7 +509,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       mbar_drain(drain, 0);
     }
     __syncwarp();
-  } else if (warp == 2) {
+  } else if (warp == 2 && Cfg::DQ) {
     // ------------------------------------------------------------------ dQ reducer
     // Adds each query tile's dQ partial, staged by the pointwise warps, to global dQ with two TMA
     // reductions; rows past the sequence hold zeros (their dS is masked), so the tile can run
@@ -498,8 +526,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         for (int i = jt; i < nt; i++, t++) {
           if (!mbar_wait(stg_full, t & 1u, abort_flag)) { ok = false; break; }
           const int y = (int)row0 + i * ATT_BM;
-          tma_reduce_add_2d(&tdq, stg_s, h * 64, y);
-          tma_reduce_add_2d(&tdq, stg_s + 128 * 128, h * 64 + 32, y);
+          tma_reduce_add_2d(&tdq, stg_s, h * HD, y);
+          tma_reduce_add_2d(&tdq, stg_s + 128 * 128, h * HD + 32, y);
           bulk_commit();
           bulk_wait_read_all();
           mbar_arrive(stg_empty);
@@ -785,12 +813,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         // dS^T into shared memory (the buffer of this tile's parity) as the MN-major A operand of
         // dQ = dS K_j: row = key r, 128-byte swizzled rows of 64 queries per panel (one panel per
         // half); this block's 16 queries are 2 units
+        if constexpr (Cfg::DQ) {
 #pragma unroll
-        for (int v = 0; v < 2; v++) {
-          const int uu = 2 * cg + v;
-          uint8_t* dst = ds_s + (t & 1u) * (2 * Cfg::BOX) + ht * Cfg::BOX + r * 128 +
-                         ((uu ^ (r & 7)) * 16);
-          *reinterpret_cast<uint4*>(dst) = make_uint4(dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]);
+          for (int v = 0; v < 2; v++) {
+            const int uu = 2 * cg + v;
+            uint8_t* dst = ds_s + (t & 1u) * (2 * Cfg::BOX) + ht * Cfg::BOX + r * 128 +
+                           ((uu ^ (r & 7)) * 16);
+            *reinterpret_cast<uint4*>(dst) =
+                make_uint4(dk[4 * v], dk[4 * v + 1], dk[4 * v + 2], dk[4 * v + 3]);
+          }
         }
         // position gradient of the block: its diagonal sums, two per lane (the global reductions
         // are issued after the arrive below: an arrive releases this warp's earlier writes, so
@@ -866,12 +897,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           if (pg1 != 0.0f && pd1 >= 0) atomicAdd(dpos_h + pd1, pg1);
         }
         // the previous tile's dQ partial, while the tensor cores work on this tile
-        if (ht == 0 && i > jt && !dq_readout(t - 1)) { ok = false; break; }
+        if (Cfg::DQ && ht == 0 && i > jt && !dq_readout(t - 1)) { ok = false; break; }
         }
       }
       if (!ok) break;
       // the item's last dQ partial
-      if (!dq_readout(t - 1)) break;
+      if (Cfg::DQ && !dq_readout(t - 1)) break;
       // the pending table-gradient sums
       if (has_time) {
         flush_time(pend_b, pend_lo);
@@ -882,44 +913,54 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         for (int o = 16; o > 0; o >>= 1) pend_p += __shfl_xor_sync(0xffffffffu, pend_p, o);
         if (lane == 0 && pend_p != 0.0f) atomicAdd(prm.dpos + (int64_t)h * P + (P - 1), pend_p);
       }
-      // dV_j and dK_j of this item: TMEM lane = key row; this warp's 16 of the 64 columns
+      // dV_j and dK_j of this item: TMEM lane = key row; this warp's columns 16 cg .. 16 cg + 15 of
+      // each 64-column panel
       if (!mbar_wait(dkv_full, k & 1u, abort_flag)) break;
       tc_fence_after();
       {
-        uint32_t vv[16], kv[16];
-        tmem_ld16(t_lane + Cfg::DV_COL + 16 * cg, vv);
-        tmem_ld16(t_lane + Cfg::DK_COL + 16 * cg, kv);
-        tmem_ld_wait16(vv);
-        tmem_ld_wait16(kv);
+        uint32_t vv[NP][16], kv[NP][16];
+#pragma unroll
+        for (int p = 0; p < NP; p++) {
+          tmem_ld16(t_lane + Cfg::DV_COL + 64 * p + 16 * cg, vv[p]);
+          tmem_ld16(t_lane + Cfg::DK_COL + 64 * p + 16 * cg, kv[p]);
+        }
+#pragma unroll
+        for (int p = 0; p < NP; p++) {
+          tmem_ld_wait16(vv[p]);
+          tmem_ld_wait16(kv[p]);
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(dkv_empty);
-        if (kvalid && prm.duvqk) {
-          // bf16 into the V and K blocks of a [T, 4 H 64] gradient of U|V|Q|K
-          bf16* base = prm.duvqk + (row0 + j) * (int64_t)(4 * H * 64) + h * 64 + 16 * cg;
-          uint32_t pv[8], pk2[8];
 #pragma unroll
-          for (int v = 0; v < 8; v++) {
-            pv[v] = pack_bf16x2(__uint_as_float(vv[2 * v]), __uint_as_float(vv[2 * v + 1]));
-            pk2[v] = pack_bf16x2(__uint_as_float(kv[2 * v]), __uint_as_float(kv[2 * v + 1]));
-          }
-          uint4* dvb = reinterpret_cast<uint4*>(base + H * 64);
-          uint4* dkb = reinterpret_cast<uint4*>(base + 3 * H * 64);
-          dvb[0] = make_uint4(pv[0], pv[1], pv[2], pv[3]);
-          dvb[1] = make_uint4(pv[4], pv[5], pv[6], pv[7]);
-          dkb[0] = make_uint4(pk2[0], pk2[1], pk2[2], pk2[3]);
-          dkb[1] = make_uint4(pk2[4], pk2[5], pk2[6], pk2[7]);
-        } else if (kvalid) {
-          float* dvr = prm.dv + (row0 + j) * (int64_t)(H * 64) + h * 64 + 16 * cg;
-          float* dkr = prm.dk + (row0 + j) * (int64_t)(H * 64) + h * 64 + 16 * cg;
+        for (int p = 0; p < NP; p++) {
+          if (kvalid && prm.duvqk) {
+            // bf16 into the V and K blocks of a [T, 4 H hd] gradient of U|V|Q|K
+            bf16* base = prm.duvqk + (row0 + j) * (int64_t)(4 * H * HD) + h * HD + 64 * p + 16 * cg;
+            uint32_t pv[8], pk2[8];
 #pragma unroll
-          for (int v = 0; v < 4; v++) {
-            reinterpret_cast<float4*>(dvr)[v] =
-                make_float4(__uint_as_float(vv[4 * v]), __uint_as_float(vv[4 * v + 1]),
-                            __uint_as_float(vv[4 * v + 2]), __uint_as_float(vv[4 * v + 3]));
-            reinterpret_cast<float4*>(dkr)[v] =
-                make_float4(__uint_as_float(kv[4 * v]), __uint_as_float(kv[4 * v + 1]),
-                            __uint_as_float(kv[4 * v + 2]), __uint_as_float(kv[4 * v + 3]));
+            for (int v = 0; v < 8; v++) {
+              pv[v] = pack_bf16x2(__uint_as_float(vv[p][2 * v]), __uint_as_float(vv[p][2 * v + 1]));
+              pk2[v] = pack_bf16x2(__uint_as_float(kv[p][2 * v]), __uint_as_float(kv[p][2 * v + 1]));
+            }
+            uint4* dvb = reinterpret_cast<uint4*>(base + H * HD);
+            uint4* dkb = reinterpret_cast<uint4*>(base + 3 * H * HD);
+            dvb[0] = make_uint4(pv[0], pv[1], pv[2], pv[3]);
+            dvb[1] = make_uint4(pv[4], pv[5], pv[6], pv[7]);
+            dkb[0] = make_uint4(pk2[0], pk2[1], pk2[2], pk2[3]);
+            dkb[1] = make_uint4(pk2[4], pk2[5], pk2[6], pk2[7]);
+          } else if (kvalid) {
+            float* dvr = prm.dv + (row0 + j) * (int64_t)(H * HD) + h * HD + 64 * p + 16 * cg;
+            float* dkr = prm.dk + (row0 + j) * (int64_t)(H * HD) + h * HD + 64 * p + 16 * cg;
+#pragma unroll
+            for (int v = 0; v < 4; v++) {
+              reinterpret_cast<float4*>(dvr)[v] =
+                  make_float4(__uint_as_float(vv[p][4 * v]), __uint_as_float(vv[p][4 * v + 1]),
+                              __uint_as_float(vv[p][4 * v + 2]), __uint_as_float(vv[p][4 * v + 3]));
+              reinterpret_cast<float4*>(dkr)[v] =
+                  make_float4(__uint_as_float(kv[p][4 * v]), __uint_as_float(kv[p][4 * v + 1]),
+                              __uint_as_float(kv[p][4 * v + 2]), __uint_as_float(kv[p][4 * v + 3]));
+            }
           }
         }
       }

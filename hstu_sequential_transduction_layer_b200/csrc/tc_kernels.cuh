@@ -8,6 +8,7 @@
 
 #include "tc_attention.cuh"
 #include "tc_attention_bwd.cuh"
+#include "tc_attention_bwd_dq.cuh"
 #include "tc_gemm.cuh"
 #include "tc_ln_f2.cuh"
 
@@ -277,27 +278,56 @@ inline size_t attention_bwd_workspace_bytes(int64_t T, int64_t B, int H) {
   return (size_t)(256 + ((16 * B + 255) / 256) * 256 + 8 * attention_bwd_capacity(T, B, H));
 }
 
-template <int BM>
+template <int BM, int HD>
 hstu_status_t launch_attention_bwd_kernel(const CUtensorMap& tm, const CUtensorMap& tdo,
                                           const CUtensorMap& tdq, const BwdParams& prm,
                                           const AttnSchedule& sch, int grid, cudaStream_t st) {
-  auto kern = attention_bwd_kernel<BM>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg::SMEM) !=
+  auto kern = attention_bwd_kernel<BM, HD>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, BwdCfg<HD>::SMEM) !=
       cudaSuccess)
     return HSTU_ERR_CUDA;
-  kern<<<grid, BWD_THREADS, BwdCfg::SMEM, st>>>(tm, tdo, tdq, prm, sch);
+  kern<<<grid, BWD_THREADS, BwdCfg<HD>::SMEM, st>>>(tm, tdo, tdq, prm, sch);
   count_launch();
-  return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+  if constexpr (!BwdCfg<HD>::DQ) {
+    // dQ from the query-stationary kernel, on the same schedule
+    auto dqk = attention_bwd_dq_kernel<BM, HD>;
+    if (cudaFuncSetAttribute(dqk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             BwdDqCfg<HD>::SMEM) != cudaSuccess)
+      return HSTU_ERR_CUDA;
+    dqk<<<grid, BWD_THREADS, BwdDqCfg<HD>::SMEM, st>>>(tm, tdo, prm, sch);
+    count_launch();
+    if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
+  }
+  return HSTU_OK;
 }
 
-// Backward of Eq. 2 (head dim 64): dq, dpos and dtime are accumulated and must be zero on entry.
-inline hstu_status_t launch_attention_bwd(int64_t T, int64_t B, int H, int64_t max_seq_len,
+template <int HD>
+hstu_status_t launch_attention_bwd_hd(const CUtensorMap& tm, const CUtensorMap& tdo,
+                                      const CUtensorMap& tdq, const BwdParams& prm,
+                                      const AttnSchedule& sch, int grid, int bm, cudaStream_t st) {
+  switch (bm) {
+    case 0: return launch_attention_bwd_kernel<0, HD>(tm, tdo, tdq, prm, sch, grid, st);
+    case BWD_POS: return launch_attention_bwd_kernel<BWD_POS, HD>(tm, tdo, tdq, prm, sch, grid, st);
+    case BWD_TIME:
+      return launch_attention_bwd_kernel<BWD_TIME, HD>(tm, tdo, tdq, prm, sch, grid, st);
+    case BWD_POS | BWD_TIME:
+      return launch_attention_bwd_kernel<BWD_POS | BWD_TIME, HD>(tm, tdo, tdq, prm, sch, grid, st);
+    default: return launch_attention_bwd_kernel<BWD_ALIBI, HD>(tm, tdo, tdq, prm, sch, grid, st);
+  }
+}
+
+// Backward of Eq. 2 (head dim 64 or 128).  dpos and dtime are accumulated and must be zero on
+// entry; so must dq at head dim 64 (reduced in fp32 across key tiles), while at head dim 128 every
+// row of dq (or of the Q block of duvqk, when given) is written once.
+inline hstu_status_t launch_attention_bwd(int64_t T, int64_t B, int H, int hd, int64_t max_seq_len,
                                           const bf16* uvqk, const int64_t* off, const int64_t* ts,
                                           const float* pos, int P, const float* tim, int Tb,
                                           const float* alibi, float scale, const bf16* dav, float* dq,
                                           float* dk, float* dv, float* dpos, float* dtime, void* ws,
                                           size_t ws_bytes, cudaStream_t st,
                                           bf16* duvqk = nullptr) {
+  if (hd != 64 && hd != 128) return HSTU_ERR_UNSUPPORTED;
   if (T >= (1LL << 31) || H >= (1 << 15)) return HSTU_ERR_UNSUPPORTED;
   if (ws_bytes < attention_bwd_workspace_bytes(T, B, H)) return HSTU_ERR_INVALID_ARG;
   const int64_t max_tiles64 = ((max_seq_len > 0 ? max_seq_len : T) + ATT_BN - 1) / ATT_BN;
@@ -313,11 +343,15 @@ inline hstu_status_t launch_attention_bwd(int64_t T, int64_t B, int H, int64_t m
   bwd_schedule_kernel<<<1, 1024, sched_smem, st>>>(off, B, T, H, max_tiles, capacity, sch);
   count_launch();
   if (cudaGetLastError() != cudaSuccess) return HSTU_ERR_CUDA;
-  const int n1 = 4 * H * 64;
+  const int n1 = 4 * H * hd;
   CUtensorMap tm, tdo, tdq;
   if (!make_map_bf16(&tm, uvqk, n1, T, n1, 64, 128)) return HSTU_ERR_CUDA;
-  if (!make_map_bf16(&tdo, dav, (uint64_t)H * 64, T, (uint64_t)H * 64, 64, 128)) return HSTU_ERR_CUDA;
-  if (!make_map_f32(&tdq, dq, (uint64_t)H * 64, T, (uint64_t)H * 64, 32, 128)) return HSTU_ERR_CUDA;
+  if (!make_map_bf16(&tdo, dav, (uint64_t)H * hd, T, (uint64_t)H * hd, 64, 128)) return HSTU_ERR_CUDA;
+  if (hd == 64) {
+    if (!make_map_f32(&tdq, dq, (uint64_t)H * hd, T, (uint64_t)H * hd, 32, 128)) return HSTU_ERR_CUDA;
+  } else {
+    tdq = tdo;   // not read: dQ is stored directly
+  }
   BwdParams prm;
   prm.ts = ts;
   prm.pos = pos;
@@ -336,14 +370,8 @@ inline hstu_status_t launch_attention_bwd(int64_t T, int64_t B, int H, int64_t m
   prm.dtime = dtime;
   const int grid = (int)(capacity < num_sms() ? capacity : num_sms());
   const int bm = alibi ? BWD_ALIBI : ((pos ? BWD_POS : 0) | (tim ? BWD_TIME : 0));
-  switch (bm) {
-    case 0: return launch_attention_bwd_kernel<0>(tm, tdo, tdq, prm, sch, grid, st);
-    case BWD_POS: return launch_attention_bwd_kernel<BWD_POS>(tm, tdo, tdq, prm, sch, grid, st);
-    case BWD_TIME: return launch_attention_bwd_kernel<BWD_TIME>(tm, tdo, tdq, prm, sch, grid, st);
-    case BWD_POS | BWD_TIME:
-      return launch_attention_bwd_kernel<BWD_POS | BWD_TIME>(tm, tdo, tdq, prm, sch, grid, st);
-    default: return launch_attention_bwd_kernel<BWD_ALIBI>(tm, tdo, tdq, prm, sch, grid, st);
-  }
+  if (hd == 64) return launch_attention_bwd_hd<64>(tm, tdo, tdq, prm, sch, grid, bm, st);
+  return launch_attention_bwd_hd<128>(tm, tdo, tdq, prm, sch, grid, bm, st);
 }
 
 // M-FALCON candidate attention workspace: header (256 B), per-user (candidate start, count,

@@ -192,9 +192,10 @@ hstu_status_t hstu_ln_f2_fwd(const hstu_shape_t* shape, const void* av, const vo
  *   dv_j = sum_{i>=j} scale*SiLU(x_ij) dAV_i,   dx_ij = scale*SiLU'(x_ij) (dAV_i . v_j),
  *   dq_i = sum_{j<=i} dx_ij k_j,   dk_j = sum_{i>=j} dx_ij q_i,
  *   dpos[h][p], dtime[h][b] = sums of dx_ij over the pairs in bucket p, b (ALiBi slopes: none).
- * bf16 with d_qk = d_v = 64 (else HSTU_ERR_UNSUPPORTED); the forward's arguments, plus
- *  dav            [T, H*64] bf16, the incoming gradient
- *  dq, dk, dv     [T, H*64] fp32 outputs (16-byte aligned, not overlapping)
+ * bf16 with d_qk = d_v = hd, hd = 64 or 128 (else HSTU_ERR_UNSUPPORTED); the forward's
+ * arguments, plus
+ *  dav            [T, H*hd] bf16, the incoming gradient
+ *  dq, dk, dv     [T, H*hd] fp32 outputs (16-byte aligned, not overlapping)
  *  dpos_table     [H, P] fp32 output, required when pos_table is given (else ignored)
  *  dtime_table    [H, Tb] fp32 output, required when time_table is given (else ignored)
  *  workspace      hstu_attention_bwd_workspace_size(shape) bytes, 256-byte aligned
@@ -257,8 +258,8 @@ void hstu_layer_pipeline_destroy(hstu_layer_pipeline_t* p);
  * The activations come from the forward: `fwd_workspace` (fwd_workspace_bytes >=
  * hstu_layer_fwd_workspace_size(shape)) is the workspace that a preceding hstu_layer_fwd call with
  * the same shape, X, offsets, timestamps, weights and tables filled, not written since; its U, V, Q,
- * K and AV are read, and X W1 + b1 and G = LayerNorm(AV) * U are recomputed.  bf16 with d_qk = d_v = 64 and
- * H*d_v <= 8192 (else HSTU_ERR_UNSUPPORTED).  Arguments as in hstu_layer_fwd (b2 is not needed),
+ * K and AV are read, and X W1 + b1 and G = LayerNorm(AV) * U are recomputed.  bf16 with d_qk = d_v = 64 or 128
+ * and H*d_v <= 8192 (else HSTU_ERR_UNSUPPORTED).  Arguments as in hstu_layer_fwd (b2 is not needed),
  * plus
  *  dY             [T, d] bf16, the incoming gradient
  *  dX             [T, d] bf16 output

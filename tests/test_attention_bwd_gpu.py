@@ -1,4 +1,4 @@
-"""Backward of Eq. 2 on the GPU (tcgen05, head dim 64) against the fp64 oracle ("Actions Speak
+"""Backward of Eq. 2 on the GPU (tcgen05, head dims 64 and 128) against the fp64 oracle ("Actions Speak
 Louder than Words" paper notes, section 3.1; training).  P and dS enter the tensor-core products in
 bf16, so dq, dk, dv are held to the bf16 criteria; the table gradients sum fp32 scores."""
 import ctypes
@@ -18,8 +18,7 @@ def hstu():
     return m
 
 
-def _run(hstu, seed, lengths, H, bias, P=96, Tb=24):
-    hd = 64
+def _run(hstu, seed, lengths, H, bias, P=96, Tb=24, hd=64):
     d = H * hd
     inp = random_case(seed, lengths, d, H, hd, P=P, Tb=Tb, dtype="bf16", alibi=(bias == "alibi"))
     if bias in ("pos", "none"):
@@ -74,13 +73,42 @@ def test_attention_backward_longer_sequences(hstu):
         assert_bf16_close(got[k], ref[k], f"{k} (2 x ~2k)")
 
 
+@pytest.mark.gpu
+@pytest.mark.parametrize("seed,lengths,H,bias", [
+    (61, [300, 1, 129, 513], 2, "rab"),
+    (62, [256, 0, 1000], 2, "pos"),
+    (63, [700, 31], 2, "alibi"),
+    (64, [128, 255, 257], 1, "none"),
+    (65, [1, 2, 127, 128, 129], 3, "rab"),
+])
+def test_attention_backward_head_dim_128(hstu, seed, lengths, H, bias):
+    """Head dim 128: dK, dV and the table gradients from the key-stationary kernel, dQ from the
+    query-stationary one; ragged lengths around the 128-row tile, an empty sequence, one token."""
+    got, ref = _run(hstu, seed, lengths, H, bias, hd=128)
+    for k in ("dq", "dk", "dv"):
+        assert_bf16_close(got[k], ref[k], f"{k} ({bias}, hd=128)")
+    for k in ("dpos", "dtime"):
+        if ref[k] is not None:
+            assert_bf16_close(got[k], ref[k], f"{k} ({bias}, hd=128)")
+
+
+@pytest.mark.gpu
+def test_attention_backward_head_dim_128_longer(hstu):
+    got, ref = _run(hstu, 66, [1800, 2100], 2, "rab", P=1024, Tb=64, hd=128)
+    for k in ("dq", "dk", "dv", "dpos", "dtime"):
+        assert_bf16_close(got[k], ref[k], f"{k} (2 x ~2k, hd=128)")
+
+
 def test_backward_host_validation(hstu):
     lib = hstu.library()
     fake = ctypes.c_void_p(1 << 20)
-    s128 = hstu.make_shape(1, 10, 10, 256, 2, 128, 128, hstu.HSTU_BF16, 16, 0)
-    rc = lib.hstu_attention_bwd(ctypes.byref(s128), fake, fake, None, fake, None, None,
-                                ctypes.c_float(1.0), fake, fake, fake, fake, fake, None, fake, 1 << 30, None)
-    assert rc == hstu.HSTU_ERR_UNSUPPORTED
+    # head dims other than 64 and 128, and d_qk != d_v
+    for hq, hv in ((32, 32), (256, 256), (64, 128)):
+        sh = hstu.make_shape(1, 10, 10, 256, 2, hq, hv, hstu.HSTU_BF16, 16, 0)
+        rc = lib.hstu_attention_bwd(ctypes.byref(sh), fake, fake, None, fake, None, None,
+                                    ctypes.c_float(1.0), fake, fake, fake, fake, fake, None, fake,
+                                    1 << 30, None)
+        assert rc == hstu.HSTU_ERR_UNSUPPORTED, (hq, hv)
     s64 = hstu.make_shape(1, 10, 10, 128, 2, 64, 64, hstu.HSTU_BF16, 16, 0)
     # a position table without a place for its gradient
     rc = lib.hstu_attention_bwd(ctypes.byref(s64), fake, fake, None, fake, None, None,

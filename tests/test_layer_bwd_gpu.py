@@ -24,8 +24,8 @@ def hstu():
 
 def _gpu_bwd(hstu, inp, dY):
     w, p = inp.workload, inp.layers[0]
-    H, d = w.num_heads, w.d_model
-    n1, wv = 4 * H * 64, H * 64
+    H, d, hd = w.num_heads, w.d_model, w.head_dim
+    n1, wv = 4 * H * hd, H * hd
     has_t = inp.time_table is not None
     ts = dev(inp.timestamps) if has_t else None
     X, off = dev(inp.X), dev(inp.seq_offsets)
@@ -33,7 +33,7 @@ def _gpu_bwd(hstu, inp, dY):
     ln_w, ln_b = dev(p.ln_w), dev(p.ln_b)
     pos, tim, ali = dev(inp.pos_table, "f32"), dev(inp.time_table, "f32"), dev(inp.alibi_slopes, "f32")
     max_len = max(1, int(inp.lengths.max(initial=1)))
-    s = hstu.shape_for(X, off, H, 64, 64, max_len, inp.pos_table, inp.time_table, inp.ln_eps)
+    s = hstu.shape_for(X, off, H, hd, hd, max_len, inp.pos_table, inp.time_table, inp.ln_eps)
     fws = hstu.alloc_workspace(s, "cuda")
     hstu.hstu_layer_fwd(X, off, ts, W1, b1, W2, b2, ln_w, ln_b, pos, tim, ali, inp.scale,
                         num_heads=H, max_seq_len=max_len, ln_eps=inp.ln_eps, workspace=fws)
@@ -52,20 +52,20 @@ def _oracle_bwd(inp, dY):
     w, p = inp.workload, inp.layers[0]
     has_t = inp.time_table is not None
     return oracle.layer_bwd(inp.seq_offsets, inp.X, p.W1, p.b1, p.W2, p.b2, p.ln_w, p.ln_b, dY,
-                            num_heads=w.num_heads, d_qk=64, d_v=64,
+                            num_heads=w.num_heads, d_qk=w.head_dim, d_v=w.head_dim,
                             timestamps=inp.timestamps if has_t else None,
                             pos_table=inp.pos_table, time_table=inp.time_table,
                             alibi_slopes=inp.alibi_slopes, scale=inp.scale, ln_eps=inp.ln_eps)
 
 
-def _case(seed, lengths, H, bias, P=96, Tb=24):
-    inp = random_case(seed, lengths, H * 64, H, 64, P=P, Tb=Tb, dtype="bf16",
+def _case(seed, lengths, H, bias, P=96, Tb=24, hd=64):
+    inp = random_case(seed, lengths, H * hd, H, hd, P=P, Tb=Tb, dtype="bf16",
                       alibi=(bias == "alibi"))
     if bias in ("pos", "none"):
         inp.time_table = None
     if bias == "none":
         inp.pos_table = None
-    dY = round_bf16(np.random.default_rng(seed + 7).normal(0, 1.0, (inp.T, H * 64)))
+    dY = round_bf16(np.random.default_rng(seed + 7).normal(0, 1.0, (inp.T, H * hd)))
     return inp, dY
 
 
@@ -90,6 +90,17 @@ def _compare(got, ref, dY, what):
 def test_layer_backward_matches_oracle(hstu, seed, lengths, H, bias):
     inp, dY = _case(seed, lengths, H, bias)
     _compare(_gpu_bwd(hstu, inp, dY), _oracle_bwd(inp, dY), dY, f"{bias}, H={H}")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("seed,lengths,H,bias", [
+    (71, [300, 1, 129, 513], 2, "rab"),
+    (72, [700, 0, 31], 2, "alibi"),
+    (73, [128, 255, 257], 1, "none"),
+])
+def test_layer_backward_head_dim_128(hstu, seed, lengths, H, bias):
+    inp, dY = _case(seed, lengths, H, bias, hd=128)
+    _compare(_gpu_bwd(hstu, inp, dY), _oracle_bwd(inp, dY), dY, f"{bias}, H={H}, hd=128")
 
 
 @pytest.mark.gpu
@@ -122,12 +133,13 @@ def test_layer_bwd_host_validation(hstu):
     lib = hstu.library()
     fake = ctypes.c_void_p(1 << 20)
     f = [fake] * 11
-    # head dim 128 is not implemented by the backward
-    s128 = hstu.make_shape(1, 10, 10, 256, 2, 128, 128, hstu.HSTU_BF16, 0, 0)
-    rc = lib.hstu_layer_bwd(ctypes.byref(s128), fake, fake, None, fake, fake, fake, fake, fake, None,
-                            None, None, ctypes.c_float(0.1), fake, 1 << 30, fake, fake, *f[:6],
-                            None, None, fake, 1 << 30, None)
-    assert rc == hstu.HSTU_ERR_UNSUPPORTED
+    # the backward takes d_qk = d_v = 64 or 128 only
+    for hq, hv in ((64, 128), (256, 256)):
+        sh = hstu.make_shape(1, 10, 10, 256, 2, hq, hv, hstu.HSTU_BF16, 0, 0)
+        rc = lib.hstu_layer_bwd(ctypes.byref(sh), fake, fake, None, fake, fake, fake, fake, fake,
+                                None, None, None, ctypes.c_float(0.1), fake, 1 << 30, fake, fake,
+                                *f[:6], None, None, fake, 1 << 30, None)
+        assert rc == hstu.HSTU_ERR_UNSUPPORTED, (hq, hv)
     s = hstu.make_shape(1, 10, 10, 128, 2, 64, 64, hstu.HSTU_BF16, 16, 0)
     # a position table without its gradient
     rc = lib.hstu_layer_bwd(ctypes.byref(s), fake, fake, None, fake, fake, fake, fake, fake, fake,
