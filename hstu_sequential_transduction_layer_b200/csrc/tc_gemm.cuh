@@ -8,6 +8,8 @@
 //   EPI_F32:            C32 = acc (fp32)                  dG = dY W2^T
 //   EPI_SILU_GRAD:      C = R * SiLU'(acc + bias)         dZ = dUVQK * SiLU'(X W1 + b1)
 //   EPI_RED_F32:        C32 += acc (fp32 reductions)      dW = X^T dZ over a split of K
+// and for the fused LayerNorm*U -> f2 kernel, whose accumulator already holds the residual:
+//   EPI_BIAS:           C = acc + bias
 // With `splits` > 1 every output tile is computed in that many parts over consecutive ranges of K
 // (split-K, for the weight gradients' short M and N and long K); only EPI_RED_F32 combines parts.
 //
@@ -31,7 +33,7 @@ namespace hstu {
 namespace tc {
 
 enum GemmEpilogue { EPI_BIAS_SILU = 0, EPI_BIAS_RESIDUAL = 1, EPI_F32 = 2, EPI_SILU_GRAD = 3,
-                    EPI_RED_F32 = 4 };
+                    EPI_RED_F32 = 4, EPI_BIAS = 5 };
 
 template <int BN>
 struct GemmCfg {

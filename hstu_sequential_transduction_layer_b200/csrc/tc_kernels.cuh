@@ -103,15 +103,17 @@ hstu_status_t launch_ln_f2_n(int64_t M, int n1, const float* av, const bf16* uvq
                              const bf16* ln_w, const bf16* ln_b, float eps, const bf16* W2,
                              const bf16* b2, const bf16* X, bf16* Y, cudaStream_t st) {
   using Cfg = LnF2Cfg<N>;
-  CUtensorMap tb;
+  CUtensorMap tb, tu, tx;
   if (!make_map_bf16(&tb, W2, N, N, N, 64, 64)) return HSTU_ERR_CUDA;
+  if (!make_map_bf16(&tu, uvqk, n1, M, n1, 64, 128)) return HSTU_ERR_CUDA;   // U: columns 0 .. N-1
+  if (!make_map_bf16(&tx, X, N, M, N, 64, 128)) return HSTU_ERR_CUDA;
   auto kern = ln_f2_kernel<N, N>;
   constexpr int smem = Cfg::SMEM + 1024;   // + alignment slack
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return HSTU_ERR_CUDA;
   const int64_t blocks = (M + Cfg::BM - 1) / Cfg::BM;
   const int grid = (int)(blocks < num_sms() ? blocks : num_sms());
-  kern<<<grid, LNF2_THREADS, smem, st>>>(tb, M, n1, av, uvqk, ln_w, ln_b, eps, b2, X, Y);
+  kern<<<grid, LNF2_THREADS, smem, st>>>(tb, tu, tx, M, n1, av, uvqk, ln_w, ln_b, eps, b2, X, Y);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
