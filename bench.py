@@ -239,8 +239,8 @@ def run_ours(args, rank, world, local_rank):
                           device=dev)
     outs = [torch.empty_like(D["X"]) for _ in range(nl)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    # hstu_layer_fwd runs LayerNorm*U and f2 as one kernel where it can (H*d_v == d in 128/256/512)
-    fused = wv == d and d in (128, 256, 512)
+    # hstu_layer_fwd runs LayerNorm*U and f2 as one kernel where that is faster (H*d_v == d in 128/256)
+    fused = wv == d and d in (128, 256)
 
     def step(evs=None):
         # every layer through the entry points hstu_layer_fwd chains, events between them

@@ -35,16 +35,25 @@ namespace tc {
 enum GemmEpilogue { EPI_BIAS_SILU = 0, EPI_BIAS_RESIDUAL = 1, EPI_F32 = 2, EPI_SILU_GRAD = 3,
                     EPI_RED_F32 = 4, EPI_BIAS = 5 };
 
-template <int BN>
+// RX: the residual R enters the accumulator on the tensor core.  In the first BN/64 K blocks of a
+// tile, stage i also holds R's 128 x 64 chunk i (TMA), and R_i times a 16 x 16 identity is added to
+// accumulator columns 64 i .. 64 i + 63 (products by 1 and fp32 sums: exact up to the order of the
+// fp32 additions), so the epilogue loads nothing but the bias.
+template <int BN, bool RX = false>
 struct GemmCfg {
   static constexpr int BM = 128, BK = 64;
-  static constexpr int STAGES = BN == 256 ? 4 : (BN == 128 ? 6 : 8);
   static constexpr int A_BYTES = BM * BK * 2;
   static constexpr int B_BYTES = BK * BN * 2;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int X_BYTES = RX ? BM * BK * 2 : 0;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + X_BYTES;
+  static constexpr int STAGES = RX ? (BN == 256 ? 3 : (BN == 128 ? 4 : 5))
+                                   : (BN == 256 ? 4 : (BN == 128 ? 6 : 8));
+  static constexpr int OFF_ID = STAGES * STAGE_BYTES;       // RX: 16 x 64 bf16, the identity
+  static constexpr int OFF_BAR = OFF_ID + (RX ? 16 * 128 : 0);
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
+  static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
   static constexpr int TMEM_COLS = 2 * BN;
+  static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 __device__ __forceinline__ void gemm_tile_coords(int64_t t, int tiles_n, int64_t tiles_m,
@@ -128,18 +137,19 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const uint32_t (&r)[32], con
 
 constexpr int kGemmThreads = 320;  // producer warp, MMA warp, 8 epilogue warps
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool RX = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   int64_t M, int N, int K, const bf16* __restrict__ bias,
-                   const bf16* __restrict__ R, bf16* __restrict__ C, float* __restrict__ C32,
-                   int splits) {
-  using Cfg = GemmCfg<BN>;
+                   const __grid_constant__ CUtensorMap tmR, int64_t M, int N, int K,
+                   const bf16* __restrict__ bias, const bf16* __restrict__ R, bf16* __restrict__ C,
+                   float* __restrict__ C32, int splits) {
+  static_assert(!RX || EPI == EPI_BIAS_RESIDUAL, "the residual on the tensor core is f2's");
+  using Cfg = GemmCfg<BN, RX>;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::STAGES * Cfg::STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::OFF_BAR);
   uint64_t* empty = full + Cfg::STAGES;
   uint64_t* tfull = empty + Cfg::STAGES;
   uint64_t* tempty = tfull + 2;
@@ -153,6 +163,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int kblocks = K / Cfg::BK;
   const int kbps = (kblocks + splits - 1) / splits;   // K blocks per split (every split non-empty)
   const int64_t num_units = tiles_m * tiles_n * splits;
+  // the residual on the tensor core needs one K block per 64 output columns, in one split
+  const bool rx = RX && splits == 1 && K >= BN;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < Cfg::STAGES; s++) {
@@ -168,6 +180,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     fence_mbar_init();
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
+    if (rx) prefetch_tensormap(&tmR);
+  }
+  if (RX) {
+    // the 16 x 16 identity as an MN-major B operand (128-byte swizzled rows of 64 columns, of
+    // which 16 are used): row k holds 1 in column k
+    uint8_t* id_s = smem + Cfg::OFF_ID;
+    for (int e = threadIdx.x; e < 16 * 128 / 16; e += blockDim.x)
+      reinterpret_cast<uint4*>(id_s)[e] = make_uint4(0, 0, 0, 0);
+    __syncthreads();
+    if (threadIdx.x < 16) {
+      const int k = threadIdx.x;
+      *reinterpret_cast<uint16_t*>(id_s + k * 128 + (((k >> 3) ^ (k & 7)) << 4) + (k & 7) * 2) =
+          0x3F80;   // bf16 1.0
+    }
+    fence_proxy_async_smem();   // read by the tensor core through the async proxy
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
@@ -196,11 +223,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
           uint8_t* a_s = smem + stage * Cfg::STAGE_BYTES;
           uint8_t* b_s = a_s + Cfg::A_BYTES;
-          mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+          const bool xload = rx && kb - kb0 < BN / 64;   // R's chunk kb - kb0 of this tile
+          mbar_arrive_expect_tx(&full[stage],
+                                Cfg::A_BYTES + Cfg::B_BYTES + (xload ? Cfg::X_BYTES : 0));
           tma_load_2d(a_s, &tmA, &full[stage], kb * Cfg::BK, m0);
 #pragma unroll
           for (int c = 0; c < BN / 64; c++)
             tma_load_2d(b_s + c * (Cfg::BK * 128), &tmB, &full[stage], n0 + c * 64, kb * Cfg::BK);
+          if (xload)
+            tma_load_2d(b_s + Cfg::B_BYTES, &tmR, &full[stage], n0 + (kb - kb0) * 64, m0);
           issued[stage] = true;
           issued_phase[stage] = phase;
           if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
@@ -231,6 +262,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint64_t ad = sdesc_sw128(a_addr + kk * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(b_addr + kk * 2048, Cfg::BK * 128, 1024);
             mma_ss(d_tmem, ad, bd, idesc, (kb != kb0 || kk != 0) ? 1u : 0u);
+          }
+          if (RX && rx && kb - kb0 < BN / 64) {
+            // + R: accumulator columns 64 i + 16 kk .. + 15 get R_i's columns times I_16 (after
+            // the first block's products, which set every column)
+            constexpr uint32_t idesc_x = idesc_bf16(128, 16, false, true);
+            const uint32_t x_addr = b_addr + Cfg::B_BYTES;
+            const uint64_t id_desc = sdesc_sw128(smem_u32(smem + Cfg::OFF_ID), Cfg::BK * 128, 1024);
+            const int i = kb - kb0;
+#pragma unroll
+            for (int kk = 0; kk < Cfg::BK / 16; kk++)
+              mma_ss(d_tmem + 64 * i + 16 * kk, sdesc_sw128(x_addr + kk * 32, 16, 1024), id_desc,
+                     idesc_x, 1u);
           }
           mma_commit(&empty[stage]);
           if (++stage == Cfg::STAGES) { stage = 0; phase ^= 1u; }
@@ -277,7 +320,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[acc]);
         }
-        gemm_epilogue_chunk<EPI>(cur, bias, R, C, C32, row, M, N, n0 + c * 32);
+        if (RX && rx)   // the residual is in the accumulator already
+          gemm_epilogue_chunk<EPI_BIAS>(cur, bias, nullptr, C, C32, row, M, N, n0 + c * 32);
+        else
+          gemm_epilogue_chunk<EPI>(cur, bias, R, C, C32, row, M, N, n0 + c * 32);
       }
       acc ^= 1u;
       if (acc == 0) acc_phase ^= 1u;
