@@ -49,8 +49,13 @@ struct GemmCfg {
   static constexpr int STAGES = RX ? (BN == 256 ? 3 : (BN == 128 ? 4 : 5))
                                    : (BN == 256 ? 4 : (BN == 128 ? 6 : 8));
   static constexpr int OFF_ID = STAGES * STAGE_BYTES;       // RX: 16 x 64 bf16, the identity
-  static constexpr int OFF_BAR = OFF_ID + (RX ? 16 * 128 : 0);
+  // bf16 outputs leave through TMA stores: per epilogue warp NSTG staging tiles of 32 rows x 32
+  // columns (2 KB, 64-byte swizzled), two when they fit
+  static constexpr int OFF_STG = OFF_ID + (RX ? 16 * 128 : 0);
+  static constexpr int STG_TILE = 32 * 32 * 2;
   static constexpr int BAR_BYTES = 256;
+  static constexpr int NSTG = OFF_STG + 8 * 2 * STG_TILE + BAR_BYTES + 1024 <= 232448 ? 2 : 1;
+  static constexpr int OFF_BAR = OFF_STG + 8 * NSTG * STG_TILE;
   static constexpr int SMEM = OFF_BAR + BAR_BYTES + 1024;  // + alignment slack
   static constexpr int TMEM_COLS = 2 * BN;
   static_assert(SMEM <= 232448, "shared memory budget");
@@ -135,12 +140,57 @@ __device__ __forceinline__ void gemm_epilogue_chunk(const uint32_t (&r)[32], con
   for (int v = 0; v < 4; v++) reinterpret_cast<uint4*>(C + row * N + n)[v] = out[v];
 }
 
+// The bf16 epilogues' 32 output values of one row as packed pairs (the math of gemm_epilogue_chunk;
+// rows past M produce values that the clipped TMA store does not write).
+template <int EPI>
+__device__ __forceinline__ void gemm_epilogue_pack(const uint32_t (&r)[32], const bf16* __restrict__ bias,
+                                                   const bf16* __restrict__ R, int64_t row, int64_t M,
+                                                   int N, int n, uint32_t (&ow)[16]) {
+  uint4 bvec[4];
+  if (bias) {
+#pragma unroll
+    for (int v = 0; v < 4; v++) bvec[v] = __ldg(reinterpret_cast<const uint4*>(bias + n) + v);
+  } else {
+#pragma unroll
+    for (int v = 0; v < 4; v++) bvec[v] = make_uint4(0, 0, 0, 0);
+  }
+  uint4 rvec[4] = {};
+  if ((EPI == EPI_BIAS_RESIDUAL || EPI == EPI_SILU_GRAD) && row < M) {
+#pragma unroll
+    for (int v = 0; v < 4; v++) rvec[v] = __ldcs(reinterpret_cast<const uint4*>(R + row * N + n) + v);
+  }
+#pragma unroll
+  for (int v = 0; v < 4; v++) {
+    const uint32_t* bw = reinterpret_cast<const uint32_t*>(&bvec[v]);
+    const uint32_t* rw = reinterpret_cast<const uint32_t*>(&rvec[v]);
+#pragma unroll
+    for (int e = 0; e < 4; e++) {
+      float lo = __uint_as_float(r[v * 8 + 2 * e]) + bf16_lo(bw[e]);
+      float hi = __uint_as_float(r[v * 8 + 2 * e + 1]) + bf16_hi(bw[e]);
+      if (EPI == EPI_BIAS_SILU) {
+        lo = silu_tanh(lo);
+        hi = silu_tanh(hi);
+      } else if (EPI == EPI_SILU_GRAD) {
+        const float sl = fmaf(0.5f, sm100::tanh_approx(0.5f * lo), 0.5f);
+        const float sh = fmaf(0.5f, sm100::tanh_approx(0.5f * hi), 0.5f);
+        lo = bf16_lo(rw[e]) * sl * fmaf(lo, 1.0f - sl, 1.0f);
+        hi = bf16_hi(rw[e]) * sh * fmaf(hi, 1.0f - sh, 1.0f);
+      } else if (EPI == EPI_BIAS_RESIDUAL) {
+        lo += bf16_lo(rw[e]);
+        hi += bf16_hi(rw[e]);
+      }
+      ow[4 * v + e] = pack_bf16x2(lo, hi);
+    }
+  }
+}
+
 constexpr int kGemmThreads = 320;  // producer warp, MMA warp, 8 epilogue warps
 
 template <int BN, int EPI, bool RX = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmR, int64_t M, int N, int K,
+                   const __grid_constant__ CUtensorMap tmR, const __grid_constant__ CUtensorMap tmC,
+                   int64_t M, int N, int K,
                    const bf16* __restrict__ bias, const bf16* __restrict__ R, bf16* __restrict__ C,
                    float* __restrict__ C32, int splits) {
   static_assert(!RX || EPI == EPI_BIAS_RESIDUAL, "the residual on the tensor core is f2's");
@@ -181,6 +231,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     prefetch_tensormap(&tmA);
     prefetch_tensormap(&tmB);
     if (rx) prefetch_tensormap(&tmR);
+    if (EPI != EPI_F32 && EPI != EPI_RED_F32) prefetch_tensormap(&tmC);
   }
   if (RX) {
     // the 16 x 16 identity as an MN-major B operand (128-byte swizzled rows of 64 columns, of
@@ -294,6 +345,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;
     constexpr int HALF = BN / 2, CHUNKS = HALF / 32;
+    // bf16 outputs: each 32 x 32 chunk goes through this warp's staging tiles and a TMA store
+    constexpr bool TS = EPI != EPI_F32 && EPI != EPI_RED_F32;
+    uint8_t* stg = smem + Cfg::OFF_STG + (warp - 2) * Cfg::NSTG * Cfg::STG_TILE;
+    uint32_t nstore = 0;
     uint32_t acc = 0, acc_phase = 0;
     for (int64_t u = blockIdx.x; u < num_units; u += gridDim.x) {
       const int64_t t = u / splits;
@@ -320,14 +375,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[acc]);
         }
-        if (RX && rx)   // the residual is in the accumulator already
-          gemm_epilogue_chunk<EPI_BIAS>(cur, bias, nullptr, C, C32, row, M, N, n0 + c * 32);
-        else
+        if constexpr (TS) {
+          uint32_t ow[16];
+          if (RX && rx)   // the residual is in the accumulator already
+            gemm_epilogue_pack<EPI_BIAS>(cur, bias, nullptr, row, M, N, n0 + c * 32, ow);
+          else
+            gemm_epilogue_pack<EPI>(cur, bias, R, row, M, N, n0 + c * 32, ow);
+          // the staging tile's previous TMA store has read it (at most NSTG - 1 still reading)
+          uint8_t* tile = stg + (nstore % Cfg::NSTG) * Cfg::STG_TILE;
+          if (lane == 0) bulk_wait_read<Cfg::NSTG - 1>();
+          __syncwarp();
+          // row `lane` of the 32 x 32 tile: 64 bytes, 16-byte unit u at u ^ ((lane >> 1) & 3)
+#pragma unroll
+          for (int u = 0; u < 4; u++)
+            *reinterpret_cast<uint4*>(tile + lane * 64 + ((u ^ ((lane >> 1) & 3)) << 4)) =
+                make_uint4(ow[4 * u], ow[4 * u + 1], ow[4 * u + 2], ow[4 * u + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmC, tile, n0 + c * 32, (int)(mb * Cfg::BM) + q * 32);
+            bulk_commit();
+          }
+          nstore++;
+        } else {
           gemm_epilogue_chunk<EPI>(cur, bias, R, C, C32, row, M, N, n0 + c * 32);
+        }
       }
       acc ^= 1u;
       if (acc == 0) acc_phase ^= 1u;
     }
+    // the stores have completed before the CTA (and its shared memory) goes away
+    if (TS && lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();

@@ -43,6 +43,21 @@ inline bool make_map_bf16(CUtensorMap* map, const void* base, uint64_t inner, ui
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D bf16 tensor map with a box of 32 x 32 elements and 64-byte swizzling: the staging tiles of
+// the GEMM epilogue's TMA stores.
+inline bool make_map_bf16_store(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                                uint64_t ld) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // The same for an fp32 matrix (box_inner * 4 must be 128).
 inline bool make_map_f32(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
                          uint64_t ld, uint32_t box_inner, uint32_t box_outer) {
@@ -69,7 +84,7 @@ hstu_status_t launch_gemm_cfg(int64_t M, int N, int K, const bf16* A, const bf16
                               const bf16* bias, const bf16* R, bf16* C, cudaStream_t st,
                               float* C32, int splits, int64_t b_rows) {
   using Cfg = GemmCfg<BN, RX>;
-  CUtensorMap ta, tb, tr;
+  CUtensorMap ta, tb, tr, tc;
   // B may hold fewer than K rows: the tensor map's zero fill stands in for the rest
   if (b_rows < 0 || b_rows > K) b_rows = K;
   if (!make_map_bf16(&ta, A, K, M, K, 64, 128)) return HSTU_ERR_CUDA;
@@ -78,6 +93,11 @@ hstu_status_t launch_gemm_cfg(int64_t M, int N, int K, const bf16* A, const bf16
     if (!make_map_bf16(&tr, R, N, M, N, 64, 128)) return HSTU_ERR_CUDA;   // the residual [M, N]
   } else {
     tr = ta;   // not read
+  }
+  if (EPI != EPI_F32 && EPI != EPI_RED_F32) {
+    if (!make_map_bf16_store(&tc, C, N, M, N)) return HSTU_ERR_CUDA;   // bf16 output [M, N]
+  } else {
+    tc = ta;   // not used: fp32 outputs are stored by the threads
   }
   auto kern = gemm_tc_kernel<BN, EPI, RX>;
   // set on every launch: the attribute is per device and the call is cheap
@@ -92,7 +112,7 @@ hstu_status_t launch_gemm_cfg(int64_t M, int N, int K, const bf16* A, const bf16
   splits = (kblocks + kbps - 1) / kbps;
   const int64_t units = ((M + 127) / 128) * (N / BN) * splits;
   const int grid = (int)(units < num_sms() ? units : num_sms());
-  kern<<<grid, kGemmThreads, Cfg::SMEM, st>>>(ta, tb, tr, M, N, K, bias, R, C, C32, splits);
+  kern<<<grid, kGemmThreads, Cfg::SMEM, st>>>(ta, tb, tr, tc, M, N, K, bias, R, C, C32, splits);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? HSTU_OK : HSTU_ERR_CUDA;
 }
