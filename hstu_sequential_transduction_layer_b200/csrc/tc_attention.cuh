@@ -38,7 +38,9 @@
 // TMEM: NSB buffers of S (128 columns each; hd = 64: three, hd = 128: two) that rotate over the
 // (query tile, key tile) slots, then O_A | O_B (hd columns each).  Each warp writes its P over the
 // first 32 of its 64 S columns once it has read them; with three buffers the S of the next slots
-// is computed while the pointwise warps work on the current one.
+// is computed while the pointwise warps work on the current one.  With two (hd = 128) each query
+// tile's next S waits for its PV product, so the PV product starts on the first half of the keys
+// as soon as their P is written.
 //
 // The pointwise stage works on pairs of scores with the sm_100 packed f32x2 instructions: per pair,
 // two 32-bit shared loads of the two halved position biases, one
@@ -634,7 +636,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
   // [2][2]: query tile x's P of its t-th computed tile is in TMEM, on barrier [x][t & 1]: with
   // three S buffers the pointwise warps can be two tiles ahead of the PV products
   uint64_t* p_full = buf_free + 2 * Cfg::NSB;
-  uint64_t* o_full = p_full + 4;             // [2]
+  // [2][2], hd = 128 (two S buffers, where the PV product is on the critical path): the P of chunk
+  // 0 of every pointwise warp of query tile x (keys 0..31 and 64..95) is in TMEM, on barrier
+  // [x][t & 1]; the PV product starts on those keys while chunk 1 is computed
+  uint64_t* p_half = p_full + 4;
+  uint64_t* o_full = p_half + 4;             // [2]
   uint64_t* o_empty = o_full + 2;            // [2]
   uint64_t* q_full = o_empty + 2;
   uint64_t* q_empty = q_full + 1;
@@ -663,6 +669,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
     for (int x = 0; x < 2; x++) {
       mbar_init(&p_full[2 * x], ATT_PW_WARPS);
       mbar_init(&p_full[2 * x + 1], ATT_PW_WARPS);
+      mbar_init(&p_half[2 * x], ATT_PW_WARPS);
+      mbar_init(&p_half[2 * x + 1], ATT_PW_WARPS);
       mbar_init(&o_full[x], 1);
       mbar_init(&o_empty[x], ATT_PW_WARPS);
     }
@@ -885,12 +893,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         for (int j = 0; j < nk && ok; j++) {
           const uint32_t gj = g + j;
           if (mine && j <= last) {
-            if (!__all_sync(FULL, mbar_wait(&p_full[2 * x + (pv_count & 1u)], (pv_count >> 1) & 1u,
-                                            abort_flag))) {
+            // hd = 128: the first half of the keys as soon as it is written (see p_half)
+            uint64_t* first = Cfg::NSB == 2 ? &p_half[2 * x + (pv_count & 1u)]
+                                            : &p_full[2 * x + (pv_count & 1u)];
+            if (!__all_sync(FULL, mbar_wait(first, (pv_count >> 1) & 1u, abort_flag))) {
               ok = false;
               break;
             }
-            pv_count++;
             if (j == 0 &&
                 !__all_sync(FULL, mbar_wait(&o_empty[x], (o_count & 1u) ^ 1u, abort_flag))) {
               ok = false;
@@ -901,11 +910,29 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             // slot's S buffer, keys 0..63 at columns 0..31 and keys 64..127 at columns 64..95
             const uint32_t b = (2 * gj + x) % Cfg::NSB;
             const uint64_t vd = v_desc0 + (uint64_t)(((gj % Cfg::NST) * Cfg::STAGE_BYTES) >> 4);
+            auto pv_keys = [&](int kk) {
+              mma_ts(o_tmem, tmem + b * 128 + (kk & 3) * 8 + (kk >> 2) * 64,
+                     vd + (uint64_t)((kk * 2048) >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+            };
+            if (Cfg::NSB == 2) {
+              // keys 0..31 and 64..95 (chunk 0 of both warps of each lane quadrant), then the rest
+              if (elect_one()) pv_keys(0), pv_keys(1), pv_keys(4), pv_keys(5);
+              __syncwarp();
+              if (!__all_sync(FULL, mbar_wait(&p_full[2 * x + (pv_count & 1u)], (pv_count >> 1) & 1u,
+                                              abort_flag))) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            pv_count++;
             if (elect_one()) {
+              if (Cfg::NSB == 2) {
+                pv_keys(2), pv_keys(3), pv_keys(6), pv_keys(7);
+              } else {
 #pragma unroll
-              for (int kk = 0; kk < ATT_BN / 16; kk++)
-                mma_ts(o_tmem, tmem + b * 128 + (kk & 3) * 8 + (kk >> 2) * 64,
-                       vd + (uint64_t)((kk * 2048) >> 4), idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                for (int kk = 0; kk < ATT_BN / 16; kk++) pv_keys(kk);
+              }
               mma_commit(&buf_free[2 * b + x]);
               if (j == last) mma_commit(&o_full[x]);
               mma_commit(&kv_empty[gj % Cfg::NST]);
@@ -1121,6 +1148,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
             }
           }
           tmem_st16(s_col + 16 * c, pk);
+          if (Cfg::NSB == 2 && c == 0) {   // hd = 128: chunk 0's P is in TMEM, the PV may start
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_half[2 * x + (tcount & 1u)]);
+          }
         }
         if (!ok) break;
         tmem_st_wait();
