@@ -337,6 +337,7 @@ struct AttnParams {
   float* av;                // [T, H*hd] fp32
   int64_t T;
   int dynamic;              // 1: CTAs claim items from the list's counter; 0: CTA b takes b, b+grid, ...
+  int zigzag;               // static assignment in alternating directions (see static_item)
   // candidate mode only: the candidates' timestamps [T_cand] and UVQK rows (for each candidate's
   // own term); ts, the K/V tensor map and the schedule's key rows are then the history's
   const int64_t* cts;
@@ -590,9 +591,15 @@ __device__ __forceinline__ bool publish_item(uint32_t k, uint64_t* item_full, ui
   return true;
 }
 
-// Static assignment: the CTA's k-th item is list entry blockIdx.x + k * gridDim.x (-1 past the end).
-__device__ __forceinline__ int64_t static_item(uint32_t k, const AttnSchedule& sch, int64_t n_items) {
-  const int64_t it = (int64_t)blockIdx.x + (int64_t)k * gridDim.x;
+// Static assignment: the CTA's k-th item is entry k * gridDim.x + blockIdx.x of the list (-1 past
+// the end); with `zigzag`, odd waves are taken in decreasing CTA order (k * gridDim.x +
+// gridDim.x - 1 - blockIdx.x), so that, the list being heaviest first, the CTA that took a wave's
+// heaviest item takes the next wave's lightest.
+__device__ __forceinline__ int64_t static_item(uint32_t k, const AttnSchedule& sch, int64_t n_items,
+                                               bool zigzag) {
+  const int64_t g = gridDim.x;
+  const bool rev = zigzag && (k & 1u);
+  const int64_t it = (int64_t)k * g + (rev ? g - 1 - (int64_t)blockIdx.x : (int64_t)blockIdx.x);
   return it < n_items ? sch.items[it] : -1;
 }
 
@@ -724,7 +731,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         ok = __shfl_sync(0xffffffffu, ok, 0);
         item = __shfl_sync(0xffffffffu, item, 0);
       } else {
-        item = static_item(k, sch, n_items);
+        item = static_item(k, sch, n_items, prm.zigzag != 0);
       }
       if (!ok || item < 0) break;
       const ItemGeom ig = item_geom<CAND>(item, sch);
@@ -837,7 +844,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         if (lane == 0) item = read_item(k, item_full, item_empty, item_ring, abort_flag);
         item = __shfl_sync(FULL, item, 0);
       } else {
-        item = static_item(k, sch, n_items);
+        item = static_item(k, sch, n_items, prm.zigzag != 0);
       }
       if (item < 0) break;
       const ItemGeom ig = item_geom<CAND>(item, sch);
@@ -983,7 +990,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 1)
         if (lane == 0) item = read_item(k, item_full, item_empty, item_ring, abort_flag);
         item = __shfl_sync(FULL, item, 0);
       } else {
-        item = static_item(k, sch, n_items);
+        item = static_item(k, sch, n_items, prm.zigzag != 0);
       }
       if (item < 0) break;
       const ItemGeom ig = item_geom<CAND>(item, sch);

@@ -64,8 +64,10 @@ def test_f1_kernel(hstu, T, d, hd):
     assert_bf16_close(host(out), ref, "f1")
 
 
+# (the residual joins the accumulator on the tensor core when K = wv is at most 512 and at least
+# the tile width; (77, 256, 128) and (260, 256, 1024) take the epilogue's residual loads instead)
 @pytest.mark.parametrize("T,d,wv", [(1, 64, 64), (300, 128, 128), (200, 192, 256), (129, 512, 512),
-                                    (260, 256, 1024)])
+                                    (77, 256, 128), (260, 256, 1024)])
 def test_f2_kernel(hstu, T, d, wv):
     rng = np.random.default_rng(T + wv)
     G = round_bf16(rng.standard_normal((T, wv)))

@@ -60,3 +60,43 @@ def test_schedule_is_a_batched_heaviest_first_permutation(hstu, lengths, hd, H):
         assert int(batch_pairs[0]) == int(group_pairs[b0]) - 1   # heaviest item first
         pos += cnt
     assert pos == n_items
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("lengths,hd,H", [([300, 1, 129, 513, 0, 2000, 256, 257], 64, 2),
+                                          ([700] * 40 + [1] * 9 + [5000], 64, 3),
+                                          ([8192] * 3 + [4000, 2500, 700, 100, 1], 64, 8),
+                                          ([4096, 4096, 100, 3000, 700], 128, 4)])
+def test_backward_schedule_is_a_heaviest_first_permutation(hstu, lengths, hd, H):
+    """The attention backward's schedule (items: sequence | key tile << 32 | head << 48): every
+    (sequence, key tile, head) item exactly once, by non-increasing cost (the query tiles the item
+    visits, tiles - key tile), which the query-stationary dQ kernel at head dim 128 reads as the
+    key tiles of query tile tiles - 1 - key tile."""
+    d = H * hd
+    lengths = np.asarray(lengths, dtype=np.int64)
+    offsets = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    T = int(offsets[-1])
+    B = len(lengths)
+    uvqk = torch.zeros((T, 4 * d), dtype=torch.bfloat16, device="cuda")
+    dav = torch.zeros((T, d), dtype=torch.bfloat16, device="cuda")
+    max_len = int(lengths.max())
+    s = hstu.make_shape(B, T, max_len, d, H, hd, hd, hstu.HSTU_BF16, 0, 0)
+    ws = torch.zeros(int(hstu.library().hstu_attention_bwd_workspace_size(s)), dtype=torch.uint8,
+                     device="cuda")
+    f = lambda: torch.empty((T, d), dtype=torch.float32, device="cuda")
+    hstu.hstu_attention_bwd(s, uvqk, dev(offsets), None, None, None, None, 1.0, dav, f(), f(), f(),
+                            None, None, ws)
+    torch.cuda.synchronize()
+    assert hstu.device_status() == hstu.HSTU_OK
+    raw = ws.cpu().numpy().view(np.int64)
+    n_items = int(raw[0])
+    seqinfo_words = ((16 * B + 255) // 256) * 256 // 8
+    items = raw[32 + seqinfo_words: 32 + seqinfo_words + n_items]
+    seq, jt, head = items & 0xFFFFFFFF, (items >> 32) & 0xFFFF, items >> 48
+    tiles = (lengths + 127) // 128
+    expected = sorted((s_, j, h) for s_ in range(B) for h in range(H) for j in range(tiles[s_]))
+    got = sorted(zip(seq.tolist(), jt.tolist(), head.tolist()))
+    assert got == expected                                # each item exactly once
+    cost = tiles[seq] - jt
+    assert np.all(np.diff(cost) <= 0), "heaviest first"
+    assert int(cost[0]) == int(tiles.max())
