@@ -340,7 +340,8 @@ def run_ours(args, rank, world, local_rank):
     result = {
         "metric": METRIC, "value": round(tokens_per_s, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32" if w.dtype == "f32" else "bf16",
         "data": "synthetic (seeded; shapes of the pages' workloads)",
         "config": {"workload": workload_text(w, max_len),
                    "global_batch_tokens": job_tokens, "seq_len": max_len,
