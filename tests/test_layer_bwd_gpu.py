@@ -12,7 +12,8 @@ import torch
 
 import oracle
 import workloads
-from tests.gpu_util import assert_bwd_close, assert_layer_part_close, dev, host, round_bf16
+from tests.gpu_util import (assert_bf16_close, assert_bwd_close, assert_layer_part_close, dev,
+                            host, round_bf16)
 from workloads import random_case
 
 
@@ -69,11 +70,20 @@ def _case(seed, lengths, H, bias, P=96, Tb=24, hd=64):
     return inp, dY
 
 
+# Outputs held to the forward's mean bound (BF16_MEAN_REL) because they meet it on every case
+# (observed mean|err|/rms(ref), all cases here: dln_b 1.2-1.4e-3, dtime 1.0-1.8e-3); the others keep
+# the chain-of-roundings bound (observed: dW1 2.6-3.0e-3, dW2 2.0-2.5e-3, db1 1.6-2.4e-3,
+# dln_w 1.7-2.4e-3, dpos 0.8-2.5e-3, dX - dY 3.9-4.0e-3; db2 is exact)
+FORWARD_BOUND = ("dln_b", "dtime")
+
+
 def _compare(got, ref, dY, what):
     assert_layer_part_close(got["dX"], ref["dX"], dY, f"dX ({what})")
     for k in ("dW1", "db1", "dW2", "db2", "dln_w", "dln_b", "dpos", "dtime"):
         if ref[k] is None:
             assert got[k] is None
+        elif k in FORWARD_BOUND:
+            assert_bf16_close(got[k], ref[k], f"{k} ({what})")
         else:
             assert_bwd_close(got[k], ref[k], f"{k} ({what})")
 
