@@ -104,15 +104,38 @@ __global__ void __launch_bounds__(SL_THREADS) sl_select_kernel(const int64_t* __
         if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
       }
       __syncthreads();
-      if (tid == 0) {
-        int64_t cum = 0;
-        uint32_t d = 0;
-        for (; d < 255; d++) {
-          if (cum + hist[d] >= k) break;
-          cum += hist[d];
+      if (tid < 32) {
+        // the digit: the first bin d < 255 at which the running count reaches k (else 255), found
+        // by one warp: lane l sums bins 8l .. 8l+7, a warp scan gives each lane's running count,
+        // and the first lane to reach k walks its eight bins
+        const int lane = tid;
+        uint32_t h[8];
+        int64_t sum = 0;
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+          h[j] = hist[8 * lane + j];
+          sum += h[j];
         }
-        sel_digit = d;
-        sel_k = k - cum;
+        int64_t incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int64_t y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, incl >= k);
+        const int first = hit ? __ffs(hit) - 1 : 31;
+        if (lane == first) {
+          int64_t cum = incl - sum;
+          uint32_t d = 8 * lane;
+#pragma unroll 1
+          for (int j = 0; j < 8; j++) {
+            d = 8 * lane + j;
+            if (d == 255 || cum + h[j] >= k) break;
+            cum += h[j];
+          }
+          sel_digit = d;
+          sel_k = k - cum;
+        }
       }
       __syncthreads();
       prefix |= sel_digit << shift;
@@ -122,20 +145,31 @@ __global__ void __launch_bounds__(SL_THREADS) sl_select_kernel(const int64_t* __
     }
     const uint32_t K = prefix;
     const int64_t take_eq = k;
-    // ordered compaction: keep key < K, and the first take_eq keys equal to K
-    int64_t carry_eq = 0, carry_keep = 0;
-    for (int64_t base = 0; base < n; base += SL_THREADS) {
-      const int64_t i = base + tid;
-      const bool valid = i < n;
-      const uint32_t key = valid ? keys[a + i] : 0xffffffffu;
-      const bool lt = valid && key < K, eq = valid && key == K;
-      int64_t eq_tot, keep_tot;
-      const int64_t eq_before = block_exclusive_scan(eq ? 1 : 0, scratch, eq_tot);
-      const bool keep = lt || (eq && carry_eq + eq_before < take_eq);
-      const int64_t keep_before = block_exclusive_scan(keep ? 1 : 0, scratch, keep_tot);
-      if (keep) dst[carry_keep + keep_before] = a + i;
-      carry_eq += eq_tot;
-      carry_keep += keep_tot;
+    // ordered compaction: keep key < K, and the first take_eq keys equal to K.  Thread t owns the
+    // contiguous segment [t * per, (t + 1) * per): one pass counts its keys equal to K, a block scan
+    // gives the equal keys before it, a second pass decides and counts what it keeps, a second scan
+    // gives the kept rows before it, and a third pass writes them in order
+    const int64_t per = (n + SL_THREADS - 1) / SL_THREADS;
+    const int64_t i0 = (int64_t)tid * per < n ? (int64_t)tid * per : n;
+    const int64_t i1 = i0 + per < n ? i0 + per : n;
+    int64_t n_eq = 0;
+    for (int64_t i = i0; i < i1; i++) n_eq += keys[a + i] == K ? 1 : 0;
+    int64_t tot;
+    const int64_t eq_before = block_exclusive_scan(n_eq, scratch, tot);
+    int64_t n_keep = 0, seen_eq = eq_before;
+    for (int64_t i = i0; i < i1; i++) {
+      const uint32_t key = keys[a + i];
+      const bool eq = key == K;
+      n_keep += (key < K || (eq && seen_eq < take_eq)) ? 1 : 0;
+      seen_eq += eq ? 1 : 0;
+    }
+    int64_t pos = block_exclusive_scan(n_keep, scratch, tot);
+    seen_eq = eq_before;
+    for (int64_t i = i0; i < i1; i++) {
+      const uint32_t key = keys[a + i];
+      const bool eq = key == K;
+      if (key < K || (eq && seen_eq < take_eq)) dst[pos++] = a + i;
+      seen_eq += eq ? 1 : 0;
     }
   }
 }
