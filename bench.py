@@ -612,7 +612,9 @@ def run_candidates(args, rank, world, local_rank):
                    "l2": "flushed between timed steps (256 MB write, outside the events)"},
         "roofline": {"bound": "tensor", "kernel": "candidate_attention",
                      "achieved": round(attn_tflops, 2), "peak": tpk, "unit": "TFLOP/s",
-                     "frac": round(attn_tflops / tpk, 4), "traffic": None,
+                     "frac": round(attn_tflops / tpk, 4),
+                     "traffic": profiled_traffic(f"{w.name}_{M // 1024}k", "candidate_attention")
+                     if M % 1024 == 0 else None,
                      "peak_source": f"{peaks_src} bf16 burst (MEASURED_PEAKS.json)"
                      if peaks_src == "measured" else "fallback 1590 TFLOP/s"},
         "kernels": kernels,

@@ -51,7 +51,7 @@ def test_bench_reads_traffic_only_for_the_source_captured():
     spec.loader.exec_module(bench)
     for path in _summaries():
         name = os.path.basename(path)[:-3]
-        m = re.fullmatch(r"(attention_tc_kernel|attention_bwd_kernel)_(\w+)", name)
+        m = re.fullmatch(r"(attention_tc_kernel|attention_bwd_kernel|candidate_attention)_(\w+)", name)
         if not m:
             continue
         f = _fields(path)
